@@ -1,0 +1,434 @@
+"""Benchmark of the KDA core on B200.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one kda_chunk_fwd over the grouped-value-head training-shape
+workload (B=4, H=16, HV=32, T=8192, Dk=Dv=128, chunk=64, bf16 activations,
+q/k L2-norm, beta sigmoid and bounded gate in-kernel), inputs resident in HBM.
+Rank 0 prints ONE JSON line with the throughput in token-heads/s, its fraction
+of the BF16 tensor-core and HBM rooflines, the end-to-end number through the
+Python API with host buffers, the decode step (B=256, H=HV=32, D=128, fp32
+state, 512 consecutive steps) in GB/s, the segmented KCP pass, and the FP64
+oracle timed on the host cores as a reported baseline.
+
+Multi-GPU (torchrun): every rank runs its own batch of the same workload (weak
+scaling, no collective on the data path); the time is the max over ranks.
+--impl reference times the FP64 oracle (the only reference this method has)
+on rank 0 on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk_kda fwd tokens·heads/s + % bf16 TC peak; kda_step decode HBM GB/s"
+UNIT = "tokens·heads/s"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def chunk_flops_per_token_head(Dk, Dv, C):
+    # 6 Dk Dv (W S, (Q Gamma) S, K^T U) + C (3 Dk + 2 Dv) (A_kk, A_qk, W, Ut, A_qk U) + C^2/3 (solve)
+    return 6 * Dk * Dv + C * (3 * Dk + 2 * Dv) + C * C / 3.0
+
+
+def chunk_bytes(w):
+    """Algorithmic HBM bytes of one kda_chunk_fwd: every input read once, o written once,
+    initial/final state once per chain."""
+    es = 2 if w.dtype == "bf16" else 4
+    ntok = w.B * w.T
+    b = ntok * w.H * w.Dk * es * 2            # q, k
+    b += ntok * w.HV * w.Dv * es * 2          # v, o
+    b += ntok * w.HV * w.Dk * es              # g (raw z)
+    b += ntok * w.HV * es                     # beta
+    b += w.B * w.HV * w.Dk * w.Dv * 4 * (1 + (1 if w.s0_std is not None else 0))  # S_T (+S0)
+    return b
+
+
+def decode_bytes(w):
+    es = 2 if w.dtype == "bf16" else 4
+    b = 2 * w.B * w.HV * w.Dk * w.Dv * 4      # state read + write
+    b += w.B * w.H * w.Dk * es * 2 + w.B * w.HV * (w.Dv * 2 + w.Dk + 1) * es   # q,k,v,o,z,beta
+    return b
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def dist_setup(n):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+def cpu_baseline(w, inp_cpu, target_s=12.0):
+    """Time the FP64 oracle, as it stands, on a bounded sample of workload w:
+    the first n_chains (b, hv) chains over the first T_s tokens."""
+    import oracle
+    import numpy as np
+    import torch
+
+    def f64(t):
+        return None if t is None else t.to(torch.float64).numpy()
+
+    cores = oracle.num_threads()
+
+    def run(nb, nh, T_s):
+        sl = {n: inp_cpu[n][:nb, :T_s] for n in ("q", "k", "v", "g", "beta")}
+        hq = max(1, nh // (w.HV // w.H))
+        t0 = time.perf_counter()
+        oracle.kda_fwd(f64(sl["q"][:, :, :hq]), f64(sl["k"][:, :, :hq]),
+                       f64(sl["v"][:, :, :nh]), f64(sl["g"][:, :, :nh]), f64(sl["beta"][:, :, :nh]),
+                       A_log=f64(inp_cpu["A_log"][:nh]),
+                       dt_bias=None if inp_cpu["dt_bias"] is None else f64(inp_cpu["dt_bias"][:nh]))
+        return time.perf_counter() - t0
+
+    # Calibrate on a small sample, then size the sample for about target_s seconds.
+    nh = min(w.HV, max(2, cores))
+    t_cal = run(1, nh, 256)
+    per_token = t_cal / (256.0)
+    T_s = int(min(w.T, max(256, target_s / max(per_token, 1e-9))))
+    T_s = max(64, (T_s // 64) * 64)
+    dt = run(1, nh, T_s)
+    units = nh * T_s
+    return {"value": units / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": "FP64 oracle, %d value heads x %d tokens of the B=4,HV=32,T=8192 workload "
+                      "(%.1f s wall)" % (nh, T_s, dt)}
+
+
+def run_reference(args):
+    """--impl reference: the FP64 oracle on rank 0, one bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    import oracle
+    import workloads
+    w = workloads.workload("gva_bf16")
+    # Only the sampled slice is generated: the first value heads of batch row 0.
+    cores = oracle.num_threads()
+    nh = min(w.HV, max(2, cores))
+    T_s = 1024
+    ws = workloads.workload("gva_bf16", B=1, T=T_s)
+    inp = workloads.chunk_inputs(ws)
+
+    def f64(t):
+        return None if t is None else t.to(torch.float64).numpy()
+
+    hq = max(1, nh // (w.HV // w.H))
+    arrays = (f64(inp["q"][:, :, :hq]), f64(inp["k"][:, :, :hq]), f64(inp["v"][:, :, :nh]),
+              f64(inp["g"][:, :, :nh]), f64(inp["beta"][:, :, :nh]))
+    kw = dict(A_log=f64(inp["A_log"][:nh]), dt_bias=f64(inp["dt_bias"][:nh]))
+    for _ in range(args.warmup):
+        oracle.kda_fwd(*arrays, **kw)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.kda_fwd(*arrays, **kw)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = nh * T_s / dt
+    sample = "FP64 oracle, %d value heads x %d tokens of the B=4,HV=32,T=8192 workload per step" % (nh, T_s)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "gva_bf16: B=4 H=16 HV=32 T=8192 Dk=Dv=128 chunk=64 (sampled)",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_launches(fn, n, stream):
+    """n launches of fn with CUDA events around each one on `stream`; returns ms per launch."""
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    evs[0].record(stream)
+    for i in range(n):
+        fn(i)
+        evs[i + 1].record(stream)
+    evs[-1].synchronize()
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(n)]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--decode-steps", type=int, default=512)
+    ap.add_argument("--no-extras", action="store_true", help="only the headline workload")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    args.warmup = max(args.warmup, 3)
+
+    import torch
+    import gated_delta_rule_157_b200 as kda
+    import workloads
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    pk = peaks()
+
+    # ---------------- headline: chunked forward, B=4 HV=32 T=8192 -------------
+    w = workloads.workload("gva_bf16")
+    inp = workloads.chunk_inputs(w, seed=w.seed + 1000 * rank, device=dev)
+    o = torch.empty((w.B, w.T, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
+    S_T = torch.empty((w.B, w.HV, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+
+    def step(_i):
+        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                          A_log=inp["A_log"], dt_bias=inp["dt_bias"], S0=inp["S0"],
+                          chunk=w.chunk, algo=args.algo, o=o, S_T=S_T, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    kda.kda_device_status(stream)
+    clocks = Clocks(local)
+    barrier(world, dev)
+    clocks.start()
+    per = time_launches(step, args.steps, stream)
+    barrier(world, dev)
+    clk = clocks.stop()
+    kda.kda_device_status(stream)
+    ms_local = sum(per) / len(per)
+    ms = max_over_ranks(ms_local, world, dev)
+    units = w.token_heads
+    value = world * units / (ms * 1e-3)
+    flops = units * chunk_flops_per_token_head(w.Dk, w.Dv, w.chunk)
+    nbytes = chunk_bytes(w)
+    achieved_gbs = nbytes / (ms_local * 1e-3) / 1e9
+    tflops = flops / (ms_local * 1e-3) / 1e12
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "gva_bf16: B=4 H=16 HV=32 T=8192 Dk=Dv=128 chunk=64 per GPU, "
+                                   "bf16 q/k/v/z/beta, fp32 state; l2norm, beta sigmoid, gate in-kernel",
+                       "algo": args.algo, "l2": "inputs larger than L2 (%.2f GB read per step)"
+                                                % (nbytes / 1e9),
+                       "parallelism": "dp%d (independent batches per GPU)" % world},
+            "tc_peak_frac": tflops / pk["bf16_tflops"],
+            "useful_tflops": tflops,
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"], "traffic": None,
+                         "kernel": "kda_chunk_fwd (%s)" % args.algo,
+                         "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst)"},
+            "gpu_launches": args.steps}
+    if clk is not None:
+        line["clocks"] = clk
+
+    # ---------------- end to end through the API with host buffers ------------
+    host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
+    dev_in = {n: torch.empty_like(inp[n]) for n in host}
+    h_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    h_S = torch.empty(S_T.shape, dtype=S_T.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_o.numel() * h_o.element_size() + h_S.numel() * h_S.element_size()
+
+    def e2e_step(_i):
+        for n in host:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        kda.kda_chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"],
+                          A_log=inp["A_log"], dt_bias=inp["dt_bias"], S0=inp["S0"],
+                          chunk=w.chunk, algo=args.algo, o=o, S_T=S_T, stream=stream)
+        h_o.copy_(o, non_blocking=True)
+        h_S.copy_(S_T, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    barrier(world, dev)
+    n_e2e = max(3, min(args.steps, 10))
+    per_e2e = time_launches(e2e_step, n_e2e, stream)
+    barrier(world, dev)
+    ms_e2e = max_over_ranks(sum(per_e2e) / len(per_e2e), world, dev)
+    line["e2e"] = {"value": world * units / (ms_e2e * 1e-3), "unit": UNIT,
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                   "ms_per_step": ms_e2e, "api": "gated_delta_rule_157_b200.kda_chunk_fwd"}
+    del host, dev_in, h_o, h_S
+
+    if not args.no_extras:
+        line["decode"] = bench_decode(args, kda, workloads, dev, stream, pk, world, rank)
+        line["kcp"] = bench_kcp(args, kda, workloads, dev, stream, world, rank)
+        line["gpu_launches_extras"] = {"decode": line["decode"]["launches"],
+                                       "kcp": line["kcp"]["launches"]}
+
+    if rank == 0 and world == 1:
+        inp_cpu = workloads.chunk_inputs(workloads.workload("gva_bf16", B=1, T=8192))
+        line["cpu_baseline"] = cpu_baseline(w, inp_cpu)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[dev.index])
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_decode(args, kda, workloads, dev, stream, pk, world, rank):
+    """512 consecutive decode steps of B=256, H=HV=32, D=128 against a resident fp32 state."""
+    import torch
+    w = workloads.workload("decode_bf16")
+    S = workloads.decode_state(w, seed=w.seed + 1000 * rank, device=dev)
+    n = args.decode_steps
+    steps = [workloads.decode_step_inputs(w, i, seed=w.seed + 1000 * rank, device=dev)
+             for i in range(n)]
+    o = torch.empty((w.B, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        d = steps[i % n]
+        kda.kda_step(S, d["q"], d["k"], d["v"], d["g"], d["beta"], A_log=d["A_log"], o=o,
+                     stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier(world, dev)
+    per = time_launches(step, n, stream)
+    barrier(world, dev)
+    ms_local = sum(per) / len(per)
+    ms = max_over_ranks(ms_local, world, dev)
+    nb = decode_bytes(w)
+    gbs = nb / (ms_local * 1e-3) / 1e9
+    return {"workload": "decode_bf16: B=256 H=HV=32 Dk=Dv=128, fp32 state, %d consecutive steps" % n,
+            "value": world * nb / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "kernel": "kda_step"},
+            "launches": n, "l2": "state 512 MiB > L2"}
+
+
+def bench_kcp(args, kda, workloads, dev, stream, world, rank):
+    """Segmented forward of B=1, HV=16, T=65536 as 8 segments of 8192: segments
+    with transitions (one batched launch), the combine, and the rerun for o."""
+    import torch
+    w = workloads.workload("kcp_bf16")
+    inp = workloads.chunk_inputs(w, seed=w.seed + 1000 * rank, device=dev)
+    L = w.T // w.n_seg
+    seg = {n: inp[n].view(w.n_seg, L, *inp[n].shape[2:]) for n in ("q", "k", "v", "g", "beta")}
+    o = torch.empty((w.n_seg, L, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
+    S_loc = torch.empty((w.n_seg, w.HV, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+    M_loc = torch.empty((w.n_seg, w.HV, w.Dk, w.Dk), dtype=torch.float32, device=dev)
+    S_in = torch.empty((w.n_seg + 1, w.HV, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+    S_init = inp["S0"].view(w.HV, w.Dk, w.Dv)
+
+    def step(_i):
+        kda.kda_chunk_fwd(seg["q"], seg["k"], seg["v"], seg["g"], seg["beta"], A_log=inp["A_log"],
+                          chunk=w.chunk, algo=args.algo, o=o, S_T=S_loc, M_T=M_loc,
+                          output_transition=True, stream=stream)
+        kda.kda_compose(M_loc, S_loc, S_init, S_in=S_in, stream=stream)
+        kda.kda_chunk_fwd(seg["q"], seg["k"], seg["v"], seg["g"], seg["beta"], A_log=inp["A_log"],
+                          S0=S_in[:w.n_seg], chunk=w.chunk, algo=args.algo, o=o,
+                          output_final_state=False, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    barrier(world, dev)
+    k = max(3, min(args.steps, 10))
+    per = time_launches(step, k, stream)
+    barrier(world, dev)
+    ms = max_over_ranks(sum(per) / len(per), world, dev)
+    return {"workload": "kcp_bf16: B=1 H=HV=16 T=65536 as 8 x 8192, Dk=Dv=128",
+            "value": world * w.token_heads / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "launches": 3 * k}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,18 @@
+"""B200-native (sm_100a) Kimi Delta Attention core.
+
+Python binding of the C ABI in include/kda.h.  The entry points keep the
+library's names:
+
+  kda_chunk_fwd  chunk-parallel forward over whole sequences (o, S_T, M_T)
+  kda_step       single-token decode, state updated in place
+  kda_compose    KCP segment prefix combine
+
+PyTorch is used for device memory and streams only; every step runs in the
+library's CUDA kernels.
+"""
+from ._lib import (ALGOS, EXPORTS, KdaError, kda_chunk_fwd, kda_compose, kda_device_status,
+                   kda_status_string, kda_step, kda_version, library_path, load)
+
+__all__ = ["kda_chunk_fwd", "kda_step", "kda_compose", "kda_device_status",
+           "kda_status_string", "kda_version", "KdaError", "ALGOS", "EXPORTS",
+           "library_path", "load"]

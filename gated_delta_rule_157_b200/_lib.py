@@ -1,0 +1,252 @@
+"""ctypes binding of libkda_b200.so (the C ABI in include/kda.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, outputs are allocated with torch when the caller passes none, and
+raw device pointers plus the current CUDA stream are handed to the library.
+Every step of the computation runs in the library's CUDA kernels; there is no
+CPU path.  If the shared object is missing it is built with nvcc; if that
+fails, the import fails.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+KDA_OK = 0
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+                3: "KDA_ERR_ALIGNMENT", 4: "KDA_ERR_ALIAS", 5: "KDA_ERR_CUDA",
+                6: "KDA_ERR_TIMEOUT"}
+DT_F32, DT_BF16 = 0, 1
+ALGOS = {"auto": 0, "simt": 1, "tc": 2}
+
+
+class KdaError(RuntimeError):
+    """A non-OK kda_status returned by the library."""
+
+    def __init__(self, fn, status):
+        self.status = int(status)
+        super().__init__("%s returned %s" % (fn, STATUS_NAMES.get(self.status, self.status)))
+
+
+class ChunkArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("HV", ctypes.c_int),
+        ("Dk", ctypes.c_int), ("Dv", ctypes.c_int), ("chunk", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("algo", ctypes.c_int),
+        ("g_min", ctypes.c_float), ("scale", ctypes.c_float), ("l2_eps", ctypes.c_float),
+        ("qk_l2norm_in_kernel", ctypes.c_int), ("beta_sigmoid_in_kernel", ctypes.c_int),
+        ("gate_in_kernel", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+        ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("S0", ctypes.c_void_p),
+        ("o", ctypes.c_void_p), ("S_T", ctypes.c_void_p), ("M_T", ctypes.c_void_p),
+    ]
+
+
+class StepArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("HV", ctypes.c_int),
+        ("Dk", ctypes.c_int), ("Dv", ctypes.c_int), ("dtype", ctypes.c_int),
+        ("g_min", ctypes.c_float), ("scale", ctypes.c_float), ("l2_eps", ctypes.c_float),
+        ("qk_l2norm_in_kernel", ctypes.c_int), ("beta_sigmoid_in_kernel", ctypes.c_int),
+        ("gate_in_kernel", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+        ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+        ("S", ctypes.c_void_p), ("o", ctypes.c_void_p),
+    ]
+
+
+EXPORTS = ["kda_chunk_fwd", "kda_step", "kda_compose", "kda_device_status",
+           "kda_status_string", "kda_version"]
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load():
+    """Load (building first if needed) the CUDA library; raises if unavailable."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.build()
+    if not os.path.exists(path):
+        raise ImportError("libkda_b200.so is missing and could not be built")
+    lib = ctypes.CDLL(path)
+    lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(ChunkArgs), ctypes.c_void_p]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
+    lib.kda_step.restype = ctypes.c_int
+    lib.kda_compose.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 5
+    lib.kda_compose.restype = ctypes.c_int
+    lib.kda_device_status.argtypes = [ctypes.c_void_p]
+    lib.kda_device_status.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr()).value
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return DT_F32
+    if t.dtype == torch.bfloat16:
+        return DT_BF16
+    raise ValueError("activations must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _check(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _raise(fn, status):
+    if status != KDA_OK:
+        raise KdaError(fn, status)
+
+
+def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=64,
+                  g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
+                  beta_sigmoid_in_kernel=True, gate_in_kernel=True,
+                  output_final_state=True, output_transition=False, algo="auto",
+                  o=None, S_T=None, M_T=None, stream=None):
+    """Chunk-parallel KDA forward.  Returns (o, S_T or None, M_T or None).
+
+    q, k [B,T,H,Dk]; v [B,T,HV,Dv]; g (log-decay or raw z) [B,T,HV,Dk];
+    beta (or logits) [B,T,HV] -- all float32 or all bfloat16, on one CUDA device.
+    A_log [HV], dt_bias [HV,Dk], S0 [B,HV,Dk,Dv]: float32.
+    """
+    lib = load()
+    if not isinstance(q, torch.Tensor) or not q.is_cuda:
+        raise ValueError("q must be a CUDA tensor")
+    dev = q.device
+    B, T, H, Dk = q.shape
+    HV, Dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    _check(q, "q", (B, T, H, Dk), dt, dev)
+    _check(k, "k", (B, T, H, Dk), dt, dev)
+    _check(v, "v", (B, T, HV, Dv), dt, dev)
+    _check(g, "g", (B, T, HV, Dk), dt, dev)
+    _check(beta, "beta", (B, T, HV), dt, dev)
+    _check(A_log, "A_log", (HV,), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (HV, Dk), torch.float32, dev)
+    _check(S0, "S0", (B, HV, Dk, Dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, T, HV, Dv), dtype=dt, device=dev)
+    _check(o, "o", (B, T, HV, Dv), dt, dev)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((B, HV, Dk, Dv), dtype=torch.float32, device=dev)
+    _check(S_T, "S_T", (B, HV, Dk, Dv), torch.float32, dev)
+    if M_T is None and output_transition:
+        M_T = torch.empty((B, HV, Dk, Dk), dtype=torch.float32, device=dev)
+    _check(M_T, "M_T", (B, HV, Dk, Dk), torch.float32, dev)
+    a = ChunkArgs()
+    a.B, a.T, a.H, a.HV, a.Dk, a.Dv, a.chunk = B, T, H, HV, Dk, Dv, int(chunk)
+    a.dtype, a.algo = _dtype_code(q), ALGOS[algo]
+    a.g_min, a.scale, a.l2_eps = float(g_min), float(scale), float(l2_eps)
+    a.qk_l2norm_in_kernel = int(bool(qk_l2norm_in_kernel))
+    a.beta_sigmoid_in_kernel = int(bool(beta_sigmoid_in_kernel))
+    a.gate_in_kernel = int(bool(gate_in_kernel))
+    a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
+    a.A_log, a.dt_bias, a.S0 = _ptr(A_log), _ptr(dt_bias), _ptr(S0)
+    a.o, a.S_T, a.M_T = _ptr(o), _ptr(S_T), _ptr(M_T)
+    _raise("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a), _stream(stream, dev)))
+    return o, S_T, M_T
+
+
+def kda_step(S, q, k, v, g, beta, *, A_log=None, dt_bias=None, g_min=-5.0, scale=1.0,
+             l2_eps=1e-6, qk_l2norm_in_kernel=True, beta_sigmoid_in_kernel=True,
+             gate_in_kernel=True, o=None, stream=None):
+    """One decode step; S [B,HV,Dk,Dv] float32 is updated in place.  Returns o [B,HV,Dv].
+
+    q, k [B,H,Dk]; v [B,HV,Dv]; g [B,HV,Dk]; beta [B,HV] (float32 or bfloat16).
+    """
+    lib = load()
+    if not isinstance(S, torch.Tensor) or not S.is_cuda:
+        raise ValueError("S must be a CUDA tensor")
+    dev = S.device
+    B, HV, Dk, Dv = S.shape
+    H = q.shape[1]
+    dt = q.dtype
+    _check(S, "S", (B, HV, Dk, Dv), torch.float32, dev)
+    _check(q, "q", (B, H, Dk), dt, dev)
+    _check(k, "k", (B, H, Dk), dt, dev)
+    _check(v, "v", (B, HV, Dv), dt, dev)
+    _check(g, "g", (B, HV, Dk), dt, dev)
+    _check(beta, "beta", (B, HV), dt, dev)
+    _check(A_log, "A_log", (HV,), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (HV, Dk), torch.float32, dev)
+    if o is None:
+        o = torch.empty((B, HV, Dv), dtype=dt, device=dev)
+    _check(o, "o", (B, HV, Dv), dt, dev)
+    a = StepArgs()
+    a.B, a.H, a.HV, a.Dk, a.Dv = B, H, HV, Dk, Dv
+    a.dtype = _dtype_code(q)
+    a.g_min, a.scale, a.l2_eps = float(g_min), float(scale), float(l2_eps)
+    a.qk_l2norm_in_kernel = int(bool(qk_l2norm_in_kernel))
+    a.beta_sigmoid_in_kernel = int(bool(beta_sigmoid_in_kernel))
+    a.gate_in_kernel = int(bool(gate_in_kernel))
+    a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
+    a.A_log, a.dt_bias, a.S, a.o = _ptr(A_log), _ptr(dt_bias), _ptr(S), _ptr(o)
+    _raise("kda_step", lib.kda_step(ctypes.byref(a), _stream(stream, dev)))
+    return o
+
+
+def kda_compose(M, S_seg, S_init=None, S_in=None, stream=None):
+    """Segment prefix combine.  M [n,BH,Dk,Dk], S_seg [n,BH,Dk,Dv], S_init [BH,Dk,Dv]
+    (float32, CUDA).  Returns S_in [n+1,BH,Dk,Dv] with S_in[s] the state entering
+    segment s and S_in[n] the final state."""
+    lib = load()
+    dev = S_seg.device
+    n, BH, Dk, Dv = S_seg.shape
+    _check(M, "M", (n, BH, Dk, Dk), torch.float32, dev)
+    _check(S_seg, "S_seg", (n, BH, Dk, Dv), torch.float32, dev)
+    _check(S_init, "S_init", (BH, Dk, Dv), torch.float32, dev)
+    if S_in is None:
+        S_in = torch.empty((n + 1, BH, Dk, Dv), dtype=torch.float32, device=dev)
+    _check(S_in, "S_in", (n + 1, BH, Dk, Dv), torch.float32, dev)
+    st = lib.kda_compose(n, BH, Dk, Dv, _ptr(M), _ptr(S_seg), _ptr(S_init), _ptr(S_in),
+                         _stream(stream, dev))
+    _raise("kda_compose", st)
+    return S_in
+
+
+def kda_device_status(stream=None, device=None):
+    """Synchronise and read/clear the device error word; raises KdaError if set."""
+    lib = load()
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _raise("kda_device_status", lib.kda_device_status(_stream(stream, dev)))
+
+
+def kda_status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> int:
+    return int(load().kda_version())

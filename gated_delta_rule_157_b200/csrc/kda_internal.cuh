@@ -1,0 +1,63 @@
+// Internal declarations shared by the CUDA translation units of the library.
+// Nothing here is part of the C ABI (include/kda.h is).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+
+namespace kda {
+
+// Element loads/stores for the two activation dtypes.
+__device__ __forceinline__ float ld_act(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ld_act(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void st_act(float *p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void st_act(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// Bounded log-decay g = g_min * sigmoid(exp(A_log) * (z + dt_bias)); `ea` is exp(A_log).
+__device__ __forceinline__ float bounded_gate(float z, float bias, float ea, float g_min) {
+    return g_min * sigmoidf_(ea * (z + bias));
+}
+
+// Validated arguments of a chunked forward, as the kernels see them.
+struct ChunkParams {
+    int B, T, H, HV, Dk, Dv, C;
+    int group;                       // HV / H
+    float g_min, scale, l2_eps;
+    int l2norm, beta_sigmoid, gate_in;
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias, *S0;
+    void *o;
+    float *S_T, *M_T;
+};
+
+struct StepParams {
+    int B, H, HV, Dk, Dv, group;
+    float g_min, scale, l2_eps;
+    int l2norm, beta_sigmoid, gate_in;
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias;
+    float *S;
+    void *o;
+};
+
+// Launchers (host).  They assume validated arguments and return the launch status.
+cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, cudaStream_t s);
+cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s);
+bool chunk_tc_supported(const ChunkParams &p, bool bf16);
+cudaError_t launch_chunk_empty(const ChunkParams &p, cudaStream_t s);   // T == 0
+cudaError_t launch_step(const StepParams &p, bool bf16, cudaStream_t s);
+cudaError_t launch_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
+                           const float *S_seg, const float *S_init, float *S_in,
+                           cudaStream_t s);
+// Device error word (set by bounded waits that gave up).  Reads and clears it.
+cudaError_t read_and_clear_device_error(cudaStream_t s, unsigned int *out);
+
+}  // namespace kda

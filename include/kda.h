@@ -1,0 +1,176 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention core.
+ *
+ * KDA keeps, per (batch b, value head hv), a state S in R^{Dk x Dv} (row c =
+ * key channel, column j = value channel) and, for every token t, applies
+ * (page "Implémenter KDA", sections "La forme récurrente de référence" and
+ * "Trois pièges"; page "KDA 模块交互式演示", section 1.3 Eq. 1):
+ *
+ *     S <- Diag(alpha_t) S                      decay, alpha_t = exp(g_t) per key channel
+ *     S <- S + beta_t k_t (v_t - S^T k_t)^T     delta-rule write of the retrieval error
+ *     o_t = scale * S^T q_t                     read AFTER the update
+ *
+ * Three optional preprocessing steps run inside the kernels (page
+ * "KDAAttention 层", section "chunk_kda 内部做了什么"; all three default on):
+ *     qk_l2norm_in_kernel:    q <- q / sqrt(|q|^2 + l2_eps), same for k
+ *     beta_sigmoid_in_kernel: beta <- 1 / (1 + exp(-beta))
+ *     gate_in_kernel:         g <- g_min * sigmoid(exp(A_log[hv]) * (g + dt_bias[hv,:]))
+ *                             (bounded decay; page "KDA 模块交互式演示" section 1.4
+ *                             Eq. 5, page "Implémenter KDA" "La décroissance bornée")
+ *
+ * Value head hv reads q/k head h = hv / (HV / H) (contiguous groups).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers (CUDA global memory on the
+ *     current device), row-major and contiguous in the stated layout.  The
+ *     caller owns every buffer; the library allocates nothing and keeps no
+ *     state across calls except one device-resident error word per device.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.
+ *   - Argument errors are detected on the host before anything is launched and
+ *     are returned as a kda_status; nothing is written in that case.  A failed
+ *     launch returns KDA_ERR_CUDA.  Device-side faults of the tensor-core
+ *     kernel (a bounded wait that ran out) are recorded in the device error
+ *     word and reported by kda_device_status().
+ *   - No entry point falls back to the CPU.
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, HV % H != 0, ... */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid request no kernel of this build handles */
+    KDA_ERR_ALIGNMENT = 3,     /* a pointer is not aligned as the layout requires */
+    KDA_ERR_ALIAS = 4,         /* an output overlaps an input or another output */
+    KDA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up (see kda_device_status) */
+} kda_status;
+
+typedef enum {
+    KDA_DT_F32 = 0,            /* IEEE binary32 */
+    KDA_DT_BF16 = 1            /* bfloat16 (rounded to nearest even by the producer) */
+} kda_dtype;
+
+typedef enum {
+    KDA_ALGO_AUTO = 0,         /* tensor-core kernel when the shape allows it, else SIMT */
+    KDA_ALGO_SIMT = 1,         /* FP32 FMA chunk kernel (any supported shape, both dtypes) */
+    KDA_ALGO_TC = 2            /* tcgen05 BF16 chunk kernel (bf16, Dk = Dv = 128, chunk = 64) */
+} kda_algo;
+
+/*
+ * kda_chunk_fwd -- chunk-parallel forward over whole sequences.
+ *
+ * Computes, for every (b, hv), the outputs o_t of the recurrence above for
+ * t = 0..T-1 from the initial state S0, the final state S_T and, optionally,
+ * the cumulative transition M_T = prod_{t=T-1..0} (I - beta_t k_t k_t^T) Diag(alpha_t)
+ * (page "Implémenter KDA", "Test 2 - l'identité de composition"), so that
+ * S_T = M_T S0 + (state reached from S0 = 0).
+ * The chunk form it uses is the one of page "KDA 模块交互式演示" section 1.5
+ * (Eqs. 3-4) with the decay-weighted UT transform: per chunk of `chunk`
+ * tokens, a cumulative sum of g, the triangular solve
+ * (I + tril(Diag(beta)(K*Gamma)(K/Gamma)^T, -1))^-1, the intra-chunk
+ * Tril[(Q*Gamma)(K/Gamma)^T] product and the serial state carry.
+ *
+ * Layouts (element type `dtype` unless stated):
+ *   q, k    [B, T, H,  Dk]
+ *   v       [B, T, HV, Dv]
+ *   g       [B, T, HV, Dk]  log-decay g, or the raw gate input z when gate_in_kernel
+ *   beta    [B, T, HV]      write strength, or its logit when beta_sigmoid_in_kernel
+ *   A_log   [HV]      fp32  read iff gate_in_kernel (must then be non-NULL)
+ *   dt_bias [HV, Dk]  fp32  read iff gate_in_kernel; NULL means 0
+ *   S0      [B, HV, Dk, Dv] fp32, or NULL for zeros
+ *   o       [B, T, HV, Dv]  output, element type `dtype` (bf16 rounded to nearest even)
+ *   S_T     [B, HV, Dk, Dv] fp32 output, or NULL; may be the same buffer as S0
+ *           (exactly, not partially overlapping)
+ *   M_T     [B, HV, Dk, Dk] fp32 output, or NULL
+ *
+ * Limits: B, T >= 0; 1 <= H <= HV, HV % H == 0; 1 <= Dk, Dv <= 128;
+ * 1 <= chunk <= 64.  q, k, v, g, beta, o must be aligned to their element size;
+ * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64 and
+ * 16-byte aligned q, k, v, g, o.  o must not overlap any input; S_T and M_T
+ * must not overlap each other, o, or any input except S_T == S0.
+ * T == 0 writes S_T = S0 (or 0) and M_T = I.
+ */
+typedef struct {
+    int B, T, H, HV, Dk, Dv, chunk;
+    int dtype;                 /* kda_dtype of q, k, v, g, beta and o */
+    int algo;                  /* kda_algo */
+    float g_min;               /* lower bound of the log-decay, -5 for Kimi K3 */
+    float scale;               /* output scale (the pages apply none: 1) */
+    float l2_eps;              /* epsilon inside the L2-norm square root */
+    int qk_l2norm_in_kernel, beta_sigmoid_in_kernel, gate_in_kernel;
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias;
+    const float *S0;
+    void *o;
+    float *S_T;
+    float *M_T;
+} kda_chunk_args;
+
+kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
+
+/*
+ * kda_step -- one decode token for B*HV independent chains against a resident
+ * state, updated in place (page "Implémenter KDA", "La forme récurrente de
+ * référence"; page "KDA 模块交互式演示" section 1.1 single-step decode).
+ *
+ * Layouts:
+ *   q, k    [B, H,  Dk]   dtype
+ *   v       [B, HV, Dv]   dtype
+ *   g       [B, HV, Dk]   dtype (log-decay, or raw z when gate_in_kernel)
+ *   beta    [B, HV]       dtype
+ *   A_log   [HV], dt_bias [HV, Dk] fp32 (as in kda_chunk_fwd)
+ *   S       [B, HV, Dk, Dv] fp32, read and written in place, 16-byte aligned
+ *   o       [B, HV, Dv]   dtype output
+ *
+ * Limits: 1 <= Dk <= 128, 4 <= Dv <= 128 with Dv % 4 == 0.  o must not overlap
+ * S or any input.  One read and one write of S per call.
+ */
+typedef struct {
+    int B, H, HV, Dk, Dv;
+    int dtype;
+    float g_min, scale, l2_eps;
+    int qk_l2norm_in_kernel, beta_sigmoid_in_kernel, gate_in_kernel;
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias;
+    float *S;
+    void *o;
+} kda_step_args;
+
+kda_status kda_step(const kda_step_args *args, void *stream);
+
+/*
+ * kda_compose -- prefix combine of segment results (KCP; page "KDA 模块交互式演示"
+ * section 1.6, page "Implémenter KDA" "Test 3 - le balayage préfixe"):
+ *
+ *     S_in[0] = S_init (or 0 when S_init is NULL)
+ *     S_in[s+1] = M[s] S_in[s] + S_seg[s],   s = 0..n_seg-1
+ *
+ * S_in[s] is the state entering segment s; S_in[n_seg] is the final state.
+ * Layouts (all fp32, device): M [n_seg, BH, Dk, Dk], S_seg [n_seg, BH, Dk, Dv],
+ * S_init [BH, Dk, Dv] or NULL, S_in [n_seg + 1, BH, Dk, Dv] output.
+ * Limits: n_seg >= 0, BH >= 0, 1 <= Dk, Dv <= 128.  S_in must not overlap the inputs.
+ */
+kda_status kda_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
+                       const float *S_seg, const float *S_init, float *S_in,
+                       void *stream);
+
+/* Reads and clears the device error word of the current device after
+ * synchronising `stream`.  Returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_CUDA. */
+kda_status kda_device_status(void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *kda_status_string(kda_status status);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_B200_H */

@@ -1,0 +1,187 @@
+"""The C-ABI library: it loads, exports every entry point include/kda.h
+declares, and its host-side validation rejects bad arguments before anything
+reaches the GPU.  No test here needs a GPU.
+
+The validation tests pass made-up pointer values; they are skipped when a CUDA
+device is present so that a validation bug can never send such a pointer to a
+kernel (the GPU tests cover the same checks with real buffers).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_delta_rule_157_b200 as kda
+from gated_delta_rule_157_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "kda.h")
+OK, INVALID, UNSUPPORTED, ALIGN, ALIAS = 0, 1, 2, 3, 4
+
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                 reason="made-up pointers are only used without a GPU")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_three_entry_points():
+    names = declared_functions()
+    for n in ("kda_chunk_fwd", "kda_step", "kda_compose"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = kda.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(_lib.EXPORTS)
+
+
+def test_library_is_in_tree_and_links_no_oracle():
+    path = kda.library_path()
+    assert os.path.dirname(path) == os.path.dirname(os.path.abspath(kda.__file__))
+    blob = open(path, "rb").read()
+    assert b"oracle_kda" not in blob
+
+
+def test_status_strings_and_version():
+    assert kda.kda_status_string(0) == "KDA_OK"
+    assert kda.kda_status_string(6) == "KDA_ERR_TIMEOUT"
+    assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+    assert kda.kda_version() >= 100
+
+
+def _chunk_args(**kw):
+    a = _lib.ChunkArgs()
+    a.B, a.T, a.H, a.HV, a.Dk, a.Dv, a.chunk = 1, 64, 2, 4, 16, 16, 16
+    a.dtype, a.algo = 0, 0
+    a.g_min, a.scale, a.l2_eps = -5.0, 1.0, 1e-6
+    a.qk_l2norm_in_kernel = a.beta_sigmoid_in_kernel = a.gate_in_kernel = 1
+    base = 0x7f0000000000
+    sizes = {"q": 1 << 20, "k": 2 << 20, "v": 3 << 20, "g": 4 << 20, "beta": 5 << 20,
+             "A_log": 6 << 20, "dt_bias": 7 << 20, "S0": 8 << 20, "o": 9 << 20,
+             "S_T": 10 << 20, "M_T": 11 << 20}
+    for name, off in sizes.items():
+        setattr(a, name, base + off)
+    a.dt_bias = None
+    a.M_T = None
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+def _fwd(a):
+    return kda.load().kda_chunk_fwd(ctypes.byref(a), None)
+
+
+def test_null_args_rejected():
+    assert kda.load().kda_chunk_fwd(None, None) == INVALID
+    assert kda.load().kda_step(None, None) == INVALID
+
+
+def test_empty_batch_is_a_no_op():
+    # B == 0: nothing to do, nothing launched (works without a GPU).
+    assert _fwd(_chunk_args(B=0)) == OK
+
+
+@no_gpu_only
+@pytest.mark.parametrize("field,value,expected", [
+    ("H", 3, INVALID),            # HV % H != 0
+    ("H", 0, INVALID),
+    ("Dk", 0, INVALID),
+    ("Dk", 129, UNSUPPORTED),
+    ("Dv", 256, UNSUPPORTED),
+    ("chunk", 0, INVALID),
+    ("chunk", 128, UNSUPPORTED),
+    ("dtype", 7, INVALID),
+    ("algo", 9, INVALID),
+    ("T", -1, INVALID),
+    ("g_min", 0.5, INVALID),
+    ("q", None, INVALID),
+    ("o", None, INVALID),
+    ("A_log", None, INVALID),     # gate_in_kernel needs A_log
+    ("q", 0x7f0000100002, ALIGN),  # fp32 needs 4-byte alignment
+    ("S0", 0x7f0000800001, ALIGN),
+])
+def test_chunk_validation(field, value, expected):
+    assert _fwd(_chunk_args(**{field: value})) == expected
+
+
+@no_gpu_only
+def test_chunk_aliasing_rejected():
+    a = _chunk_args()
+    assert _fwd(_chunk_args(o=a.q)) == ALIAS                  # o over an input
+    assert _fwd(_chunk_args(o=a.v + 64)) == ALIAS             # partial overlap
+    assert _fwd(_chunk_args(S_T=a.o)) == ALIAS
+    assert _fwd(_chunk_args(S_T=a.S0 + 4)) == ALIAS           # partial S_T/S0 overlap
+    assert _fwd(_chunk_args(M_T=a.S_T)) == ALIAS
+
+
+@no_gpu_only
+def test_chunk_tc_request_on_unsupported_shape():
+    # The tensor-core kernel needs bf16, Dk = Dv = 128, chunk = 64.
+    assert _fwd(_chunk_args(algo=2)) == UNSUPPORTED
+
+
+@no_gpu_only
+def test_valid_request_without_gpu_reports_cuda_error():
+    # Passes validation, so the launch is attempted and fails: no CPU fallback.
+    a = _chunk_args(S_T=_chunk_args().S_T)
+    assert _fwd(a) == 5
+
+
+def _step_args(**kw):
+    a = _lib.StepArgs()
+    a.B, a.H, a.HV, a.Dk, a.Dv, a.dtype = 2, 2, 4, 16, 16, 1
+    a.g_min, a.scale, a.l2_eps = -5.0, 1.0, 1e-6
+    a.qk_l2norm_in_kernel = a.beta_sigmoid_in_kernel = a.gate_in_kernel = 1
+    base = 0x7f1000000000
+    for i, name in enumerate(["q", "k", "v", "g", "beta", "A_log", "S", "o"]):
+        setattr(a, name, base + (i + 1) * (1 << 20))
+    a.dt_bias = None
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+@no_gpu_only
+@pytest.mark.parametrize("field,value,expected", [
+    ("Dv", 6, UNSUPPORTED),       # Dv % 4 != 0
+    ("Dk", 200, UNSUPPORTED),
+    ("HV", 3, INVALID),
+    ("S", None, INVALID),
+    ("S", 0x7f1000700008, ALIGN),  # state needs 16-byte alignment
+    ("q", 0x7f1000100001, ALIGN),  # bf16 needs 2-byte alignment
+])
+def test_step_validation(field, value, expected):
+    assert kda.load().kda_step(ctypes.byref(_step_args(**{field: value})), None) == expected
+
+
+@no_gpu_only
+def test_step_aliasing_rejected():
+    a = _step_args()
+    assert kda.load().kda_step(ctypes.byref(_step_args(o=a.S + 32)), None) == ALIAS
+    assert kda.load().kda_step(ctypes.byref(_step_args(S=a.v)), None) == ALIAS
+
+
+@no_gpu_only
+def test_compose_validation():
+    lib = kda.load()
+    p = 0x7f2000000000
+    assert lib.kda_compose(-1, 1, 8, 8, p, p + (1 << 20), None, p + (2 << 20), None) == INVALID
+    assert lib.kda_compose(2, 1, 8, 200, p, p + (1 << 20), None, p + (2 << 20), None) == UNSUPPORTED
+    assert lib.kda_compose(2, 1, 8, 8, p, p + (1 << 20), None, None, None) == INVALID
+    assert lib.kda_compose(2, 1, 8, 8, p, p + (1 << 20), None, p + 64, None) == ALIAS
+    assert lib.kda_compose(0, 0, 8, 8, None, None, None, None, None) == OK
+
+
+def test_binding_rejects_cpu_tensors():
+    x = torch.zeros(1, 4, 1, 16)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))

@@ -1,0 +1,155 @@
+"""GPU parity of kda_chunk_fwd against the FP64 oracle on identical seeded inputs.
+
+Bars: FP32 inputs <= 1e-4 max relative error (o, S_T, M_T); BF16 inputs <= 2e-2 of
+max|o| and <= 2e-2 relative Frobenius error of S_T.  The SIMT kernel computes
+in FP32 from the exact inputs, so its fp32 outputs (S_T, M_T) are also held to
+1e-4 when the inputs are bf16.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_157_b200 as kda
+import workloads
+from helpers import TOL_BF16, TOL_F32, fro_rel, max_rel, oracle_chunk, to_device, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(inp, w, algo, flags=True, want_M=False, out_state=True, **kw):
+    return kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                             A_log=inp["A_log"], dt_bias=inp["dt_bias"], S0=inp["S0"],
+                             chunk=w.chunk, qk_l2norm_in_kernel=flags,
+                             beta_sigmoid_in_kernel=flags, gate_in_kernel=flags,
+                             output_final_state=out_state, output_transition=want_M,
+                             algo=algo, **kw)
+
+
+def check(o, S_T, M_T, ref, dtype, algo):
+    if dtype == "f32":
+        assert max_rel(to_np(o), ref["o"]) <= TOL_F32
+        if S_T is not None:
+            assert max_rel(to_np(S_T), ref["S_T"]) <= TOL_F32
+        if M_T is not None:
+            assert max_rel(to_np(M_T), ref["M_T"]) <= TOL_F32
+    else:
+        assert max_rel(to_np(o), ref["o"]) <= TOL_BF16
+        if S_T is not None:
+            assert fro_rel(to_np(S_T), ref["S_T"]) <= TOL_BF16
+            if algo == "simt":
+                assert max_rel(to_np(S_T), ref["S_T"]) <= TOL_F32
+        if M_T is not None:
+            assert fro_rel(to_np(M_T), ref["M_T"]) <= TOL_BF16
+            if algo == "simt":
+                assert max_rel(to_np(M_T), ref["M_T"]) <= TOL_F32
+
+
+def test_tiny_fp32_workload(cuda_device):
+    """B=1, H=HV=2, T=64, Dk=Dv=16, chunk=16, fp32, seed 0, A_log=0, S0=0."""
+    w = workloads.workload("tiny_fp32")
+    inp = workloads.chunk_inputs(w)
+    ref = oracle_chunk(inp, want_M=True)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "auto", want_M=True)
+    check(o, S_T, M_T, ref, "f32", "simt")
+
+
+SHAPES = [
+    # B, T, H, HV, Dk, Dv, chunk, dtype, s0
+    (1, 100, 1, 1, 16, 16, 16, "f32", None),     # ragged tail
+    (2, 77, 2, 4, 32, 24, 32, "f32", 0.1),        # Dk != Dv, grouped heads, ragged
+    (1, 130, 1, 4, 48, 40, 64, "f32", 0.05),      # HV/H = 4, ragged, C=64
+    (1, 64, 2, 2, 128, 128, 64, "f32", 0.02),     # full head size, one chunk
+    (2, 200, 2, 2, 64, 128, 64, "bf16", 0.02),    # bf16 activations
+    (1, 33, 1, 2, 8, 12, 16, "bf16", None),       # tiny odd sizes
+    (1, 5, 1, 1, 4, 4, 64, "f32", 0.3),           # T < chunk
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B%d_T%d_H%d_HV%d_K%d_V%d_C%d_%s" % s[:8])
+@pytest.mark.parametrize("want_M", [False, True])
+def test_simt_shapes(cuda_device, shape, want_M):
+    B, T, H, HV, Dk, Dv, C, dt, s0 = shape
+    w = workloads.Workload("case", B=B, T=T, H=H, HV=HV, Dk=Dk, Dv=Dv, chunk=C, dtype=dt,
+                           seed=T + Dk, a_log="uniform", dt_bias_std=0.5, s0_std=s0)
+    inp = workloads.chunk_inputs(w)
+    ref = oracle_chunk(inp, want_M=want_M)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "simt", want_M=want_M)
+    check(o, S_T, M_T, ref, dt, "simt")
+
+
+def test_switches_off_path(cuda_device):
+    """Inputs already in activated form (log-decay g, beta in (0,1), near-unit keys)."""
+    w = workloads.Workload("act", B=2, T=90, H=1, HV=2, Dk=32, Dv=32, chunk=32, dtype="f32",
+                           seed=11, s0_std=0.1)
+    inp = workloads.activated_inputs(w)
+    ref = oracle_chunk(inp, flags=False, want_M=True)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "simt", flags=False, want_M=True)
+    check(o, S_T, M_T, ref, "f32", "simt")
+
+
+@pytest.mark.parametrize("z_mean", [-12.0, 12.0])
+def test_extreme_gates(cuda_device, z_mean):
+    """z far negative: alpha -> 1 (no forgetting, long memory); z far positive:
+    g -> g_min every token, so a 64-token chunk decays by e^-320 (the case
+    that overflows an unguarded K/Gamma factorisation in fp32)."""
+    w = workloads.Workload("gate", B=1, T=192, H=1, HV=2, Dk=64, Dv=64, chunk=64, dtype="f32",
+                           seed=21, s0_std=0.1)
+    inp = workloads.chunk_inputs(w, z_mean=z_mean, z_std=0.5)
+    ref = oracle_chunk(inp, want_M=True)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "simt", want_M=True)
+    assert torch.isfinite(o).all() and torch.isfinite(S_T).all() and torch.isfinite(M_T).all()
+    check(o, S_T, M_T, ref, "f32", "simt")
+
+
+def test_scale_and_null_state_outputs(cuda_device):
+    w = workloads.Workload("sc", B=1, T=40, H=1, HV=1, Dk=16, Dv=16, chunk=16, dtype="f32",
+                           seed=5, s0_std=0.2)
+    inp = workloads.chunk_inputs(w)
+    ref = oracle_chunk(inp, scale=0.125)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "simt", out_state=False, scale=0.125)
+    assert S_T is None and M_T is None
+    assert max_rel(to_np(o), ref["o"]) <= TOL_F32
+
+
+def test_state_in_place(cuda_device):
+    """S_T may be the same buffer as S0."""
+    w = workloads.Workload("ip", B=2, T=50, H=1, HV=2, Dk=16, Dv=32, chunk=16, dtype="f32",
+                           seed=6, s0_std=0.3)
+    inp = workloads.chunk_inputs(w)
+    ref = oracle_chunk(inp)
+    d = to_device(inp, cuda_device)
+    S = d["S0"].clone()
+    d["S0"] = S
+    o, S_T, _ = run_gpu(d, w, "simt", S_T=S)
+    assert S_T.data_ptr() == S.data_ptr()
+    assert max_rel(to_np(S), ref["S_T"]) <= TOL_F32
+    assert max_rel(to_np(o), ref["o"]) <= TOL_F32
+
+
+def test_empty_sequence(cuda_device):
+    w = workloads.Workload("e", B=2, T=0, H=1, HV=2, Dk=8, Dv=4, chunk=16, dtype="f32", seed=7,
+                           s0_std=1.0)
+    d = to_device(workloads.chunk_inputs(w), cuda_device)
+    o, S_T, M_T = run_gpu(d, w, "auto", want_M=True)
+    assert o.numel() == 0
+    torch.testing.assert_close(S_T, d["S0"], rtol=0, atol=0)
+    eye = torch.eye(8, device=cuda_device).expand(2, 2, 8, 8)
+    torch.testing.assert_close(M_T, eye, rtol=0, atol=0)
+
+
+def test_aliasing_rejected_with_real_buffers(cuda_device):
+    w = workloads.Workload("al", B=1, T=16, H=1, HV=1, Dk=16, Dv=16, chunk=16, dtype="f32",
+                           seed=8)
+    d = to_device(workloads.chunk_inputs(w), cuda_device)
+    with pytest.raises(kda.KdaError) as ei:
+        run_gpu(d, w, "simt", o=d["v"])
+    assert ei.value.status == 4
+
+
+def test_prefill_bf16_workload_simt(cuda_device):
+    """B=1, H=HV=16, T=4096, Dk=Dv=128, chunk=64, bf16, S0 ~ N(0, 0.02), on the SIMT kernel."""
+    w = workloads.workload("prefill_bf16")
+    inp = workloads.chunk_inputs(w)
+    ref = oracle_chunk(inp)
+    o, S_T, _ = run_gpu(to_device(inp, cuda_device), w, "simt")
+    check(o, S_T, None, ref, "bf16", "simt")
