@@ -34,10 +34,11 @@ __global__ void __launch_bounds__(kThreads)
 chunk_simt_kernel(ChunkParams p) {
     extern __shared__ float smem[];
     const int C = p.C, Dk = p.Dk, Dv = p.Dv;
-    float *Qs = smem;                      // [C][Dk]  q, then q*exp(G)
-    float *Ks = Qs + C * Dk;               // [C][Dk]  k, then k*exp(G)
-    float *Gs = Ks + C * Dk;               // [C][Dk]  g -> G -> k*exp(G_last - G)
-    float *Vs = Gs + C * Dk;               // [C][kVT] v -> X -> U
+    const int L = Dk | 1;                  // padded row stride of the [C][Dk] tiles
+    float *Qs = smem;                      // [C][L]  q, then q*exp(G)
+    float *Ks = Qs + C * L;                // [C][L]  k, then k*exp(G)
+    float *Gs = Ks + C * L;                // [C][L]  g -> G -> k*exp(G_last - G)
+    float *Vs = Gs + C * L;                // [C][kVT] v -> X -> U
     float *Akk = Vs + C * kVT;             // [C][C]
     float *Aqk = Akk + C * C;              // [C][C]
     float *Ss = Aqk + C * C;               // [Dk][kVT] state slice
@@ -50,6 +51,7 @@ chunk_simt_kernel(ChunkParams p) {
     const int b = chain / p.HV, hv = chain % p.HV, h = hv / p.group;
     const int col0 = blockIdx.y * kVT;     // first state column of this CTA
     const int ncol_state = Dv;             // columns [0, Dv) are the state, [Dv, Dv+Dk) carry M
+    const int ncol = Dv + (p.M_T ? Dk : 0);  // columns that exist in this launch
     const Tin *q = static_cast<const Tin *>(p.q);
     const Tin *k = static_cast<const Tin *>(p.k);
     const Tin *v = static_cast<const Tin *>(p.v);
@@ -64,7 +66,7 @@ chunk_simt_kernel(ChunkParams p) {
         float s = 0.f;
         if (col < ncol_state) {
             if (p.S0) s = p.S0[((size_t)chain * Dk + c) * Dv + col];
-        } else if (col < ncol_state + Dk) {
+        } else if (col < ncol) {
             s = (c == col - ncol_state) ? 1.f : 0.f;
         }
         Ss[idx] = s;
@@ -77,14 +79,14 @@ chunk_simt_kernel(ChunkParams p) {
         for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
             int r = idx / Dk, c = idx % Dk;
             size_t tok = (size_t)b * p.T + t0 + r;
-            Qs[r * Dk + c] = ld_act(q, (tok * p.H + h) * Dk + c);
-            Ks[r * Dk + c] = ld_act(k, (tok * p.H + h) * Dk + c);
+            Qs[r * L + c] = ld_act(q, (tok * p.H + h) * Dk + c);
+            Ks[r * L + c] = ld_act(k, (tok * p.H + h) * Dk + c);
             float gz = ld_act(g, (tok * p.HV + hv) * Dk + c);
             if (p.gate_in) {
                 float bias = p.dt_bias ? p.dt_bias[(size_t)hv * Dk + c] : 0.f;
                 gz = bounded_gate(gz, bias, ea, p.g_min);
             }
-            Gs[r * Dk + c] = gz;
+            Gs[r * L + c] = gz;
         }
         for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
             int r = idx / kVT, jj = idx % kVT, col = col0 + jj;
@@ -100,7 +102,7 @@ chunk_simt_kernel(ChunkParams p) {
             for (int r = warp; r < Cc; r += kThreads / 32) {
                 float sq = 0.f, sk = 0.f;
                 for (int c = lane; c < Dk; c += 32) {
-                    float a = Qs[r * Dk + c], bb = Ks[r * Dk + c];
+                    float a = Qs[r * L + c], bb = Ks[r * L + c];
                     sq = fmaf(a, a, sq);
                     sk = fmaf(bb, bb, sk);
                 }
@@ -110,8 +112,8 @@ chunk_simt_kernel(ChunkParams p) {
                 }
                 float rq = rsqrtf(sq + p.l2_eps), rk = rsqrtf(sk + p.l2_eps);
                 for (int c = lane; c < Dk; c += 32) {
-                    Qs[r * Dk + c] *= rq;
-                    Ks[r * Dk + c] *= rk;
+                    Qs[r * L + c] *= rq;
+                    Ks[r * L + c] *= rk;
                 }
             }
         }
@@ -119,8 +121,8 @@ chunk_simt_kernel(ChunkParams p) {
         for (int c = tid; c < Dk; c += kThreads) {
             float run = 0.f;
             for (int r = 0; r < Cc; ++r) {
-                run += Gs[r * Dk + c];
-                Gs[r * Dk + c] = run;
+                run += Gs[r * L + c];
+                Gs[r * L + c] = run;
             }
             Glast[c] = run;
         }
@@ -130,8 +132,8 @@ chunk_simt_kernel(ChunkParams p) {
             int r = pidx / Cc, i = pidx % Cc;
             float akk = 0.f, aqk = 0.f;
             if (i <= r) {
-                const float *kr = Ks + r * Dk, *ki = Ks + i * Dk, *qr = Qs + r * Dk;
-                const float *gr = Gs + r * Dk, *gi = Gs + i * Dk;
+                const float *kr = Ks + r * L, *ki = Ks + i * L, *qr = Qs + r * L;
+                const float *gr = Gs + r * L, *gi = Gs + i * L;
                 for (int c = 0; c < Dk; ++c) {
                     float e = expf(gr[c] - gi[c]);
                     float kie = ki[c] * e;
@@ -146,20 +148,20 @@ chunk_simt_kernel(ChunkParams p) {
         __syncthreads();
         // ---- decay-weighted operands (in place) ----------------------------
         for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
-            int c = idx % Dk;
-            float G = Gs[idx];
+            int r = idx / Dk, c = idx % Dk, a = r * L + c;
+            float G = Gs[a];
             float e = expf(G);
-            float kd = Ks[idx] * expf(Glast[c] - G);
-            Qs[idx] *= e;
-            Ks[idx] *= e;
-            Gs[idx] = kd;
+            float kd = Ks[a] * expf(Glast[c] - G);
+            Qs[a] *= e;
+            Ks[a] *= e;
+            Gs[a] = kd;
         }
         __syncthreads();
         // ---- X = V - (K*exp(G)) S ------------------------------------------
         for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
             int r = idx / kVT, jj = idx % kVT;
             float acc = Vs[idx];
-            const float *kr = Ks + r * Dk;
+            const float *kr = Ks + r * L;
             for (int c = 0; c < Dk; ++c) acc = fmaf(-kr[c], Ss[c * kVT + jj], acc);
             Vs[idx] = acc;
         }
@@ -180,7 +182,7 @@ chunk_simt_kernel(ChunkParams p) {
                 int r = idx / kVT, jj = idx % kVT, col = col0 + jj;
                 if (col >= ncol_state) continue;
                 float acc = 0.f;
-                const float *qr = Qs + r * Dk;
+                const float *qr = Qs + r * L;
                 for (int c = 0; c < Dk; ++c) acc = fmaf(qr[c], Ss[c * kVT + jj], acc);
                 const float *ar = Aqk + r * C;
                 for (int i = 0; i <= r; ++i) acc = fmaf(ar[i], Vs[i * kVT + jj], acc);
@@ -193,7 +195,7 @@ chunk_simt_kernel(ChunkParams p) {
         for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
             int c = idx / kVT, jj = idx % kVT;
             float acc = expf(Glast[c]) * Ss[idx];
-            for (int r = 0; r < Cc; ++r) acc = fmaf(Gs[r * Dk + c], Vs[r * kVT + jj], acc);
+            for (int r = 0; r < Cc; ++r) acc = fmaf(Gs[r * L + c], Vs[r * kVT + jj], acc);
             Ss[idx] = acc;
         }
     }
@@ -203,14 +205,14 @@ chunk_simt_kernel(ChunkParams p) {
         int c = idx / kVT, jj = idx % kVT, col = col0 + jj;
         if (col < ncol_state) {
             if (p.S_T) p.S_T[((size_t)chain * Dk + c) * Dv + col] = Ss[idx];
-        } else if (col < ncol_state + Dk) {
+        } else if (col < ncol) {
             p.M_T[((size_t)chain * Dk + c) * Dk + (col - ncol_state)] = Ss[idx];
         }
     }
 }
 
 size_t simt_smem_bytes(int C, int Dk) {
-    size_t f = (size_t)3 * C * Dk + (size_t)C * kVT + (size_t)2 * C * C + (size_t)Dk * kVT + C +
+    size_t f = (size_t)3 * C * (Dk | 1) + (size_t)C * kVT + (size_t)2 * C * C + (size_t)Dk * kVT + C +
                Dk + 2 * kThreads / 32;
     return f * sizeof(float);
 }
