@@ -22,6 +22,8 @@ REL_FLOOR = 1e-30
 def to_np(t):
     if t is None:
         return None
+    if isinstance(t, np.ndarray):
+        return t.astype(np.float64, copy=False)
     return t.detach().to("cpu", torch.float64).numpy()
 
 
