@@ -1,21 +1,626 @@
-// tcgen05 BF16 chunk kernel (placeholder until the tensor-core path lands) and
-// the device error word used by bounded waits.
+// tcgen05 BF16 chunk kernel for Dk = Dv = 128, chunk C = 64.
+//
+// One CTA (256 threads) per (b, hv) chain walks the chunks in order with the
+// state kept on chip: fp32 S^T in tensor memory (lane j = value channel,
+// column c = key channel) plus a bf16 copy in shared memory as the MMA operand.
+// Per chunk, with G the in-chunk cumulative sum of the log-decay, tiles of 16
+// tokens and P_R the cumulative sum before tile R (page "KDA 模块交互式演示"
+// section 1.5, Eqs. 3-4, with the decay-weighted UT transform; page
+// "Implémenter KDA", "La forme par blocs", for U = Ut - W S):
+//
+//   prep (CUDA cores)   L2-norm of q,k; beta = sigmoid; bounded gate
+//                       g = g_min sigmoid(exp(A_log)(z + dt_bias)); G, P_R;
+//                       bf16 operands scaled by exp(G_r - P_R) <= 1 and
+//                       exp(P_R' - G_i) (<= e^80 inside a tile, <= 1 before it)
+//   (I)   MMA  [K e^L ; Q e^L] x [K_R' e^{P_R'-G}]^T -> A_kk, A_qk, all tiles at once
+//   solve      T = (I + tril(Diag(beta) A_kk, -1))^-1   (blocked, fp32 CUDA cores)
+//   (II)  MMA  Ut^T = V^T (T Diag(beta))^T
+//   (III) MMA  W^T  = (K Gamma)^T (T Diag(beta))^T
+//   (IV)  MMA  U^T  = Ut^T - S^T W^T                       (serial carry)
+//   (V)   MMA  O^T  = S^T (Q Gamma)^T + U^T A_qk^T
+//   (VI)  MMA  S^T <- S^T Diag(gamma_C) + U^T K'            K' = K exp(G_C - G)
+//
+// Every exponent is bounded: within a 16-token tile |G_r - P_R| <= 16 |g_min| = 80
+// (e^80 ~ 5.5e34 < bf16/fp32 max, page "Implémenter KDA" "La décroissance
+// bornée"), and across tiles the factors are decays <= 1.
+//
+// All MMAs are cta_group::1, M = 128, BF16 operands from shared memory in the
+// K-major 128-byte-swizzle layout (tc_ptx.cuh), FP32 accumulators in TMEM.
+// When M_T is requested a second CTA per chain (blockIdx.y == 1) runs the same
+// recurrence on the transition columns: v = 0 and S0 = I, no o.
+//
+// Every wait on an MMA completion is bounded; if one gives up the CTA records
+// the device error word, stops, frees its TMEM and returns.
 #include "kda_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace kda {
 
 __device__ unsigned int g_device_error = 0;
 
+namespace {
+
+using namespace tc;
+
+constexpr int kThreads = 256;
+constexpr int C = 64;
+constexpr int D = 128;
+
+// Shared-memory map (bytes from a 1024-aligned base).
+constexpr uint32_t OFF_AINTRA = 0;        // [128 rows][K=128]  K e^L (rows 0-63), Q e^L (64-127)
+constexpr uint32_t OFF_KRCAT = 32768;     // [160 rows][K=128]  K_R' e^{P_R'-G}, R' = 0..3
+constexpr uint32_t OFF_AKK = 0;           //   alias: fp32 [64][65] A_kk (after MMA I)
+constexpr uint32_t OFF_TINV = 16640;      //   alias: fp32 [64][65] T
+constexpr uint32_t OFF_W = 34816;         //   alias: [64 rows][K=128] W (after the solve)
+constexpr uint32_t OFF_QG = 73728;        // [64 rows][K=128]   Q Gamma
+constexpr uint32_t OFF_KGT = 90112;       // [128 rows][K=64]   (K Gamma)^T
+constexpr uint32_t OFF_KP = 106496;       // [128 rows][K=64]   K'^T
+constexpr uint32_t OFF_VT = 122880;       // [128 rows][K=64]   V^T
+constexpr uint32_t OFF_TB = 139264;       // [64 rows][K=64]    T Diag(beta)
+constexpr uint32_t OFF_AQK = 147456;      // [64 rows][K=64]    A_qk (lower, diagonal kept)
+constexpr uint32_t OFF_ST = 155648;       // [128 rows][K=128]  S^T bf16
+constexpr uint32_t OFF_UT = 188416;       // [128 rows][K=64]   U^T bf16
+constexpr uint32_t OFF_MISC = 204800;
+constexpr uint32_t MISC_RQ = 0;           // float[64]
+constexpr uint32_t MISC_RK = 256;         // float[64]
+constexpr uint32_t MISC_BETA = 512;       // float[64]
+constexpr uint32_t MISC_RED = 768;        // float[8 warps][16][2]
+constexpr uint32_t MISC_TSUM = 1792;      // float[4][128]
+constexpr uint32_t MISC_GAMMA = 3840;     // float[128]
+constexpr uint32_t MISC_X = 4352;         // float[3][16][17] solve scratch
+constexpr uint32_t MISC_MBAR = 7680;      // uint64
+constexpr uint32_t MISC_TMEM = 7688;      // uint32
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 7696 + 1024;   // + alignment slack
+
+// TMEM columns.
+constexpr uint32_t COL_INTRA = 0;         // 160 columns
+constexpr uint32_t COL_WT = 160;          // 64
+constexpr uint32_t COL_UT = 224;          // 64
+constexpr uint32_t COL_OT = 288;          // 64
+constexpr uint32_t COL_ST = 384;          // 128
+constexpr uint32_t TMEM_COLS = 512;
+
+// Row offset of block R' in the concatenated B operand: 16 * R' * (R' + 1) / 2.
+__host__ __device__ constexpr int kr_off(int r) { return 8 * r * (r + 1); }
+constexpr uint32_t kWaitLimit = 1u << 24;
+
+__device__ __forceinline__ float fast_sigmoid(float x) {
+    return __fdividef(1.0f, 1.0f + __expf(-x));
+}
+
+__device__ __forceinline__ void st_u32(uint8_t *base, uint32_t off, uint32_t v) {
+    *reinterpret_cast<uint32_t *>(base + off) = v;
+}
+__device__ __forceinline__ void st_u128(uint8_t *base, uint32_t off, uint4 v) {
+    *reinterpret_cast<uint4 *>(base + off) = v;
+}
+
+// Wait for the MMA barrier; every thread of the CTA learns whether any gave up.
+__device__ __forceinline__ bool wait_mma(uint32_t mbar, uint32_t &phase) {
+    bool ok = mbar_wait(mbar, phase, kWaitLimit);
+    phase ^= 1u;
+    int failed = __syncthreads_or(ok ? 0 : 1);
+    fence_after_sync();
+    return failed == 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_tc_kernel(ChunkParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const uint32_t sbase = smem_addr(sm);
+    float *rq_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_RQ);
+    float *rk_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_RK);
+    float *beta_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_BETA);
+    float *red_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_RED);
+    float *tsum_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_TSUM);
+    float *gam_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GAMMA);
+    float *X_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_X);
+    float *Akk = reinterpret_cast<float *>(sm + OFF_AKK);
+    float *Tm = reinterpret_cast<float *>(sm + OFF_TINV);
+    const uint32_t mbar = sbase + OFF_MISC + MISC_MBAR;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TMEM);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chain = blockIdx.x;
+    const bool trans = blockIdx.y == 1;     // transition columns (v = 0, S0 = I)
+    const int b = chain / p.HV, hv = chain % p.HV, h = hv / p.group;
+    const int T = p.T;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
+    const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
+    const __nv_bfloat16 *gz = static_cast<const __nv_bfloat16 *>(p.g);
+    const __nv_bfloat16 *bl = static_cast<const __nv_bfloat16 *>(p.beta);
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
+
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        fence_mbar_init();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;   // this warp's TMEM quadrant
+    uint32_t phase = 0;
+    bool aborted = false;
+
+    // ---- initial state: S^T (TMEM fp32) and its bf16 copy (smem) ----------
+    if (warp >= 4) {
+        const int j = (warp - 4) * 32 + lane;
+        for (int m = 0; m < D / 16; ++m) {
+            float vals[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int c = m * 16 + u;
+                float s0 = 0.f;
+                if (trans) s0 = (c == j) ? 1.f : 0.f;
+                else if (p.S0) s0 = p.S0[((size_t)chain * D + c) * D + j];
+                vals[u] = s0;
+            }
+            tmem_st16(tm + lane_base + COL_ST + m * 16, vals);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint4 w4;
+                w4.x = pack_bf16x2(vals[hh * 8 + 0], vals[hh * 8 + 1]);
+                w4.y = pack_bf16x2(vals[hh * 8 + 2], vals[hh * 8 + 3]);
+                w4.z = pack_bf16x2(vals[hh * 8 + 4], vals[hh * 8 + 5]);
+                w4.w = pack_bf16x2(vals[hh * 8 + 6], vals[hh * 8 + 7]);
+                st_u128(sm, OFF_ST + kmaj_chunk_off(j, m * 2 + hh, 128), w4);
+            }
+        }
+        tmem_st_wait();
+    }
+
+    const float ea = p.gate_in ? __expf(p.A_log[hv]) : 0.f;
+    const int R = tid >> 6;            // prep: 16-token tile
+    const int cp = tid & 63;           // prep: channel pair
+    const int c0 = 2 * cp;
+    const float bias0 = (p.gate_in && p.dt_bias) ? p.dt_bias[(size_t)hv * D + c0] : 0.f;
+    const float bias1 = (p.gate_in && p.dt_bias) ? p.dt_bias[(size_t)hv * D + c0 + 1] : 0.f;
+
+    const int nchunks = (T + C - 1) / C;
+    for (int n = 0; n < nchunks && !aborted; ++n) {
+        const int t0 = n * C;
+        const int Cc = min(C, T - t0);
+        // =============== Phase A: load + preprocess (all 256 threads) ======
+        float qv[16][2], kv[16][2], gv[16][2];
+        float sq[16], sk[16];
+        float tile0 = 0.f, tile1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = R * 16 + i;
+            float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, g0 = 0.f, g1 = 0.f;
+            if (t < Cc) {
+                const size_t tok = (size_t)b * T + t0 + t;
+                const __nv_bfloat162 qq =
+                    *reinterpret_cast<const __nv_bfloat162 *>(q + (tok * p.H + h) * D + c0);
+                const __nv_bfloat162 kk =
+                    *reinterpret_cast<const __nv_bfloat162 *>(k + (tok * p.H + h) * D + c0);
+                const __nv_bfloat162 zz =
+                    *reinterpret_cast<const __nv_bfloat162 *>(gz + (tok * p.HV + hv) * D + c0);
+                q0 = __low2float(qq); q1 = __high2float(qq);
+                k0 = __low2float(kk); k1 = __high2float(kk);
+                g0 = __low2float(zz); g1 = __high2float(zz);
+                if (p.gate_in) {
+                    g0 = p.g_min * fast_sigmoid(ea * (g0 + bias0));
+                    g1 = p.g_min * fast_sigmoid(ea * (g1 + bias1));
+                }
+            }
+            qv[i][0] = q0; qv[i][1] = q1; kv[i][0] = k0; kv[i][1] = k1;
+            gv[i][0] = g0; gv[i][1] = g1;
+            sq[i] = q0 * q0 + q1 * q1;
+            sk[i] = k0 * k0 + k1 * k1;
+            tile0 += g0;
+            tile1 += g1;
+        }
+        if (p.l2norm) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], off);
+                    sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], off);
+                }
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    red_s[(warp * 16 + i) * 2 + 0] = sq[i];
+                    red_s[(warp * 16 + i) * 2 + 1] = sk[i];
+                }
+            }
+        }
+        tsum_s[R * D + c0] = tile0;
+        tsum_s[R * D + c0 + 1] = tile1;
+        if (cp < 16) {
+            const int t = R * 16 + cp;
+            float bb = 0.f;
+            if (t < Cc) {
+                bb = __bfloat162float(bl[((size_t)b * T + t0 + t) * p.HV + hv]);
+                if (p.beta_sigmoid) bb = fast_sigmoid(bb);
+            }
+            beta_s[t] = bb;
+        }
+        __syncthreads();
+        if (tid < 64) {
+            const int t = tid, w0 = (t >> 4) * 2, i = t & 15;
+            float rq = 1.f, rk = 1.f;
+            if (p.l2norm) {
+                rq = rsqrtf(red_s[(w0 * 16 + i) * 2 + 0] + red_s[((w0 + 1) * 16 + i) * 2 + 0] + p.l2_eps);
+                rk = rsqrtf(red_s[(w0 * 16 + i) * 2 + 1] + red_s[((w0 + 1) * 16 + i) * 2 + 1] + p.l2_eps);
+            }
+            rq_s[t] = rq;
+            rk_s[t] = rk;
+        }
+        // Tile-start cumulative sums P_R' for this channel pair.
+        float P[4][2], GC[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            float run = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                P[rr][x] = run;
+                run += tsum_s[rr * D + c0 + x];
+            }
+            GC[x] = run;
+        }
+        __syncthreads();
+        if (R == 0) {
+            gam_s[c0] = __expf(GC[0]);
+            gam_s[c0 + 1] = __expf(GC[1]);
+        }
+        float eP[2], eCP[2], Dn[4][2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const float PR = (R == 0) ? P[0][x] : (R == 1) ? P[1][x] : (R == 2) ? P[2][x] : P[3][x];
+            eP[x] = __expf(PR);
+            eCP[x] = __expf(GC[x] - PR);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) Dn[rr][x] = (rr >= R) ? __expf(P[rr][x] - PR) : 0.f;
+        }
+        float kg[2][16], kpv[2][16], vv[2][16];
+        float L0 = 0.f, L1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int t = R * 16 + i;
+            const float rq = rq_s[t], rk = rk_s[t];
+            L0 += gv[i][0];
+            L1 += gv[i][1];
+            const float e0 = __expf(L0), e1 = __expf(L1);
+            const float ei0 = __expf(-L0), ei1 = __expf(-L1);
+            const float kh0 = kv[i][0] * rk, kh1 = kv[i][1] * rk;
+            const float qh0 = qv[i][0] * rq, qh1 = qv[i][1] * rq;
+            st_u32(sm, OFF_AINTRA + kmaj_off(t, c0, 128), pack_bf16x2(kh0 * e0, kh1 * e1));
+            st_u32(sm, OFF_AINTRA + kmaj_off(64 + t, c0, 128), pack_bf16x2(qh0 * e0, qh1 * e1));
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                if (rr >= R)
+                    st_u32(sm, OFF_KRCAT + kmaj_off(kr_off(rr) + t, c0, 160),
+                           pack_bf16x2(kh0 * ei0 * Dn[rr][0], kh1 * ei1 * Dn[rr][1]));
+            }
+            st_u32(sm, OFF_QG + kmaj_off(t, c0, 64), pack_bf16x2(qh0 * e0 * eP[0], qh1 * e1 * eP[1]));
+            kg[0][i] = kh0 * e0 * eP[0];
+            kg[1][i] = kh1 * e1 * eP[1];
+            kpv[0][i] = kh0 * ei0 * eCP[0];
+            kpv[1][i] = kh1 * ei1 * eCP[1];
+            float v0 = 0.f, v1 = 0.f;
+            if (!trans && t < Cc) {
+                const __nv_bfloat162 vv2 = *reinterpret_cast<const __nv_bfloat162 *>(
+                    v + (((size_t)b * T + t0 + t) * p.HV + hv) * D + c0);
+                v0 = __low2float(vv2);
+                v1 = __high2float(vv2);
+            }
+            vv[0][i] = v0;
+            vv[1][i] = v1;
+        }
+        // Channel-major tiles: rows c0, c0+1; this thread's 16 tokens are chunks 2R, 2R+1.
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int ch = 2 * R + hh;
+                uint4 a, bq, cq;
+                a.x = pack_bf16x2(kg[x][hh * 8 + 0], kg[x][hh * 8 + 1]);
+                a.y = pack_bf16x2(kg[x][hh * 8 + 2], kg[x][hh * 8 + 3]);
+                a.z = pack_bf16x2(kg[x][hh * 8 + 4], kg[x][hh * 8 + 5]);
+                a.w = pack_bf16x2(kg[x][hh * 8 + 6], kg[x][hh * 8 + 7]);
+                bq.x = pack_bf16x2(kpv[x][hh * 8 + 0], kpv[x][hh * 8 + 1]);
+                bq.y = pack_bf16x2(kpv[x][hh * 8 + 2], kpv[x][hh * 8 + 3]);
+                bq.z = pack_bf16x2(kpv[x][hh * 8 + 4], kpv[x][hh * 8 + 5]);
+                bq.w = pack_bf16x2(kpv[x][hh * 8 + 6], kpv[x][hh * 8 + 7]);
+                cq.x = pack_bf16x2(vv[x][hh * 8 + 0], vv[x][hh * 8 + 1]);
+                cq.y = pack_bf16x2(vv[x][hh * 8 + 2], vv[x][hh * 8 + 3]);
+                cq.z = pack_bf16x2(vv[x][hh * 8 + 4], vv[x][hh * 8 + 5]);
+                cq.w = pack_bf16x2(vv[x][hh * 8 + 6], vv[x][hh * 8 + 7]);
+                st_u128(sm, OFF_KGT + kmaj_chunk_off(c0 + x, ch, 128), a);
+                st_u128(sm, OFF_KP + kmaj_chunk_off(c0 + x, ch, 128), bq);
+                st_u128(sm, OFF_VT + kmaj_chunk_off(c0 + x, ch, 128), cq);
+            }
+        }
+        fence_async_smem();
+        __syncthreads();
+
+        // =============== (I) intra-chunk products ============================
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id = idesc_bf16(128, 160);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tm + COL_INTRA, kmaj_desc(sbase + OFF_AINTRA, 128, s),
+                         kmaj_desc(sbase + OFF_KRCAT, 160, s), id, s > 0);
+            mma_commit(mbar);
+        }
+        if (!wait_mma(mbar, phase)) { aborted = true; break; }
+
+        // =============== read A_kk (fp32 smem) and A_qk (bf16 operand) ======
+        if (warp < 4) {
+            const int rr = (warp & 1) * 32 + lane;         // row within A_kk / A_qk
+            const int Rr = rr >> 4;
+            const int nvalid = 16 * (Rr + 1);
+            const int off = kr_off(Rr);
+            const bool is_qk = warp >= 2;
+            const int cbeg = (warp & 1) ? 48 : 0;
+            const int nld = (warp & 1) ? 7 : 3;
+            const float br = beta_s[rr];
+            for (int m = 0; m < nld; ++m) {
+                float vals[16];
+                tmem_ld16(tm + lane_base + COL_INTRA + cbeg + m * 16, vals);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = cbeg + m * 16 + u - off;
+                    if (i >= 0 && i < nvalid) {
+                        if (is_qk) {
+                            const float a = (i <= rr) ? vals[u] : 0.f;
+                            *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_AQK + kmaj_off(rr, i, 64)) =
+                                __float2bfloat16_rn(a);
+                        } else {
+                            Akk[rr * 65 + i] = (i < rr) ? br * vals[u] : 0.f;
+                        }
+                    }
+                }
+            }
+            for (int i = nvalid; i < C; ++i) {
+                if (is_qk)
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_AQK + kmaj_off(rr, i, 64)) =
+                        __float2bfloat16_rn(0.f);
+                else
+                    Akk[rr * 65 + i] = 0.f;
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+
+        // =============== solve T = (I + A_kk)^-1, blocked ===================
+        if (tid < 64) {
+            const int bb = tid >> 4, j = tid & 15;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int r = 1; r < 16; ++r) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < r; ++i) acc = fmaf(Akk[(16 * bb + r) * 65 + 16 * bb + i], x[i], acc);
+                if (r > j) x[r] = -acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tm[(16 * bb + r) * 65 + 16 * bb + j] = (r >= j) ? x[r] : 0.f;
+        }
+        __syncthreads();
+        for (int d = 1; d < 4; ++d) {
+            const int er = tid >> 4, ec = tid & 15;
+            for (int I = d; I < 4; ++I) {
+                const int J = I - d;
+                float acc = 0.f;
+                for (int K = J; K < I; ++K) {
+#pragma unroll
+                    for (int m = 0; m < 16; ++m)
+                        acc = fmaf(Akk[(16 * I + er) * 65 + 16 * K + m], Tm[(16 * K + m) * 65 + 16 * J + ec], acc);
+                }
+                X_s[((I - d) * 16 + er) * 17 + ec] = acc;
+            }
+            __syncthreads();
+            for (int I = d; I < 4; ++I) {
+                const int J = I - d;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(Tm[(16 * I + er) * 65 + 16 * I + m], X_s[((I - d) * 16 + m) * 17 + ec], acc);
+                Tm[(16 * I + er) * 65 + 16 * J + ec] = -acc;
+            }
+            __syncthreads();
+        }
+        // T Diag(beta) -> bf16 K-major [r][i]
+        {
+            const int r = tid >> 2, ib = (tid & 3) * 16;
+#pragma unroll
+            for (int u = 0; u < 16; u += 2) {
+                const int i = ib + u;
+                const float a0 = (i <= r) ? Tm[r * 65 + i] * beta_s[i] : 0.f;
+                const float a1 = (i + 1 <= r) ? Tm[r * 65 + i + 1] * beta_s[i + 1] : 0.f;
+                st_u32(sm, OFF_TB + kmaj_off(r, i, 64), pack_bf16x2(a0, a1));
+            }
+        }
+        fence_async_smem();
+        __syncthreads();
+
+        // =============== (II) Ut^T = V^T TB^T, (III) W^T = KG^T TB^T ========
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id = idesc_bf16(128, 64);
+            if (!trans) {
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tm + COL_UT, kmaj_desc(sbase + OFF_VT, 128, s),
+                             kmaj_desc(sbase + OFF_TB, 64, s), id, s > 0);
+            }
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tm + COL_WT, kmaj_desc(sbase + OFF_KGT, 128, s),
+                         kmaj_desc(sbase + OFF_TB, 64, s), id, s > 0);
+            mma_commit(mbar);
+        }
+        if (!wait_mma(mbar, phase)) { aborted = true; break; }
+
+        // W^T (lane = channel c) -> W [t][c] bf16
+        if (warp < 4) {
+            const int c = warp * 32 + lane;
+            for (int m = 0; m < C / 16; ++m) {
+                float vals[16];
+                tmem_ld16(tm + lane_base + COL_WT + m * 16, vals);
+#pragma unroll
+                for (int u = 0; u < 16; ++u)
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_W + kmaj_off(m * 16 + u, c, 64)) =
+                        __float2bfloat16_rn(vals[u]);
+            }
+        }
+        fence_before_sync();
+        fence_async_smem();
+        __syncthreads();
+
+        // =============== (IV) U^T = Ut^T - S^T W^T ==========================
+        if (tid == 0) {
+            fence_after_sync();
+            const uint32_t id = idesc_bf16(128, 64, /*negate_a=*/true);
+#pragma unroll
+            for (int s = 0; s < D / 16; ++s)
+                mma_bf16(tm + COL_UT, kmaj_desc(sbase + OFF_ST, 128, s),
+                         kmaj_desc(sbase + OFF_W, 64, s), id, (trans && s == 0) ? 0u : 1u);
+            mma_commit(mbar);
+        }
+        if (!wait_mma(mbar, phase)) { aborted = true; break; }
+
+        if (warp < 4) {
+            // U^T row j -> bf16 operand
+            const int j = warp * 32 + lane;
+            for (int m = 0; m < C / 16; ++m) {
+                float vals[16];
+                tmem_ld16(tm + lane_base + COL_UT + m * 16, vals);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint4 w4;
+                    w4.x = pack_bf16x2(vals[hh * 8 + 0], vals[hh * 8 + 1]);
+                    w4.y = pack_bf16x2(vals[hh * 8 + 2], vals[hh * 8 + 3]);
+                    w4.z = pack_bf16x2(vals[hh * 8 + 4], vals[hh * 8 + 5]);
+                    w4.w = pack_bf16x2(vals[hh * 8 + 6], vals[hh * 8 + 7]);
+                    st_u128(sm, OFF_UT + kmaj_chunk_off(j, m * 2 + hh, 64), w4);
+                }
+            }
+        } else {
+            // S^T <- S^T Diag(gamma_C) in place (fp32, TMEM)
+            for (int m = 0; m < D / 16; ++m) {
+                float vals[16];
+                tmem_ld16(tm + lane_base + COL_ST + m * 16, vals);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) vals[u] *= gam_s[m * 16 + u];
+                tmem_st16(tm + lane_base + COL_ST + m * 16, vals);
+            }
+            tmem_st_wait();
+        }
+        fence_before_sync();
+        fence_async_smem();
+        __syncthreads();
+
+        // =============== (V) O^T, (VI) S^T += U^T K' ========================
+        if (tid == 0) {
+            fence_after_sync();
+            if (!trans) {
+                const uint32_t id = idesc_bf16(128, 64);
+#pragma unroll
+                for (int s = 0; s < D / 16; ++s)
+                    mma_bf16(tm + COL_OT, kmaj_desc(sbase + OFF_ST, 128, s),
+                             kmaj_desc(sbase + OFF_QG, 64, s), id, s > 0);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(tm + COL_OT, kmaj_desc(sbase + OFF_UT, 128, s),
+                             kmaj_desc(sbase + OFF_AQK, 64, s), id, 1u);
+            }
+            const uint32_t id2 = idesc_bf16(128, 128);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tm + COL_ST, kmaj_desc(sbase + OFF_UT, 128, s),
+                         kmaj_desc(sbase + OFF_KP, 128, s), id2, 1u);
+            mma_commit(mbar);
+        }
+        if (!wait_mma(mbar, phase)) { aborted = true; break; }
+
+        if (warp < 4) {
+            if (!trans) {
+                const int j = warp * 32 + lane;
+                for (int m = 0; m < C / 16; ++m) {
+                    float vals[16];
+                    tmem_ld16(tm + lane_base + COL_OT + m * 16, vals);
+    #pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        const int t = m * 16 + u;
+                        if (t < Cc)
+                            o[(((size_t)b * T + t0 + t) * p.HV + hv) * D + j] =
+                                __float2bfloat16_rn(p.scale * vals[u]);
+                    }
+                }
+            }
+        } else {
+            const int j = (warp - 4) * 32 + lane;
+            for (int m = 0; m < D / 16; ++m) {
+                float vals[16];
+                tmem_ld16(tm + lane_base + COL_ST + m * 16, vals);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint4 w4;
+                    w4.x = pack_bf16x2(vals[hh * 8 + 0], vals[hh * 8 + 1]);
+                    w4.y = pack_bf16x2(vals[hh * 8 + 2], vals[hh * 8 + 3]);
+                    w4.z = pack_bf16x2(vals[hh * 8 + 4], vals[hh * 8 + 5]);
+                    w4.w = pack_bf16x2(vals[hh * 8 + 6], vals[hh * 8 + 7]);
+                    st_u128(sm, OFF_ST + kmaj_chunk_off(j, m * 2 + hh, 128), w4);
+                }
+            }
+        }
+        fence_before_sync();
+        fence_async_smem();
+        __syncthreads();
+    }
+
+    // ---- final state -------------------------------------------------------
+    if (!aborted && warp >= 4) {
+        const int j = (warp - 4) * 32 + lane;
+        float *out = trans ? p.M_T : p.S_T;
+        if (out) {
+            for (int m = 0; m < D / 16; ++m) {
+                float vals[16];
+                tmem_ld16(tm + lane_base + COL_ST + m * 16, vals);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) out[((size_t)chain * D + m * 16 + u) * D + j] = vals[u];
+            }
+        }
+    }
+    if (aborted && tid == 0) atomicOr(&g_device_error, 1u);
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tm, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
 bool chunk_tc_supported(const ChunkParams &p, bool bf16) {
-    (void)p;
-    (void)bf16;
-    return false;
+    return bf16 && p.Dk == D && p.Dv == D && p.C == C;
 }
 
 cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s) {
-    (void)p;
-    (void)s;
-    return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.B * p.HV, p.M_T ? 2 : 1);
+    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t s, unsigned int *out) {

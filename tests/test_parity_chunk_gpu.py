@@ -153,3 +153,97 @@ def test_prefill_bf16_workload_simt(cuda_device):
     ref = oracle_chunk(inp)
     o, S_T, _ = run_gpu(to_device(inp, cuda_device), w, "simt")
     check(o, S_T, None, ref, "bf16", "simt")
+
+
+# ---------------------------------------------------------------------------
+# Tensor-core kernel (bf16, Dk = Dv = 128, chunk = 64)
+# ---------------------------------------------------------------------------
+TC_CASES = [
+    # B, T, H, HV, s0_std, want_M, z_mean
+    (1, 64, 1, 1, None, False, 0.0),      # one chunk, no initial state
+    (1, 192, 1, 2, 0.02, False, 0.0),     # three chunks, carried state
+    (2, 200, 2, 4, 0.02, True, 0.0),      # ragged tail, grouped heads, transition
+    (1, 256, 1, 2, 0.05, True, -8.0),     # slow decay: long memory, M_T far from 0
+    (1, 128, 1, 1, 0.05, False, 12.0),    # g = g_min every token: e^-320 per chunk
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "B%d_T%d_H%d_HV%d_M%d_z%g" % (
+    c[0], c[1], c[2], c[3], c[5], c[6]))
+def test_tc_small(cuda_device, case):
+    B, T, H, HV, s0, want_M, z_mean = case
+    w = workloads.Workload("tc", B=B, T=T, H=H, HV=HV, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                           seed=31 + T, a_log="uniform", dt_bias_std=0.5, s0_std=s0)
+    inp = workloads.chunk_inputs(w, z_mean=z_mean)
+    ref = oracle_chunk(inp, want_M=want_M)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "tc", want_M=want_M)
+    check(o, S_T, M_T, ref, "bf16", "tc")
+
+
+def test_tc_switches_off(cuda_device):
+    w = workloads.Workload("tcoff", B=1, T=130, H=1, HV=2, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                           seed=41, s0_std=0.05)
+    inp = workloads.activated_inputs(w)
+    ref = oracle_chunk(inp, flags=False, want_M=True)
+    o, S_T, M_T = run_gpu(to_device(inp, cuda_device), w, "tc", flags=False, want_M=True)
+    check(o, S_T, M_T, ref, "bf16", "tc")
+
+
+def test_tc_is_the_default_for_its_shape(cuda_device):
+    """algo='auto' picks the tensor-core kernel for bf16 / 128 / chunk 64: its
+    result equals the explicit 'tc' call bit for bit."""
+    w = workloads.Workload("auto", B=1, T=128, H=1, HV=1, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                           seed=43, s0_std=0.02)
+    d = to_device(workloads.chunk_inputs(w), cuda_device)
+    o1, S1, _ = run_gpu(d, w, "auto")
+    o2, S2, _ = run_gpu(d, w, "tc")
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_prefill_bf16_workload_tc(cuda_device):
+    """B=1, H=HV=16, T=4096, Dk=Dv=128, chunk=64, bf16, S0 ~ N(0, 0.02)."""
+    w = workloads.workload("prefill_bf16")
+    inp = workloads.chunk_inputs(w)
+    ref = oracle_chunk(inp)
+    o, S_T, _ = run_gpu(to_device(inp, cuda_device), w, "tc")
+    check(o, S_T, None, ref, "bf16", "tc")
+
+
+def test_gva_bf16_workload_sampled(cuda_device):
+    """B=4, H=16, HV=32, T=8192, Dk=Dv=128, chunk=64, in-kernel switches, in the
+    launch configuration the benchmark times; the oracle checks sampled chains
+    (first, last and two grouped value heads of one q/k head)."""
+    w = workloads.workload("gva_bf16")
+    inp = workloads.chunk_inputs(w)
+    o, S_T, _ = run_gpu(to_device(inp, cuda_device), w, "auto")
+    chains = [(0, 0), (0, 1), (2, 17), (3, 31)]
+    refs = oracle_chunk(inp, chains=chains)
+    o_np, S_np = o.float().cpu(), S_T.cpu()
+    for (b, hv), r in refs.items():
+        assert max_rel(to_np(o_np[b:b + 1, :, hv:hv + 1]), r["o"]) <= TOL_BF16
+        assert fro_rel(to_np(S_np[b:b + 1, hv:hv + 1]), r["S_T"]) <= TOL_BF16
+
+
+def test_kcp_workload_segmented_tc(cuda_device):
+    """B=1, H=HV=16, T=65536 as 8 segments of 8192: segments with transitions in
+    one batched launch, the combine, and the rerun from the combined states give
+    the unsegmented pass (compared on sampled heads with the oracle, and in full
+    with the unsegmented GPU pass)."""
+    w = workloads.workload("kcp_bf16")
+    inp = workloads.chunk_inputs(w)
+    d = to_device(inp, cuda_device)
+    L = w.T // w.n_seg
+    seg = {n: d[n].view(w.n_seg, L, *d[n].shape[2:]) for n in ("q", "k", "v", "g", "beta")}
+    kw = dict(A_log=d["A_log"], chunk=w.chunk, algo="tc")
+    _, S_loc, M_loc = kda.kda_chunk_fwd(seg["q"], seg["k"], seg["v"], seg["g"], seg["beta"],
+                                        output_transition=True, **kw)
+    S_in = kda.kda_compose(M_loc, S_loc, d["S0"].view(w.HV, 128, 128))
+    o_seg, _, _ = kda.kda_chunk_fwd(seg["q"], seg["k"], seg["v"], seg["g"], seg["beta"],
+                                    S0=S_in[:w.n_seg].contiguous(), output_final_state=False, **kw)
+    o_full, S_full, _ = kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S0=d["S0"], **kw)
+    assert fro_rel(to_np(S_in[-1]), to_np(S_full[0])) <= TOL_BF16
+    assert max_rel(to_np(o_seg.reshape(o_full.shape)), to_np(o_full)) <= TOL_BF16
+    refs = oracle_chunk(inp, chains=[(0, 0), (0, 9)])
+    for (b, hv), r in refs.items():
+        assert max_rel(to_np(o_seg.reshape(o_full.shape)[:, :, hv:hv + 1]), r["o"]) <= TOL_BF16
+        assert fro_rel(to_np(S_in[-1][hv:hv + 1]), r["S_T"][0]) <= TOL_BF16
