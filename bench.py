@@ -153,39 +153,28 @@ def barrier(world, device):
     torch.cuda.synchronize(device)
 
 
-def cpu_baseline(w, inp_cpu, target_s=12.0):
-    """Time the FP64 oracle, as it stands, on a bounded sample of workload w:
-    the first n_chains (b, hv) chains over the first T_s tokens."""
+def cpu_baseline(w):
+    """Time the FP64 oracle, as it stands, on the host cores: the whole
+    workload w (every chain, every token) generated on the CPU with the same
+    recipe, so no sampling is needed; the oracle parallelises over chains."""
     import oracle
-    import numpy as np
     import torch
+    import workloads
 
     def f64(t):
         return None if t is None else t.to(torch.float64).numpy()
 
-    cores = oracle.num_threads()
-
-    def run(nb, nh, T_s):
-        sl = {n: inp_cpu[n][:nb, :T_s] for n in ("q", "k", "v", "g", "beta")}
-        hq = max(1, nh // (w.HV // w.H))
-        t0 = time.perf_counter()
-        oracle.kda_fwd(f64(sl["q"][:, :, :hq]), f64(sl["k"][:, :, :hq]),
-                       f64(sl["v"][:, :, :nh]), f64(sl["g"][:, :, :nh]), f64(sl["beta"][:, :, :nh]),
-                       A_log=f64(inp_cpu["A_log"][:nh]),
-                       dt_bias=None if inp_cpu["dt_bias"] is None else f64(inp_cpu["dt_bias"][:nh]))
-        return time.perf_counter() - t0
-
-    # Calibrate on a small sample, then size the sample for about target_s seconds.
-    nh = min(w.HV, max(2, cores))
-    t_cal = run(1, nh, 256)
-    per_token = t_cal / (256.0)
-    T_s = int(min(w.T, max(256, target_s / max(per_token, 1e-9))))
-    T_s = max(64, (T_s // 64) * 64)
-    dt = run(1, nh, T_s)
-    units = nh * T_s
-    return {"value": units / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": "FP64 oracle, %d value heads x %d tokens of the B=4,HV=32,T=8192 workload "
-                      "(%.1f s wall)" % (nh, T_s, dt)}
+    inp = workloads.chunk_inputs(w)
+    arrays = [f64(inp[n]) for n in ("q", "k", "v", "g", "beta")]
+    kw = dict(A_log=f64(inp["A_log"]), dt_bias=f64(inp["dt_bias"]), S0=f64(inp["S0"]))
+    del inp
+    t0 = time.perf_counter()
+    oracle.kda_fwd(*arrays, **kw)
+    dt = time.perf_counter() - t0
+    return {"value": w.token_heads / dt, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "FP64 oracle on the whole B=%d,HV=%d,T=%d workload (%d chains, %.1f s wall)"
+                      % (w.B, w.HV, w.T, w.B * w.HV, dt)}
 
 
 def run_reference(args):
@@ -253,6 +242,9 @@ def main():
     ap.add_argument("--algo", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--decode-steps", type=int, default=512)
     ap.add_argument("--no-extras", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override B of the headline workload (small cases for profiling)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -270,6 +262,8 @@ def main():
 
     # ---------------- headline: chunked forward, B=4 HV=32 T=8192 -------------
     w = workloads.workload("gva_bf16")
+    if args.batch is not None:
+        w = workloads.workload("gva_bf16", B=args.batch)
     inp = workloads.chunk_inputs(w, seed=w.seed + 1000 * rank, device=dev)
     o = torch.empty((w.B, w.T, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((w.B, w.HV, w.Dk, w.Dv), dtype=torch.float32, device=dev)
@@ -302,7 +296,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": "gva_bf16: B=4 H=16 HV=32 T=8192 Dk=Dv=128 chunk=64 per GPU, "
+            "config": {"workload": "gva_bf16: B=%d H=16 HV=32 T=8192 Dk=Dv=128 chunk=64 per GPU, " % w.B +
                                    "bf16 q/k/v/z/beta, fp32 state; l2norm, beta sigmoid, gate in-kernel",
                        "algo": args.algo, "l2": "inputs larger than L2 (%.2f GB read per step)"
                                                 % (nbytes / 1e9),
@@ -352,9 +346,8 @@ def main():
         line["gpu_launches_extras"] = {"decode": line["decode"]["launches"],
                                        "kcp": line["kcp"]["launches"]}
 
-    if rank == 0 and world == 1:
-        inp_cpu = workloads.chunk_inputs(workloads.workload("gva_bf16", B=1, T=8192))
-        line["cpu_baseline"] = cpu_baseline(w, inp_cpu)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -73,11 +73,13 @@ constexpr uint32_t MISC_TMEM = 7688;      // uint32
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 7696 + 1024;   // + alignment slack
 
 // TMEM columns.
-constexpr uint32_t COL_INTRA = 0;         // 160 columns
-constexpr uint32_t COL_WT = 160;          // 64
-constexpr uint32_t COL_UT = 224;          // 64
-constexpr uint32_t COL_OT = 288;          // 64
-constexpr uint32_t COL_ST = 384;          // 128
+constexpr uint32_t COL_INTRA = 0;         // 160 columns: A_kk / A_qk products
+constexpr uint32_t COL_WT = 0;            // 64: W^T (after the A readout)
+constexpr uint32_t COL_UT = 160;          // 64: Ut^T, then U^T
+constexpr uint32_t COL_OT = 224;          // 64: O^T
+constexpr uint32_t COL_SBF = 288;         // 64: S^T as packed bf16 (MMA A operand)
+constexpr uint32_t COL_UBF = 352;         // 32: U^T as packed bf16 (MMA A operand)
+constexpr uint32_t COL_ST = 384;          // 128: S^T fp32
 constexpr uint32_t TMEM_COLS = 512;
 
 // Row offset of block R' in the concatenated B operand: 16 * R' * (R' + 1) / 2.
@@ -164,15 +166,10 @@ chunk_tc_kernel(ChunkParams p) {
                 vals[u] = s0;
             }
             tmem_st16(tm + lane_base + COL_ST + m * 16, vals);
+            uint32_t pk[8];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint4 w4;
-                w4.x = pack_bf16x2(vals[hh * 8 + 0], vals[hh * 8 + 1]);
-                w4.y = pack_bf16x2(vals[hh * 8 + 2], vals[hh * 8 + 3]);
-                w4.z = pack_bf16x2(vals[hh * 8 + 4], vals[hh * 8 + 5]);
-                w4.w = pack_bf16x2(vals[hh * 8 + 6], vals[hh * 8 + 7]);
-                st_u128(sm, OFF_ST + kmaj_chunk_off(j, m * 2 + hh, 128), w4);
-            }
+            for (int u = 0; u < 8; ++u) pk[u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+            tmem_st8(tm + lane_base + COL_SBF + m * 8, pk);
         }
         tmem_st_wait();
     }
@@ -468,16 +465,21 @@ chunk_tc_kernel(ChunkParams p) {
         }
         if (!wait_mma(mbar, phase)) { aborted = true; break; }
 
-        // W^T (lane = channel c) -> W [t][c] bf16
+        // W^T (lane = channel c) -> -W as an MN-major operand: row c holds t = 0..63
         if (warp < 4) {
             const int c = warp * 32 + lane;
             for (int m = 0; m < C / 16; ++m) {
                 float vals[16];
                 tmem_ld16(tm + lane_base + COL_WT + m * 16, vals);
 #pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_W + kmaj_off(m * 16 + u, c, 64)) =
-                        __float2bfloat16_rn(vals[u]);
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint4 w4;
+                    w4.x = pack_bf16x2(-vals[hh * 8 + 0], -vals[hh * 8 + 1]);
+                    w4.y = pack_bf16x2(-vals[hh * 8 + 2], -vals[hh * 8 + 3]);
+                    w4.z = pack_bf16x2(-vals[hh * 8 + 4], -vals[hh * 8 + 5]);
+                    w4.w = pack_bf16x2(-vals[hh * 8 + 6], -vals[hh * 8 + 7]);
+                    st_u128(sm, OFF_W + mnmaj_chunk_off(c, m * 2 + hh), w4);
+                }
             }
         }
         fence_before_sync();
@@ -487,31 +489,26 @@ chunk_tc_kernel(ChunkParams p) {
         // =============== (IV) U^T = Ut^T - S^T W^T ==========================
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t id = idesc_bf16(128, 64, /*negate_a=*/true);
+            const uint32_t id = idesc_bf16(128, 64, false, /*b_mn_major=*/true);
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
-                mma_bf16(tm + COL_UT, kmaj_desc(sbase + OFF_ST, 128, s),
-                         kmaj_desc(sbase + OFF_W, 64, s), id, (trans && s == 0) ? 0u : 1u);
+                mma_bf16_tmem_a(tm + COL_UT, tm + COL_SBF + s * 8, mnmaj_desc(sbase + OFF_W, s), id,
+                                (trans && s == 0) ? 0u : 1u);
             mma_commit(mbar);
         }
         if (!wait_mma(mbar, phase)) { aborted = true; break; }
 
         if (warp < 4) {
-            // U^T row j -> bf16 operand
-            const int j = warp * 32 + lane;
+            // U^T row j -> packed bf16 A operand in TMEM
             for (int m = 0; m < C / 16; ++m) {
                 float vals[16];
                 tmem_ld16(tm + lane_base + COL_UT + m * 16, vals);
+                uint32_t pk[8];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint4 w4;
-                    w4.x = pack_bf16x2(vals[hh * 8 + 0], vals[hh * 8 + 1]);
-                    w4.y = pack_bf16x2(vals[hh * 8 + 2], vals[hh * 8 + 3]);
-                    w4.z = pack_bf16x2(vals[hh * 8 + 4], vals[hh * 8 + 5]);
-                    w4.w = pack_bf16x2(vals[hh * 8 + 6], vals[hh * 8 + 7]);
-                    st_u128(sm, OFF_UT + kmaj_chunk_off(j, m * 2 + hh, 64), w4);
-                }
+                for (int u = 0; u < 8; ++u) pk[u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+                tmem_st8(tm + lane_base + COL_UBF + m * 8, pk);
             }
+            tmem_st_wait();
         } else {
             // S^T <- S^T Diag(gamma_C) in place (fp32, TMEM)
             for (int m = 0; m < D / 16; ++m) {
@@ -534,18 +531,18 @@ chunk_tc_kernel(ChunkParams p) {
                 const uint32_t id = idesc_bf16(128, 64);
 #pragma unroll
                 for (int s = 0; s < D / 16; ++s)
-                    mma_bf16(tm + COL_OT, kmaj_desc(sbase + OFF_ST, 128, s),
-                             kmaj_desc(sbase + OFF_QG, 64, s), id, s > 0);
+                    mma_bf16_tmem_a(tm + COL_OT, tm + COL_SBF + s * 8,
+                                    kmaj_desc(sbase + OFF_QG, 64, s), id, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(tm + COL_OT, kmaj_desc(sbase + OFF_UT, 128, s),
-                             kmaj_desc(sbase + OFF_AQK, 64, s), id, 1u);
+                    mma_bf16_tmem_a(tm + COL_OT, tm + COL_UBF + s * 8,
+                                    kmaj_desc(sbase + OFF_AQK, 64, s), id, 1u);
             }
             const uint32_t id2 = idesc_bf16(128, 128);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16(tm + COL_ST, kmaj_desc(sbase + OFF_UT, 128, s),
-                         kmaj_desc(sbase + OFF_KP, 128, s), id2, 1u);
+                mma_bf16_tmem_a(tm + COL_ST, tm + COL_UBF + s * 8,
+                                kmaj_desc(sbase + OFF_KP, 128, s), id2, 1u);
             mma_commit(mbar);
         }
         if (!wait_mma(mbar, phase)) { aborted = true; break; }
@@ -566,20 +563,15 @@ chunk_tc_kernel(ChunkParams p) {
                 }
             }
         } else {
-            const int j = (warp - 4) * 32 + lane;
             for (int m = 0; m < D / 16; ++m) {
                 float vals[16];
                 tmem_ld16(tm + lane_base + COL_ST + m * 16, vals);
+                uint32_t pk[8];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint4 w4;
-                    w4.x = pack_bf16x2(vals[hh * 8 + 0], vals[hh * 8 + 1]);
-                    w4.y = pack_bf16x2(vals[hh * 8 + 2], vals[hh * 8 + 3]);
-                    w4.z = pack_bf16x2(vals[hh * 8 + 4], vals[hh * 8 + 5]);
-                    w4.w = pack_bf16x2(vals[hh * 8 + 6], vals[hh * 8 + 7]);
-                    st_u128(sm, OFF_ST + kmaj_chunk_off(j, m * 2 + hh, 128), w4);
-                }
+                for (int u = 0; u < 8; ++u) pk[u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+                tmem_st8(tm + lane_base + COL_SBF + m * 8, pk);
             }
+            tmem_st_wait();
         }
         fence_before_sync();
         fence_async_smem();

@@ -43,12 +43,33 @@ __device__ __forceinline__ uint64_t kmaj_desc(uint32_t base, int rows, int s) {
     return d;
 }
 
-// Instruction descriptor: BF16 x BF16 -> FP32, both operands K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false) {
+// MN-major SW128 operand (the non-reduced index contiguous): a tile with K rows
+// of 64 MN-elements (128 B each), eight K-rows per 1024-byte atom, 16-byte
+// chunk j of K-row r at position j ^ (r % 8).  Used for an N = 64 operand, so
+// there is a single 64-element MN block.  k-step s (16 K-rows) starts 2048 * s
+// bytes in; SBO (between 8-row K groups) = 1024 B.
+__device__ __forceinline__ uint32_t mnmaj_chunk_off(int krow, int chunk) {
+    return (uint32_t)(krow * 128 + ((chunk ^ (krow & 7)) << 4));
+}
+__device__ __forceinline__ uint64_t mnmaj_desc(uint32_t base, int s) {
+    const uint32_t addr = base + (uint32_t)(s * 2048);
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(8192u >> 4) << 16;       // leading byte offset: next 64-element MN block
+    d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset: 8 K-rows x 128 B
+    d |= (uint64_t)1u << 46;                 // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                 // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: BF16 x BF16 -> FP32.  A and B are K-major unless
+// `b_mn_major`; an A operand read from TMEM is always K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false,
+                                                  bool b_mn_major = false) {
     return (1u << 4)                          // D format: f32
            | (1u << 7)                        // A format: bf16
            | (1u << 10)                       // B format: bf16
            | ((negate_a ? 1u : 0u) << 13)     // negate A
+           | ((b_mn_major ? 1u : 0u) << 16)   // B major-ness
            | ((uint32_t)(N >> 3) << 17)       // N / 8
            | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
@@ -61,6 +82,19 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
         :
         : "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// A operand from tensor memory (M = 128 lanes; 16 bf16 K-elements packed in 8
+// columns, lower K index in the lower half of each 32-bit cell).
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -152,6 +186,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
           "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
           "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
           "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        :
+        : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+          "r"(v[7])
         : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() {
