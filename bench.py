@@ -121,7 +121,12 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def dist_setup(n):
+def dist_setup(n, backend="nccl"):
+    """Rank/world from the torchrun environment; one process group per job.
+
+    Ranks shard the work by batch (each runs its own independent batch of the
+    workload, seeded by rank_seed), so the only collectives are the timing
+    barrier and the max-over-ranks reduction."""
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -129,13 +134,26 @@ def dist_setup(n):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=300), **kw)
     return world, rank, local
 
 
+def rank_seed(w, rank):
+    """Seed of rank `rank`'s batch: every rank draws an independent batch."""
+    return w.seed + 1000 * rank
+
+
+def whole_job_value(units_per_rank, world, ms):
+    """Throughput of the whole job: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def max_over_ranks(x, world, device):
+    """Max of a host float over the ranks (on `device`: cuda for NCCL, cpu for gloo)."""
     if world == 1:
         return x
     import torch
@@ -149,8 +167,12 @@ def barrier(world, device):
     import torch
     if world > 1:
         import torch.distributed as dist
-        dist.barrier(device_ids=[device.index])
-    torch.cuda.synchronize(device)
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+    if device.type == "cuda":
+        torch.cuda.synchronize(device)
 
 
 def cpu_baseline(w):
@@ -264,7 +286,7 @@ def main():
     w = workloads.workload("gva_bf16")
     if args.batch is not None:
         w = workloads.workload("gva_bf16", B=args.batch)
-    inp = workloads.chunk_inputs(w, seed=w.seed + 1000 * rank, device=dev)
+    inp = workloads.chunk_inputs(w, seed=rank_seed(w, rank), device=dev)
     o = torch.empty((w.B, w.T, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
     S_T = torch.empty((w.B, w.HV, w.Dk, w.Dv), dtype=torch.float32, device=dev)
 
@@ -286,7 +308,7 @@ def main():
     ms_local = sum(per) / len(per)
     ms = max_over_ranks(ms_local, world, dev)
     units = w.token_heads
-    value = world * units / (ms * 1e-3)
+    value = whole_job_value(units, world, ms)
     flops = units * chunk_flops_per_token_head(w.Dk, w.Dv, w.chunk)
     nbytes = chunk_bytes(w)
     achieved_gbs = nbytes / (ms_local * 1e-3) / 1e9
@@ -335,7 +357,7 @@ def main():
     per_e2e = time_launches(e2e_step, n_e2e, stream)
     barrier(world, dev)
     ms_e2e = max_over_ranks(sum(per_e2e) / len(per_e2e), world, dev)
-    line["e2e"] = {"value": world * units / (ms_e2e * 1e-3), "unit": UNIT,
+    line["e2e"] = {"value": whole_job_value(units, world, ms_e2e), "unit": UNIT,
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "ms_per_step": ms_e2e, "api": "gated_delta_rule_157_b200.kda_chunk_fwd"}
     del host, dev_in, h_o, h_S
@@ -361,9 +383,9 @@ def bench_decode(args, kda, workloads, dev, stream, pk, world, rank):
     """512 consecutive decode steps of B=256, H=HV=32, D=128 against a resident fp32 state."""
     import torch
     w = workloads.workload("decode_bf16")
-    S = workloads.decode_state(w, seed=w.seed + 1000 * rank, device=dev)
+    S = workloads.decode_state(w, seed=rank_seed(w, rank), device=dev)
     n = args.decode_steps
-    steps = [workloads.decode_step_inputs(w, i, seed=w.seed + 1000 * rank, device=dev)
+    steps = [workloads.decode_step_inputs(w, i, seed=rank_seed(w, rank), device=dev)
              for i in range(n)]
     o = torch.empty((w.B, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
 
@@ -393,7 +415,7 @@ def bench_kcp(args, kda, workloads, dev, stream, world, rank):
     with transitions (one batched launch), the combine, and the rerun for o."""
     import torch
     w = workloads.workload("kcp_bf16")
-    inp = workloads.chunk_inputs(w, seed=w.seed + 1000 * rank, device=dev)
+    inp = workloads.chunk_inputs(w, seed=rank_seed(w, rank), device=dev)
     L = w.T // w.n_seg
     seg = {n: inp[n].view(w.n_seg, L, *inp[n].shape[2:]) for n in ("q", "k", "v", "g", "beta")}
     o = torch.empty((w.n_seg, L, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
@@ -419,7 +441,7 @@ def bench_kcp(args, kda, workloads, dev, stream, world, rank):
     barrier(world, dev)
     ms = max_over_ranks(sum(per) / len(per), world, dev)
     return {"workload": "kcp_bf16: B=1 H=HV=16 T=65536 as 8 x 8192, Dk=Dv=128",
-            "value": world * w.token_heads / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "value": whole_job_value(w.token_heads, world, ms), "unit": UNIT, "ms_per_step": ms,
             "launches": 3 * k}
 
 

@@ -1,6 +1,6 @@
 // tcgen05 BF16 chunk kernel for Dk = Dv = 128, chunk C = 64, warp-specialised.
 //
-// One CTA (384 threads) per (b, hv) chain walks the chunks in order with the
+// One CTA (640 threads) per (b, hv) chain walks the chunks in order with the
 // state on chip: fp32 S^T in tensor memory (lane j = value channel, column c =
 // key channel) and a packed-bf16 copy in tensor memory as the MMA A operand.
 // With G the in-chunk cumulative sum of the log-decay, tiles of 16 tokens and
@@ -8,7 +8,7 @@
 // Eqs. 3-4, with the decay-weighted UT transform; page "Implémenter KDA",
 // "La forme par blocs", for U = Ut - W S), the work per chunk splits in two:
 //
-// prep warps 0-7 (state-independent; run one chunk ahead of the state warps)
+// prep warps 0-15 (state-independent; run one chunk ahead of the state warps)
 //   loads        q, k, z, v, beta of the chunk
 //   prologue     L2 norm of q,k; beta = sigmoid; g = g_min sigmoid(exp(A_log)(z + dt_bias))
 //   operands     bf16 tiles scaled by exp(G_r - P_R) <= 1 and exp(P_R' - G_i)
@@ -17,7 +17,7 @@
 //   solve        T = (I + tril(Diag(beta) A_kk, -1))^-1    (blocked, fp32)
 //   (II)  MMA    Ut^T = V^T (T Diag(beta))^T              -> TMEM buffer of the chunk
 //   (III) MMA    W^T  = (K Gamma)^T (T Diag(beta))^T      -> -W (MN-major smem)
-// state warps 8-11 (the serial carry, one TMEM lane per value channel)
+// state warps 16-19 (the serial carry, one TMEM lane per value channel)
 //   (IV)  MMA    U^T = Ut^T - S^T W^T        while the state is scaled by gamma_C
 //   (VI)  MMA    S^T <- S^T Diag(gamma_C) + U^T K',   K' = K exp(G_C - G)
 //   (V)   MMA    O^T = S^T (Q Gamma)^T + U^T A_qk^T   -> o
@@ -48,7 +48,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kPrepThreads = 256;
+constexpr int kPrepThreads = 512;
 constexpr int kStateThreads = 128;
 constexpr int kThreads = kPrepThreads + kStateThreads;
 constexpr int C = 64;
@@ -72,18 +72,17 @@ constexpr uint32_t OFF_W = 196608;        // [128 K-rows][N=64] MN-major, -W
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_RK = 0;           // float[64]
 constexpr uint32_t MISC_BETA = 256;       // float[64]
-constexpr uint32_t MISC_RED = 512;        // float[8 warps][16 tokens][2]
-constexpr uint32_t MISC_TSUM = 1536;      // float[4][128] tile sums (log2 units)
-constexpr uint32_t MISC_GAM = 3584;       // float[2][128] gamma_C per buffer
-constexpr uint32_t MISC_X = 4608;         // float[3][16][17] solve scratch
-constexpr uint32_t MISC_RQ = 7872;        // float[64]
-constexpr uint32_t MISC_BAR = 8192;       // 8 mbarriers
-constexpr uint32_t MISC_TMEM = 8256;      // uint32
-constexpr uint32_t MISC_ABORT = 8260;     // int
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 8320 + 1024;   // + alignment slack
+constexpr uint32_t MISC_QSUM = 512;       // float[16 quarters][128] (log2 units)
+constexpr uint32_t MISC_GAM = 8704;       // float[2][128] gamma_C per buffer
+constexpr uint32_t MISC_RQ = 9728;        // float[64]
+constexpr uint32_t MISC_TSUM = 9984;      // float[4][128] tile sums (log2 units)
+constexpr uint32_t MISC_BAR = 12032;      // 8 mbarriers
+constexpr uint32_t MISC_TMEM = 12096;     // uint32
+constexpr uint32_t MISC_ABORT = 12100;    // int
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 12160 + 1024;   // + alignment slack
 constexpr int LDA = 68;                   // fp32 row stride of A_kk / T
 
-constexpr int MB_MMA_P = 0, MB_MMA_S = 1, MB_READY = 2, MB_FREE = 4, MB_WFREE = 6;
+constexpr int MB_MMA_P = 0, MB_MMA_S = 1, MB_READY = 2, MB_FREE = 4, MB_WFREE = 6, MB_ODONE = 7;
 
 // TMEM columns.
 constexpr uint32_t COL_ST = 0;            // 128: S^T fp32
@@ -96,7 +95,6 @@ constexpr uint32_t TMEM_COLS = 512;
 
 // Row offset of block R' in the concatenated B operand of (I): 16 * R' (R' + 1) / 2.
 __host__ __device__ constexpr int kr_off(int r) { return 8 * r * (r + 1); }
-constexpr uint32_t kWaitLimit = 1u << 24;
 
 struct Ctx {
     uint8_t *sm;
@@ -110,20 +108,20 @@ __device__ __forceinline__ uint32_t bar_addr(const Ctx &x, int i) {
     return x.sbase + OFF_MISC + MISC_BAR + 8u * (uint32_t)i;
 }
 
-// Bounded wait that also gives up when the other role has aborted.
+// Bounded wait that also gives up when the other role has aborted.  Each try
+// may suspend the thread for up to 0.5 ms; about 4000 tries bound the wait to
+// roughly two seconds.
+constexpr uint32_t kSuspendNs = 500000;
+constexpr uint32_t kWaitTries = 4000;
 __device__ __forceinline__ bool wait_bar(const Ctx &x, uint32_t mbar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try_wait(mbar, parity)) return true;
+    for (uint32_t i = 0; i < kWaitTries; ++i) {
+        if (mbar_try_wait_suspend(mbar, parity, kSuspendNs)) return true;
         if (*x.abort_flag) return false;
-        if (i >= 16) __nanosleep(128);
     }
     *x.abort_flag = 1;
     return false;
 }
 
-__device__ __forceinline__ void st_u32(uint8_t *base, uint32_t off, uint32_t v) {
-    *reinterpret_cast<uint32_t *>(base + off) = v;
-}
 __device__ __forceinline__ void st_u128(uint8_t *base, uint32_t off, uint4 v) {
     *reinterpret_cast<uint4 *>(base + off) = v;
 }
@@ -139,24 +137,40 @@ __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w <<
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // =====================================================================
-// Prep role: warps 0-7.
+// Prep role: warps 0-15.  Thread (R, qt, cq) owns tokens 16R + 4qt .. +3 and
+// key/value channels 4cq .. 4cq+3 of each chunk; warp w = (R, qt) covers whole
+// 128-channel rows, so every global load is one contiguous 256-byte row.
 // =====================================================================
+__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
+    return make_uint2(pack_bf16x2(a, b), pack_bf16x2(c, d));
+}
+// Elementwise bf16 x bf16 product of two packed 4-element groups (rounded to nearest).
+__device__ __forceinline__ uint2 bmul4(uint2 a, uint2 b) {
+    __nv_bfloat162 r0 = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a.x), *reinterpret_cast<__nv_bfloat162 *>(&b.x));
+    __nv_bfloat162 r1 = __hmul2(*reinterpret_cast<__nv_bfloat162 *>(&a.y), *reinterpret_cast<__nv_bfloat162 *>(&b.y));
+    return make_uint2(*reinterpret_cast<uint32_t *>(&r0), *reinterpret_cast<uint32_t *>(&r1));
+}
+__device__ __forceinline__ void st_u64(uint8_t *base, uint32_t off, uint2 v) {
+    *reinterpret_cast<uint2 *>(base + off) = v;
+}
+
 __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, int tid) {
     uint8_t *sm = x.sm;
     const int lane = tid & 31, warp = tid >> 5;
-    const int R = tid >> 6;                 // 16-token tile
-    const int cp = tid & 63;                // channel pair
-    const int c0 = 2 * cp;
-    const int kb = c0 >> 6;                 // K block of this channel pair in K=128 tiles
-    const uint32_t sw_base = (uint32_t)((c0 & 63) >> 3);
-    const uint32_t within = (uint32_t)((c0 & 7) * 2);
+    const int R = warp >> 2;                // 16-token tile
+    const int qt = warp & 3;                // quarter of the tile: tokens 16R + 4qt .. +3
+    const int cq = lane;                    // channel quad: 4cq .. 4cq+3
+    const int c0 = 4 * cq;
+    const int kb = cq >> 4;                 // K block of the quad in K=128 tiles
+    const uint32_t chunk_c = (uint32_t)((cq & 15) >> 1);
+    const uint32_t within = (uint32_t)((cq & 1) * 8);
+    const int tq = R * 16 + qt * 4;         // first token of this thread
     float *rk_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_RK);
     float *rq_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_RQ);
     float *beta_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_BETA);
-    float *red_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_RED);
+    float *qsum_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_QSUM);
     float *tsum_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_TSUM);
     float *gam_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GAM);
-    float *X_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_X);
     float *Akk = reinterpret_cast<float *>(sm + OFF_AKK);
     float *Tm = reinterpret_cast<float *>(sm + OFF_TINV);
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
@@ -167,63 +181,85 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
 
     // Gate in log2 units: g2 = g_min log2(e) / (1 + 2^-(A1 z + B1)), A1 = exp(A_log) log2(e).
     const float A1 = p.gate_in ? expf(p.A_log[x.hv]) * kLog2e : 0.f;
-    const float b0 = (p.gate_in && p.dt_bias) ? p.dt_bias[(size_t)x.hv * D + c0] : 0.f;
-    const float b1 = (p.gate_in && p.dt_bias) ? p.dt_bias[(size_t)x.hv * D + c0 + 1] : 0.f;
-    const float B10 = b0 * A1, B11 = b1 * A1;
+    float B1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        B1[u] = (p.gate_in && p.dt_bias) ? p.dt_bias[(size_t)x.hv * D + c0 + u] * A1 : 0.f;
     const float gmin2 = p.g_min * kLog2e;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t ph_mma = 0;
 
+    // Raw q, k, z, v of one chunk for this thread (4 tokens x 4 channels), all
+    // loads issued together.
+    uint2 qw[4], kw[4], zw[4], vw[4];
+    auto load_chunk = [&](int mc) {
+        const int lt0 = mc * C, lCc = min(C, x.T - lt0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = tq + i;
+            uint2 a = make_uint2(0, 0), bb = a, z = a, vv = a;
+            if (t < lCc) {
+                const size_t tok = (size_t)x.b * x.T + lt0 + t;
+                a = __ldg(reinterpret_cast<const uint2 *>(q + (tok * p.H + x.h) * D + c0));
+                bb = __ldg(reinterpret_cast<const uint2 *>(k + (tok * p.H + x.h) * D + c0));
+                z = __ldg(reinterpret_cast<const uint2 *>(gz + (tok * p.HV + x.hv) * D + c0));
+                if (!x.trans) vv = __ldg(reinterpret_cast<const uint2 *>(v + (tok * p.HV + x.hv) * D + c0));
+            }
+            qw[i] = a;
+            kw[i] = bb;
+            zw[i] = z;
+            vw[i] = vv;
+        }
+    };
     for (int m = 0; m < x.nchunks; ++m) {
         const int t0 = m * C;
         const int Cc = min(C, x.T - t0);
         const int buf = m & 1;
+        load_chunk(m);
 
-        // ---------------- loads + gate + norm partials --------------------
-        uint32_t qw[16], kw[16], vw[16];
-        float g2[16][2];
+        // The double-buffered operands (and the Ut^T accumulator) of chunk m-2
+        // are free once the state warps have finished that chunk.
+        bool ok = true;
+        if (m >= 2) ok = wait_bar(x, bar_addr(x, MB_FREE + buf), (uint32_t)(((m - 2) >> 1) & 1));
+        if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
+        fence_after_sync();
+
+        // ---------------- gate, quarter sums, norms -----------------------
+        float g2[4][4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = R * 16 + i;
-            uint32_t a = 0, bb = 0, z = 0, vv = 0;
-            if (t < Cc) {
-                const size_t tok = (size_t)x.b * x.T + t0 + t;
-                a = *reinterpret_cast<const uint32_t *>(q + (tok * p.H + x.h) * D + c0);
-                bb = *reinterpret_cast<const uint32_t *>(k + (tok * p.H + x.h) * D + c0);
-                z = *reinterpret_cast<const uint32_t *>(gz + (tok * p.HV + x.hv) * D + c0);
-                if (!x.trans)
-                    vv = *reinterpret_cast<const uint32_t *>(v + (tok * p.HV + x.hv) * D + c0);
+        for (int i = 0; i < 4; ++i) {
+            const float zz[4] = {bf_lo(zw[i].x), bf_hi(zw[i].x), bf_lo(zw[i].y), bf_hi(zw[i].y)};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float g;
+                if (p.gate_in) g = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(zz[u], A1, B1[u])));
+                else g = zz[u] * kLog2e;
+                g2[i][u] = (tq + i < Cc) ? g : 0.f;
             }
-            qw[i] = a;
-            kw[i] = bb;
-            vw[i] = vv;
-            const float z0 = bf_lo(z), z1 = bf_hi(z);
-            float ga, gb;
-            if (p.gate_in) {
-                ga = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(z0, A1, B10)));
-                gb = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(z1, A1, B11)));
-            } else {
-                ga = z0 * kLog2e;
-                gb = z1 * kLog2e;
-            }
-            g2[i][0] = (t < Cc) ? ga : 0.f;
-            g2[i][1] = (t < Cc) ? gb : 0.f;
+        }
+        {
+            float4 qs;
+            qs.x = g2[0][0] + g2[1][0] + g2[2][0] + g2[3][0];
+            qs.y = g2[0][1] + g2[1][1] + g2[2][1] + g2[3][1];
+            qs.z = g2[0][2] + g2[1][2] + g2[2][2] + g2[3][2];
+            qs.w = g2[0][3] + g2[1][3] + g2[2][3] + g2[3][3];
+            *reinterpret_cast<float4 *>(qsum_s + (R * 4 + qt) * D + c0) = qs;
         }
         if (p.l2norm) {
-            // Per-token sums of squares over the warp's 64 channels: transpose
-            // reduction, 16 values over 32 lanes in 16 shuffles per quantity.
-            float sq[16], sk[16];
+            // Per-token sums of squares over the warp's 128 channels: 4 values
+            // over 32 lanes by transpose reduction (6 shuffles per quantity).
+            float sq[4], sk[4];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float qa = bf_lo(qw[i]), qb = bf_hi(qw[i]);
-                const float ka = bf_lo(kw[i]), kb2 = bf_hi(kw[i]);
-                sq[i] = fmaf(qa, qa, qb * qb);
-                sk[i] = fmaf(ka, ka, kb2 * kb2);
+            for (int i = 0; i < 4; ++i) {
+                const float q0 = bf_lo(qw[i].x), q1 = bf_hi(qw[i].x), q2 = bf_lo(qw[i].y), q3 = bf_hi(qw[i].y);
+                const float k0 = bf_lo(kw[i].x), k1 = bf_hi(kw[i].x), k2 = bf_lo(kw[i].y), k3 = bf_hi(kw[i].y);
+                sq[i] = fmaf(q0, q0, fmaf(q1, q1, fmaf(q2, q2, q3 * q3)));
+                sk[i] = fmaf(k0, k0, fmaf(k1, k1, fmaf(k2, k2, k3 * k3)));
             }
 #pragma unroll
-            for (int step = 0; step < 4; ++step) {
-                const int half = 8 >> step;            // values kept after this step
-                const int bit = 16 >> step;            // lane bit exchanged
+            for (int step = 0; step < 2; ++step) {
+                const int half = 2 >> step;
+                const int bit = 16 >> step;
                 const bool hi = (lane & bit) != 0;
 #pragma unroll
                 for (int i = 0; i < half; ++i) {
@@ -235,26 +271,23 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
                     sk[i] = sk_keep + __shfl_xor_sync(0xffffffffu, sk_send, bit);
                 }
             }
-            sq[0] += __shfl_xor_sync(0xffffffffu, sq[0], 1);
-            sk[0] += __shfl_xor_sync(0xffffffffu, sk[0], 1);
-            // Lane l now holds token ((l>>4)&1)*8 + ((l>>3)&1)*4 + ((l>>2)&1)*2 + ((l>>1)&1).
-            if ((lane & 1) == 0) {
-                const int tok = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-                                ((lane >> 1) & 1);
-                red_s[(warp * 16 + tok) * 2 + 0] = sq[0];
-                red_s[(warp * 16 + tok) * 2 + 1] = sk[0];
-            }
-        }
-        float ts0 = 0.f, ts1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            ts0 += g2[i][0];
-            ts1 += g2[i][1];
+            for (int bit = 4; bit > 0; bit >>= 1) {
+                sq[0] += __shfl_xor_sync(0xffffffffu, sq[0], bit);
+                sk[0] += __shfl_xor_sync(0xffffffffu, sk[0], bit);
+            }
+            // Lane l holds token ((l >> 4) & 1) * 2 + ((l >> 3) & 1) of this thread's four.
+            if ((lane & 7) == 0) {
+                const int t = tq + ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+                rq_s[t] = rsqrtf(sq[0] + p.l2_eps);
+                rk_s[t] = rsqrtf(sk[0] + p.l2_eps);
+            }
+        } else if (lane < 4) {
+            rq_s[tq + lane] = 1.f;
+            rk_s[tq + lane] = 1.f;
         }
-        tsum_s[R * D + c0] = ts0;
-        tsum_s[R * D + c0 + 1] = ts1;
-        if (cp < 16) {
-            const int t = R * 16 + cp;
+        if (lane >= 28) {
+            const int t = tq + (lane - 28);
             float bb = 0.f;
             if (t < Cc) {
                 bb = __bfloat162float(bl[((size_t)x.b * x.T + t0 + t) * p.HV + x.hv]);
@@ -263,99 +296,90 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
             beta_s[t] = bb;
         }
         named_bar(BAR_PREP, kPrepThreads);
-        if (tid < 64) {
-            const int t = tid, w0 = (t >> 4) * 2, i = t & 15;
-            float rq = 1.f, rk = 1.f;
-            if (p.l2norm) {
-                rq = rsqrtf(red_s[(w0 * 16 + i) * 2 + 0] + red_s[((w0 + 1) * 16 + i) * 2 + 0] + p.l2_eps);
-                rk = rsqrtf(red_s[(w0 * 16 + i) * 2 + 1] + red_s[((w0 + 1) * 16 + i) * 2 + 1] + p.l2_eps);
+
+        // Per channel: tile-start prefixes P_R', the chunk total, and the start of
+        // this thread's quarter inside its tile (log2 units).
+        if (qt == 0) {
+            // Tile sums of this warp's tile, for all 128 channels.
+            float4 ts = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(qsum_s + (R * 4 + qq) * D + c0);
+                ts.x += s4.x; ts.y += s4.y; ts.z += s4.z; ts.w += s4.w;
             }
-            rq_s[t] = rq;
-            rk_s[t] = rk;
+            *reinterpret_cast<float4 *>(tsum_s + R * D + c0) = ts;
         }
-        // Tile-start prefixes P_R' and the chunk total, per channel (log2 units).
-        float P2[4][2], GC2[2];
+        float Lst[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int xx = 0; xx < 2; ++xx) {
-            float run = 0.f;
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                P2[rr][xx] = run;
-                run += tsum_s[rr * D + c0 + xx];
+        for (int qq = 0; qq < 3; ++qq) {
+            if (qq < qt) {
+                const float4 s4 = *reinterpret_cast<const float4 *>(qsum_s + (R * 4 + qq) * D + c0);
+                Lst[0] += s4.x; Lst[1] += s4.y; Lst[2] += s4.z; Lst[3] += s4.w;
             }
-            GC2[xx] = run;
         }
-        // The double-buffered operands of this chunk overwrite those of chunk m-2.
-        bool ok = true;
-        if (m >= 2) ok = wait_bar(x, bar_addr(x, MB_FREE + buf), (uint32_t)(((m - 2) >> 1) & 1));
-        if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;   // also orders rq/rk writes
-        if (R == 0) {
-            gam_s[buf * D + c0] = ex2_approx(GC2[0]);
-            gam_s[buf * D + c0 + 1] = ex2_approx(GC2[1]);
+        named_bar(BAR_PREP, kPrepThreads);
+        float Pc[4][4], GC[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(tsum_s + rr * D + c0);
+            Pc[rr][0] = GC[0]; Pc[rr][1] = GC[1]; Pc[rr][2] = GC[2]; Pc[rr][3] = GC[3];
+            GC[0] += t4.x; GC[1] += t4.y; GC[2] += t4.z; GC[3] += t4.w;
         }
-        float eP[2], eCP[2], Dn[4][2];
+        // Decay factors, packed as bf16 pairs for the derived operands.
+        uint2 ePp, eCPp, Dnp[4];
+        {
+            float eP[4], eCP[4], Dn[4][4];
 #pragma unroll
-        for (int xx = 0; xx < 2; ++xx) {
-            const float PR = (R == 0) ? P2[0][xx] : (R == 1) ? P2[1][xx] : (R == 2) ? P2[2][xx] : P2[3][xx];
-            eP[xx] = ex2_approx(PR);
-            eCP[xx] = ex2_approx(GC2[xx] - PR);
+            for (int u = 0; u < 4; ++u) {
+                const float PR = (R == 0) ? Pc[0][u] : (R == 1) ? Pc[1][u] : (R == 2) ? Pc[2][u] : Pc[3][u];
+                eP[u] = ex2_approx(PR);
+                eCP[u] = ex2_approx(GC[u] - PR);
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) Dn[rr][xx] = (rr >= R) ? ex2_approx(P2[rr][xx] - PR) : 0.f;
+                for (int rr = 0; rr < 4; ++rr) Dn[rr][u] = (rr >= R) ? ex2_approx(Pc[rr][u] - PR) : 0.f;
+                if (R == 0 && qt == 0) gam_s[buf * D + c0 + u] = ex2_approx(GC[u]);
+            }
+            ePp = pack4(eP[0], eP[1], eP[2], eP[3]);
+            eCPp = pack4(eCP[0], eCP[1], eCP[2], eCP[3]);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) Dnp[rr] = pack4(Dn[rr][0], Dn[rr][1], Dn[rr][2], Dn[rr][3]);
         }
 
         // ---------------- operand tiles -----------------------------------
-        const uint32_t rowR = (uint32_t)(R * 16 * 128);
-        const uint32_t a_base = OFF_AINTRA + (uint32_t)kb * 16384u + rowR + within;
-        const uint32_t kr_base = OFF_KRCAT + (uint32_t)kb * 20480u + rowR + within;
-        const uint32_t qg_base = OFF_QG + (uint32_t)buf * 16384u + (uint32_t)kb * 8192u + rowR + within;
-        float kg[2][8], kpv[2][8];
-        uint32_t vlo[4], vhi[4];
-        float L0 = 0.f, L1 = 0.f;
+        // Base operands in fp32, rounded once: K e^L, Q e^L, K e^-L (tile anchors).
+        // Derived operands are bf16 x bf16 products of those with the decay
+        // factors: K_R' (x e^{P_R'-P_R}), Q Gamma and K Gamma (x e^{P_R}), K' (x e^{G_C-P_R}).
+        // The operands of MMA (I) are written first; the rest while it runs.
+        const uint32_t a_base = OFF_AINTRA + (uint32_t)kb * 16384u + within;
+        const uint32_t kr_base = OFF_KRCAT + (uint32_t)kb * 20480u + within;
+        const uint32_t qg_base = OFF_QG + (uint32_t)buf * 16384u + (uint32_t)kb * 8192u + within;
+        uint2 klp[4], qlp[4], krp[4];
+        {
+            float L[4] = {Lst[0], Lst[1], Lst[2], Lst[3]};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int t = R * 16 + i;
-            const uint32_t sw = ((sw_base ^ (uint32_t)(i & 7)) << 4) + (uint32_t)(i * 128);
-            const float rq = rq_s[t], rk = rk_s[t];
-            L0 += g2[i][0];
-            L1 += g2[i][1];
-            const float e0 = ex2_approx(L0), e1 = ex2_approx(L1);
-            const float ei0 = ex2_approx(-L0), ei1 = ex2_approx(-L1);
-            const float kh0 = bf_lo(kw[i]) * rk, kh1 = bf_hi(kw[i]) * rk;
-            const float qh0 = bf_lo(qw[i]) * rq, qh1 = bf_hi(qw[i]) * rq;
-            const float kl0 = kh0 * e0, kl1 = kh1 * e1;
-            const float ql0 = qh0 * e0, ql1 = qh1 * e1;
-            const float kr0 = kh0 * ei0, kr1 = kh1 * ei1;
-            st_u32(sm, a_base + sw, pack_bf16x2(kl0, kl1));
-            st_u32(sm, a_base + 8192u + sw, pack_bf16x2(ql0, ql1));
+            for (int i = 0; i < 4; ++i) {
+                const int t = tq + i;
+                const uint32_t roff = (uint32_t)(t * 128) + ((chunk_c ^ (uint32_t)(t & 7)) << 4);
+                const float rq = rq_s[t], rk = rk_s[t];
+                const float kv4[4] = {bf_lo(kw[i].x), bf_hi(kw[i].x), bf_lo(kw[i].y), bf_hi(kw[i].y)};
+                const float qv4[4] = {bf_lo(qw[i].x), bf_hi(qw[i].x), bf_lo(qw[i].y), bf_hi(qw[i].y)};
+                float kl[4], ql[4], kr[4];
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                if (rr >= R)
-                    st_u32(sm, kr_base + (uint32_t)(kr_off(rr) * 128) + sw,
-                           pack_bf16x2(kr0 * Dn[rr][0], kr1 * Dn[rr][1]));
-            }
-            st_u32(sm, qg_base + sw, pack_bf16x2(ql0 * eP[0], ql1 * eP[1]));
-            kg[0][i & 7] = kl0 * eP[0];
-            kg[1][i & 7] = kl1 * eP[1];
-            kpv[0][i & 7] = kr0 * eCP[0];
-            kpv[1][i & 7] = kr1 * eCP[1];
-            if ((i & 1) == 1) {
-                // value channels c0 (low halves) and c0+1 (high halves) of tokens i-1, i
-                vlo[(i & 7) >> 1] = (vw[i - 1] & 0xFFFFu) | (vw[i] << 16);
-                vhi[(i & 7) >> 1] = (vw[i - 1] >> 16) | (vw[i] & 0xFFFF0000u);
-            }
-            if ((i & 7) == 7) {
-                const int ch = 2 * R + (i >> 3);
-#pragma unroll
-                for (int xx = 0; xx < 2; ++xx) {
-                    const int row = c0 + xx;
-                    const uint32_t o = (uint32_t)(row * 128) + (uint32_t)(((ch ^ (row & 7))) << 4);
-                    st_u128(sm, OFF_KGT + o, pack8(kg[xx]));
-                    st_u128(sm, OFF_KP + (uint32_t)buf * 16384u + o, pack8(kpv[xx]));
-                    if (!x.trans) {
-                        const uint32_t *vsrc = xx ? vhi : vlo;
-                        st_u128(sm, OFF_VT + o, make_uint4(vsrc[0], vsrc[1], vsrc[2], vsrc[3]));
-                    }
+                for (int u = 0; u < 4; ++u) {
+                    L[u] += g2[i][u];
+                    const float e = ex2_approx(L[u]), ei = ex2_approx(-L[u]);
+                    const float kh = kv4[u] * rk;
+                    kl[u] = kh * e;
+                    ql[u] = qv4[u] * rq * e;
+                    kr[u] = kh * ei;
                 }
+                klp[i] = pack4(kl[0], kl[1], kl[2], kl[3]);
+                qlp[i] = pack4(ql[0], ql[1], ql[2], ql[3]);
+                krp[i] = pack4(kr[0], kr[1], kr[2], kr[3]);
+                st_u64(sm, a_base + roff, klp[i]);
+                st_u64(sm, a_base + 8192u + roff, qlp[i]);
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr)
+                    if (rr >= R) st_u64(sm, kr_base + (uint32_t)(kr_off(rr) * 128) + roff, bmul4(krp[i], Dnp[rr]));
             }
         }
         fence_async_smem();
@@ -371,6 +395,42 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
                          kmaj_desc(x.sbase + OFF_KRCAT, 160, s), id, s > 0);
             mma_commit(bar_addr(x, MB_MMA_P));
         }
+        // Meanwhile: Q Gamma (token-major) and the channel-major tiles [c][t]:
+        // rows c0..c0+3, tokens tq..tq+3 (8 bytes per row; row u's word pair holds
+        // tokens (tq, tq+1), (tq+2, tq+3)), rows visited in a lane-rotated order
+        // to spread shared-memory banks.
+        {
+            uint2 kgp[4], kpp[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = tq + i;
+                const uint32_t roff = (uint32_t)(t * 128) + ((chunk_c ^ (uint32_t)(t & 7)) << 4);
+                st_u64(sm, qg_base + roff, bmul4(qlp[i], ePp));
+                kgp[i] = bmul4(klp[i], ePp);
+                kpp[i] = bmul4(krp[i], eCPp);
+            }
+            const uint32_t tchunk = (uint32_t)(tq >> 3), tbyte = (uint32_t)((tq & 7) * 2);
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const int u = (s + (cq >> 1)) & 3;
+                const int row = c0 + u;
+                const uint32_t off = (uint32_t)(row * 128) + (((tchunk ^ (uint32_t)(row & 7))) << 4) + tbyte;
+                // halfword u of the 4-channel group: word (u >> 1), half (u & 1)
+                const bool hiw = (u & 2) != 0;
+                const uint32_t sel = (u & 1) ? 0x7632u : 0x5410u;    // high or low halves
+                st_u64(sm, OFF_KGT + off,
+                       make_uint2(__byte_perm(hiw ? kgp[0].y : kgp[0].x, hiw ? kgp[1].y : kgp[1].x, sel),
+                                  __byte_perm(hiw ? kgp[2].y : kgp[2].x, hiw ? kgp[3].y : kgp[3].x, sel)));
+                st_u64(sm, OFF_KP + (uint32_t)buf * 16384u + off,
+                       make_uint2(__byte_perm(hiw ? kpp[0].y : kpp[0].x, hiw ? kpp[1].y : kpp[1].x, sel),
+                                  __byte_perm(hiw ? kpp[2].y : kpp[2].x, hiw ? kpp[3].y : kpp[3].x, sel)));
+                if (!x.trans)
+                    st_u64(sm, OFF_VT + off,
+                           make_uint2(__byte_perm(hiw ? vw[0].y : vw[0].x, hiw ? vw[1].y : vw[1].x, sel),
+                                      __byte_perm(hiw ? vw[2].y : vw[2].x, hiw ? vw[3].y : vw[3].x, sel)));
+            }
+        }
+        fence_async_smem();
         ok = wait_bar(x, bar_addr(x, MB_MMA_P), ph_mma);
         ph_mma ^= 1u;
         if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
@@ -432,6 +492,11 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         named_bar(BAR_PREP, kPrepThreads);
 
         // ---------------- T = (I + A_kk)^-1, blocked ----------------------
+        // (a) the four diagonal 16x16 blocks by forward substitution, one
+        //     column per thread; (b) the two 32x32 diagonal blocks:
+        //     T_{I,I-1} = -T_II (A_{I,I-1} T_{I-1,I-1}) for I = 1, 3; (c) the
+        //     lower-left 32x32 block: T_{23,01} = -T_{23,23} (A_{23,01} T_{01,01}).
+        // The products' intermediates live in the (never read) upper triangle of T.
         if (tid < 64) {
             const int bb = tid >> 4, j = tid & 15;
             float xv[16];
@@ -439,39 +504,112 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
             for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
             for (int r = 1; r < 16; ++r) {
-                float acc = 0.f;
+                const float *arow = Akk + (16 * bb + r) * LDA + 16 * bb;
+                float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < r; ++i) acc = fmaf(Akk[(16 * bb + r) * LDA + 16 * bb + i], xv[i], acc);
-                if (r > j) xv[r] = -acc;
+                for (int i4 = 0; i4 < r; i4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + i4);
+                    if (i4 + 0 < r) acc0 = fmaf(a4.x, xv[i4 + 0], acc0);
+                    if (i4 + 1 < r) acc1 = fmaf(a4.y, xv[i4 + 1], acc1);
+                    if (i4 + 2 < r) acc0 = fmaf(a4.z, xv[i4 + 2], acc0);
+                    if (i4 + 3 < r) acc1 = fmaf(a4.w, xv[i4 + 3], acc1);
+                }
+                if (r > j) xv[r] = -(acc0 + acc1);
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) Tm[(16 * bb + r) * LDA + 16 * bb + j] = (r >= j) ? xv[r] : 0.f;
         }
         named_bar(BAR_PREP, kPrepThreads);
-        for (int d = 1; d < 4; ++d) {
-            const int er = tid >> 4, ec = tid & 15;
-            for (int I = d; I < 4; ++I) {
-                const int J = I - d;
-                float acc = 0.f;
-                for (int K = J; K < I; ++K) {
+        if (tid < 256) {
+            // (b) thread: block I = 1 + 2 (tid >> 7), row er, columns ec..ec+1
+            const int I = 1 + 2 * (tid >> 7), g = tid & 127;
+            const int er = g >> 3, ec = (g & 7) * 2;
+            const float *arow = Akk + (16 * I + er) * LDA + 16 * (I - 1);
+            float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-                    for (int mm = 0; mm < 16; ++mm)
-                        acc = fmaf(Akk[(16 * I + er) * LDA + 16 * K + mm], Tm[(16 * K + mm) * LDA + 16 * J + ec], acc);
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const float2 t2 = *reinterpret_cast<const float2 *>(
+                        Tm + (16 * (I - 1) + m4 + mm) * LDA + 16 * (I - 1) + ec);
+                    x0 = fmaf(av[mm], t2.x, x0);
+                    x1 = fmaf(av[mm], t2.y, x1);
                 }
-                X_s[((I - d) * 16 + er) * 17 + ec] = acc;
             }
-            named_bar(BAR_PREP, kPrepThreads);
-            for (int I = d; I < 4; ++I) {
-                const int J = I - d;
-                float acc = 0.f;
-#pragma unroll
-                for (int mm = 0; mm < 16; ++mm)
-                    acc = fmaf(Tm[(16 * I + er) * LDA + 16 * I + mm], X_s[((I - d) * 16 + mm) * 17 + ec], acc);
-                Tm[(16 * I + er) * LDA + 16 * J + ec] = -acc;
-            }
-            named_bar(BAR_PREP, kPrepThreads);
+            // scratch: block (I-1, I) of T (upper triangle)
+            *reinterpret_cast<float2 *>(Tm + (16 * (I - 1) + er) * LDA + 16 * I + ec) = make_float2(x0, x1);
         }
-        {
+        named_bar(BAR_PREP, kPrepThreads);
+        if (tid < 256) {
+            const int I = 1 + 2 * (tid >> 7), g = tid & 127;
+            const int er = g >> 3, ec = (g & 7) * 2;
+            const float *trow = Tm + (16 * I + er) * LDA + 16 * I;
+            float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(trow + m4);
+                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const float2 x2 = *reinterpret_cast<const float2 *>(
+                        Tm + (16 * (I - 1) + m4 + mm) * LDA + 16 * I + ec);
+                    y0 = fmaf(tv[mm], x2.x, y0);     // T_II is lower triangular: zeros above
+                    y1 = fmaf(tv[mm], x2.y, y1);
+                }
+            }
+            *reinterpret_cast<float2 *>(Tm + (16 * I + er) * LDA + 16 * (I - 1) + ec) = make_float2(-y0, -y1);
+        }
+        named_bar(BAR_PREP, kPrepThreads);
+        // (c) 256 threads: row er (0..31), columns ec..ec+3.  The (b) scratch
+        // sits in the upper triangles of T_{01,01} and T_{23,23} (blocks (0,1) and
+        // (2,3)), so the sums below skip those blocks.
+        if (tid < 256) {
+            const int er = tid >> 3, ec = (tid & 7) * 4;
+            const float *arow = Akk + (32 + er) * LDA;
+            float4 xacc = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int mstart = ec >= 16 ? 16 : 0;        // T_{01,01}: no rows 0-15 in columns 16-31
+#pragma unroll
+            for (int m4 = 0; m4 < 32; m4 += 4) {
+                if (m4 < mstart) continue;
+                const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(Tm + (m4 + mm) * LDA + ec);
+                    xacc.x = fmaf(av[mm], t4.x, xacc.x);
+                    xacc.y = fmaf(av[mm], t4.y, xacc.y);
+                    xacc.z = fmaf(av[mm], t4.z, xacc.z);
+                    xacc.w = fmaf(av[mm], t4.w, xacc.w);
+                }
+            }
+            *reinterpret_cast<float4 *>(Tm + er * LDA + 32 + ec) = xacc;   // upper-right scratch
+        }
+        named_bar(BAR_PREP, kPrepThreads);
+        if (tid < 256) {
+            const int er = tid >> 3, ec = (tid & 7) * 4;
+            const float *trow = Tm + (32 + er) * LDA + 32;
+            const int mend = (er & ~3) + 4;               // T_{23,23} lower triangular
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m4 = 0; m4 < 32; m4 += 4) {
+                if (m4 >= mend) continue;
+                const float4 t4 = *reinterpret_cast<const float4 *>(trow + m4);
+                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const float4 x4 = *reinterpret_cast<const float4 *>(Tm + (m4 + mm) * LDA + 32 + ec);
+                    y.x = fmaf(tv[mm], x4.x, y.x);
+                    y.y = fmaf(tv[mm], x4.y, y.y);
+                    y.z = fmaf(tv[mm], x4.z, y.z);
+                    y.w = fmaf(tv[mm], x4.w, y.w);
+                }
+            }
+            *reinterpret_cast<float4 *>(Tm + (32 + er) * LDA + ec) = make_float4(-y.x, -y.y, -y.z, -y.w);
+        }
+        named_bar(BAR_PREP, kPrepThreads);
+        if (tid < 256) {
             // T Diag(beta) -> bf16 K-major [r][i]; row r, columns 16*qq .. 16*qq+15
             const int r = tid >> 2, qq = tid & 3;
             float vv[16];
@@ -511,9 +649,9 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         if (ok && m >= 1) ok = wait_bar(x, bar_addr(x, MB_WFREE), (uint32_t)((m - 1) & 1));
         if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
         fence_after_sync();
-        if (warp < 4) {
-            const int c = warp * 32 + lane;
-            for (int mm = 0; mm < C / 16; ++mm) {
+        if (warp < 8) {
+            const int c = (warp & 3) * 32 + lane;
+            for (int mm = 2 * (warp >> 2); mm < 2 * (warp >> 2) + 2; ++mm) {
                 float vals[16];
                 tmem_ld16(x.tm + lane_base + COL_WT + mm * 16, vals);
 #pragma unroll
@@ -531,7 +669,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
 }
 
 // =====================================================================
-// State role: warps 8-11, thread j <-> TMEM lane j <-> value channel j.
+// State role: warps 16-19, thread j <-> TMEM lane j <-> value channel j.
 // =====================================================================
 __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, int tid) {
     uint8_t *sm = x.sm;
@@ -540,7 +678,6 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
     const int j = ts;                        // (warp - 8) * 32 + lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const float *gam_s = reinterpret_cast<const float *>(sm + OFF_MISC + MISC_GAM);
-    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
 
     // Initial state: S0^T (or the identity for the transition columns, or 0).
     for (int mm = 0; mm < D / 16; ++mm) {
@@ -563,10 +700,13 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
     fence_before_sync();
     named_bar(BAR_STATE, kStateThreads);
 
-    uint32_t ph_s = 0;
+    // Descriptors: start-address fields advance by compile-time offsets per k-step.
+    const uint64_t dW0 = mnmaj_desc(x.sbase + OFF_W, 0);
+    const uint32_t id_iv = idesc_bf16(128, 64, false, /*b_mn_major=*/true);
+    const uint32_t id_vi = idesc_bf16(128, 128);
+    const uint32_t id_v = idesc_bf16(128, 64);
+    uint32_t ph_s = 0, ph_o = 0;
     for (int n = 0; n < x.nchunks; ++n) {
-        const int t0 = n * C;
-        const int Cc = min(C, x.T - t0);
         const int buf = n & 1;
         const uint32_t col_ut = COL_UT + 64u * (uint32_t)buf;
         bool ok = wait_bar(x, bar_addr(x, MB_READY + buf), (uint32_t)((n >> 1) & 1));
@@ -575,11 +715,10 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
 
         // (IV) U^T = Ut^T + S^T (-W)
         if (ts == 0) {
-            const uint32_t id = idesc_bf16(128, 64, false, /*b_mn_major=*/true);
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
-                mma_bf16_tmem_a(x.tm + col_ut, x.tm + COL_SBF + s * 8, mnmaj_desc(x.sbase + OFF_W, s),
-                                id, (x.trans && s == 0) ? 0u : 1u);
+                mma_bf16_tmem_a(x.tm + col_ut, x.tm + COL_SBF + s * 8, dW0 + (uint64_t)(s * 2048 / 16),
+                                id_iv, (x.trans && s == 0) ? 0u : 1u);
             mma_commit(bar_addr(x, MB_MMA_S));
             mma_commit(bar_addr(x, MB_WFREE));
         }
@@ -587,8 +726,15 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
         for (int mm = 0; mm < D / 16; ++mm) {
             float vals[16];
             tmem_ld16(x.tm + lane_base + COL_ST + mm * 16, vals);
+            const float4 *g4 = reinterpret_cast<const float4 *>(gam_s + buf * D + mm * 16);
 #pragma unroll
-            for (int u = 0; u < 16; ++u) vals[u] *= gam_s[buf * D + mm * 16 + u];
+            for (int u4 = 0; u4 < 4; ++u4) {
+                const float4 g = g4[u4];
+                vals[4 * u4 + 0] *= g.x;
+                vals[4 * u4 + 1] *= g.y;
+                vals[4 * u4 + 2] *= g.z;
+                vals[4 * u4 + 3] *= g.w;
+            }
             tmem_st16(x.tm + lane_base + COL_ST + mm * 16, vals);
         }
         tmem_st_wait();
@@ -610,33 +756,38 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
         fence_before_sync();
         named_bar(BAR_STATE, kStateThreads);
 
-        // (VI) S^T += U^T K'  then  (V) O^T = S^T (Q Gamma)^T + U^T A_qk^T
+        // (VI) S^T += U^T K' (the serial carry), then (V) O^T = S^T (Q Gamma)^T + U^T A_qk^T
+        // with its own completion barrier so the next S^T operand is built meanwhile.
         if (ts == 0) {
             fence_after_sync();
-            const uint32_t id2 = idesc_bf16(128, 128);
+            const uint64_t dKP = kmaj_desc(x.sbase + OFF_KP + 16384u * buf, 128, 0);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16_tmem_a(x.tm + COL_ST, x.tm + COL_UBF + s * 8,
-                                kmaj_desc(x.sbase + OFF_KP + 16384u * buf, 128, s), id2, 1u);
+                mma_bf16_tmem_a(x.tm + COL_ST, x.tm + COL_UBF + s * 8, dKP + (uint64_t)(s * 32 / 16), id_vi, 1u);
+            mma_commit(bar_addr(x, MB_MMA_S));
             if (!x.trans) {
-                const uint32_t id = idesc_bf16(128, 64);
+                const uint64_t dQG = kmaj_desc(x.sbase + OFF_QG + 16384u * buf, 64, 0);
+                const uint64_t dAQ = kmaj_desc(x.sbase + OFF_AQK + 8192u * buf, 64, 0);
 #pragma unroll
                 for (int s = 0; s < D / 16; ++s)
                     mma_bf16_tmem_a(x.tm + col_ut, x.tm + COL_SBF + s * 8,
-                                    kmaj_desc(x.sbase + OFF_QG + 16384u * buf, 64, s), id, s > 0);
+                                    dQG + (uint64_t)(((s >> 2) * 64 * 128 + (s & 3) * 32) / 16), id_v, s > 0);
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    mma_bf16_tmem_a(x.tm + col_ut, x.tm + COL_UBF + s * 8,
-                                    kmaj_desc(x.sbase + OFF_AQK + 8192u * buf, 64, s), id, 1u);
+                    mma_bf16_tmem_a(x.tm + col_ut, x.tm + COL_UBF + s * 8, dAQ + (uint64_t)(s * 32 / 16), id_v, 1u);
             }
-            mma_commit(bar_addr(x, MB_MMA_S));
+            mma_commit(bar_addr(x, MB_ODONE));
         }
         ok = wait_bar(x, bar_addr(x, MB_MMA_S), ph_s);
         ph_s ^= 1u;
         if (named_bar_any(BAR_STATE, kStateThreads, !ok)) break;
         fence_after_sync();
-
-        // New S^T as the bf16 operand of the next chunk, then the outputs.
+        // The new S^T as the bf16 operand of the next chunk.  (V) still reads
+        // the old operand: wait for it before overwriting.
+        ok = wait_bar(x, bar_addr(x, MB_ODONE), ph_o);
+        ph_o ^= 1u;
+        if (named_bar_any(BAR_STATE, kStateThreads, !ok)) break;
+        fence_after_sync();
         for (int mm = 0; mm < D / 16; ++mm) {
             float vals[16];
             tmem_ld16(x.tm + lane_base + COL_ST + mm * 16, vals);
@@ -646,16 +797,17 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
             tmem_st8(x.tm + lane_base + COL_SBF + mm * 8, pk);
         }
         if (!x.trans) {
+            // o rows of this chunk: thread j writes value channel j of each token.
+            const int t0 = n * C, Cc = min(C, x.T - t0);
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) +
+                                  (((size_t)x.b * x.T + t0) * p.HV + x.hv) * D + j;
+            const size_t tstride = (size_t)p.HV * D;
             for (int mm = 0; mm < C / 16; ++mm) {
                 float vals[16];
                 tmem_ld16(x.tm + lane_base + col_ut + mm * 16, vals);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const int t = mm * 16 + u;
-                    if (t < Cc)
-                        o[(((size_t)x.b * x.T + t0 + t) * p.HV + x.hv) * D + j] =
-                            __float2bfloat16_rn(p.scale * vals[u]);
-                }
+                for (int u = 0; u < 16; ++u)
+                    if (mm * 16 + u < Cc) orow[(mm * 16 + u) * tstride] = __float2bfloat16_rn(p.scale * vals[u]);
             }
         }
         tmem_st_wait();
@@ -701,7 +853,7 @@ chunk_tc_kernel(ChunkParams p) {
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(bar_addr(x, i), 1);
+        for (int i = 0; i < 8; ++i) mbar_init(bar_addr(x, i), 1);
         *x.abort_flag = 0;
         fence_mbar_init();
     }

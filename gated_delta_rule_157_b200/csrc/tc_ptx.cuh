@@ -133,6 +133,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that lets the hardware suspend the thread for up to `suspend_ns`
+// while the phase is incomplete (no busy polling).
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t mbar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: gives up after roughly `limit` polls (with back-off), so a
 // phase that never completes ends the wait instead of hanging the GPU.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint32_t limit) {
@@ -223,6 +237,11 @@ __device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
         "{\n\t.reg .b64 st;\n\t"
         "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n" ::"r"(mbar)
         : "memory");
+}
+
+// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void prefetch_l2(const void *gptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");
 }
 
 // 2^x and 1/x on the special-function unit (PTX approximate instructions).
