@@ -154,6 +154,34 @@ __device__ __forceinline__ void st_u64(uint8_t *base, uint32_t off, uint2 v) {
     *reinterpret_cast<uint2 *>(base + off) = v;
 }
 
+// One warp: d (a 16x8 tile) += A (16 x 8KS) B (8KS x 8), both fp32 in shared
+// memory with row stride LDA, on the tensor cores in tf32 (mma.sync m16n8k8).
+template <int KS>
+__device__ __forceinline__ void warp_mm16x8(float d[4], const float *A, const float *B, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+        const float *a = A + g * LDA + 8 * kk + t;
+        const float *b = B + (8 * kk + t) * LDA + g;
+        const uint32_t af[4] = {to_tf32(a[0]), to_tf32(a[8 * LDA]), to_tf32(a[4]), to_tf32(a[8 * LDA + 4])};
+        const uint32_t bf[2] = {to_tf32(b[0]), to_tf32(b[4 * LDA])};
+        mma_tf32_16x8x8(d, af, bf);
+    }
+}
+// D (16x8 tile in shared memory) = sgn * d, or D += sgn * d.
+__device__ __forceinline__ void warp_st16x8(float *D, const float d[4], float sgn, bool accumulate, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float2 *p0 = reinterpret_cast<float2 *>(D + g * LDA + 2 * t);
+    float2 *p1 = reinterpret_cast<float2 *>(D + (g + 8) * LDA + 2 * t);
+    float2 v0 = make_float2(sgn * d[0], sgn * d[1]), v1 = make_float2(sgn * d[2], sgn * d[3]);
+    if (accumulate) {
+        const float2 o0 = *p0, o1 = *p1;
+        v0.x += o0.x; v0.y += o0.y; v1.x += o1.x; v1.y += o1.y;
+    }
+    *p0 = v0;
+    *p1 = v1;
+}
+
 __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, int tid) {
     uint8_t *sm = x.sm;
     const int lane = tid & 31, warp = tid >> 5;
@@ -216,6 +244,20 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         const int Cc = min(C, x.T - t0);
         const int buf = m & 1;
         load_chunk(m);
+        // Chunk m+1's rows stream into L2 during this chunk (one 256-byte row of
+        // q, k, z or v per thread), so its loads above hit L2 instead of
+        // competing for HBM all at once.
+        if (tid < 256 && m + 1 < x.nchunks) {
+            const int which = tid >> 6, t = (m + 1) * C + (tid & 63);
+            if (t < x.T && !(which == 3 && x.trans)) {
+                const size_t tok = (size_t)x.b * x.T + t;
+                const __nv_bfloat16 *row = which == 0 ? q + (tok * p.H + x.h) * D
+                                         : which == 1 ? k + (tok * p.H + x.h) * D
+                                         : which == 2 ? gz + (tok * p.HV + x.hv) * D
+                                                      : v + (tok * p.HV + x.hv) * D;
+                prefetch_l2(row, D * 2);
+            }
+        }
 
         // The double-buffered operands (and the Ut^T accumulator) of chunk m-2
         // are free once the state warps have finished that chunk.
@@ -437,192 +479,145 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         fence_after_sync();
 
         // ---------------- A_kk (fp32) and A_qk (bf16 operand) -------------
-        if (warp < 4) {
-            const int rr = (warp & 1) * 32 + lane;        // row of A_kk / A_qk
+        {
+            // All 16 warps: warp w reads TMEM lane quarter q = w % 4 (A_kk rows for
+            // q < 2, A_qk rows for q >= 2) and column blocks sub, sub + 4 of that
+            // quarter's range (rows 0-31 need blocks 0-2, rows 32-63 blocks 3-9).
+            const int q = warp & 3, sub = warp >> 2;
+            const int rr = (q & 1) * 32 + lane;           // row of A_kk / A_qk
             const int Rr = rr >> 4;
-            const bool is_qk = warp >= 2;
-            const int cbeg = (warp & 1) ? 48 : 0;
-            const int nld = (warp & 1) ? 7 : 3;
+            const bool is_qk = q >= 2;
+            const int nblk = (q & 1) ? 7 : 3;
+            const int cb0 = (q & 1) ? 48 : 0;
             const float br = beta_s[rr];
             uint8_t *aqk = sm + OFF_AQK + buf * 8192;
-            for (int mm = 0; mm < nld; ++mm) {
-                const int cb = cbeg + mm * 16;               // warp-uniform column
-                const int Rb = cb < 16 ? 0 : cb < 48 ? 1 : cb < 96 ? 2 : 3;   // its block
-                float vals[16];
-                tmem_ld16(x.tm + lane_base + COL_INTRA + cb, vals);
-                if (Rb == Rr) {
-                    const int i0 = cb - kr_off(Rb);           // first column index i of the slice
-                    if (is_qk) {
-                        float vv[16];
-#pragma unroll
-                        for (int u = 0; u < 16; ++u) vv[u] = (i0 + u <= rr) ? vals[u] : 0.f;
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int ch = (i0 >> 3) + hh;
-                            st_u128(aqk, (uint32_t)(rr * 128 + ((ch ^ (rr & 7)) << 4)), pack8(vv + 8 * hh));
-                        }
-                    } else {
-#pragma unroll
-                        for (int u4 = 0; u4 < 4; ++u4) {
-                            float4 f;
-                            f.x = (i0 + 4 * u4 + 0 < rr) ? br * vals[4 * u4 + 0] : 0.f;
-                            f.y = (i0 + 4 * u4 + 1 < rr) ? br * vals[4 * u4 + 1] : 0.f;
-                            f.z = (i0 + 4 * u4 + 2 < rr) ? br * vals[4 * u4 + 2] : 0.f;
-                            f.w = (i0 + 4 * u4 + 3 < rr) ? br * vals[4 * u4 + 3] : 0.f;
-                            *reinterpret_cast<float4 *>(Akk + rr * LDA + i0 + 4 * u4) = f;
-                        }
-                    }
-                }
-            }
-            // Columns past this row's tile are zero.
-            for (int i0 = 16 * (Rr + 1); i0 < C; i0 += 16) {
+            auto emit = [&](int cb, const float (&vals)[16]) {
+                const int Rb = cb < 16 ? 0 : cb < 48 ? 1 : cb < 96 ? 2 : 3;   // block of the slice
+                if (Rb != Rr) return;
+                const int i0 = cb - kr_off(Rb);               // first column index i of the slice
                 if (is_qk) {
+                    float vv[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) vv[u] = (i0 + u <= rr) ? vals[u] : 0.f;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int ch = (i0 >> 3) + hh;
+                        st_u128(aqk, (uint32_t)(rr * 128 + ((ch ^ (rr & 7)) << 4)), pack8(vv + 8 * hh));
+                    }
+                } else {
+                    // Only the strictly lower part is read by the solve.
+#pragma unroll
+                    for (int u4 = 0; u4 < 4; ++u4)
+                        *reinterpret_cast<float4 *>(Akk + rr * LDA + i0 + 4 * u4) =
+                            make_float4(br * vals[4 * u4 + 0], br * vals[4 * u4 + 1],
+                                        br * vals[4 * u4 + 2], br * vals[4 * u4 + 3]);
+                }
+            };
+            if (sub + 4 < nblk) {
+                float v0[16], v1[16];
+                const int cba = cb0 + 16 * sub, cbb = cb0 + 16 * (sub + 4);
+                tmem_ld16x2(x.tm + lane_base + COL_INTRA + cba, x.tm + lane_base + COL_INTRA + cbb, v0, v1);
+                emit(cba, v0);
+                emit(cbb, v1);
+            } else if (sub < nblk) {
+                float v0[16];
+                const int cba = cb0 + 16 * sub;
+                tmem_ld16(x.tm + lane_base + COL_INTRA + cba, v0);
+                emit(cba, v0);
+            }
+            // A_qk columns past this row's tile are zero.
+            if (is_qk && sub == 3) {
+                for (int i0 = 16 * (Rr + 1); i0 < C; i0 += 16) {
                     const uint4 z4 = make_uint4(0, 0, 0, 0);
                     st_u128(aqk, (uint32_t)(rr * 128 + ((((i0 >> 3) + 0) ^ (rr & 7)) << 4)), z4);
                     st_u128(aqk, (uint32_t)(rr * 128 + ((((i0 >> 3) + 1) ^ (rr & 7)) << 4)), z4);
-                } else {
-#pragma unroll
-                    for (int u4 = 0; u4 < 4; ++u4)
-                        *reinterpret_cast<float4 *>(Akk + rr * LDA + i0 + 4 * u4) = make_float4(0, 0, 0, 0);
                 }
             }
         }
+        // (A_qk reaches the async proxy through the fence before the READY hand-off.)
         fence_before_sync();
-        fence_async_smem();
         named_bar(BAR_PREP, kPrepThreads);
 
         // ---------------- T = (I + A_kk)^-1, blocked ----------------------
-        // (a) the four diagonal 16x16 blocks by forward substitution, one
-        //     column per thread; (b) the two 32x32 diagonal blocks:
-        //     T_{I,I-1} = -T_II (A_{I,I-1} T_{I-1,I-1}) for I = 1, 3; (c) the
-        //     lower-left 32x32 block: T_{23,01} = -T_{23,23} (A_{23,01} T_{01,01}).
-        // The products' intermediates live in the (never read) upper triangle of T.
-        if (tid < 64) {
-            const int bb = tid >> 4, j = tid & 15;
-            float xv[16];
+        // Diagonal 16x16 blocks T_II = (I + A_II)^-1 first; the rest follows from
+        // (I + A) T = I, i.e. T_IJ = -T_II sum_{J<=K<I} A_IK T_KJ, in three steps:
+        //   (1) X10 = A10 T00, X32 = A32 T22, Xc = A_{23,01} T_{01,01} without its T10 term;
+        //   (2) T10 = -T11 X10, T32 = -T33 X32, Xc[:, 0:16] -= Xc[:, 16:32] X10
+        //       (the missing term A_{23,1} T10 equals -(A_{23,1} T11) X10);
+        //   (3) T_{23,01} = -T_{23,23} Xc.
+        // The products run on the tensor cores in tf32 (warp-level mma); X10, X32
+        // and Xc live in the upper triangle of T, which is never read as T.
+        if (warp < 2) {
+            // Diagonal blocks: lane = (block 2 warp + lane / 16, column j = lane % 16),
+            // right-looking substitution down the column: once x_i is final, every
+            // later row takes its term, so the dependent chain is one FMA per row.
+            const int b = 2 * warp + (lane >> 4), j = lane & 15;
+            const float *Ab = Akk + 16 * b * LDA + 16 * b;
+            float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) xv[r] = (r == j) ? 1.f : 0.f;
+            for (int r = 0; r < 16; ++r) x[r] = 0.f;
 #pragma unroll
-            for (int r = 1; r < 16; ++r) {
-                const float *arow = Akk + (16 * bb + r) * LDA + 16 * bb;
-                float acc0 = 0.f, acc1 = 0.f;
+            for (int i = 0; i < 16; ++i) {
+                x[i] = (i == j) ? 1.f : x[i];                // rows above j stay 0
 #pragma unroll
-                for (int i4 = 0; i4 < r; i4 += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + i4);
-                    if (i4 + 0 < r) acc0 = fmaf(a4.x, xv[i4 + 0], acc0);
-                    if (i4 + 1 < r) acc1 = fmaf(a4.y, xv[i4 + 1], acc1);
-                    if (i4 + 2 < r) acc0 = fmaf(a4.z, xv[i4 + 2], acc0);
-                    if (i4 + 3 < r) acc1 = fmaf(a4.w, xv[i4 + 3], acc1);
-                }
-                if (r > j) xv[r] = -(acc0 + acc1);
+                for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-Ab[r * LDA + i], x[i], x[r]);
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tm[(16 * bb + r) * LDA + 16 * bb + j] = (r >= j) ? xv[r] : 0.f;
+            for (int r = 0; r < 16; ++r) Tm[(16 * b + r) * LDA + 16 * b + j] = x[r];
         }
         named_bar(BAR_PREP, kPrepThreads);
-        if (tid < 256) {
-            // (b) thread: block I = 1 + 2 (tid >> 7), row er, columns ec..ec+1
-            const int I = 1 + 2 * (tid >> 7), g = tid & 127;
-            const int er = g >> 3, ec = (g & 7) * 2;
-            const float *arow = Akk + (16 * I + er) * LDA + 16 * (I - 1);
-            float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-            for (int m4 = 0; m4 < 16; m4 += 4) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
-                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                for (int mm = 0; mm < 4; ++mm) {
-                    const float2 t2 = *reinterpret_cast<const float2 *>(
-                        Tm + (16 * (I - 1) + m4 + mm) * LDA + 16 * (I - 1) + ec);
-                    x0 = fmaf(av[mm], t2.x, x0);
-                    x1 = fmaf(av[mm], t2.y, x1);
-                }
-            }
-            // scratch: block (I-1, I) of T (upper triangle)
-            *reinterpret_cast<float2 *>(Tm + (16 * (I - 1) + er) * LDA + 16 * I + ec) = make_float2(x0, x1);
+        if (warp < 12) {
+            // (1) one 16x8 tile per warp: X10 = A10 T00, X32 = A32 T22,
+            //     Xc[:, 16:32] = A_{23,1} T11, Xc[:, 0:16] = A_{23,0} T00.
+            const int blk = warp >> 1, nh = (warp & 1) * 8;
+            const int arow = blk == 0 ? 16 : blk == 1 ? 48 : (blk == 2 || blk == 4) ? 32 : 48;
+            const int kc = blk == 1 ? 32 : (blk == 2 || blk == 3) ? 16 : 0;
+            const int drow = blk == 1 ? 32 : (blk == 3 || blk == 5) ? 16 : 0;
+            const int dcol = blk == 0 ? 16 : blk == 4 || blk == 5 ? 32 : 48;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_mm16x8<2>(d, Akk + arow * LDA + kc, Tm + kc * LDA + kc + nh, lane);
+            warp_st16x8(Tm + drow * LDA + dcol + nh, d, 1.f, false, lane);
         }
         named_bar(BAR_PREP, kPrepThreads);
-        if (tid < 256) {
-            const int I = 1 + 2 * (tid >> 7), g = tid & 127;
-            const int er = g >> 3, ec = (g & 7) * 2;
-            const float *trow = Tm + (16 * I + er) * LDA + 16 * I;
-            float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-            for (int m4 = 0; m4 < 16; m4 += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(trow + m4);
-                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                for (int mm = 0; mm < 4; ++mm) {
-                    const float2 x2 = *reinterpret_cast<const float2 *>(
-                        Tm + (16 * (I - 1) + m4 + mm) * LDA + 16 * I + ec);
-                    y0 = fmaf(tv[mm], x2.x, y0);     // T_II is lower triangular: zeros above
-                    y1 = fmaf(tv[mm], x2.y, y1);
-                }
-            }
-            *reinterpret_cast<float2 *>(Tm + (16 * I + er) * LDA + 16 * (I - 1) + ec) = make_float2(-y0, -y1);
+        if (warp < 8) {
+            // (2) T10 = -T11 X10, T32 = -T33 X32, Xc[:, 0:16] -= Xc[:, 16:32] X10.
+            const int task = warp >> 1, nh = (warp & 1) * 8;
+            const int arow = task == 0 ? 16 : task == 1 ? 48 : 16 * (task - 2);
+            const int acol = task == 0 ? 16 : 48;
+            const int brow = task == 1 ? 32 : 0;
+            const int bcol = task == 1 ? 48 : 16;
+            const int drow = task == 0 ? 16 : task == 1 ? 48 : 16 * (task - 2);
+            const int dcol = task == 0 ? 0 : 32;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            warp_mm16x8<2>(d, Tm + arow * LDA + acol, Tm + brow * LDA + bcol + nh, lane);
+            warp_st16x8(Tm + drow * LDA + dcol + nh, d, -1.f, task >= 2, lane);
         }
         named_bar(BAR_PREP, kPrepThreads);
-        // (c) 256 threads: row er (0..31), columns ec..ec+3.  The (b) scratch
-        // sits in the upper triangles of T_{01,01} and T_{23,23} (blocks (0,1) and
-        // (2,3)), so the sums below skip those blocks.
-        if (tid < 256) {
-            const int er = tid >> 3, ec = (tid & 7) * 4;
-            const float *arow = Akk + (32 + er) * LDA;
-            float4 xacc = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int mstart = ec >= 16 ? 16 : 0;        // T_{01,01}: no rows 0-15 in columns 16-31
-#pragma unroll
-            for (int m4 = 0; m4 < 32; m4 += 4) {
-                if (m4 < mstart) continue;
-                const float4 a4 = *reinterpret_cast<const float4 *>(arow + m4);
-                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-                for (int mm = 0; mm < 4; ++mm) {
-                    const float4 t4 = *reinterpret_cast<const float4 *>(Tm + (m4 + mm) * LDA + ec);
-                    xacc.x = fmaf(av[mm], t4.x, xacc.x);
-                    xacc.y = fmaf(av[mm], t4.y, xacc.y);
-                    xacc.z = fmaf(av[mm], t4.z, xacc.z);
-                    xacc.w = fmaf(av[mm], t4.w, xacc.w);
-                }
-            }
-            *reinterpret_cast<float4 *>(Tm + er * LDA + 32 + ec) = xacc;   // upper-right scratch
+        if (warp < 8) {
+            // (3) T_{23,01} = -T_{23,23} Xc, 16x8 tiles; rows 32-47 of T_{23,23}
+            //     reach only K = 16 (their upper-right block holds X32).
+            const int mt = warp >> 2, n0 = 8 * (warp & 3);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            const float *A = Tm + (32 + 16 * mt) * LDA + 32;
+            const float *B = Tm + 32 + n0;
+            if (mt == 0) warp_mm16x8<2>(d, A, B, lane);
+            else warp_mm16x8<4>(d, A, B, lane);
+            warp_st16x8(Tm + (32 + 16 * mt) * LDA + n0, d, -1.f, false, lane);
         }
         named_bar(BAR_PREP, kPrepThreads);
-        if (tid < 256) {
-            const int er = tid >> 3, ec = (tid & 7) * 4;
-            const float *trow = Tm + (32 + er) * LDA + 32;
-            const int mend = (er & ~3) + 4;               // T_{23,23} lower triangular
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+        {
+            // T Diag(beta) -> bf16 K-major [r][i]; row r, columns 8 ch .. 8 ch + 7
+            const int r = tid >> 3, ch = tid & 7;
+            const float4 t0 = *reinterpret_cast<const float4 *>(Tm + r * LDA + 8 * ch);
+            const float4 t1 = *reinterpret_cast<const float4 *>(Tm + r * LDA + 8 * ch + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(beta_s + 8 * ch);
+            const float4 b1 = *reinterpret_cast<const float4 *>(beta_s + 8 * ch + 4);
+            const float tv[8] = {t0.x * b0.x, t0.y * b0.y, t0.z * b0.z, t0.w * b0.w,
+                                 t1.x * b1.x, t1.y * b1.y, t1.z * b1.z, t1.w * b1.w};
+            float vv[8];
 #pragma unroll
-            for (int m4 = 0; m4 < 32; m4 += 4) {
-                if (m4 >= mend) continue;
-                const float4 t4 = *reinterpret_cast<const float4 *>(trow + m4);
-                const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                for (int mm = 0; mm < 4; ++mm) {
-                    const float4 x4 = *reinterpret_cast<const float4 *>(Tm + (m4 + mm) * LDA + 32 + ec);
-                    y.x = fmaf(tv[mm], x4.x, y.x);
-                    y.y = fmaf(tv[mm], x4.y, y.y);
-                    y.z = fmaf(tv[mm], x4.z, y.z);
-                    y.w = fmaf(tv[mm], x4.w, y.w);
-                }
-            }
-            *reinterpret_cast<float4 *>(Tm + (32 + er) * LDA + ec) = make_float4(-y.x, -y.y, -y.z, -y.w);
-        }
-        named_bar(BAR_PREP, kPrepThreads);
-        if (tid < 256) {
-            // T Diag(beta) -> bf16 K-major [r][i]; row r, columns 16*qq .. 16*qq+15
-            const int r = tid >> 2, qq = tid & 3;
-            float vv[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = 16 * qq + u;
-                vv[u] = (i <= r) ? Tm[r * LDA + i] * beta_s[i] : 0.f;
-            }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int ch = 2 * qq + hh;
-                st_u128(sm, OFF_TB + (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)), pack8(vv + 8 * hh));
-            }
+            for (int u = 0; u < 8; ++u) vv[u] = (8 * ch + u <= r) ? tv[u] : 0.f;
+            st_u128(sm, OFF_TB + (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)), pack8(vv));
         }
         fence_async_smem();
         named_bar(BAR_PREP, kPrepThreads);
@@ -649,17 +644,16 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         if (ok && m >= 1) ok = wait_bar(x, bar_addr(x, MB_WFREE), (uint32_t)((m - 1) & 1));
         if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
         fence_after_sync();
-        if (warp < 8) {
-            const int c = (warp & 3) * 32 + lane;
-            for (int mm = 2 * (warp >> 2); mm < 2 * (warp >> 2) + 2; ++mm) {
-                float vals[16];
-                tmem_ld16(x.tm + lane_base + COL_WT + mm * 16, vals);
+        {
+            // -W^T rows c (TMEM lane quarter warp % 4), 16 columns per warp.
+            const int c = (warp & 3) * 32 + lane, mm = warp >> 2;
+            float vals[16];
+            tmem_ld16(x.tm + lane_base + COL_WT + mm * 16, vals);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) vals[u] = -vals[u];
+            for (int u = 0; u < 16; ++u) vals[u] = -vals[u];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh)
-                    st_u128(sm, OFF_W + mnmaj_chunk_off(c, mm * 2 + hh), pack8(vals + 8 * hh));
-            }
+            for (int hh = 0; hh < 2; ++hh)
+                st_u128(sm, OFF_W + mnmaj_chunk_off(c, mm * 2 + hh), pack8(vals + 8 * hh));
         }
         fence_before_sync();
         fence_async_smem();
