@@ -37,6 +37,9 @@
 // operands use the K-major (or, for W, MN-major) 128-byte-swizzle layouts of
 // tc_ptx.cuh.  When M_T is requested a second CTA per chain (blockIdx.y == 1)
 // runs the same recurrence on the transition columns: v = 0 and S0 = I, no o.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kda_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -61,6 +64,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t OFF_AINTRA = 0;        // [128 rows][K=128]  K e^L (rows 0-63), Q e^L (64-127)
 constexpr uint32_t OFF_KRCAT = 32768;     // [160 rows][K=128]  K_R' e^{P_R'-G}, R' = 0..3
 constexpr uint32_t OFF_AKK = 0;           //   alias after (I): fp32 [64][68] beta-scaled A_kk
+constexpr uint32_t OFF_STAGE_Z = 0;       //   alias after the solve: raw z rows of the next chunk [64][256 B]
+constexpr uint32_t OFF_STAGE_V = 16384;   //   ... raw v rows
+constexpr uint32_t OFF_STAGE_Q = 36864;   //   alias after (I): raw q rows of the next chunk
+constexpr uint32_t OFF_STAGE_K = 53248;   //   ... raw k rows
 constexpr uint32_t OFF_TINV = 17408;      //   alias after (I): fp32 [64][68] T
 constexpr uint32_t OFF_KGT = 73728;       // [128 rows][K=64]   (K Gamma)^T
 constexpr uint32_t OFF_VT = 90112;        // [128 rows][K=64]   V^T
@@ -76,13 +83,15 @@ constexpr uint32_t MISC_QSUM = 512;       // float[16 quarters][128] (log2 units
 constexpr uint32_t MISC_GAM = 8704;       // float[2][128] gamma_C per buffer
 constexpr uint32_t MISC_RQ = 9728;        // float[64]
 constexpr uint32_t MISC_TSUM = 9984;      // float[4][128] tile sums (log2 units)
-constexpr uint32_t MISC_BAR = 12032;      // 8 mbarriers
-constexpr uint32_t MISC_TMEM = 12096;     // uint32
-constexpr uint32_t MISC_ABORT = 12100;    // int
+constexpr uint32_t MISC_BAR = 12032;      // 10 mbarriers
+constexpr uint32_t MISC_TMEM = 12120;     // uint32
+constexpr uint32_t MISC_ABORT = 12124;    // int
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 12160 + 1024;   // + alignment slack
 constexpr int LDA = 68;                   // fp32 row stride of A_kk / T
 
 constexpr int MB_MMA_P = 0, MB_MMA_S = 1, MB_READY = 2, MB_FREE = 4, MB_WFREE = 6, MB_ODONE = 7;
+constexpr int MB_LZV = 8, MB_LQK = 9;      // raw z, v rows / raw q, k rows of a chunk
+constexpr int kNumBars = 10;
 
 // TMEM columns.
 constexpr uint32_t COL_ST = 0;            // 128: S^T fp32
@@ -95,6 +104,14 @@ constexpr uint32_t TMEM_COLS = 512;
 
 // Row offset of block R' in the concatenated B operand of (I): 16 * R' (R' + 1) / 2.
 __host__ __device__ constexpr int kr_off(int r) { return 8 * r * (r + 1); }
+
+// Kernel parameters: the chunk arguments plus tensor maps of q, k (per key head)
+// and z, v (per value head), each viewed as [B*T tokens][heads][128 channels]
+// with a [64 tokens][1][128] box.
+struct TcParams {
+    ChunkParams p;
+    CUtensorMap tm[4];   // q, k, z, v
+};
 
 struct Ctx {
     uint8_t *sm;
@@ -168,6 +185,19 @@ __device__ __forceinline__ void warp_mm16x8(float d[4], const float *A, const fl
         mma_tf32_16x8x8(d, af, bf);
     }
 }
+// Element (r, i) of the bf16 K-major 64 x 64 tile T Diag(beta).
+__device__ __forceinline__ uint32_t tb_off(int r, int i) {
+    return OFF_TB + (uint32_t)(r * 128 + ((((i >> 3) ^ (r & 7))) << 4) + (i & 7) * 2);
+}
+// A 16x8 fragment of T (rows row0.., columns col0..), times -1 and Diag(beta),
+// into the bf16 tile (one 32-bit store per row pair of columns).
+__device__ __forceinline__ void warp_tb16x8(uint8_t *sm, int row0, int col0, const float d[4], const float *beta_s,
+                                            int lane) {
+    const int g = lane >> 2, t = lane & 3, c = col0 + 2 * t;
+    const float b0 = beta_s[c], b1 = beta_s[c + 1];
+    *reinterpret_cast<uint32_t *>(sm + tb_off(row0 + g, c)) = pack_bf16x2(-d[0] * b0, -d[1] * b1);
+    *reinterpret_cast<uint32_t *>(sm + tb_off(row0 + g + 8, c)) = pack_bf16x2(-d[2] * b0, -d[3] * b1);
+}
 // D (16x8 tile in shared memory) = sgn * d, or D += sgn * d.
 __device__ __forceinline__ void warp_st16x8(float *D, const float d[4], float sgn, bool accumulate, int lane) {
     const int g = lane >> 2, t = lane & 3;
@@ -182,7 +212,7 @@ __device__ __forceinline__ void warp_st16x8(float *D, const float d[4], float sg
     *p1 = v1;
 }
 
-__device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, int tid) {
+__device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMap *tmaps, const Ctx &x, int tid) {
     uint8_t *sm = x.sm;
     const int lane = tid & 31, warp = tid >> 5;
     const int R = warp >> 2;                // 16-token tile
@@ -201,10 +231,6 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
     float *gam_s = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GAM);
     float *Akk = reinterpret_cast<float *>(sm + OFF_AKK);
     float *Tm = reinterpret_cast<float *>(sm + OFF_TINV);
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(p.q);
-    const __nv_bfloat16 *k = static_cast<const __nv_bfloat16 *>(p.k);
-    const __nv_bfloat16 *v = static_cast<const __nv_bfloat16 *>(p.v);
-    const __nv_bfloat16 *gz = static_cast<const __nv_bfloat16 *>(p.g);
     const __nv_bfloat16 *bl = static_cast<const __nv_bfloat16 *>(p.beta);
 
     // Gate in log2 units: g2 = g_min log2(e) / (1 + 2^-(A1 z + B1)), A1 = exp(A_log) log2(e).
@@ -217,76 +243,75 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t ph_mma = 0;
 
-    // Raw q, k, z, v of one chunk for this thread (4 tokens x 4 channels), all
-    // loads issued together.
+    // Raw rows of each chunk arrive in shared memory by tensor-map copies (one
+    // [64 x 128] box per tensor) issued one chunk ahead: q, k as soon as MMA (I)
+    // has finished with its operand tiles (counted on MB_LQK), z, v once the
+    // solve no longer needs its workspace (MB_LZV).  Whole boxes are counted,
+    // rows past the tensor included (zero-filled).
+    // Issued by one lane of the last prep warp, which has no part in the
+    // diagonal blocks of the solve nor in issuing MMAs.
+    auto issue_rows = [&](int mc, bool zv) {
+        if (tid != kPrepThreads - 32) return;
+        const int row0 = x.b * x.T + mc * C;
+        if (zv) {
+            const uint32_t bar = bar_addr(x, MB_LZV);
+            mbar_arrive_expect_tx(bar, (uint32_t)((x.trans ? 1 : 2) * C * D * 2));
+            tma_load_3d(x.sbase + OFF_STAGE_Z, &tmaps[2], 0, x.hv, row0, bar);
+            if (!x.trans) tma_load_3d(x.sbase + OFF_STAGE_V, &tmaps[3], 0, x.hv, row0, bar);
+        } else {
+            const uint32_t bar = bar_addr(x, MB_LQK);
+            mbar_arrive_expect_tx(bar, (uint32_t)(2 * C * D * 2));
+            tma_load_3d(x.sbase + OFF_STAGE_Q, &tmaps[0], 0, x.h, row0, bar);
+            tma_load_3d(x.sbase + OFF_STAGE_K, &tmaps[1], 0, x.h, row0, bar);
+        }
+    };
     uint2 qw[4], kw[4], zw[4], vw[4];
-    auto load_chunk = [&](int mc) {
-        const int lt0 = mc * C, lCc = min(C, x.T - lt0);
+    auto read_zv = [&](int lCc) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = tq + i;
-            uint2 a = make_uint2(0, 0), bb = a, z = a, vv = a;
-            if (t < lCc) {
-                const size_t tok = (size_t)x.b * x.T + lt0 + t;
-                a = __ldg(reinterpret_cast<const uint2 *>(q + (tok * p.H + x.h) * D + c0));
-                bb = __ldg(reinterpret_cast<const uint2 *>(k + (tok * p.H + x.h) * D + c0));
-                z = __ldg(reinterpret_cast<const uint2 *>(gz + (tok * p.HV + x.hv) * D + c0));
-                if (!x.trans) vv = __ldg(reinterpret_cast<const uint2 *>(v + (tok * p.HV + x.hv) * D + c0));
-            }
-            qw[i] = a;
-            kw[i] = bb;
-            zw[i] = z;
-            vw[i] = vv;
+            const uint32_t off = (uint32_t)t * 256u + 8u * (uint32_t)cq;
+            const bool in = t < lCc;
+            zw[i] = in ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_Z + off) : make_uint2(0, 0);
+            vw[i] = (in && !x.trans) ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_V + off) : make_uint2(0, 0);
         }
     };
+    auto read_qk = [&](int lCc) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = tq + i;
+            const uint32_t off = (uint32_t)t * 256u + 8u * (uint32_t)cq;
+            const bool in = t < lCc;
+            qw[i] = in ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_Q + off) : make_uint2(0, 0);
+            kw[i] = in ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_K + off) : make_uint2(0, 0);
+        }
+    };
+    // Chunks whose rows were requested / have arrived, per barrier.
+    int issued_zv = 0, landed_zv = 0, issued_qk = 0, landed_qk = 0;
+    if (tid == kPrepThreads - 32)
+        for (int i = 0; i < 4; ++i) prefetch_tensormap(&tmaps[i]);
+    if (x.nchunks > 0) {
+        issue_rows(0, true);
+        issue_rows(0, false);
+        issued_zv = issued_qk = 1;
+    }
+    // T Diag(beta) keeps a zero upper triangle; the solve writes only the lower one.
+    st_u128(sm, OFF_TB + 16u * (uint32_t)tid, make_uint4(0, 0, 0, 0));   // 512 x 16 B
     for (int m = 0; m < x.nchunks; ++m) {
         const int t0 = m * C;
         const int Cc = min(C, x.T - t0);
         const int buf = m & 1;
-        load_chunk(m);
-        // Chunk m+1's rows stream into L2 during this chunk (one 256-byte row of
-        // q, k, z or v per thread), so its loads above hit L2 instead of
-        // competing for HBM all at once.
-        if (tid < 256 && m + 1 < x.nchunks) {
-            const int which = tid >> 6, t = (m + 1) * C + (tid & 63);
-            if (t < x.T && !(which == 3 && x.trans)) {
-                const size_t tok = (size_t)x.b * x.T + t;
-                const __nv_bfloat16 *row = which == 0 ? q + (tok * p.H + x.h) * D
-                                         : which == 1 ? k + (tok * p.H + x.h) * D
-                                         : which == 2 ? gz + (tok * p.HV + x.hv) * D
-                                                      : v + (tok * p.HV + x.hv) * D;
-                prefetch_l2(row, D * 2);
-            }
-        }
-
-        // The double-buffered operands (and the Ut^T accumulator) of chunk m-2
-        // are free once the state warps have finished that chunk.
-        bool ok = true;
-        if (m >= 2) ok = wait_bar(x, bar_addr(x, MB_FREE + buf), (uint32_t)(((m - 2) >> 1) & 1));
+        // This chunk's raw q, k rows have landed; the double-buffered operands
+        // (and the Ut^T accumulator) of chunk m-2 are free once the state warps
+        // have finished that chunk.
+        bool ok = wait_bar(x, bar_addr(x, MB_LQK), (uint32_t)(m & 1));
+        if (ok) landed_qk = m + 1;
+        if (ok && m >= 2) ok = wait_bar(x, bar_addr(x, MB_FREE + buf), (uint32_t)(((m - 2) >> 1) & 1));
         if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
         fence_after_sync();
+        read_qk(Cc);
 
-        // ---------------- gate, quarter sums, norms -----------------------
-        float g2[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float zz[4] = {bf_lo(zw[i].x), bf_hi(zw[i].x), bf_lo(zw[i].y), bf_hi(zw[i].y)};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float g;
-                if (p.gate_in) g = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(zz[u], A1, B1[u])));
-                else g = zz[u] * kLog2e;
-                g2[i][u] = (tq + i < Cc) ? g : 0.f;
-            }
-        }
-        {
-            float4 qs;
-            qs.x = g2[0][0] + g2[1][0] + g2[2][0] + g2[3][0];
-            qs.y = g2[0][1] + g2[1][1] + g2[2][1] + g2[3][1];
-            qs.z = g2[0][2] + g2[1][2] + g2[2][2] + g2[3][2];
-            qs.w = g2[0][3] + g2[1][3] + g2[2][3] + g2[3][3];
-            *reinterpret_cast<float4 *>(qsum_s + (R * 4 + qt) * D + c0) = qs;
-        }
+        // ---------------- norms, gate, quarter sums ----------------------
         if (p.l2norm) {
             // Per-token sums of squares over the warp's 128 channels: 4 values
             // over 32 lanes by transpose reduction (6 shuffles per quantity).
@@ -328,6 +353,31 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
             rq_s[tq + lane] = 1.f;
             rk_s[tq + lane] = 1.f;
         }
+        // The z, v rows (requested after the previous chunk's solve) arrive while
+        // the norms are computed.
+        const bool ok_zv = wait_bar(x, bar_addr(x, MB_LZV), (uint32_t)(m & 1));
+        if (ok_zv) landed_zv = m + 1;
+        read_zv(Cc);
+        float g2[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float zz[4] = {bf_lo(zw[i].x), bf_hi(zw[i].x), bf_lo(zw[i].y), bf_hi(zw[i].y)};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float g;
+                if (p.gate_in) g = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(zz[u], A1, B1[u])));
+                else g = zz[u] * kLog2e;
+                g2[i][u] = (tq + i < Cc) ? g : 0.f;
+            }
+        }
+        {
+            float4 qs;
+            qs.x = g2[0][0] + g2[1][0] + g2[2][0] + g2[3][0];
+            qs.y = g2[0][1] + g2[1][1] + g2[2][1] + g2[3][1];
+            qs.z = g2[0][2] + g2[1][2] + g2[2][2] + g2[3][2];
+            qs.w = g2[0][3] + g2[1][3] + g2[2][3] + g2[3][3];
+            *reinterpret_cast<float4 *>(qsum_s + (R * 4 + qt) * D + c0) = qs;
+        }
         if (lane >= 28) {
             const int t = tq + (lane - 28);
             float bb = 0.f;
@@ -337,7 +387,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
             }
             beta_s[t] = bb;
         }
-        named_bar(BAR_PREP, kPrepThreads);
+        if (named_bar_any(BAR_PREP, kPrepThreads, !ok_zv)) break;
 
         // Per channel: tile-start prefixes P_R', the chunk total, and the start of
         // this thread's quarter inside its tile (log2 units).
@@ -537,6 +587,10 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         // (A_qk reaches the async proxy through the fence before the READY hand-off.)
         fence_before_sync();
         named_bar(BAR_PREP, kPrepThreads);
+        if (m + 1 < x.nchunks) {           // MMA (I) is done with its operand tiles
+            issue_rows(m + 1, false);
+            issued_qk = m + 2;
+        }
 
         // ---------------- T = (I + A_kk)^-1, blocked ----------------------
         // Diagonal 16x16 blocks T_II = (I + A_II)^-1 first; the rest follows from
@@ -546,7 +600,9 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         //       (the missing term A_{23,1} T10 equals -(A_{23,1} T11) X10);
         //   (3) T_{23,01} = -T_{23,23} Xc.
         // The products run on the tensor cores in tf32 (warp-level mma); X10, X32
-        // and Xc live in the upper triangle of T, which is never read as T.
+        // and Xc live in the upper triangle of T, which is never read as T.  Each
+        // block of T goes to the bf16 operand T Diag(beta) as it is produced; the
+        // operand's upper triangle is zeroed once, before the first chunk.
         if (warp < 2) {
             // Diagonal blocks: lane = (block 2 warp + lane / 16, column j = lane % 16),
             // right-looking substitution down the column: once x_i is final, every
@@ -562,8 +618,13 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
 #pragma unroll
                 for (int r = i + 1; r < 16; ++r) x[r] = fmaf(-Ab[r * LDA + i], x[i], x[r]);
             }
+            const int col = 16 * b + j;
+            const float bj = beta_s[col];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tm[(16 * b + r) * LDA + 16 * b + j] = x[r];
+            for (int r = 0; r < 16; ++r) {
+                Tm[(16 * b + r) * LDA + col] = x[r];
+                *reinterpret_cast<__nv_bfloat16 *>(sm + tb_off(16 * b + r, col)) = __float2bfloat16_rn(x[r] * bj);
+            }
         }
         named_bar(BAR_PREP, kPrepThreads);
         if (warp < 12) {
@@ -590,7 +651,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
             const int dcol = task == 0 ? 0 : 32;
             float d[4] = {0.f, 0.f, 0.f, 0.f};
             warp_mm16x8<2>(d, Tm + arow * LDA + acol, Tm + brow * LDA + bcol + nh, lane);
-            warp_st16x8(Tm + drow * LDA + dcol + nh, d, -1.f, task >= 2, lane);
+            if (task != 0) warp_st16x8(Tm + drow * LDA + dcol + nh, d, -1.f, task >= 2, lane);
+            if (task < 2) warp_tb16x8(sm, drow, dcol + nh, d, beta_s, lane);   // T10, T32
         }
         named_bar(BAR_PREP, kPrepThreads);
         if (warp < 8) {
@@ -602,25 +664,14 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
             const float *B = Tm + 32 + n0;
             if (mt == 0) warp_mm16x8<2>(d, A, B, lane);
             else warp_mm16x8<4>(d, A, B, lane);
-            warp_st16x8(Tm + (32 + 16 * mt) * LDA + n0, d, -1.f, false, lane);
-        }
-        named_bar(BAR_PREP, kPrepThreads);
-        {
-            // T Diag(beta) -> bf16 K-major [r][i]; row r, columns 8 ch .. 8 ch + 7
-            const int r = tid >> 3, ch = tid & 7;
-            const float4 t0 = *reinterpret_cast<const float4 *>(Tm + r * LDA + 8 * ch);
-            const float4 t1 = *reinterpret_cast<const float4 *>(Tm + r * LDA + 8 * ch + 4);
-            const float4 b0 = *reinterpret_cast<const float4 *>(beta_s + 8 * ch);
-            const float4 b1 = *reinterpret_cast<const float4 *>(beta_s + 8 * ch + 4);
-            const float tv[8] = {t0.x * b0.x, t0.y * b0.y, t0.z * b0.z, t0.w * b0.w,
-                                 t1.x * b1.x, t1.y * b1.y, t1.z * b1.z, t1.w * b1.w};
-            float vv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) vv[u] = (8 * ch + u <= r) ? tv[u] : 0.f;
-            st_u128(sm, OFF_TB + (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)), pack8(vv));
+            warp_tb16x8(sm, 32 + 16 * mt, n0, d, beta_s, lane);
         }
         fence_async_smem();
         named_bar(BAR_PREP, kPrepThreads);
+        if (m + 1 < x.nchunks) {           // the solve workspace is free
+            issue_rows(m + 1, true);
+            issued_zv = m + 2;
+        }
 
         // ---------------- (II) Ut^T = V^T TB^T, (III) W^T = KG^T TB^T -----
         if (tid == 0) {
@@ -659,6 +710,20 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const Ctx &x, in
         fence_async_smem();
         named_bar(BAR_PREP, kPrepThreads);
         if (tid == 0) mbar_arrive(bar_addr(x, MB_READY + buf));
+    }
+    // After an abort, bulk copies may still be writing into shared memory: let
+    // the requested rows land (bounded) before the CTA can exit.
+    if (tid == 0) {
+        if (issued_zv > landed_zv) {
+            const uint32_t par = (uint32_t)((issued_zv - 1) & 1);
+            for (uint32_t i = 0; i < kWaitTries; ++i)
+                if (mbar_try_wait_suspend(bar_addr(x, MB_LZV), par, kSuspendNs)) break;
+        }
+        if (issued_qk > landed_qk) {
+            const uint32_t par = (uint32_t)((issued_qk - 1) & 1);
+            for (uint32_t i = 0; i < kWaitTries; ++i)
+                if (mbar_try_wait_suspend(bar_addr(x, MB_LQK), par, kSuspendNs)) break;
+        }
     }
 }
 
@@ -824,7 +889,8 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(ChunkParams p) {
+chunk_tc_kernel(const __grid_constant__ TcParams tp) {
+    const ChunkParams &p = tp.p;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -847,7 +913,7 @@ chunk_tc_kernel(ChunkParams p) {
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(bar_addr(x, i), 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar_addr(x, i), 1);
         *x.abort_flag = 0;
         fence_mbar_init();
     }
@@ -856,7 +922,7 @@ chunk_tc_kernel(ChunkParams p) {
     fence_after_sync();
     x.tm = *tmem_slot;
 
-    if (warp < kPrepThreads / 32) prep_role(p, x, tid);
+    if (warp < kPrepThreads / 32) prep_role(p, tp.tm, x, tid);
     else state_role(p, x, tid);
 
     fence_before_sync();
@@ -874,12 +940,39 @@ bool chunk_tc_supported(const ChunkParams &p, bool bf16) {
     return bf16 && p.Dk == D && p.Dv == D && p.C == C;
 }
 
+// Tensor map of a [B*T][heads][128] bf16 tensor with a [64][1][128] box.
+static cudaError_t make_row_map(CUtensorMap *map, const void *base, int heads, long long rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    TcParams tp;
+    tp.p = p;
+    const long long rows = (long long)p.B * p.T;
+    if ((e = make_row_map(&tp.tm[0], p.q, p.H, rows)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tp.tm[1], p.k, p.H, rows)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tp.tm[2], p.g, p.HV, rows)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tp.tm[3], p.v, p.HV, rows)) != cudaSuccess) return e;
     dim3 grid(p.B * p.HV, p.M_T ? 2 : 1);
-    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(p);
+    chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tp);
     return cudaGetLastError();
 }
 

@@ -261,9 +261,35 @@ __device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
         : "memory");
 }
 
-// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned) into L2.
-__device__ __forceinline__ void prefetch_l2(const void *gptr, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gptr), "r"(bytes) : "memory");
+// Bulk copy global -> shared memory through the tensor-memory-access engine:
+// `bytes` (a multiple of 16) from a 16-byte aligned global address to a
+// 16-byte aligned shared address; completion is counted on `mbar` as bytes.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void *src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst_smem), "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+// Tiled 3-D tensor load (no multicast) of one box into shared memory; `tmap`
+// is the generic address of a CUtensorMap kernel parameter; completion is
+// counted on `mbar` in bytes (out-of-range elements are zero-filled and counted).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void *tmap, int c0, int c1, int c2,
+                                            uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst_smem), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
+        : "memory");
+}
+// Bring a tensor map (kernel parameter) into the descriptor cache ahead of its first use.
+__device__ __forceinline__ void prefetch_tensormap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+// Arrive on `mbar` and expect `bytes` more bytes of bulk copies in this phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\t"
+        "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}\n" ::"r"(mbar), "r"(bytes)
+        : "memory");
 }
 
 // 2^x and 1/x on the special-function unit (PTX approximate instructions).
