@@ -65,15 +65,14 @@ constexpr uint32_t OFF_AINTRA = 0;        // [128 rows][K=128]  K e^L (rows 0-63
 constexpr uint32_t OFF_KRCAT = 32768;     // [160 rows][K=128]  K_R' e^{P_R'-G}, R' = 0..3
 constexpr uint32_t OFF_AKK = 0;           //   alias after (I): fp32 [64][68] beta-scaled A_kk
 constexpr uint32_t OFF_STAGE_Z = 0;       //   alias after the solve: raw z rows of the next chunk [64][256 B]
-constexpr uint32_t OFF_STAGE_V = 16384;   //   ... raw v rows
 constexpr uint32_t OFF_STAGE_Q = 36864;   //   alias after (I): raw q rows of the next chunk
 constexpr uint32_t OFF_STAGE_K = 53248;   //   ... raw k rows
 constexpr uint32_t OFF_TINV = 17408;      //   alias after (I): fp32 [64][68] T
-constexpr uint32_t OFF_KGT = 73728;       // [128 rows][K=64]   (K Gamma)^T
-constexpr uint32_t OFF_VT = 90112;        // [128 rows][K=64]   V^T
+constexpr uint32_t OFF_KGT = 73728;       // K Gamma, token-major (MN-major A of (III): M = 128 channels, K = 64)
+constexpr uint32_t OFF_VT = 90112;        // V, token-major (MN-major A of (II)), loaded by TMA with the 128-byte swizzle
 constexpr uint32_t OFF_TB = 106496;       // [64 rows][K=64]    T Diag(beta)
 constexpr uint32_t OFF_QG = 114688;       // 2 x [64 rows][K=128]  Q Gamma
-constexpr uint32_t OFF_KP = 147456;       // 2 x [128 rows][K=64]  K'^T
+constexpr uint32_t OFF_KP = 147456;       // 2 x K', token-major (MN-major B of (VI): N = 128 channels, K = 64)
 constexpr uint32_t OFF_AQK = 180224;      // 2 x [64 rows][K=64]   A_qk (lower, diagonal kept)
 constexpr uint32_t OFF_W = 196608;        // [128 K-rows][N=64] MN-major, -W
 constexpr uint32_t OFF_MISC = 212992;
@@ -83,15 +82,15 @@ constexpr uint32_t MISC_QSUM = 512;       // float[16 quarters][128] (log2 units
 constexpr uint32_t MISC_GAM = 8704;       // float[2][128] gamma_C per buffer
 constexpr uint32_t MISC_RQ = 9728;        // float[64]
 constexpr uint32_t MISC_TSUM = 9984;      // float[4][128] tile sums (log2 units)
-constexpr uint32_t MISC_BAR = 12032;      // 10 mbarriers
+constexpr uint32_t MISC_BAR = 12032;      // 11 mbarriers
 constexpr uint32_t MISC_TMEM = 12120;     // uint32
 constexpr uint32_t MISC_ABORT = 12124;    // int
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 12160 + 1024;   // + alignment slack
 constexpr int LDA = 68;                   // fp32 row stride of A_kk / T
 
 constexpr int MB_MMA_P = 0, MB_MMA_S = 1, MB_READY = 2, MB_FREE = 4, MB_WFREE = 6, MB_ODONE = 7;
-constexpr int MB_LZV = 8, MB_LQK = 9;      // raw z, v rows / raw q, k rows of a chunk
-constexpr int kNumBars = 10;
+constexpr int MB_LZV = 8, MB_LQK = 9, MB_LV = 10;   // raw z rows / raw q, k rows / V tile of a chunk
+constexpr int kNumBars = 11;
 
 // TMEM columns.
 constexpr uint32_t COL_ST = 0;            // 128: S^T fp32
@@ -255,9 +254,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         const int row0 = x.b * x.T + mc * C;
         if (zv) {
             const uint32_t bar = bar_addr(x, MB_LZV);
-            mbar_arrive_expect_tx(bar, (uint32_t)((x.trans ? 1 : 2) * C * D * 2));
+            mbar_arrive_expect_tx(bar, (uint32_t)(C * D * 2));
             tma_load_3d(x.sbase + OFF_STAGE_Z, &tmaps[2], 0, x.hv, row0, bar);
-            if (!x.trans) tma_load_3d(x.sbase + OFF_STAGE_V, &tmaps[3], 0, x.hv, row0, bar);
         } else {
             const uint32_t bar = bar_addr(x, MB_LQK);
             mbar_arrive_expect_tx(bar, (uint32_t)(2 * C * D * 2));
@@ -265,15 +263,23 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             tma_load_3d(x.sbase + OFF_STAGE_K, &tmaps[1], 0, x.h, row0, bar);
         }
     };
-    uint2 qw[4], kw[4], zw[4], vw[4];
-    auto read_zv = [&](int lCc) {
+    // V goes straight into the operand tile of MMA (II): two [64 tokens x 64
+    // channels] boxes whose 128-byte swizzle is the operand layout.
+    auto issue_v = [&](int mc) {
+        if (tid != kPrepThreads - 32 || x.trans) return;
+        const int row0 = x.b * x.T + mc * C;
+        const uint32_t bar = bar_addr(x, MB_LV);
+        mbar_arrive_expect_tx(bar, (uint32_t)(C * D * 2));
+        tma_load_3d(x.sbase + OFF_VT, &tmaps[3], 0, x.hv, row0, bar);
+        tma_load_3d(x.sbase + OFF_VT + 8192u, &tmaps[3], 64, x.hv, row0, bar);
+    };
+    uint2 qw[4], kw[4], zw[4];
+    auto read_z = [&](int lCc) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = tq + i;
             const uint32_t off = (uint32_t)t * 256u + 8u * (uint32_t)cq;
-            const bool in = t < lCc;
-            zw[i] = in ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_Z + off) : make_uint2(0, 0);
-            vw[i] = (in && !x.trans) ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_V + off) : make_uint2(0, 0);
+            zw[i] = t < lCc ? *reinterpret_cast<const uint2 *>(sm + OFF_STAGE_Z + off) : make_uint2(0, 0);
         }
     };
     auto read_qk = [&](int lCc) {
@@ -287,14 +293,21 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         }
     };
     // Chunks whose rows were requested / have arrived, per barrier.
-    int issued_zv = 0, landed_zv = 0, issued_qk = 0, landed_qk = 0;
+    int issued = 0;                        // chunks whose rows were requested
     if (tid == kPrepThreads - 32)
         for (int i = 0; i < 4; ++i) prefetch_tensormap(&tmaps[i]);
     if (x.nchunks > 0) {
         issue_rows(0, true);
         issue_rows(0, false);
-        issued_zv = issued_qk = 1;
+        issue_v(0);
+        issued = 1;
     }
+    // beta of this thread's token (lanes 28-31), loaded one chunk ahead.
+    auto load_beta = [&](int mc) {
+        const int t = mc * C + tq + (lane - 28);
+        return (lane >= 28 && t < x.T) ? bl[((size_t)x.b * x.T + t) * p.HV + x.hv] : __float2bfloat16_rn(0.f);
+    };
+    __nv_bfloat16 beta_next = load_beta(0);
     // T Diag(beta) keeps a zero upper triangle; the solve writes only the lower one.
     st_u128(sm, OFF_TB + 16u * (uint32_t)tid, make_uint4(0, 0, 0, 0));   // 512 x 16 B
     for (int m = 0; m < x.nchunks; ++m) {
@@ -305,7 +318,6 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         // (and the Ut^T accumulator) of chunk m-2 are free once the state warps
         // have finished that chunk.
         bool ok = wait_bar(x, bar_addr(x, MB_LQK), (uint32_t)(m & 1));
-        if (ok) landed_qk = m + 1;
         if (ok && m >= 2) ok = wait_bar(x, bar_addr(x, MB_FREE + buf), (uint32_t)(((m - 2) >> 1) & 1));
         if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
         fence_after_sync();
@@ -353,11 +365,10 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             rq_s[tq + lane] = 1.f;
             rk_s[tq + lane] = 1.f;
         }
-        // The z, v rows (requested after the previous chunk's solve) arrive while
+        // The z rows (requested after the previous chunk's solve) arrive while
         // the norms are computed.
         const bool ok_zv = wait_bar(x, bar_addr(x, MB_LZV), (uint32_t)(m & 1));
-        if (ok_zv) landed_zv = m + 1;
-        read_zv(Cc);
+        read_z(Cc);
         float g2[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -382,7 +393,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             const int t = tq + (lane - 28);
             float bb = 0.f;
             if (t < Cc) {
-                bb = __bfloat162float(bl[((size_t)x.b * x.T + t0 + t) * p.HV + x.hv]);
+                bb = __bfloat162float(beta_next);
                 if (p.beta_sigmoid) bb = rcp_approx(1.f + ex2_approx(-bb * kLog2e));
             }
             beta_s[t] = bb;
@@ -487,39 +498,18 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
                          kmaj_desc(x.sbase + OFF_KRCAT, 160, s), id, s > 0);
             mma_commit(bar_addr(x, MB_MMA_P));
         }
-        // Meanwhile: Q Gamma (token-major) and the channel-major tiles [c][t]:
-        // rows c0..c0+3, tokens tq..tq+3 (8 bytes per row; row u's word pair holds
-        // tokens (tq, tq+1), (tq+2, tq+3)), rows visited in a lane-rotated order
-        // to spread shared-memory banks.
+        // Meanwhile: Q Gamma, K Gamma and K', all token-major (K Gamma and K'
+        // serve as MN-major operands, whose byte image is the same).
         {
-            uint2 kgp[4], kpp[4];
+            const uint32_t kg_base = OFF_KGT + (uint32_t)kb * 8192u + within;
+            const uint32_t kp_base = OFF_KP + (uint32_t)buf * 16384u + (uint32_t)kb * 8192u + within;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = tq + i;
                 const uint32_t roff = (uint32_t)(t * 128) + ((chunk_c ^ (uint32_t)(t & 7)) << 4);
                 st_u64(sm, qg_base + roff, bmul4(qlp[i], ePp));
-                kgp[i] = bmul4(klp[i], ePp);
-                kpp[i] = bmul4(krp[i], eCPp);
-            }
-            const uint32_t tchunk = (uint32_t)(tq >> 3), tbyte = (uint32_t)((tq & 7) * 2);
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const int u = (s + (cq >> 1)) & 3;
-                const int row = c0 + u;
-                const uint32_t off = (uint32_t)(row * 128) + (((tchunk ^ (uint32_t)(row & 7))) << 4) + tbyte;
-                // halfword u of the 4-channel group: word (u >> 1), half (u & 1)
-                const bool hiw = (u & 2) != 0;
-                const uint32_t sel = (u & 1) ? 0x7632u : 0x5410u;    // high or low halves
-                st_u64(sm, OFF_KGT + off,
-                       make_uint2(__byte_perm(hiw ? kgp[0].y : kgp[0].x, hiw ? kgp[1].y : kgp[1].x, sel),
-                                  __byte_perm(hiw ? kgp[2].y : kgp[2].x, hiw ? kgp[3].y : kgp[3].x, sel)));
-                st_u64(sm, OFF_KP + (uint32_t)buf * 16384u + off,
-                       make_uint2(__byte_perm(hiw ? kpp[0].y : kpp[0].x, hiw ? kpp[1].y : kpp[1].x, sel),
-                                  __byte_perm(hiw ? kpp[2].y : kpp[2].x, hiw ? kpp[3].y : kpp[3].x, sel)));
-                if (!x.trans)
-                    st_u64(sm, OFF_VT + off,
-                           make_uint2(__byte_perm(hiw ? vw[0].y : vw[0].x, hiw ? vw[1].y : vw[1].x, sel),
-                                      __byte_perm(hiw ? vw[2].y : vw[2].x, hiw ? vw[3].y : vw[3].x, sel)));
+                st_u64(sm, kg_base + roff, bmul4(klp[i], ePp));
+                st_u64(sm, kp_base + roff, bmul4(krp[i], eCPp));
             }
         }
         fence_async_smem();
@@ -589,8 +579,9 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         named_bar(BAR_PREP, kPrepThreads);
         if (m + 1 < x.nchunks) {           // MMA (I) is done with its operand tiles
             issue_rows(m + 1, false);
-            issued_qk = m + 2;
         }
+
+        beta_next = load_beta(m + 1);     // in flight during the solve (beta_s holds this chunk's)
 
         // ---------------- T = (I + A_kk)^-1, blocked ----------------------
         // Diagonal 16x16 blocks T_II = (I + A_II)^-1 first; the rest follows from
@@ -670,22 +661,23 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         named_bar(BAR_PREP, kPrepThreads);
         if (m + 1 < x.nchunks) {           // the solve workspace is free
             issue_rows(m + 1, true);
-            issued_zv = m + 2;
+            issued = m + 2;
         }
 
         // ---------------- (II) Ut^T = V^T TB^T, (III) W^T = KG^T TB^T -----
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t id = idesc_bf16(128, 64);
-            if (!x.trans) {
+            const uint32_t id = idesc_bf16(128, 64, false, false, /*a_mn_major=*/true);
+            // (The V tile was requested a chunk ago; a failed wait has set the abort flag.)
+            if (!x.trans && wait_bar(x, bar_addr(x, MB_LV), (uint32_t)(m & 1))) {
 #pragma unroll
                 for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(x.tm + COL_UT + 64u * (uint32_t)buf, kmaj_desc(x.sbase + OFF_VT, 128, s),
+                    mma_bf16(x.tm + COL_UT + 64u * (uint32_t)buf, mnmaj_desc(x.sbase + OFF_VT, s),
                              kmaj_desc(x.sbase + OFF_TB, 64, s), id, s > 0);
             }
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16(x.tm + COL_WT, kmaj_desc(x.sbase + OFF_KGT, 128, s),
+                mma_bf16(x.tm + COL_WT, mnmaj_desc(x.sbase + OFF_KGT, s),
                          kmaj_desc(x.sbase + OFF_TB, 64, s), id, s > 0);
             mma_commit(bar_addr(x, MB_MMA_P));
         }
@@ -695,6 +687,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         if (ok && m >= 1) ok = wait_bar(x, bar_addr(x, MB_WFREE), (uint32_t)((m - 1) & 1));
         if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
         fence_after_sync();
+        if (m + 1 < x.nchunks) issue_v(m + 1);   // MMA (II) is done with the V tile
         {
             // -W^T rows c (TMEM lane quarter warp % 4), 16 columns per warp.
             const int c = (warp & 3) * 32 + lane, mm = warp >> 2;
@@ -711,18 +704,16 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         named_bar(BAR_PREP, kPrepThreads);
         if (tid == 0) mbar_arrive(bar_addr(x, MB_READY + buf));
     }
-    // After an abort, bulk copies may still be writing into shared memory: let
-    // the requested rows land (bounded) before the CTA can exit.
-    if (tid == 0) {
-        if (issued_zv > landed_zv) {
-            const uint32_t par = (uint32_t)((issued_zv - 1) & 1);
+    // After an abort, tensor copies may still be writing into shared memory: let
+    // the last requested phase of each load barrier complete (bounded) before
+    // the CTA can exit.  (Waiting on a phase that already completed returns at
+    // once.)
+    if (tid == kPrepThreads - 32 && issued > 0) {
+        const int bars[3] = {MB_LQK, MB_LZV, MB_LV};
+        for (int b = 0; b < (x.trans ? 2 : 3); ++b) {
+            const uint32_t par = (uint32_t)((issued - 1) & 1);
             for (uint32_t i = 0; i < kWaitTries; ++i)
-                if (mbar_try_wait_suspend(bar_addr(x, MB_LZV), par, kSuspendNs)) break;
-        }
-        if (issued_qk > landed_qk) {
-            const uint32_t par = (uint32_t)((issued_qk - 1) & 1);
-            for (uint32_t i = 0; i < kWaitTries; ++i)
-                if (mbar_try_wait_suspend(bar_addr(x, MB_LQK), par, kSuspendNs)) break;
+                if (mbar_try_wait_suspend(bar_addr(x, bars[b]), par, kSuspendNs)) break;
         }
     }
 }
@@ -762,7 +753,7 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
     // Descriptors: start-address fields advance by compile-time offsets per k-step.
     const uint64_t dW0 = mnmaj_desc(x.sbase + OFF_W, 0);
     const uint32_t id_iv = idesc_bf16(128, 64, false, /*b_mn_major=*/true);
-    const uint32_t id_vi = idesc_bf16(128, 128);
+    const uint32_t id_vi = idesc_bf16(128, 128, false, /*b_mn_major=*/true);
     const uint32_t id_v = idesc_bf16(128, 64);
     uint32_t ph_s = 0, ph_o = 0;
     for (int n = 0; n < x.nchunks; ++n) {
@@ -819,10 +810,10 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
         // with its own completion barrier so the next S^T operand is built meanwhile.
         if (ts == 0) {
             fence_after_sync();
-            const uint64_t dKP = kmaj_desc(x.sbase + OFF_KP + 16384u * buf, 128, 0);
+            const uint64_t dKP = mnmaj_desc(x.sbase + OFF_KP + 16384u * buf, 0);
 #pragma unroll
             for (int s = 0; s < C / 16; ++s)
-                mma_bf16_tmem_a(x.tm + COL_ST, x.tm + COL_UBF + s * 8, dKP + (uint64_t)(s * 32 / 16), id_vi, 1u);
+                mma_bf16_tmem_a(x.tm + COL_ST, x.tm + COL_UBF + s * 8, dKP + (uint64_t)(s * 2048 / 16), id_vi, 1u);
             mma_commit(bar_addr(x, MB_MMA_S));
             if (!x.trans) {
                 const uint64_t dQG = kmaj_desc(x.sbase + OFF_QG + 16384u * buf, 64, 0);
@@ -940,8 +931,10 @@ bool chunk_tc_supported(const ChunkParams &p, bool bf16) {
     return bf16 && p.Dk == D && p.Dv == D && p.C == C;
 }
 
-// Tensor map of a [B*T][heads][128] bf16 tensor with a [64][1][128] box.
-static cudaError_t make_row_map(CUtensorMap *map, const void *base, int heads, long long rows) {
+// Tensor map of a [B*T][heads][128] bf16 tensor with a [64][1][128] box, or
+// with a [64][1][64] box in the 128-byte swizzle (the MMA operand layout).
+static cudaError_t make_row_map(CUtensorMap *map, const void *base, int heads, long long rows,
+                                bool swizzle128 = false) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         void *fn = nullptr;
@@ -952,10 +945,12 @@ static cudaError_t make_row_map(CUtensorMap *map, const void *base, int heads, l
     }
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)C};
+    const cuuint32_t box[3] = {(cuuint32_t)(swizzle128 ? 64 : D), 1, (cuuint32_t)C};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -970,7 +965,7 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s) {
     if ((e = make_row_map(&tp.tm[0], p.q, p.H, rows)) != cudaSuccess) return e;
     if ((e = make_row_map(&tp.tm[1], p.k, p.H, rows)) != cudaSuccess) return e;
     if ((e = make_row_map(&tp.tm[2], p.g, p.HV, rows)) != cudaSuccess) return e;
-    if ((e = make_row_map(&tp.tm[3], p.v, p.HV, rows)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tp.tm[3], p.v, p.HV, rows, /*swizzle128=*/true)) != cudaSuccess) return e;
     dim3 grid(p.B * p.HV, p.M_T ? 2 : 1);
     chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tp);
     return cudaGetLastError();

@@ -43,10 +43,11 @@ __device__ __forceinline__ uint64_t kmaj_desc(uint32_t base, int rows, int s) {
     return d;
 }
 
-// MN-major SW128 operand (the non-reduced index contiguous): a tile with K rows
-// of 64 MN-elements (128 B each), eight K-rows per 1024-byte atom, 16-byte
-// chunk j of K-row r at position j ^ (r % 8).  Used for an N = 64 operand, so
-// there is a single 64-element MN block.  k-step s (16 K-rows) starts 2048 * s
+// MN-major SW128 operand (the non-reduced index contiguous): blocks of 64
+// MN-elements, each block K rows of 128 B (eight K-rows per 1024-byte atom,
+// 16-byte chunk j of K-row r at position j ^ (r % 8)); a 128-wide operand has
+// its second 64-element block 8192 B after the first (LBO), which is the byte
+// image of a K-major [K rows][128] tile.  k-step s (16 K-rows) starts 2048 * s
 // bytes in; SBO (between 8-row K groups) = 1024 B.
 __device__ __forceinline__ uint32_t mnmaj_chunk_off(int krow, int chunk) {
     return (uint32_t)(krow * 128 + ((chunk ^ (krow & 7)) << 4));
@@ -62,13 +63,14 @@ __device__ __forceinline__ uint64_t mnmaj_desc(uint32_t base, int s) {
 }
 
 // Instruction descriptor: BF16 x BF16 -> FP32.  A and B are K-major unless
-// `b_mn_major`; an A operand read from TMEM is always K-major.
+// `a_mn_major` / `b_mn_major`; an A operand read from TMEM is always K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool negate_a = false,
-                                                  bool b_mn_major = false) {
+                                                  bool b_mn_major = false, bool a_mn_major = false) {
     return (1u << 4)                          // D format: f32
            | (1u << 7)                        // A format: bf16
            | (1u << 10)                       // B format: bf16
            | ((negate_a ? 1u : 0u) << 13)     // negate A
+           | ((a_mn_major ? 1u : 0u) << 15)   // A major-ness
            | ((b_mn_major ? 1u : 0u) << 16)   // B major-ness
            | ((uint32_t)(N >> 3) << 17)       // N / 8
            | ((uint32_t)(M >> 4) << 24);      // M / 16
