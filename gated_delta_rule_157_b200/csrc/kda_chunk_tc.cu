@@ -82,15 +82,18 @@ constexpr uint32_t MISC_QSUM = 512;       // float[16 quarters][128] (log2 units
 constexpr uint32_t MISC_GAM = 8704;       // float[2][128] gamma_C per buffer
 constexpr uint32_t MISC_RQ = 9728;        // float[64]
 constexpr uint32_t MISC_TSUM = 9984;      // float[4][128] tile sums (log2 units)
-constexpr uint32_t MISC_BAR = 12032;      // 11 mbarriers
-constexpr uint32_t MISC_TMEM = 12120;     // uint32
-constexpr uint32_t MISC_ABORT = 12124;    // int
+constexpr uint32_t MISC_BAR = 12032;      // 13 mbarriers
+constexpr uint32_t MISC_TMEM = 12136;     // uint32
+constexpr uint32_t MISC_ABORT = 12140;    // int
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 12160 + 1024;   // + alignment slack
 constexpr int LDA = 68;                   // fp32 row stride of A_kk / T
 
-constexpr int MB_MMA_P = 0, MB_MMA_S = 1, MB_READY = 2, MB_FREE = 4, MB_WFREE = 6, MB_ODONE = 7;
-constexpr int MB_LZV = 8, MB_LQK = 9, MB_LV = 10;   // raw z rows / raw q, k rows / V tile of a chunk
-constexpr int kNumBars = 11;
+// Barriers used by both roles in every chunk are double-buffered by chunk
+// parity (READY, FREE, MMA_W), so neither role can fall two phases behind.
+constexpr int MB_MMA_P = 0, MB_MMA_S = 1, MB_READY = 2, MB_FREE = 4, MB_MMA_W = 6, MB_ODONE = 8;
+constexpr int MB_LZV = 9, MB_LQK = 10, MB_LV = 11;  // raw z rows / raw q, k rows / V tile of a chunk
+constexpr int MB_WTFREE = 12;             // W^T read out of TMEM by the state warps
+constexpr int kNumBars = 13;
 
 // TMEM columns.
 constexpr uint32_t COL_ST = 0;            // 128: S^T fp32
@@ -294,13 +297,15 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
     };
     // Chunks whose rows were requested / have arrived, per barrier.
     int issued = 0;                        // chunks whose rows were requested
+    int mw_issued = 0;                     // chunks whose MMAs (II)/(III) were issued
+    int v_issued = 0;                      // chunks whose V tile was requested
     if (tid == kPrepThreads - 32)
         for (int i = 0; i < 4; ++i) prefetch_tensormap(&tmaps[i]);
     if (x.nchunks > 0) {
         issue_rows(0, true);
         issue_rows(0, false);
         issue_v(0);
-        issued = 1;
+        issued = v_issued = 1;
     }
     // beta of this thread's token (lanes 28-31), loaded one chunk ahead.
     auto load_beta = [&](int mc) {
@@ -489,7 +494,9 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         named_bar(BAR_PREP, kPrepThreads);
 
         // ---------------- (I) intra-chunk products -------------------------
-        if (tid == 0) {
+        // MMA (I) overwrites the TMEM columns of W^T: the state warps must have
+        // read out chunk m-1's.
+        if (tid == 0 && (m == 0 || wait_bar(x, bar_addr(x, MB_WTFREE), (uint32_t)((m - 1) & 1)))) {
             fence_after_sync();
             const uint32_t id = idesc_bf16(128, 160);
 #pragma unroll
@@ -499,7 +506,15 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             mma_commit(bar_addr(x, MB_MMA_P));
         }
         // Meanwhile: Q Gamma, K Gamma and K', all token-major (K Gamma and K'
-        // serve as MN-major operands, whose byte image is the same).
+        // serve as MN-major operands, whose byte image is the same).  K Gamma
+        // and V were read by MMAs (II)/(III) of chunk m-1, finished long ago.
+        if (m >= 1) {
+            // MMA (II) of chunk m-1 has released the V tile: load this chunk's.
+            if (wait_bar(x, bar_addr(x, MB_MMA_W + ((m - 1) & 1)), (uint32_t)(((m - 1) >> 1) & 1))) {
+                issue_v(m);
+                v_issued = m + 1;
+            }
+        }
         {
             const uint32_t kg_base = OFF_KGT + (uint32_t)kb * 8192u + within;
             const uint32_t kp_base = OFF_KP + (uint32_t)buf * 16384u + (uint32_t)kb * 8192u + within;
@@ -665,6 +680,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         }
 
         // ---------------- (II) Ut^T = V^T TB^T, (III) W^T = KG^T TB^T -----
+        // Issued, not waited for: the state warps wait for their completion and
+        // read W^T out of TMEM themselves.
         if (tid == 0) {
             fence_after_sync();
             const uint32_t id = idesc_bf16(128, 64, false, false, /*a_mn_major=*/true);
@@ -679,30 +696,18 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             for (int s = 0; s < C / 16; ++s)
                 mma_bf16(x.tm + COL_WT, mnmaj_desc(x.sbase + OFF_KGT, s),
                          kmaj_desc(x.sbase + OFF_TB, 64, s), id, s > 0);
-            mma_commit(bar_addr(x, MB_MMA_P));
+            mma_commit(bar_addr(x, MB_MMA_W + buf));
+            mbar_arrive(bar_addr(x, MB_READY + buf));
+            mw_issued = m + 1;
         }
-        ok = wait_bar(x, bar_addr(x, MB_MMA_P), ph_mma);
-        ph_mma ^= 1u;
-        // -W overwrites the buffer MMA (IV) of chunk m-1 reads.
-        if (ok && m >= 1) ok = wait_bar(x, bar_addr(x, MB_WFREE), (uint32_t)((m - 1) & 1));
-        if (named_bar_any(BAR_PREP, kPrepThreads, !ok)) break;
-        fence_after_sync();
-        if (m + 1 < x.nchunks) issue_v(m + 1);   // MMA (II) is done with the V tile
-        {
-            // -W^T rows c (TMEM lane quarter warp % 4), 16 columns per warp.
-            const int c = (warp & 3) * 32 + lane, mm = warp >> 2;
-            float vals[16];
-            tmem_ld16(x.tm + lane_base + COL_WT + mm * 16, vals);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) vals[u] = -vals[u];
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                st_u128(sm, OFF_W + mnmaj_chunk_off(c, mm * 2 + hh), pack8(vals + 8 * hh));
-        }
-        fence_before_sync();
-        fence_async_smem();
-        named_bar(BAR_PREP, kPrepThreads);
-        if (tid == 0) mbar_arrive(bar_addr(x, MB_READY + buf));
+    }
+    // MMAs (II)/(III) are not waited for in the loop: make sure the last ones
+    // have completed (bounded) before the TMEM can be freed.
+    if (tid == 0 && mw_issued > 0) {
+        const int last = mw_issued - 1;
+        for (uint32_t i = 0; i < kWaitTries; ++i)
+            if (mbar_try_wait_suspend(bar_addr(x, MB_MMA_W + (last & 1)), (uint32_t)((last >> 1) & 1), kSuspendNs))
+                break;
     }
     // After an abort, tensor copies may still be writing into shared memory: let
     // the last requested phase of each load barrier complete (bounded) before
@@ -710,8 +715,9 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
     // once.)
     if (tid == kPrepThreads - 32 && issued > 0) {
         const int bars[3] = {MB_LQK, MB_LZV, MB_LV};
+        const int last[3] = {issued, issued, v_issued};
         for (int b = 0; b < (x.trans ? 2 : 3); ++b) {
-            const uint32_t par = (uint32_t)((issued - 1) & 1);
+            const uint32_t par = (uint32_t)((last[b] - 1) & 1);
             for (uint32_t i = 0; i < kWaitTries; ++i)
                 if (mbar_try_wait_suspend(bar_addr(x, bars[b]), par, kSuspendNs)) break;
         }
@@ -760,17 +766,41 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
         const int buf = n & 1;
         const uint32_t col_ut = COL_UT + 64u * (uint32_t)buf;
         bool ok = wait_bar(x, bar_addr(x, MB_READY + buf), (uint32_t)((n >> 1) & 1));
+        if (ok) ok = wait_bar(x, bar_addr(x, MB_MMA_W + buf), (uint32_t)((n >> 1) & 1));
         if (named_bar_any(BAR_STATE, kStateThreads, !ok)) break;
         fence_after_sync();
 
+        // -W^T (row j = TMEM lane j) -> MN-major bf16 operand; then the W^T
+        // columns are free for the prep warps' next MMA (I).
+        {
+            float v0[16], v1[16];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                tmem_ld16x2(x.tm + lane_base + COL_WT + hf * 32, x.tm + lane_base + COL_WT + hf * 32 + 16, v0, v1);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    v0[u] = -v0[u];
+                    v1[u] = -v1[u];
+                }
+                st_u128(sm, OFF_W + mnmaj_chunk_off(j, 4 * hf + 0), pack8(v0));
+                st_u128(sm, OFF_W + mnmaj_chunk_off(j, 4 * hf + 1), pack8(v0 + 8));
+                st_u128(sm, OFF_W + mnmaj_chunk_off(j, 4 * hf + 2), pack8(v1));
+                st_u128(sm, OFF_W + mnmaj_chunk_off(j, 4 * hf + 3), pack8(v1 + 8));
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        named_bar(BAR_STATE, kStateThreads);
+
         // (IV) U^T = Ut^T + S^T (-W)
         if (ts == 0) {
+            fence_after_sync();
+            mbar_arrive(bar_addr(x, MB_WTFREE));
 #pragma unroll
             for (int s = 0; s < D / 16; ++s)
                 mma_bf16_tmem_a(x.tm + col_ut, x.tm + COL_SBF + s * 8, dW0 + (uint64_t)(s * 2048 / 16),
                                 id_iv, (x.trans && s == 0) ? 0u : 1u);
             mma_commit(bar_addr(x, MB_MMA_S));
-            mma_commit(bar_addr(x, MB_WFREE));
         }
         // Meanwhile: S^T <- S^T Diag(gamma_C) (fp32, in TMEM).
         for (int mm = 0; mm < D / 16; ++mm) {
