@@ -297,8 +297,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
     };
     // Chunks whose rows were requested / have arrived, per barrier.
     int issued = 0;                        // chunks whose rows were requested
-    int mw_issued = 0;                     // chunks whose MMAs (II)/(III) were issued
     int v_issued = 0;                      // chunks whose V tile was requested
+    int mi_issued = 0;                     // chunks whose MMA (I) was issued (by this thread)
     if (tid == kPrepThreads - 32)
         for (int i = 0; i < 4; ++i) prefetch_tensormap(&tmaps[i]);
     if (x.nchunks > 0) {
@@ -494,9 +494,11 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         named_bar(BAR_PREP, kPrepThreads);
 
         // ---------------- (I) intra-chunk products -------------------------
-        // MMA (I) overwrites the TMEM columns of W^T: the state warps must have
-        // read out chunk m-1's.
-        if (tid == 0 && (m == 0 || wait_bar(x, bar_addr(x, MB_WTFREE), (uint32_t)((m - 1) & 1)))) {
+        // Issued by lane 0 of the last prep warp, whose own share of the work
+        // below overlaps the MMA.  MMA (I) overwrites the TMEM columns of W^T:
+        // the state warps must have read out chunk m-1's.
+        if (tid == kPrepThreads - 32 &&
+            (m == 0 || wait_bar(x, bar_addr(x, MB_WTFREE), (uint32_t)((m - 1) & 1)))) {
             fence_after_sync();
             const uint32_t id = idesc_bf16(128, 160);
 #pragma unroll
@@ -504,6 +506,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
                 mma_bf16(x.tm + COL_INTRA, kmaj_desc(x.sbase + OFF_AINTRA, 128, s),
                          kmaj_desc(x.sbase + OFF_KRCAT, 160, s), id, s > 0);
             mma_commit(bar_addr(x, MB_MMA_P));
+            mi_issued = m + 1;
         }
         // Meanwhile: Q Gamma, K Gamma and K', all token-major (K Gamma and K'
         // serve as MN-major operands, whose byte image is the same).  K Gamma
@@ -679,40 +682,18 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             issued = m + 2;
         }
 
-        // ---------------- (II) Ut^T = V^T TB^T, (III) W^T = KG^T TB^T -----
-        // Issued, not waited for: the state warps wait for their completion and
-        // read W^T out of TMEM themselves.
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t id = idesc_bf16(128, 64, false, false, /*a_mn_major=*/true);
-            // (The V tile was requested a chunk ago; a failed wait has set the abort flag.)
-            if (!x.trans && wait_bar(x, bar_addr(x, MB_LV), (uint32_t)(m & 1))) {
-#pragma unroll
-                for (int s = 0; s < C / 16; ++s)
-                    mma_bf16(x.tm + COL_UT + 64u * (uint32_t)buf, mnmaj_desc(x.sbase + OFF_VT, s),
-                             kmaj_desc(x.sbase + OFF_TB, 64, s), id, s > 0);
-            }
-#pragma unroll
-            for (int s = 0; s < C / 16; ++s)
-                mma_bf16(x.tm + COL_WT, mnmaj_desc(x.sbase + OFF_KGT, s),
-                         kmaj_desc(x.sbase + OFF_TB, 64, s), id, s > 0);
-            mma_commit(bar_addr(x, MB_MMA_W + buf));
-            mbar_arrive(bar_addr(x, MB_READY + buf));
-            mw_issued = m + 1;
-        }
-    }
-    // MMAs (II)/(III) are not waited for in the loop: make sure the last ones
-    // have completed (bounded) before the TMEM can be freed.
-    if (tid == 0 && mw_issued > 0) {
-        const int last = mw_issued - 1;
-        for (uint32_t i = 0; i < kWaitTries; ++i)
-            if (mbar_try_wait_suspend(bar_addr(x, MB_MMA_W + (last & 1)), (uint32_t)((last >> 1) & 1), kSuspendNs))
-                break;
+        // Everything of chunk m is in shared memory: the state warps take the
+        // chunk, starting with MMAs (II)/(III).
+        if (tid == 0) mbar_arrive(bar_addr(x, MB_READY + buf));
     }
     // After an abort, tensor copies may still be writing into shared memory: let
     // the last requested phase of each load barrier complete (bounded) before
     // the CTA can exit.  (Waiting on a phase that already completed returns at
     // once.)
+    if (tid == kPrepThreads - 32 && mi_issued > 0) {
+        for (uint32_t i = 0; i < kWaitTries; ++i)
+            if (mbar_try_wait_suspend(bar_addr(x, MB_MMA_P), (uint32_t)((mi_issued - 1) & 1), kSuspendNs)) break;
+    }
     if (tid == kPrepThreads - 32 && issued > 0) {
         const int bars[3] = {MB_LQK, MB_LZV, MB_LV};
         const int last[3] = {issued, issued, v_issued};
@@ -761,11 +742,33 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
     const uint32_t id_iv = idesc_bf16(128, 64, false, /*b_mn_major=*/true);
     const uint32_t id_vi = idesc_bf16(128, 128, false, /*b_mn_major=*/true);
     const uint32_t id_v = idesc_bf16(128, 64);
+    const uint32_t id_w = idesc_bf16(128, 64, false, false, /*a_mn_major=*/true);
     uint32_t ph_s = 0, ph_o = 0;
+    int w_issued = 0;                      // chunks whose MMAs (II)/(III) were issued (by ts 0)
     for (int n = 0; n < x.nchunks; ++n) {
         const int buf = n & 1;
         const uint32_t col_ut = COL_UT + 64u * (uint32_t)buf;
         bool ok = wait_bar(x, bar_addr(x, MB_READY + buf), (uint32_t)((n >> 1) & 1));
+        // (II) Ut^T = V^T TB^T and (III) W^T = (K Gamma)^T TB^T of this chunk,
+        // once its V tile has landed.
+        if (ts == 0 && ok) {
+            if (!x.trans) ok = wait_bar(x, bar_addr(x, MB_LV), (uint32_t)(n & 1));
+            if (ok) {
+                fence_after_sync();
+                if (!x.trans) {
+#pragma unroll
+                    for (int s = 0; s < C / 16; ++s)
+                        mma_bf16(x.tm + col_ut, mnmaj_desc(x.sbase + OFF_VT, s), kmaj_desc(x.sbase + OFF_TB, 64, s),
+                                 id_w, s > 0);
+                }
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16(x.tm + COL_WT, mnmaj_desc(x.sbase + OFF_KGT, s), kmaj_desc(x.sbase + OFF_TB, 64, s),
+                             id_w, s > 0);
+                mma_commit(bar_addr(x, MB_MMA_W + buf));
+                w_issued = n + 1;
+            }
+        }
         if (ok) ok = wait_bar(x, bar_addr(x, MB_MMA_W + buf), (uint32_t)((n >> 1) & 1));
         if (named_bar_any(BAR_STATE, kStateThreads, !ok)) break;
         fence_after_sync();
@@ -896,6 +899,14 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
         if (ts == 0) mbar_arrive(bar_addr(x, MB_FREE + buf));
     }
 
+    // After an abort, let this role's last MMAs (II)/(III) complete (bounded)
+    // before the TMEM can be freed.
+    if (ts == 0 && w_issued > 0) {
+        const int last = w_issued - 1;
+        for (uint32_t i = 0; i < kWaitTries; ++i)
+            if (mbar_try_wait_suspend(bar_addr(x, MB_MMA_W + (last & 1)), (uint32_t)((last >> 1) & 1), kSuspendNs))
+                break;
+    }
     if (!*x.abort_flag) {
         float *out = x.trans ? p.M_T : p.S_T;
         if (out) {
