@@ -60,7 +60,7 @@ class StepArgs(ctypes.Structure):
 
 
 EXPORTS = ["kda_chunk_fwd", "kda_step", "kda_compose", "kda_device_status",
-           "kda_status_string", "kda_version"]
+           "kda_status_string", "kda_version", "kda_debug_chunk_stall"]
 
 _lib = None
 
@@ -80,6 +80,8 @@ def load():
     lib = ctypes.CDLL(path)
     lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(ChunkArgs), ctypes.c_void_p]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_debug_chunk_stall.argtypes = [ctypes.POINTER(ChunkArgs), ctypes.c_void_p]
+    lib.kda_debug_chunk_stall.restype = ctypes.c_int
     lib.kda_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
     lib.kda_step.restype = ctypes.c_int
     lib.kda_compose.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 5
@@ -135,8 +137,10 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
                   g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
                   beta_sigmoid_in_kernel=True, gate_in_kernel=True,
                   output_final_state=True, output_transition=False, algo="auto",
-                  o=None, S_T=None, M_T=None, stream=None):
+                  o=None, S_T=None, M_T=None, stream=None, _withhold_ready=False):
     """Chunk-parallel KDA forward.  Returns (o, S_T or None, M_T or None).
+
+    (_withhold_ready routes to kda_debug_chunk_stall, the failure-path test hook.)
 
     q, k [B,T,H,Dk]; v [B,T,HV,Dv]; g (log-decay or raw z) [B,T,HV,Dk];
     beta (or logits) [B,T,HV] -- all float32 or all bfloat16, on one CUDA device.
@@ -176,7 +180,10 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
     a.A_log, a.dt_bias, a.S0 = _ptr(A_log), _ptr(dt_bias), _ptr(S0)
     a.o, a.S_T, a.M_T = _ptr(o), _ptr(S_T), _ptr(M_T)
-    _raise("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a), _stream(stream, dev)))
+    if _withhold_ready:
+        _raise("kda_debug_chunk_stall", lib.kda_debug_chunk_stall(ctypes.byref(a), _stream(stream, dev)))
+    else:
+        _raise("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a), _stream(stream, dev)))
     return o, S_T, M_T
 
 

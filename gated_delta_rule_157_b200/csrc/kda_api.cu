@@ -31,7 +31,7 @@ kda_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_E
 
 extern "C" {
 
-kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
+static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold_ready) {
     if (!a) return KDA_ERR_INVALID_ARG;
     if (a->B < 0 || a->T < 0 || a->H < 1 || a->HV < 1 || a->HV % a->H != 0)
         return KDA_ERR_INVALID_ARG;
@@ -90,11 +90,13 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.S0 = a->S0;
     p.o = a->o; p.S_T = a->S_T; p.M_T = a->M_T;
+    p.withhold_ready = withhold_ready ? 1 : 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     if (a->T == 0) return cuda_status(kda::launch_chunk_empty(p, s));
 
     const bool tc_ok = kda::chunk_tc_supported(p, bf16);
+    if (withhold_ready && (a->algo != KDA_ALGO_TC || !tc_ok)) return KDA_ERR_UNSUPPORTED;
     if (a->algo == KDA_ALGO_TC) {
         if (!tc_ok) return KDA_ERR_UNSUPPORTED;
         const void *v16[] = {a->q, a->k, a->v, a->g, a->o};
@@ -110,6 +112,10 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     }
     return cuda_status(kda::launch_chunk_simt(p, bf16, s));
 }
+
+kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) { return chunk_fwd(a, stream, false); }
+
+kda_status kda_debug_chunk_stall(const kda_chunk_args *a, void *stream) { return chunk_fwd(a, stream, true); }
 
 kda_status kda_step(const kda_step_args *a, void *stream) {
     if (!a) return KDA_ERR_INVALID_ARG;

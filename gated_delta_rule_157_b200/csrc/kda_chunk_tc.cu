@@ -127,18 +127,24 @@ __device__ __forceinline__ uint32_t bar_addr(const Ctx &x, int i) {
     return x.sbase + OFF_MISC + MISC_BAR + 8u * (uint32_t)i;
 }
 
-// Bounded wait that also gives up when the other role has aborted.  Each try
-// may suspend the thread for up to 0.5 ms; about 4000 tries bound the wait to
-// roughly two seconds.
+// Bounded wait that also gives up when the other role has aborted: spins on
+// the mbarrier (a suspend-hinted wait wakes up measurably later) for at most
+// about two seconds of SM clock.  The exit drains below use the suspend hint
+// (kSuspendNs per try, kWaitTries tries).
 constexpr uint32_t kSuspendNs = 500000;
 constexpr uint32_t kWaitTries = 4000;
+constexpr long long kWaitCycles = 4000000000LL;
 __device__ __forceinline__ bool wait_bar(const Ctx &x, uint32_t mbar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitTries; ++i) {
-        if (mbar_try_wait_suspend(mbar, parity, kSuspendNs)) return true;
+    if (mbar_try_wait(mbar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(mbar, parity)) {
         if (*x.abort_flag) return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *x.abort_flag = 1;
+            return false;
+        }
     }
-    *x.abort_flag = 1;
-    return false;
+    return true;
 }
 
 __device__ __forceinline__ void st_u128(uint8_t *base, uint32_t off, uint4 v) {
@@ -684,7 +690,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
 
         // Everything of chunk m is in shared memory: the state warps take the
         // chunk, starting with MMAs (II)/(III).
-        if (tid == 0) mbar_arrive(bar_addr(x, MB_READY + buf));
+        if (tid == 0 && !p.withhold_ready) mbar_arrive(bar_addr(x, MB_READY + buf));
     }
     // After an abort, tensor copies may still be writing into shared memory: let
     // the last requested phase of each load barrier complete (bounded) before

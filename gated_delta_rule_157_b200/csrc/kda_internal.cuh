@@ -36,6 +36,7 @@ struct ChunkParams {
     const float *A_log, *dt_bias, *S0;
     void *o;
     float *S_T, *M_T;
+    int withhold_ready;              // test hook: the tensor-core kernel's prep warps never hand a chunk over
 };
 
 struct StepParams {

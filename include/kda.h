@@ -164,6 +164,17 @@ kda_status kda_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
  * synchronising `stream`.  Returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_CUDA. */
 kda_status kda_device_status(void *stream);
 
+/* Test hook for the failure path of the tensor-core chunk kernel (no
+ * counterpart in the method): validates and launches exactly like
+ * kda_chunk_fwd with algo KDA_ALGO_TC, except that the kernel's prep warps
+ * never hand a chunk over to its state warps.  The state warps' bounded wait
+ * then gives up after about two seconds, every CTA records the device error
+ * word, frees its tensor memory and returns; the outputs are unspecified.
+ * kda_device_status() afterwards reports KDA_ERR_TIMEOUT and the context stays
+ * usable.  Returns KDA_ERR_UNSUPPORTED unless the arguments select the
+ * tensor-core kernel; otherwise as kda_chunk_fwd. */
+kda_status kda_debug_chunk_stall(const kda_chunk_args *args, void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *kda_status_string(kda_status status);
 
