@@ -28,6 +28,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "chunk_kda fwd tokens·heads/s + % bf16 TC peak; kda_step decode HBM GB/s"
+# DRAM bytes (read + write) per launch from ncu captures of the current kernels
+# (profiles/chunk_tc_kernel_gva_b1.md: one B=1 launch, 32 chains, scaled by 4 to
+# the 128 chains of the B=4 launch; profiles/step_kernel_decode_bf16.md).
+CHUNK_TC_TRAFFIC_B4 = 4 * (201.988864e6 + 49.091328e6)
+STEP_TRAFFIC = 545.3e6 + 485.3e6
 UNIT = "tokens·heads/s"
 
 
@@ -326,7 +331,9 @@ def main():
             "tc_peak_frac": tflops / pk["bf16_tflops"],
             "useful_tflops": tflops,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"], "traffic": None,
+                         "unit": "GB/s", "frac": achieved_gbs / pk["hbm_gbs"],
+                         "traffic": CHUNK_TC_TRAFFIC_B4 if (w.B == 4 and args.algo != "simt") else None,
+                         "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "kernel": "kda_chunk_fwd (%s)" % args.algo,
                          "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst)"},
             "gpu_launches": args.steps}
@@ -406,7 +413,8 @@ def bench_decode(args, kda, workloads, dev, stream, pk, world, rank):
     return {"workload": "decode_bf16: B=256 H=HV=32 Dk=Dv=128, fp32 state, %d consecutive steps" % n,
             "value": world * nb / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm_gbs"], "traffic": None, "kernel": "kda_step"},
+                         "frac": gbs / pk["hbm_gbs"], "traffic": STEP_TRAFFIC,
+                         "traffic_unit": "bytes per launch (ncu dram read + write)", "kernel": "kda_step"},
             "launches": n, "l2": "state 512 MiB > L2"}
 
 
