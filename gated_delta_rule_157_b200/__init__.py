@@ -6,13 +6,15 @@ library's names:
   kda_chunk_fwd  chunk-parallel forward over whole sequences (o, S_T, M_T)
   kda_step       single-token decode, state updated in place
   kda_compose    KCP segment prefix combine
+  kcp_chunk_fwd  context-parallel forward across the ranks of a process group
 
 PyTorch is used for device memory and streams only; every step runs in the
 library's CUDA kernels.
 """
 from ._lib import (ALGOS, EXPORTS, KdaError, kda_chunk_fwd, kda_compose, kda_device_status,
                    kda_status_string, kda_step, kda_version, library_path, load)
+from .kcp import kcp_chunk_fwd
 
-__all__ = ["kda_chunk_fwd", "kda_step", "kda_compose", "kda_device_status",
+__all__ = ["kda_chunk_fwd", "kda_step", "kda_compose", "kcp_chunk_fwd", "kda_device_status",
            "kda_status_string", "kda_version", "KdaError", "ALGOS", "EXPORTS",
            "library_path", "load"]

@@ -1,0 +1,83 @@
+"""Context-parallel KDA forward across ranks (KCP).
+
+A sequence too long for one GPU is split into contiguous segments, one per
+rank of a process group.  The state recurrence is affine in the state
+(page "Implémenter KDA", the composition test: running a segment from S0 gives
+M S0 plus its run from zero), so each rank
+
+  1. runs its segment from the zero state, keeping the final state S_seg and
+     the cumulative transition M_seg (kda_chunk_fwd with output_transition),
+  2. all-gathers (M_seg, S_seg) from every rank (the only exchange: a
+     Dk x (Dk + Dv) fp32 block per chain),
+  3. combines them in segment order into the state entering each segment
+     (kda_compose: S_in[s+1] = M_s S_in[s] + S_seg[s], S_in[0] = the initial
+     state), and
+  4. reruns its segment from S_in[rank] for its output rows.
+
+Every rank returns its own segment's o and the final state of the whole
+sequence.  The compute steps run in the library's kernels; the exchange is a
+process-group all-gather (NCCL between GPUs).
+"""
+import torch
+import torch.distributed as dist
+
+from . import _lib
+
+
+class _KernelOps:
+    """The library's kernels and the process group's all-gather."""
+
+    @staticmethod
+    def forward(q, k, v, g, beta, S0, want_M, **kw):
+        o, S_T, M_T = _lib.kda_chunk_fwd(q, k, v, g, beta, S0=S0, output_final_state=True,
+                                         output_transition=want_M, **kw)
+        return o, S_T, M_T
+
+    @staticmethod
+    def compose(M, S_seg, S_init):
+        return _lib.kda_compose(M, S_seg, S_init)
+
+    @staticmethod
+    def all_gather(t, world, group):
+        if world == 1:
+            return t.unsqueeze(0)
+        parts = [torch.empty_like(t) for _ in range(world)]
+        dist.all_gather(parts, t.contiguous(), group=group)
+        return torch.stack(parts)
+
+
+def _group_shape(group):
+    if dist.is_available() and dist.is_initialized():
+        return dist.get_world_size(group), dist.get_rank(group)
+    return 1, 0
+
+
+def kcp_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=64, group=None,
+                  g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
+                  beta_sigmoid_in_kernel=True, gate_in_kernel=True, algo="auto", ops=None):
+    """Forward of this rank's segment of a sequence split across `group`.
+
+    q, k [B,L,H,Dk]; v [B,L,HV,Dv]; g [B,L,HV,Dk]; beta [B,L,HV]: segment
+    `rank` of the sequence (segments in rank order, any lengths).  A_log,
+    dt_bias and the initial state S0 [B,HV,Dk,Dv] (or None) are the same on
+    every rank.  Returns (o [B,L,HV,Dv] of this segment, S_T [B,HV,Dk,Dv] of
+    the whole sequence).  Every rank must call this collectively.
+    """
+    ops = ops or _KernelOps
+    world, rank = _group_shape(group)
+    B, _, _, Dk = q.shape
+    HV, Dv = v.shape[2], v.shape[3]
+    kw = dict(A_log=A_log, dt_bias=dt_bias, chunk=chunk, g_min=g_min, scale=scale, l2_eps=l2_eps,
+              qk_l2norm_in_kernel=qk_l2norm_in_kernel, beta_sigmoid_in_kernel=beta_sigmoid_in_kernel,
+              gate_in_kernel=gate_in_kernel, algo=algo)
+    # 1. this segment from the zero state
+    _, S_seg, M_seg = ops.forward(q, k, v, g, beta, None, True, **kw)
+    # 2. exchange: [world, B*HV, Dk, Dk] and [world, B*HV, Dk, Dv]
+    M_all = ops.all_gather(M_seg.reshape(B * HV, Dk, Dk), world, group)
+    S_all = ops.all_gather(S_seg.reshape(B * HV, Dk, Dv), world, group)
+    # 3. state entering every segment, and the final state
+    S_init = None if S0 is None else S0.reshape(B * HV, Dk, Dv)
+    S_in = ops.compose(M_all, S_all, S_init)
+    # 4. this segment's rows from its incoming state
+    o, _, _ = ops.forward(q, k, v, g, beta, S_in[rank].reshape(B, HV, Dk, Dv).contiguous(), False, **kw)
+    return o, S_in[world].reshape(B, HV, Dk, Dv)
