@@ -372,8 +372,10 @@ def main():
     if not args.no_extras:
         line["decode"] = bench_decode(args, kda, workloads, dev, stream, pk, world, rank)
         line["kcp"] = bench_kcp(args, kda, workloads, dev, stream, world, rank)
+        line["layer"] = bench_layer(args, kda, dev, stream, pk, world)
         line["gpu_launches_extras"] = {"decode": line["decode"]["launches"],
-                                       "kcp": line["kcp"]["launches"]}
+                                       "kcp": line["kcp"]["launches"],
+                                       "layer": line["layer"]["launches"]}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
@@ -451,6 +453,52 @@ def bench_kcp(args, kda, workloads, dev, stream, world, rank):
     return {"workload": "kcp_bf16: B=1 H=HV=16 T=65536 as 8 x 8192, Dk=Dv=128",
             "value": whole_job_value(w.token_heads, world, ms), "unit": UNIT, "ms_per_step": ms,
             "launches": 3 * k}
+
+
+def bench_layer(args, kda, dev, stream, pk, world):
+    """Layer prologue (short convolution + SiLU (+ per-head L2 norm) of q, k, v)
+    and epilogue (RMSNorm + sigmoid gate of o) at the headline shapes (B=4,
+    T=8192, H=16 q/k heads, HV=32 value heads, 128 channels).  Both stream
+    bf16 in and out once: bytes = 2 B x (elements read + elements written)."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(5)
+    B, T, H, HV, D = 4, 8192, 16, 32, 128
+    xq = torch.randn((B, T, H * D), device=dev, generator=g).to(torch.bfloat16)
+    xk = torch.randn((B, T, H * D), device=dev, generator=g).to(torch.bfloat16)
+    xv = torch.randn((B, T, HV * D), device=dev, generator=g).to(torch.bfloat16)
+    wq, wk = (torch.randn((H * D, 4), device=dev, generator=g) * 0.5 for _ in range(2))
+    wv = torch.randn((HV * D, 4), device=dev, generator=g) * 0.5
+    yq, yk, yv = torch.empty_like(xq), torch.empty_like(xk), torch.empty_like(xv)
+    o = torch.randn((B * T, HV, D), device=dev, generator=g).to(torch.bfloat16)
+    gate = torch.randn((B * T, HV, D), device=dev, generator=g).to(torch.bfloat16)
+    yo = torch.empty_like(o)
+
+    def pro(_i):
+        kda.kda_short_conv(xq, wq, head_dim=D, y=yq, stream=stream)
+        kda.kda_short_conv(xk, wk, head_dim=D, y=yk, stream=stream)
+        kda.kda_short_conv(xv, wv, y=yv, stream=stream)
+
+    def epi(_i):
+        kda.kda_output_gate(o, gate, y=yo, stream=stream)
+
+    out = {"workload": "B=4 T=8192: prologue of q, k (16 x 128 channels, head L2 norm) and "
+                       "v (32 x 128); epilogue of o (32 heads x 128)", "launches": 0}
+    for name, fn, nbytes, nl in (("prologue", pro, 2 * 2 * (xq.numel() + xk.numel() + xv.numel()), 3),
+                                 ("epilogue", epi, 2 * 3 * o.numel(), 1)):
+        for i in range(args.warmup):
+            fn(i)
+        barrier(world, dev)
+        k = max(3, min(args.steps, 10))
+        per = time_launches(fn, k, stream)
+        barrier(world, dev)
+        ms_local = sum(per) / len(per)
+        ms = max_over_ranks(ms_local, world, dev)
+        gbs = nbytes / (ms_local * 1e-3) / 1e9
+        out[name] = {"ms_per_step": ms, "value": world * nbytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": gbs / pk["hbm_gbs"], "traffic": None}}
+        out["launches"] += nl * k
+    return out
 
 
 if __name__ == "__main__":

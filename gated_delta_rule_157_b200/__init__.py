@@ -7,14 +7,17 @@ library's names:
   kda_step       single-token decode, state updated in place
   kda_compose    KCP segment prefix combine
   kcp_chunk_fwd  context-parallel forward across the ranks of a process group
+  kda_short_conv, kda_output_gate   layer prologue / epilogue around the core
 
 PyTorch is used for device memory and streams only; every step runs in the
 library's CUDA kernels.
 """
 from ._lib import (ALGOS, EXPORTS, KdaError, kda_chunk_fwd, kda_compose, kda_device_status,
-                   kda_status_string, kda_step, kda_version, library_path, load)
+                   kda_output_gate, kda_short_conv, kda_status_string, kda_step, kda_version,
+                   library_path, load)
 from .kcp import kcp_chunk_fwd
 
-__all__ = ["kda_chunk_fwd", "kda_step", "kda_compose", "kcp_chunk_fwd", "kda_device_status",
+__all__ = ["kda_chunk_fwd", "kda_step", "kda_compose", "kcp_chunk_fwd", "kda_short_conv",
+           "kda_output_gate", "kda_device_status",
            "kda_status_string", "kda_version", "KdaError", "ALGOS", "EXPORTS",
            "library_path", "load"]

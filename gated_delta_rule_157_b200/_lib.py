@@ -59,8 +59,26 @@ class StepArgs(ctypes.Structure):
     ]
 
 
+class ConvArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("C", ctypes.c_int), ("K", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("silu", ctypes.c_int), ("l2_eps", ctypes.c_float),
+        ("x", ctypes.c_void_p), ("w", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+        ("state_in", ctypes.c_void_p), ("y", ctypes.c_void_p), ("state_out", ctypes.c_void_p),
+    ]
+
+
+class GateArgs(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int), ("HV", ctypes.c_int), ("D", ctypes.c_int), ("eps", ctypes.c_float),
+        ("o", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("weight", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
 EXPORTS = ["kda_chunk_fwd", "kda_step", "kda_compose", "kda_device_status",
-           "kda_status_string", "kda_version", "kda_debug_chunk_stall"]
+           "kda_status_string", "kda_version", "kda_debug_chunk_stall",
+           "kda_short_conv", "kda_output_gate"]
 
 _lib = None
 
@@ -82,6 +100,10 @@ def load():
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_debug_chunk_stall.argtypes = [ctypes.POINTER(ChunkArgs), ctypes.c_void_p]
     lib.kda_debug_chunk_stall.restype = ctypes.c_int
+    lib.kda_short_conv.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
+    lib.kda_short_conv.restype = ctypes.c_int
+    lib.kda_output_gate.argtypes = [ctypes.POINTER(GateArgs), ctypes.c_void_p]
+    lib.kda_output_gate.restype = ctypes.c_int
     lib.kda_step.argtypes = [ctypes.POINTER(StepArgs), ctypes.c_void_p]
     lib.kda_step.restype = ctypes.c_int
     lib.kda_compose.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 5
@@ -242,6 +264,60 @@ def kda_compose(M, S_seg, S_init=None, S_in=None, stream=None):
                          _stream(stream, dev))
     _raise("kda_compose", st)
     return S_in
+
+
+def kda_short_conv(x, w, bias=None, *, head_dim=0, silu=True, l2_eps=1e-6, state_in=None,
+                   y=None, state_out=None, want_state=False, stream=None):
+    """Layer prologue: causal depthwise short convolution (K = w.shape[1] taps,
+    tap K-1 on the current token), then SiLU and per-128-channel L2 norm when
+    asked.  x [B,T,C] bf16 (C % 128 == 0); w [C,K], bias [C] float32;
+    state_in [B,K-1,C] bf16 (tokens before x, oldest first) or None.
+    Returns y [B,T,C] bf16, or (y, state_out) with want_state."""
+    lib = load()
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise ValueError("x must be a CUDA tensor")
+    dev = x.device
+    B, T, C = x.shape
+    K = w.shape[1]
+    _check(x, "x", (B, T, C), torch.bfloat16, dev)
+    _check(w, "w", (C, K), torch.float32, dev)
+    _check(bias, "bias", (C,), torch.float32, dev)
+    _check(state_in, "state_in", (B, K - 1, C), torch.bfloat16, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", (B, T, C), torch.bfloat16, dev)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, K - 1, C), dtype=torch.bfloat16, device=dev)
+    _check(state_out, "state_out", (B, K - 1, C), torch.bfloat16, dev)
+    a = ConvArgs()
+    a.B, a.T, a.C, a.K = B, T, C, K
+    a.head_dim, a.silu, a.l2_eps = int(head_dim), int(bool(silu)), float(l2_eps)
+    a.x, a.w, a.bias, a.state_in = _ptr(x), _ptr(w), _ptr(bias), _ptr(state_in)
+    a.y, a.state_out = _ptr(y), _ptr(state_out)
+    _raise("kda_short_conv", lib.kda_short_conv(ctypes.byref(a), _stream(stream, dev)))
+    return (y, state_out) if want_state else y
+
+
+def kda_output_gate(o, gate, weight=None, *, eps=1e-6, y=None, stream=None):
+    """Layer epilogue: sigmoid(gate) * weight * RMSNorm over each head's D = 128
+    channels of o.  o, gate [..., HV, D] bf16; weight [D] float32 or None."""
+    lib = load()
+    if not isinstance(o, torch.Tensor) or not o.is_cuda:
+        raise ValueError("o must be a CUDA tensor")
+    dev = o.device
+    HV, D = o.shape[-2], o.shape[-1]
+    N = o.numel() // (HV * D)
+    _check(o, "o", tuple(o.shape), torch.bfloat16, dev)
+    _check(gate, "gate", tuple(o.shape), torch.bfloat16, dev)
+    _check(weight, "weight", (D,), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(o)
+    _check(y, "y", tuple(o.shape), torch.bfloat16, dev)
+    a = GateArgs()
+    a.N, a.HV, a.D, a.eps = N, HV, D, float(eps)
+    a.o, a.gate, a.weight, a.y = _ptr(o), _ptr(gate), _ptr(weight), _ptr(y)
+    _raise("kda_output_gate", lib.kda_output_gate(ctypes.byref(a), _stream(stream, dev)))
+    return y
 
 
 def kda_device_status(stream=None, device=None):

@@ -178,6 +178,54 @@ kda_status kda_compose(int n_seg, int BH, int Dk, int Dv, const float *M, const 
                                            static_cast<cudaStream_t>(stream)));
 }
 
+kda_status kda_short_conv(const kda_conv_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARG;
+    if (a->B < 0 || a->T < 0 || a->C < 1 || a->K < 1 || a->K > 4 || !(a->l2_eps >= 0.f))
+        return KDA_ERR_INVALID_ARG;
+    if (a->head_dim != 0 && a->head_dim != 128) return KDA_ERR_UNSUPPORTED;
+    if (a->C % 128 != 0) return KDA_ERR_UNSUPPORTED;
+    if (a->B == 0) return KDA_OK;
+    const size_t ntok = (size_t)a->B * a->T, es = 2;
+    if (!a->w || (ntok > 0 && (!a->x || !a->y))) return KDA_ERR_INVALID_ARG;
+    const void *p8[] = {a->x, a->y, a->state_in, a->state_out};
+    for (const void *p : p8)
+        if (p && !aligned(p, 8)) return KDA_ERR_ALIGNMENT;
+    if (!aligned(a->w, 4) || (a->bias && !aligned(a->bias, 4))) return KDA_ERR_ALIGNMENT;
+    const size_t nx = ntok * a->C * es, ns = (size_t)a->B * (a->K - 1) * a->C * es;
+    Range r_y = range_of(a->y, ntok ? nx : 0), r_so = range_of(a->state_out, a->state_out ? ns : 0);
+    Range r_in[] = {range_of(a->x, ntok ? nx : 0), range_of(a->state_in, a->state_in ? ns : 0),
+                    range_of(a->w, (size_t)a->C * a->K * 4), range_of(a->bias, a->bias ? (size_t)a->C * 4 : 0)};
+    for (Range r : r_in)
+        if (overlaps(r_y, r) || overlaps(r_so, r)) return KDA_ERR_ALIAS;
+    if (overlaps(r_y, r_so)) return KDA_ERR_ALIAS;
+    kda::ConvParams p;
+    p.B = a->B; p.T = a->T; p.C = a->C; p.K = a->K; p.head_dim = a->head_dim; p.silu = a->silu != 0;
+    p.l2_eps = a->l2_eps;
+    p.x = a->x; p.w = a->w; p.bias = a->bias; p.state_in = a->state_in; p.y = a->y; p.state_out = a->state_out;
+    return cuda_status(kda::launch_short_conv(p, static_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_output_gate(const kda_gate_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARG;
+    if (a->N < 0 || a->HV < 1 || a->D < 1 || !(a->eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    if (a->D != 128) return KDA_ERR_UNSUPPORTED;
+    if (a->N == 0) return KDA_OK;
+    if (!a->o || !a->gate || !a->y) return KDA_ERR_INVALID_ARG;
+    const void *p8[] = {a->o, a->gate, a->y};
+    for (const void *p : p8)
+        if (!aligned(p, 8)) return KDA_ERR_ALIGNMENT;
+    if (a->weight && !aligned(a->weight, 4)) return KDA_ERR_ALIGNMENT;
+    const size_t n = (size_t)a->N * a->HV * a->D * 2;
+    Range r_y = range_of(a->y, n);
+    if (overlaps(r_y, range_of(a->o, n)) || overlaps(r_y, range_of(a->gate, n)) ||
+        overlaps(r_y, range_of(a->weight, a->weight ? (size_t)a->D * 4 : 0)))
+        return KDA_ERR_ALIAS;
+    kda::GateParams p;
+    p.N = a->N; p.HV = a->HV; p.D = a->D; p.eps = a->eps;
+    p.o = a->o; p.gate = a->gate; p.weight = a->weight; p.y = a->y;
+    return cuda_status(kda::launch_output_gate(p, static_cast<cudaStream_t>(stream)));
+}
+
 kda_status kda_device_status(void *stream) {
     unsigned int word = 0;
     cudaError_t e = kda::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &word);

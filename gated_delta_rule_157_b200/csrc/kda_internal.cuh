@@ -49,12 +49,31 @@ struct StepParams {
     void *o;
 };
 
+struct ConvParams {
+    int B, T, C, K, head_dim, silu;
+    float l2_eps;
+    const void *x;
+    const float *w, *bias;
+    const void *state_in;
+    void *y, *state_out;
+};
+
+struct GateParams {
+    int N, HV, D;
+    float eps;
+    const void *o, *gate;
+    const float *weight;
+    void *y;
+};
+
 // Launchers (host).  They assume validated arguments and return the launch status.
 cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s);
 bool chunk_tc_supported(const ChunkParams &p, bool bf16);
 cudaError_t launch_chunk_empty(const ChunkParams &p, cudaStream_t s);   // T == 0
 cudaError_t launch_step(const StepParams &p, bool bf16, cudaStream_t s);
+cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s);
+cudaError_t launch_output_gate(const GateParams &p, cudaStream_t s);
 cudaError_t launch_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
                            const float *S_seg, const float *S_init, float *S_in,
                            cudaStream_t s);

@@ -1,0 +1,168 @@
+// Layer prologue and epilogue around the KDA core (page "KDA 模块交互式演示",
+// sections 1.1 ShortConv and 1.7 the complete layer; page "Implémenter KDA",
+// "La paramétrisation" and "La porte de sortie de rang plein"):
+//
+//   short_conv_kernel   u = bias + causal depthwise K-tap convolution of x,
+//                       y = SiLU(u) (optional), L2-normalised per 128-channel
+//                       head (optional); carries a K-1 token window across
+//                       calls (decode, or a sequence run in pieces).
+//   output_gate_kernel  y = sigmoid(gate) * weight * o / sqrt(mean(o^2) + eps)
+//                       per (token, head) of 128 channels.
+//
+// Both are HBM-bound streams: one warp covers 128 channels of a token (lane =
+// 4 channels, 8-byte loads and stores, 256 contiguous bytes per warp), the
+// per-head reductions are warp shuffles, and nothing is read twice.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kConvTokens = 32;     // tokens per warp (sliding window in registers)
+constexpr int kLayerThreads = 256;
+
+__device__ __forceinline__ void unpack4(uint2 w, float (&f)[4]) {
+    f[0] = __uint_as_float(w.x << 16);
+    f[1] = __uint_as_float(w.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(w.y << 16);
+    f[3] = __uint_as_float(w.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ uint2 pack4(const float (&f)[4]) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]);
+    __nv_bfloat162 b = __floats2bfloat162_rn(f[2], f[3]);
+    return make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float silu(float u) { return u / (1.f + __expf(-u)); }
+
+// Warp w of the grid: batch b, 128-channel group grp, tokens [t0, t0 + kConvTokens).
+template <int K>
+__global__ void __launch_bounds__(kLayerThreads)
+short_conv_kernel(ConvParams p) {
+    const int lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * (kLayerThreads / 32) + (threadIdx.x >> 5);
+    const int ngrp = p.C / 128;
+    const int nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
+    if (gw >= (long long)p.B * ngrp * nblk) return;
+    const int blk = (int)(gw % nblk);
+    const int grp = (int)((gw / nblk) % ngrp);
+    const int b = (int)(gw / ((long long)nblk * ngrp));
+    const int c0 = grp * 128 + 4 * lane;
+    const int t0 = blk * kConvTokens, t1 = min(p.T, t0 + kConvTokens);
+    const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(p.x);
+    const __nv_bfloat16 *sin = static_cast<const __nv_bfloat16 *>(p.state_in);
+    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.y);
+
+    float w[4][4], bias[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        bias[u] = p.bias ? p.bias[c0 + u] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[u][j] = j < K ? p.w[(size_t)(c0 + u) * K + j] : 0.f;
+    }
+    // win[s]: token t - 3 + s, s = 0..2 (only the last K-1 slots are used).
+    auto fetch = [&](int tok, float (&f)[4]) {
+        if (tok >= 0) {
+            unpack4(*reinterpret_cast<const uint2 *>(x + ((size_t)b * p.T + tok) * p.C + c0), f);
+        } else if (sin && tok >= -(K - 1)) {
+            unpack4(*reinterpret_cast<const uint2 *>(sin + ((size_t)b * (K - 1) + (K - 1) + tok) * p.C + c0), f);
+        } else {
+            f[0] = f[1] = f[2] = f[3] = 0.f;
+        }
+    };
+    float win[3][4];
+#pragma unroll
+    for (int s = 0; s < 3; ++s) fetch(t0 - 3 + s, win[s]);
+
+    float nxt[4];
+    if (t0 < t1) fetch(t0, nxt);
+    for (int t = t0; t < t1; ++t) {
+        float cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+        if (t + 1 < t1) fetch(t + 1, nxt);          // one token ahead
+        float out[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            // taps j = 0..K-2 read win[4 - K + j]; tap K-1 reads the current token
+            float acc = bias[u];
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+                if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
+            acc = fmaf(w[u][K - 1], cur[u], acc);
+            out[u] = p.silu ? silu(acc) : acc;
+        }
+        if (p.head_dim) {
+            const float ss = warp_sum(out[0] * out[0] + out[1] * out[1] + out[2] * out[2] + out[3] * out[3]);
+            const float r = rsqrtf(ss + p.l2_eps);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) out[u] *= r;
+        }
+        *reinterpret_cast<uint2 *>(y + ((size_t)b * p.T + t) * p.C + c0) = pack4(out);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            win[0][u] = win[1][u];
+            win[1][u] = win[2][u];
+            win[2][u] = cur[u];
+        }
+    }
+    // The last K-1 tokens of state_in ++ x, oldest first.
+    if (p.state_out && t1 == p.T) {
+        __nv_bfloat16 *so = static_cast<__nv_bfloat16 *>(p.state_out);
+#pragma unroll
+        for (int r = 0; r < K - 1; ++r)
+            *reinterpret_cast<uint2 *>(so + ((size_t)b * (K - 1) + r) * p.C + c0) = pack4(win[4 - K + r]);
+    }
+}
+
+// Warp per (row n, head h), lane = 4 channels of the head's 128.
+__global__ void __launch_bounds__(kLayerThreads)
+output_gate_kernel(GateParams p) {
+    const int lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * (kLayerThreads / 32) + (threadIdx.x >> 5);
+    if (gw >= (long long)p.N * p.HV) return;
+    const size_t off = (size_t)gw * p.D + 4 * lane;
+    float o[4], g[4], wv[4] = {1.f, 1.f, 1.f, 1.f};
+    unpack4(*reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.o) + off), o);
+    unpack4(*reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.gate) + off), g);
+    if (p.weight) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) wv[u] = p.weight[4 * lane + u];
+    }
+    const float ms = warp_sum(o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3]) * (1.f / 128.f);
+    const float r = rsqrtf(ms + p.eps);
+    float out[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) out[u] = o[u] * r * wv[u] / (1.f + __expf(-g[u]));
+    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.y) + off) = pack4(out);
+}
+
+}  // namespace
+
+cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s) {
+    const long long nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
+    const long long warps = (long long)p.B * (p.C / 128) * nblk;
+    if (warps == 0) return cudaSuccess;
+    const long long blocks = (warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32);
+    switch (p.K) {
+        case 1: short_conv_kernel<1><<<(unsigned)blocks, kLayerThreads, 0, s>>>(p); break;
+        case 2: short_conv_kernel<2><<<(unsigned)blocks, kLayerThreads, 0, s>>>(p); break;
+        case 3: short_conv_kernel<3><<<(unsigned)blocks, kLayerThreads, 0, s>>>(p); break;
+        default: short_conv_kernel<4><<<(unsigned)blocks, kLayerThreads, 0, s>>>(p); break;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_output_gate(const GateParams &p, cudaStream_t s) {
+    const long long warps = (long long)p.N * p.HV;
+    if (warps == 0) return cudaSuccess;
+    const long long blocks = (warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32);
+    output_gate_kernel<<<(unsigned)blocks, kLayerThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

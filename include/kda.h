@@ -160,6 +160,64 @@ kda_status kda_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
                        const float *S_seg, const float *S_init, float *S_in,
                        void *stream);
 
+/* ---------------------------------------------------------------------------
+ * Layer prologue and epilogue around the core (page "KDA 模块交互式演示",
+ * sections 1.1 and 1.7; page "Implémenter KDA", "La paramétrisation" and
+ * "La porte de sortie de rang plein"): the parts of the KDA layer that need no
+ * projection weights.
+ * ------------------------------------------------------------------------- */
+
+/* Causal depthwise short convolution, then optional SiLU and per-head L2
+ * norm (the q / k / v prologue: q = L2Norm(SiLU(ShortConv(x)))):
+ *
+ *     u[t, c] = bias[c] + sum_{j=0}^{K-1} w[c, j] * x[t - (K-1) + j, c]
+ *     y[t, c] = silu ? u / (1 + exp(-u)) : u
+ *     y[t, c] <- y[t, c] / sqrt(sum_{c' in head(c)} y[t, c']^2 + l2_eps)   if head_dim > 0
+ *
+ * Tap K-1 multiplies the current token, so w[:, K-1] = 1 (zero elsewhere,
+ * bias 0) is the identity the pages initialise with.  Tokens before the first
+ * one come from state_in (the K-1 previous tokens, oldest first) or are zero;
+ * state_out receives the last K-1 tokens of state_in ++ x, so a sequence run
+ * in pieces (or one token at a time for decode) matches one run over the
+ * whole sequence. */
+typedef struct {
+    int B, T, C;               /* tokens [B, T]; C channels per token, C % 128 == 0 */
+    int K;                     /* taps, 1..4 (4 on the pages) */
+    int head_dim;              /* 0 (no norm) or 128: L2-normalise every 128 channels */
+    int silu;                  /* apply SiLU after the convolution */
+    float l2_eps;              /* 1e-6 */
+    const void *x;             /* [B, T, C] bf16 */
+    const float *w;            /* [C, K] fp32 */
+    const float *bias;         /* [C] fp32, or NULL (= 0) */
+    const void *state_in;      /* [B, K-1, C] bf16, or NULL (= zeros) */
+    void *y;                   /* [B, T, C] bf16 */
+    void *state_out;           /* [B, K-1, C] bf16, or NULL */
+} kda_conv_args;
+
+/* Runs the prologue above.  T may be 0 (only state_out is written).  x, y,
+ * state_in and state_out must be 8-byte aligned; y and state_out must not
+ * overlap any input or each other.  Errors as for kda_chunk_fwd. */
+kda_status kda_short_conv(const kda_conv_args *args, void *stream);
+
+/* Output gate of the layer (the epilogue before the output projection):
+ *
+ *     y[n, h, :] = sigmoid(gate[n, h, :]) * weight * o[n, h, :] / sqrt(mean(o[n, h, :]^2) + eps)
+ *
+ * per row n (token), head h: RMSNorm over the D channels of each head with a
+ * per-channel scale shared by the heads, times the sigmoid gate. */
+typedef struct {
+    int N, HV, D;              /* rows (B * T), heads, channels per head (D == 128) */
+    float eps;                 /* 1e-6 */
+    const void *o;             /* [N, HV, D] bf16 (the core's output) */
+    const void *gate;          /* [N, HV, D] bf16, before the sigmoid */
+    const float *weight;       /* [D] fp32, or NULL (= 1) */
+    void *y;                   /* [N, HV, D] bf16 */
+} kda_gate_args;
+
+/* Runs the epilogue above.  o, gate and y must be 8-byte aligned; y must not
+ * overlap o or gate.  Errors as for kda_chunk_fwd. */
+kda_status kda_output_gate(const kda_gate_args *args, void *stream);
+
 /* Reads and clears the device error word of the current device after
  * synchronising `stream`.  Returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_CUDA. */
 kda_status kda_device_status(void *stream);

@@ -13,6 +13,9 @@ Contents:
   * ``chunkwise`` -- FP64 NumPy restatement of the chunk-parallel form (page
     "KDA 模块交互式演示" section 1.5, Eqs. 3-4) used only to pin the reading of
     the chunk algebra against the recurrence.
+  * ``layer`` -- FP64 NumPy restatements of the layer prologue (short
+    convolution, SiLU, per-head L2 norm) and epilogue (per-head RMSNorm and the
+    sigmoid output gate).
 
 Inputs are NumPy arrays (any float dtype; they are widened to float64 exactly).
 """
