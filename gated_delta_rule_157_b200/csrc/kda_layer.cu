@@ -20,7 +20,7 @@
 namespace kda {
 namespace {
 
-constexpr int kConvTokens = 32;     // tokens per warp (sliding window in registers)
+constexpr int kConvTokens = 64;     // tokens per warp (sliding window in registers)
 constexpr int kLayerThreads = 256;
 
 __device__ __forceinline__ void unpack4(uint2 w, float (&f)[4]) {
@@ -39,9 +39,10 @@ __device__ __forceinline__ float warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
-__device__ __forceinline__ float silu(float u) { return u / (1.f + __expf(-u)); }
+__device__ __forceinline__ float silu(float u) { return __fdividef(u, 1.f + __expf(-u)); }
 
-// Warp w of the grid: batch b, 128-channel group grp, tokens [t0, t0 + kConvTokens).
+// Warp w of the grid: batch b, 128-channel group grp, tokens [t0, t0 + kConvTokens)
+// (only the 3 halo tokens before t0 are read twice).
 template <int K>
 __global__ void __launch_bounds__(kLayerThreads)
 short_conv_kernel(ConvParams p) {
@@ -50,8 +51,10 @@ short_conv_kernel(ConvParams p) {
     const int ngrp = p.C / 128;
     const int nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
     if (gw >= (long long)p.B * ngrp * nblk) return;
-    const int blk = (int)(gw % nblk);
-    const int grp = (int)((gw / nblk) % ngrp);
+    // Consecutive warps take consecutive channel groups of the same tokens, so
+    // a thread block streams whole contiguous spans of each token row.
+    const int grp = (int)(gw % ngrp);
+    const int blk = (int)((gw / ngrp) % nblk);
     const int b = (int)(gw / ((long long)nblk * ngrp));
     const int c0 = grp * 128 + 4 * lane;
     const int t0 = blk * kConvTokens, t1 = min(p.T, t0 + kConvTokens);
@@ -80,65 +83,110 @@ short_conv_kernel(ConvParams p) {
 #pragma unroll
     for (int s = 0; s < 3; ++s) fetch(t0 - 3 + s, win[s]);
 
-    float nxt[4];
-    if (t0 < t1) fetch(t0, nxt);
-    for (int t = t0; t < t1; ++t) {
-        float cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
-        if (t + 1 < t1) fetch(t + 1, nxt);          // one token ahead
-        float out[4];
+    // Groups of 8 tokens, double-buffered: the 8 row loads of the next group
+    // are in flight while the current group is computed.  Rows past the block
+    // are computed from zeros and not stored.  state_out (the last K-1 tokens of
+    // state_in ++ x, oldest first) is written at the sequence's last token.
+    constexpr int G = 8;
+    __nv_bfloat16 *so = static_cast<__nv_bfloat16 *>(p.state_out);
+    auto put_state = [&](const float (&s0)[4], const float (&s1)[4], const float (&s2)[4]) {
+        const float *rows[3] = {s0, s1, s2};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            // taps j = 0..K-2 read win[4 - K + j]; tap K-1 reads the current token
-            float acc = bias[u];
-#pragma unroll
-            for (int j = 0; j < 3; ++j)
-                if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
-            acc = fmaf(w[u][K - 1], cur[u], acc);
-            out[u] = p.silu ? silu(acc) : acc;
+        for (int r = 0; r < K - 1; ++r) {
+            const float *src = rows[4 - K + r];
+            const float f[4] = {src[0], src[1], src[2], src[3]};
+            *reinterpret_cast<uint2 *>(so + ((size_t)b * (K - 1) + r) * p.C + c0) = pack4(f);
         }
-        if (p.head_dim) {
-            const float ss = warp_sum(out[0] * out[0] + out[1] * out[1] + out[2] * out[2] + out[3] * out[3]);
-            const float r = rsqrtf(ss + p.l2_eps);
+    };
+    auto load_group = [&](int tg, uint2 (&r)[G]) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) out[u] *= r;
+        for (int i = 0; i < G; ++i)
+            r[i] = tg + i < t1 ? *reinterpret_cast<const uint2 *>(x + ((size_t)b * p.T + tg + i) * p.C + c0)
+                               : make_uint2(0, 0);
+    };
+    auto process = [&](int tg, const uint2 (&r)[G]) {
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+            float cur[4];
+            unpack4(r[i], cur);
+            float out[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                // taps j = 0..K-2 read win[4 - K + j]; tap K-1 reads the current token
+                float acc = bias[u];
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
+                acc = fmaf(w[u][K - 1], cur[u], acc);
+                out[u] = p.silu ? silu(acc) : acc;
+            }
+            if (p.head_dim) {
+                const float ss = warp_sum(out[0] * out[0] + out[1] * out[1] + out[2] * out[2] + out[3] * out[3]);
+                const float rn = rsqrtf(ss + p.l2_eps);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) out[u] *= rn;
+            }
+            if (tg + i < t1) *reinterpret_cast<uint2 *>(y + ((size_t)b * p.T + tg + i) * p.C + c0) = pack4(out);
+            if (so && tg + i + 1 == p.T) put_state(win[1], win[2], cur);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                win[0][u] = win[1][u];
+                win[1][u] = win[2][u];
+                win[2][u] = cur[u];
+            }
         }
-        *reinterpret_cast<uint2 *>(y + ((size_t)b * p.T + t) * p.C + c0) = pack4(out);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            win[0][u] = win[1][u];
-            win[1][u] = win[2][u];
-            win[2][u] = cur[u];
+    };
+    uint2 ra[G], rb[G];
+    if (t0 < t1) load_group(t0, ra);
+    for (int tg = t0; tg < t1; tg += 2 * G) {
+        if (tg + G < t1) load_group(tg + G, rb);
+        process(tg, ra);
+        if (tg + G < t1) {
+            if (tg + 2 * G < t1) load_group(tg + 2 * G, ra);
+            process(tg + G, rb);
         }
     }
-    // The last K-1 tokens of state_in ++ x, oldest first.
-    if (p.state_out && t1 == p.T) {
-        __nv_bfloat16 *so = static_cast<__nv_bfloat16 *>(p.state_out);
-#pragma unroll
-        for (int r = 0; r < K - 1; ++r)
-            *reinterpret_cast<uint2 *>(so + ((size_t)b * (K - 1) + r) * p.C + c0) = pack4(win[4 - K + r]);
-    }
+    if (so && p.T == 0) put_state(win[0], win[1], win[2]);   // no token: state_in passes through
 }
 
-// Warp per (row n, head h), lane = 4 channels of the head's 128.
+// Warp per 4 consecutive (row n, head h) pairs, lane = 4 channels of the
+// head's 128; the 8 loads of the four pairs are in flight together.
+constexpr int kGateRows = 4;
 __global__ void __launch_bounds__(kLayerThreads)
 output_gate_kernel(GateParams p) {
     const int lane = threadIdx.x & 31;
     const long long gw = (long long)blockIdx.x * (kLayerThreads / 32) + (threadIdx.x >> 5);
-    if (gw >= (long long)p.N * p.HV) return;
-    const size_t off = (size_t)gw * p.D + 4 * lane;
-    float o[4], g[4], wv[4] = {1.f, 1.f, 1.f, 1.f};
-    unpack4(*reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.o) + off), o);
-    unpack4(*reinterpret_cast<const uint2 *>(static_cast<const __nv_bfloat16 *>(p.gate) + off), g);
+    const long long rows = (long long)p.N * p.HV;
+    const long long r0 = gw * kGateRows;
+    if (r0 >= rows) return;
+    float wv[4] = {1.f, 1.f, 1.f, 1.f};
     if (p.weight) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) wv[u] = p.weight[4 * lane + u];
     }
-    const float ms = warp_sum(o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3]) * (1.f / 128.f);
-    const float r = rsqrtf(ms + p.eps);
-    float out[4];
+    const __nv_bfloat16 *po = static_cast<const __nv_bfloat16 *>(p.o);
+    const __nv_bfloat16 *pg = static_cast<const __nv_bfloat16 *>(p.gate);
+    uint2 ro[kGateRows], rg[kGateRows];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) out[u] = o[u] * r * wv[u] / (1.f + __expf(-g[u]));
-    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.y) + off) = pack4(out);
+    for (int i = 0; i < kGateRows; ++i) {
+        const bool in = r0 + i < rows;
+        const size_t off = (size_t)(r0 + i) * p.D + 4 * lane;
+        ro[i] = in ? *reinterpret_cast<const uint2 *>(po + off) : make_uint2(0, 0);
+        rg[i] = in ? *reinterpret_cast<const uint2 *>(pg + off) : make_uint2(0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < kGateRows; ++i) {
+        float o[4], g[4];
+        unpack4(ro[i], o);
+        unpack4(rg[i], g);
+        const float ms = warp_sum(o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3]) * (1.f / 128.f);
+        const float r = rsqrtf(ms + p.eps);
+        float out[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) out[u] = __fdividef(o[u] * r * wv[u], 1.f + __expf(-g[u]));
+        if (r0 + i < rows)
+            *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.y) + (size_t)(r0 + i) * p.D + 4 * lane) = pack4(out);
+    }
 }
 
 }  // namespace
@@ -158,7 +206,7 @@ cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s) {
 }
 
 cudaError_t launch_output_gate(const GateParams &p, cudaStream_t s) {
-    const long long warps = (long long)p.N * p.HV;
+    const long long warps = ((long long)p.N * p.HV + kGateRows - 1) / kGateRows;
     if (warps == 0) return cudaSuccess;
     const long long blocks = (warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32);
     output_gate_kernel<<<(unsigned)blocks, kLayerThreads, 0, s>>>(p);
