@@ -9,15 +9,19 @@
 // "La forme par blocs", for U = Ut - W S), the work per chunk splits in two:
 //
 // prep warps 0-15 (state-independent; run one chunk ahead of the state warps)
-//   loads        q, k, z, v, beta of the chunk
+//   inputs       q, k, z rows of the chunk by tensor-map TMA (requested a chunk
+//                ahead), beta prefetched in a register
 //   prologue     L2 norm of q,k; beta = sigmoid; g = g_min sigmoid(exp(A_log)(z + dt_bias))
 //   operands     bf16 tiles scaled by exp(G_r - P_R) <= 1 and exp(P_R' - G_i)
 //                (<= e^80 inside a tile, <= 1 before it)
-//   (I)   MMA    [K e^L ; Q e^L] x [K_R' e^{P_R'-G}]^T    -> A_kk, A_qk (all tiles at once)
-//   solve        T = (I + tril(Diag(beta) A_kk, -1))^-1    (blocked, fp32)
-//   (II)  MMA    Ut^T = V^T (T Diag(beta))^T              -> TMEM buffer of the chunk
-//   (III) MMA    W^T  = (K Gamma)^T (T Diag(beta))^T      -> -W (MN-major smem)
+//   (I)   MMA    [K e^L ; Q e^L] x [K_R' e^{P_R'-G}]^T    -> A_kk, A_qk (all tiles at once),
+//                issued by one lane of warp 15
+//   solve        T = (I + tril(Diag(beta) A_kk, -1))^-1: fp32 substitution on the
+//                diagonal 16 x 16 blocks, tf32 warp-level MMAs for the rest,
+//                written as the bf16 operand T Diag(beta)
 // state warps 16-19 (the serial carry, one TMEM lane per value channel)
+//   (II)  MMA    Ut^T = V^T (T Diag(beta))^T   (V tile by swizzled TMA) -> TMEM buffer
+//   (III) MMA    W^T  = (K Gamma)^T (T Diag(beta))^T, read out as -W (MN-major smem)
 //   (IV)  MMA    U^T = Ut^T - S^T W^T        while the state is scaled by gamma_C
 //   (VI)  MMA    S^T <- S^T Diag(gamma_C) + U^T K',   K' = K exp(G_C - G)
 //   (V)   MMA    O^T = S^T (Q Gamma)^T + U^T A_qk^T   -> o
@@ -27,16 +31,18 @@
 // bornée"); across tiles the factors are decays <= 1.  Exponentials use base 2:
 // the log-decay is carried in log2 units.
 //
-// Hand-off between the two roles uses mbarriers; the operands the state warps
-// read (Q Gamma, K', A_qk, gamma_C and the Ut^T accumulator) are double
-// buffered, -W is single buffered and released as soon as MMA (IV) completes.
-// Every wait is bounded; if one gives up, the CTA records the device error
-// word, both roles leave their loops, the TMEM is freed and the CTA returns.
+// Hand-off between the two roles uses mbarriers (READY / FREE and the MMA
+// (II)/(III) completion double-buffered by chunk parity); the operands the
+// state warps read (Q Gamma, K', A_qk, gamma_C and the Ut^T accumulator) are
+// double buffered.  Every wait is bounded; if one gives up, the CTA records the
+// device error word, both roles leave their loops, in-flight MMAs and tensor
+// copies are drained (bounded), the TMEM is freed and the CTA returns.
 //
 // All MMAs are cta_group::1, M = 128, BF16 x BF16 -> FP32 in TMEM; shared
-// operands use the K-major (or, for W, MN-major) 128-byte-swizzle layouts of
-// tc_ptx.cuh.  When M_T is requested a second CTA per chain (blockIdx.y == 1)
-// runs the same recurrence on the transition columns: v = 0 and S0 = I, no o.
+// operands use the 128-byte-swizzle layouts of tc_ptx.cuh (K-major, or
+// MN-major for V, K Gamma, K' and -W).  When M_T is requested a second CTA per
+// chain (blockIdx.y == 1) runs the same recurrence on the transition columns:
+// v = 0 and S0 = I, no o.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
