@@ -8,8 +8,9 @@ q/k L2-norm, beta sigmoid and bounded gate in-kernel), inputs resident in HBM.
 Rank 0 prints ONE JSON line with the throughput in token-heads/s, its fraction
 of the BF16 tensor-core and HBM rooflines, the end-to-end number through the
 Python API with host buffers, the decode step (B=256, H=HV=32, D=128, fp32
-state, 512 consecutive steps) in GB/s, the segmented KCP pass, and the FP64
-oracle timed on the host cores as a reported baseline.
+state, 512 consecutive steps) in GB/s, the segmented KCP pass, the layer
+prologue / epilogue kernels in GB/s, and the FP64 oracle timed on the host
+cores as a reported baseline.
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload (weak
 scaling, no collective on the data path); the time is the max over ranks.
