@@ -437,38 +437,13 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
                 Lst[0] += s4.x; Lst[1] += s4.y; Lst[2] += s4.z; Lst[3] += s4.w;
             }
         }
-        named_bar(BAR_PREP, kPrepThreads);
-        float Pc[4][4], GC[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const float4 t4 = *reinterpret_cast<const float4 *>(tsum_s + rr * D + c0);
-            Pc[rr][0] = GC[0]; Pc[rr][1] = GC[1]; Pc[rr][2] = GC[2]; Pc[rr][3] = GC[3];
-            GC[0] += t4.x; GC[1] += t4.y; GC[2] += t4.z; GC[3] += t4.w;
-        }
-        // Decay factors, packed as bf16 pairs for the derived operands.
-        uint2 ePp, eCPp, Dnp[4];
-        {
-            float eP[4], eCP[4], Dn[4][4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float PR = (R == 0) ? Pc[0][u] : (R == 1) ? Pc[1][u] : (R == 2) ? Pc[2][u] : Pc[3][u];
-                eP[u] = ex2_approx(PR);
-                eCP[u] = ex2_approx(GC[u] - PR);
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) Dn[rr][u] = (rr >= R) ? ex2_approx(Pc[rr][u] - PR) : 0.f;
-                if (R == 0 && qt == 0) gam_s[buf * D + c0 + u] = ex2_approx(GC[u]);
-            }
-            ePp = pack4(eP[0], eP[1], eP[2], eP[3]);
-            eCPp = pack4(eCP[0], eCP[1], eCP[2], eCP[3]);
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) Dnp[rr] = pack4(Dn[rr][0], Dn[rr][1], Dn[rr][2], Dn[rr][3]);
-        }
-
         // ---------------- operand tiles -----------------------------------
         // Base operands in fp32, rounded once: K e^L, Q e^L, K e^-L (tile anchors).
-        // Derived operands are bf16 x bf16 products of those with the decay
-        // factors: K_R' (x e^{P_R'-P_R}), Q Gamma and K Gamma (x e^{P_R}), K' (x e^{G_C-P_R}).
-        // The operands of MMA (I) are written first; the rest while it runs.
+        // They need only this tile's prefix, so they are built while the tile
+        // sums of the other warps land; the anchored block of this tile
+        // (factor e^0 = 1) is stored with them.  Derived operands are bf16 x
+        // bf16 products with the decay factors: K_R' (x e^{P_R'-P_R}, R' > R)
+        // below, Q Gamma and K Gamma (x e^{P_R}), K' (x e^{G_C-P_R}) while MMA (I) runs.
         const uint32_t a_base = OFF_AINTRA + (uint32_t)kb * 16384u + within;
         const uint32_t kr_base = OFF_KRCAT + (uint32_t)kb * 20480u + within;
         const uint32_t qg_base = OFF_QG + (uint32_t)buf * 16384u + (uint32_t)kb * 8192u + within;
@@ -497,10 +472,43 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
                 krp[i] = pack4(kr[0], kr[1], kr[2], kr[3]);
                 st_u64(sm, a_base + roff, klp[i]);
                 st_u64(sm, a_base + 8192u + roff, qlp[i]);
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-                    if (rr >= R) st_u64(sm, kr_base + (uint32_t)(kr_off(rr) * 128) + roff, bmul4(krp[i], Dnp[rr]));
+                st_u64(sm, kr_base + (uint32_t)(kr_off(R) * 128) + roff, krp[i]);
             }
+        }
+        named_bar(BAR_PREP, kPrepThreads);
+        float Pc[4][4], GC[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(tsum_s + rr * D + c0);
+            Pc[rr][0] = GC[0]; Pc[rr][1] = GC[1]; Pc[rr][2] = GC[2]; Pc[rr][3] = GC[3];
+            GC[0] += t4.x; GC[1] += t4.y; GC[2] += t4.z; GC[3] += t4.w;
+        }
+        // Decay factors, packed as bf16 pairs for the derived operands.
+        uint2 ePp, eCPp, Dnp[4];
+        {
+            float eP[4], eCP[4], Dn[4][4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float PR = (R == 0) ? Pc[0][u] : (R == 1) ? Pc[1][u] : (R == 2) ? Pc[2][u] : Pc[3][u];
+                eP[u] = ex2_approx(PR);
+                eCP[u] = ex2_approx(GC[u] - PR);
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) Dn[rr][u] = (rr > R) ? ex2_approx(Pc[rr][u] - PR) : 0.f;
+                if (R == 0 && qt == 0) gam_s[buf * D + c0 + u] = ex2_approx(GC[u]);
+            }
+            ePp = pack4(eP[0], eP[1], eP[2], eP[3]);
+            eCPp = pack4(eCP[0], eCP[1], eCP[2], eCP[3]);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) Dnp[rr] = pack4(Dn[rr][0], Dn[rr][1], Dn[rr][2], Dn[rr][3]);
+        }
+        // The later tiles' anchored blocks K_R' (R' > R) of this thread's tokens.
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = tq + i;
+            const uint32_t roff = (uint32_t)(t * 128) + ((chunk_c ^ (uint32_t)(t & 7)) << 4);
+#pragma unroll
+            for (int rr = 1; rr < 4; ++rr)
+                if (rr > R) st_u64(sm, kr_base + (uint32_t)(kr_off(rr) * 128) + roff, bmul4(krp[i], Dnp[rr]));
         }
         fence_async_smem();
         named_bar(BAR_PREP, kPrepThreads);
