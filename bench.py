@@ -32,7 +32,7 @@ METRIC = "chunk_kda fwd tokens·heads/s + % bf16 TC peak; kda_step decode HBM GB
 # DRAM bytes (read + write) per launch from ncu captures of the current kernels
 # (profiles/chunk_tc_kernel_gva_b1.md: one B=1 launch, 32 chains, scaled by 4 to
 # the 128 chains of the B=4 launch; profiles/step_kernel_decode_bf16.md).
-CHUNK_TC_TRAFFIC_B4 = 4 * (201.988864e6 + 49.091328e6)
+CHUNK_TC_TRAFFIC_B4 = 4 * (202.115584e6 + 48.679168e6)
 STEP_TRAFFIC = 545.3e6 + 485.3e6
 UNIT = "tokens·heads/s"
 
