@@ -185,3 +185,71 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 4, 1, 16)
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+# --- layer prologue / epilogue entry points ---------------------------------
+def _conv_args(**kw):
+    a = _lib.ConvArgs()
+    a.B, a.T, a.C, a.K, a.head_dim, a.silu, a.l2_eps = 2, 64, 256, 4, 128, 1, 1e-6
+    base = 0x7f0000000000
+    a.x, a.w, a.bias = base + (1 << 20), base + (2 << 20), base + (3 << 20)
+    a.state_in, a.y, a.state_out = base + (4 << 20), base + (5 << 20), base + (6 << 20)
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+def _gate_args(**kw):
+    a = _lib.GateArgs()
+    a.N, a.HV, a.D, a.eps = 64, 4, 128, 1e-6
+    base = 0x7f0000000000
+    a.o, a.gate, a.weight, a.y = base + (1 << 20), base + (2 << 20), base + (3 << 20), base + (4 << 20)
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+def test_layer_null_and_empty():
+    lib = kda.load()
+    assert lib.kda_short_conv(None, None) == INVALID
+    assert lib.kda_output_gate(None, None) == INVALID
+    assert lib.kda_short_conv(ctypes.byref(_conv_args(B=0)), None) == OK
+    assert lib.kda_output_gate(ctypes.byref(_gate_args(N=0)), None) == OK
+
+
+@no_gpu_only
+@pytest.mark.parametrize("field,value,expected", [
+    ("K", 0, INVALID),
+    ("K", 5, INVALID),
+    ("T", -1, INVALID),
+    ("C", 192, UNSUPPORTED),          # not a multiple of 128
+    ("head_dim", 64, UNSUPPORTED),
+    ("w", None, INVALID),
+    ("x", None, INVALID),
+    ("x", 0x7f0000100004, ALIGN),     # 8-byte rows
+    ("state_out", 0x7f0000600002, ALIGN),
+    ("y", 0x7f0000100000, ALIAS),     # y == x
+    ("state_out", 0x7f0000500000, ALIAS),   # state_out == y
+])
+def test_short_conv_validation(field, value, expected):
+    assert kda.load().kda_short_conv(ctypes.byref(_conv_args(**{field: value})), None) == expected
+
+
+@no_gpu_only
+@pytest.mark.parametrize("field,value,expected", [
+    ("D", 64, UNSUPPORTED),
+    ("HV", 0, INVALID),
+    ("N", -1, INVALID),
+    ("gate", None, INVALID),
+    ("o", 0x7f0000100004, ALIGN),
+    ("y", 0x7f0000200000, ALIAS),     # y == gate
+])
+def test_output_gate_validation(field, value, expected):
+    assert kda.load().kda_output_gate(ctypes.byref(_gate_args(**{field: value})), None) == expected
+
+
+@no_gpu_only
+def test_layer_valid_calls_reach_the_launch_without_a_gpu():
+    """Valid arguments pass validation and the launch itself fails without a GPU."""
+    assert kda.load().kda_short_conv(ctypes.byref(_conv_args()), None) == 5      # KDA_ERR_CUDA
+    assert kda.load().kda_output_gate(ctypes.byref(_gate_args()), None) == 5
