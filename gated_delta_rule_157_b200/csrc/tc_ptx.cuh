@@ -1,6 +1,8 @@
 // Thin wrappers over the sm_100a instructions the tensor-core kernel uses:
 // mbarriers, TMEM allocation, tcgen05.mma (BF16 -> FP32, operands in shared
-// memory), tcgen05.commit, tcgen05.ld / tcgen05.st and the proxy fences.
+// memory or TMEM), tcgen05.commit, tcgen05.ld / tcgen05.st, the proxy fences,
+// tensor-map TMA loads (cp.async.bulk.tensor, no multicast) and the warp-level
+// tf32 mma used for the small products of the triangular solve.
 //
 // Shared-memory operand layout used throughout ("K-major, 128-byte swizzle"):
 // a tile of R rows (R % 8 == 0) and K bf16 elements per row is stored as
@@ -17,18 +19,6 @@ namespace tc {
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Byte offset of element (row, k) inside a K-major SW128 tile of `rows` rows.
-__device__ __forceinline__ uint32_t kmaj_off(int row, int k, int rows) {
-    const int kb = k >> 6, kk = k & 63;
-    return (uint32_t)(kb * rows * 128 + row * 128 + ((((kk >> 3) ^ (row & 7))) << 4) + (kk & 7) * 2);
-}
-
-// Byte offset of 16-byte chunk `chunk` (elements 8*chunk..) of `row`.
-__device__ __forceinline__ uint32_t kmaj_chunk_off(int row, int chunk, int rows) {
-    const int kb = chunk >> 3, cc = chunk & 7;
-    return (uint32_t)(kb * rows * 128 + row * 128 + ((cc ^ (row & 7)) << 4));
 }
 
 // Shared-memory matrix descriptor for k-step `s` (16 elements) of a K-major
@@ -149,16 +139,6 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t mbar, uint32_t pa
     return ok != 0;
 }
 
-// Bounded wait: gives up after roughly `limit` polls (with back-off), so a
-// phase that never completes ends the wait instead of hanging the GPU.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint32_t limit) {
-    for (uint32_t i = 0; i < limit; ++i) {
-        if (mbar_try_wait(mbar, parity)) return true;
-        if (i >= 16) __nanosleep(128);
-    }
-    return false;
-}
-
 // TMEM allocation: executed by one full warp.  The address is written to smem.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -263,14 +243,6 @@ __device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
         : "memory");
 }
 
-// Bulk copy global -> shared memory through the tensor-memory-access engine:
-// `bytes` (a multiple of 16) from a 16-byte aligned global address to a
-// 16-byte aligned shared address; completion is counted on `mbar` as bytes.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void *src, uint32_t bytes, uint32_t mbar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst_smem), "l"(src), "r"(bytes), "r"(mbar)
-                 : "memory");
-}
 // Tiled 3-D tensor load (no multicast) of one box into shared memory; `tmap`
 // is the generic address of a CUtensorMap kernel parameter; completion is
 // counted on `mbar` in bytes (out-of-range elements are zero-filled and counted).
