@@ -16,6 +16,8 @@ Contents:
   * ``layer`` -- FP64 NumPy restatements of the layer prologue (short
     convolution, SiLU, per-head L2 norm) and epilogue (per-head RMSNorm and the
     sigmoid output gate).
+  * ``backward`` -- FP64 NumPy reverse-mode gradient of the forward (token by
+    token, in reverse), pinned by finite differences of the C oracle.
 
 Inputs are NumPy arrays (any float dtype; they are widened to float64 exactly).
 """

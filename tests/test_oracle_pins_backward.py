@@ -1,0 +1,121 @@
+"""Pins of the backward oracle (oracle/backward.py).
+
+The gradient is checked against central finite differences of the C forward
+oracle (an independent implementation of the recurrence), and the gradient
+w.r.t. the initial state against the closed form dS0 = M_T^T dS_T, M_T being
+the cumulative transition the C oracle returns (the state recurrence is
+affine in S0: page "Implémenter KDA", the composition test)."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import backward
+
+RNG = np.random.default_rng(2024)
+H_FD = 1e-6
+
+
+def _inputs(B=1, T=6, H=1, HV=2, Dk=4, Dv=3, seed=0):
+    r = np.random.default_rng(seed)
+    return dict(
+        q=r.standard_normal((B, T, H, Dk)), k=r.standard_normal((B, T, H, Dk)),
+        v=r.standard_normal((B, T, HV, Dv)), g=r.standard_normal((B, T, HV, Dk)),
+        beta=r.standard_normal((B, T, HV)), A_log=0.3 * r.standard_normal(HV),
+        dt_bias=0.5 * r.standard_normal((HV, Dk)), S0=r.standard_normal((B, HV, Dk, Dv)),
+    ), r.standard_normal((B, T, HV, Dv)), r.standard_normal((B, HV, Dk, Dv))
+
+
+def _loss(x, do, dS, **sw):
+    f = oracle.kda_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], A_log=x["A_log"],
+                       dt_bias=x["dt_bias"], S0=x["S0"], **sw)
+    return float((f["o"] * do).sum() + (f["S_T"] * dS).sum())
+
+
+def _grads(x, do, dS, **sw):
+    return backward.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], A_log=x["A_log"],
+                                 dt_bias=x["dt_bias"], S0=x["S0"], do=do, dS_T=dS, **sw)
+
+
+SWITCHES = [
+    dict(),
+    dict(scale=0.5, g_min=-3.0),
+    dict(qk_l2norm=False, beta_sigmoid=False, gate_in=False),
+]
+_GRAD_NAME = {"q": "q", "k": "k", "v": "v", "g": "g", "beta": "beta", "S0": "S0",
+              "A_log": "A_log", "dt_bias": "dt_bias"}
+
+
+@pytest.mark.parametrize("sw", SWITCHES, ids=["default", "scaled", "switches_off"])
+def test_directional_derivatives_match_finite_differences(sw):
+    """<grad_X, U> equals (L(X + hU) - L(X - hU)) / 2h for a random U, per input X."""
+    x, do, dS = _inputs(seed=1)
+    if not sw.get("beta_sigmoid", True):
+        x["beta"] = 1.0 / (1.0 + np.exp(-x["beta"]))     # activated betas in (0, 1)
+    if not sw.get("gate_in", True):
+        x["g"] = -np.abs(x["g"])                           # log-decays <= 0
+    gr = _grads(x, do, dS, **sw)
+    names = ["q", "k", "v", "g", "beta", "S0"] + (["A_log", "dt_bias"] if sw.get("gate_in", True) else [])
+    for name in names:
+        U = RNG.standard_normal(x[name].shape)
+        xp = dict(x); xp[name] = x[name] + H_FD * U
+        xm = dict(x); xm[name] = x[name] - H_FD * U
+        fd = (_loss(xp, do, dS, **sw) - _loss(xm, do, dS, **sw)) / (2 * H_FD)
+        an = float((gr[_GRAD_NAME[name]] * U).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, fd, an)
+
+
+def test_elementwise_finite_differences_tiny():
+    """Every entry of every gradient on a 3-token, Dk = Dv = 2 problem."""
+    x, do, dS = _inputs(T=3, HV=1, Dk=2, Dv=2, seed=3)
+    gr = _grads(x, do, dS)
+    for name in ["q", "k", "v", "g", "beta", "S0", "A_log", "dt_bias"]:
+        fd = np.zeros_like(x[name])
+        for idx in np.ndindex(*x[name].shape):
+            xp = dict(x); xp[name] = x[name].copy(); xp[name][idx] += H_FD
+            xm = dict(x); xm[name] = x[name].copy(); xm[name][idx] -= H_FD
+            fd[idx] = (_loss(xp, do, dS) - _loss(xm, do, dS)) / (2 * H_FD)
+        assert np.allclose(gr[name], fd, rtol=1e-6, atol=1e-7), name
+
+
+def test_initial_state_gradient_is_the_transposed_transition():
+    """With do = 0, dS0 = M_T^T dS_T exactly (S_T = M_T S0 + run from zero)."""
+    x, _, dS = _inputs(B=2, T=9, H=2, HV=4, Dk=5, Dv=3, seed=5)
+    do = np.zeros((2, 9, 4, 3))
+    f = oracle.kda_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], A_log=x["A_log"],
+                       dt_bias=x["dt_bias"], S0=x["S0"], want_M=True)
+    gr = _grads(x, do, dS)
+    expect = np.einsum("bhij,bhiv->bhjv", f["M_T"], dS)
+    assert np.allclose(gr["S0"], expect, rtol=1e-12, atol=1e-12)
+
+
+def test_chain_forward_matches_the_c_oracle():
+    """The reverse pass replays its own forward; it must be the C oracle's."""
+    x, _, _ = _inputs(T=7, HV=1, Dk=4, Dv=3, seed=7)
+    f = oracle.kda_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], S0=x["S0"],
+                       qk_l2norm=False, beta_sigmoid=False, gate_in=False)
+    o, S_T, _ = backward.chain_forward(x["q"][0, :, 0], x["k"][0, :, 0], x["v"][0, :, 0],
+                                       x["g"][0, :, 0], x["beta"][0, :, 0], x["S0"][0, 0])
+    assert np.allclose(o, f["o"][0, :, 0], rtol=1e-12, atol=1e-12)
+    assert np.allclose(S_T, f["S_T"][0, 0], rtol=1e-12, atol=1e-12)
+
+
+def test_zero_beta_passes_no_gradient_to_v_and_k_through_the_write():
+    """beta = 0 (activated): the state only decays, so dv = 0 and dk = 0."""
+    x, do, dS = _inputs(seed=9)
+    x["beta"] = np.zeros_like(x["beta"])
+    gr = _grads(x, do, dS, beta_sigmoid=False)
+    assert np.array_equal(gr["v"], np.zeros_like(gr["v"]))
+    assert np.allclose(gr["k"], 0.0, atol=0.0)
+
+
+def test_gva_heads_sum_into_the_shared_qk_gradient():
+    """With HV = 2 H, dq of a q/k head is the sum over the value heads that read it."""
+    x, do, dS = _inputs(HV=2, seed=11)
+    both = _grads(x, do, dS)
+    parts = []
+    for hv in range(2):
+        do1 = do.copy(); do1[:, :, 1 - hv] = 0
+        dS1 = dS.copy(); dS1[:, 1 - hv] = 0
+        parts.append(_grads(x, do1, dS1))
+    assert np.allclose(both["q"], parts[0]["q"] + parts[1]["q"], rtol=1e-12, atol=1e-12)
+    assert np.allclose(both["k"], parts[0]["k"] + parts[1]["k"], rtol=1e-12, atol=1e-12)
