@@ -119,3 +119,21 @@ def test_gva_heads_sum_into_the_shared_qk_gradient():
         parts.append(_grads(x, do1, dS1))
     assert np.allclose(both["q"], parts[0]["q"] + parts[1]["q"], rtol=1e-12, atol=1e-12)
     assert np.allclose(both["k"], parts[0]["k"] + parts[1]["k"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,chunk", [(16, 16), (37, 16), (40, 8), (5, 16)])
+def test_chunk_backward_equals_the_token_backward(T, chunk):
+    """The chunk-parallel reverse pass (the algebra a chunk kernel follows) gives
+    the token-by-token gradient, ragged last chunk included."""
+    from oracle import chunkwise
+    r = np.random.default_rng(T * 31 + chunk)
+    Dk, Dv = 6, 5
+    q = r.standard_normal((T, Dk)); k = r.standard_normal((T, Dk))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = r.standard_normal((T, Dv)); g = -0.3 * np.abs(r.standard_normal((T, Dk)))
+    b = r.uniform(0.1, 0.9, T); S0 = r.standard_normal((Dk, Dv))
+    do = r.standard_normal((T, Dv)); dS = r.standard_normal((Dk, Dv))
+    ref = backward.chain_backward(q, k, v, g, b, S0, do, dS, scale=0.7)
+    got = chunkwise.chunk_backward(q, k, v, g, b, S0, do, dS, chunk=chunk, scale=0.7)
+    for name in ref:
+        assert np.allclose(got[name], ref[name], rtol=1e-9, atol=1e-10), name
