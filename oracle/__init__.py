@@ -18,6 +18,8 @@ Contents:
     sigmoid output gate).
   * ``backward`` -- FP64 NumPy reverse-mode gradient of the forward (token by
     token, in reverse), pinned by finite differences of the C oracle.
+  * ``gates`` -- the decay gates of the family (bounded KDA v2 gate, unbounded
+    softplus v1 gate, per-head Gated DeltaNet gate) as maps z -> log-decay.
 
 Inputs are NumPy arrays (any float dtype; they are widened to float64 exactly).
 """
