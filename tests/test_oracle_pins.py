@@ -5,6 +5,9 @@ formula: they use special cases with closed forms, an independent dense
 restatement (oracle.brute), the chunk-parallel form (oracle.chunkwise), library
 routines (scipy.special.expit, numpy.linalg.norm) and identities.
 """
+import json
+import os
+
 import numpy as np
 import pytest
 from scipy.special import expit
@@ -13,6 +16,8 @@ import oracle
 from oracle import brute, chunkwise
 
 RNG = np.random.default_rng(12345)
+with open(os.path.join(os.path.dirname(__file__), "golden", "composition_tests.json")) as _f:
+    COMPOSITION = json.load(_f)
 
 
 def _chain(T, Dk, Dv, rng, g_lo=-5.0, g_hi=0.0, unit_keys=True):
@@ -162,7 +167,8 @@ def test_kcp_composition_identity():
     S0 = rng.standard_normal((Dk, Dv))
     o_direct, S_direct, M = _run(q, k, v, g, beta, S0=S0, want_M=True)
     _, S_zero, _ = _run(q, k, v, g, beta)
-    assert np.max(np.abs(S_direct - (S_zero + M @ S0))) < 1e-12
+    err = np.max(np.abs(S_direct - (S_zero + M @ S0)))
+    assert err < COMPOSITION["asserted_bound"] and err < 1e-12
     # M is the product of the page's transition matrices, newest on the left.
     Md = np.eye(Dk)
     for t in range(T):
@@ -192,7 +198,8 @@ def test_prefix_scan_over_segments_matches_full_run():
         Ms.append(M_loc)
         Ss.append(S_loc)
     S_in = oracle.kda_compose(np.stack(Ms)[:, None], np.stack(Ss)[:, None], S_init[None])
-    assert np.max(np.abs(S_in[-1, 0] - S_full)) < 1e-12
+    err = np.max(np.abs(S_in[-1, 0] - S_full))
+    assert err < COMPOSITION["asserted_bound"] and err < 1e-12
     # Every intermediate entry is the state at that segment boundary.
     for s in range(1, nseg):
         _, S_b, _ = _run(q[: s * L], k[: s * L], v[: s * L], g[: s * L], beta[: s * L], S0=S_init)

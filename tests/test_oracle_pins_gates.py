@@ -1,5 +1,8 @@
 """Pins of the gate variants (oracle/gates.py) against what the pages print
 and the mathematics fixes, independent of the oracle's own code."""
+import json
+import os
+
 import numpy as np
 import pytest
 from scipy.special import expit
@@ -8,6 +11,8 @@ import oracle
 from oracle import brute, gates
 
 Z = np.linspace(-6.0, 6.0, 24001)
+with open(os.path.join(os.path.dirname(__file__), "golden", "gate_curves_tab3.json")) as f:
+    TAB3 = json.load(f)["printed"]
 
 
 def _alpha_and_slope(gfun):
@@ -31,19 +36,21 @@ def test_tab3_v1_curve():
     """Page "线性注意力交互式演示", Tab 3: v1 alpha falls from ~1.0 at z = -6 to
     ~0 at z = 6; its slope is most negative, ~-0.25, at z ~ 0."""
     a, d = _alpha_and_slope(_v1)
-    assert a[0] > 0.99 and a[-1] < 0.005
+    assert abs(a[0] - TAB3["v1_alpha_at_z_minus6"]) < 0.005
+    assert abs(a[-1] - TAB3["v1_alpha_at_z_plus6"]) < 0.005
     assert np.all(np.diff(a) < 0)
     i = d.argmin()
-    assert abs(d[i] + 0.25) < 0.005 and abs(Z[i]) < 0.05
+    assert abs(d[i] - TAB3["v1_slope_min"]) < 0.005 and abs(Z[i] - TAB3["v1_slope_min_at_z"]) < 0.05
 
 
 def test_tab3_v2_curve_with_floor_001():
     """Tab 3 with the floor alpha = 0.01: v2 flattens onto the floor at z = 6,
     never crosses it, and its slope is most negative, ~-0.29, near z ~ -1.5."""
     a, d = _alpha_and_slope(_v2_floor_001)
-    assert np.all(a > 0.01) and abs(a[-1] - 0.01) < 5e-4
+    floor = TAB3["v2_floor_alpha"]
+    assert np.all(a > floor) and abs(a[-1] - floor) < 5e-4
     i = d.argmin()
-    assert abs(d[i] + 0.29) < 0.01 and -2.0 < Z[i] < -1.4
+    assert abs(d[i] - TAB3["v2_slope_min"]) < 0.01 and abs(Z[i] - TAB3["v2_slope_min_at_z"]) < 0.5
     # v1 goes below the floor, v2 does not (the two separate for z > 0)
     a1, _ = _alpha_and_slope(_v1)
     assert a1[-1] < 0.01 < a[-1]
