@@ -4,6 +4,8 @@ Python binding of the C ABI in include/kda.h.  The entry points keep the
 library's names:
 
   kda_chunk_fwd  chunk-parallel forward over whole sequences (o, S_T, M_T)
+  kda_chunk_bwd  its gradient, from the per-chunk states the forward keeps
+  kda_chunk      the two as a torch.autograd function (o, S_T)
   kda_step       single-token decode, state updated in place
   kda_compose    KCP segment prefix combine
   kcp_chunk_fwd  context-parallel forward across the ranks of a process group
@@ -12,12 +14,13 @@ library's names:
 PyTorch is used for device memory and streams only; every step runs in the
 library's CUDA kernels.
 """
-from ._lib import (ALGOS, EXPORTS, KdaError, kda_chunk_fwd, kda_compose, kda_device_status,
-                   kda_output_gate, kda_short_conv, kda_status_string, kda_step, kda_version,
-                   library_path, load)
+from ._lib import (ALGOS, EXPORTS, KdaError, kda_chunk_bwd, kda_chunk_fwd, kda_compose,
+                   kda_device_status, kda_output_gate, kda_short_conv, kda_status_string, kda_step,
+                   kda_version, library_path, load)
+from .autograd import kda_chunk
 from .kcp import kcp_chunk_fwd
 
-__all__ = ["kda_chunk_fwd", "kda_step", "kda_compose", "kcp_chunk_fwd", "kda_short_conv",
+__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "kda_chunk", "kda_step", "kda_compose", "kcp_chunk_fwd", "kda_short_conv",
            "kda_output_gate", "kda_device_status",
            "kda_status_string", "kda_version", "KdaError", "ALGOS", "EXPORTS",
            "library_path", "load"]

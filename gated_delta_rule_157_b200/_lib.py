@@ -42,6 +42,25 @@ class ChunkArgs(ctypes.Structure):
         ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p),
         ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("S0", ctypes.c_void_p),
         ("o", ctypes.c_void_p), ("S_T", ctypes.c_void_p), ("M_T", ctypes.c_void_p),
+        ("S_chunks", ctypes.c_void_p),
+    ]
+
+
+class ChunkBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("HV", ctypes.c_int),
+        ("Dk", ctypes.c_int), ("Dv", ctypes.c_int), ("chunk", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("algo", ctypes.c_int),
+        ("g_min", ctypes.c_float), ("scale", ctypes.c_float), ("l2_eps", ctypes.c_float),
+        ("qk_l2norm_in_kernel", ctypes.c_int), ("beta_sigmoid_in_kernel", ctypes.c_int),
+        ("gate_in_kernel", ctypes.c_int),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+        ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("S_chunks", ctypes.c_void_p),
+        ("dout", ctypes.c_void_p), ("dS_T", ctypes.c_void_p),
+        ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+        ("dg", ctypes.c_void_p), ("dbeta", ctypes.c_void_p), ("dS0", ctypes.c_void_p),
+        ("dA_log", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p),
     ]
 
 
@@ -76,7 +95,7 @@ class GateArgs(ctypes.Structure):
     ]
 
 
-EXPORTS = ["kda_chunk_fwd", "kda_step", "kda_compose", "kda_device_status",
+EXPORTS = ["kda_chunk_fwd", "kda_chunk_bwd", "kda_step", "kda_compose", "kda_device_status",
            "kda_status_string", "kda_version", "kda_debug_chunk_stall",
            "kda_short_conv", "kda_output_gate"]
 
@@ -98,6 +117,8 @@ def load():
     lib = ctypes.CDLL(path)
     lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(ChunkArgs), ctypes.c_void_p]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_bwd.argtypes = [ctypes.POINTER(ChunkBwdArgs), ctypes.c_void_p]
+    lib.kda_chunk_bwd.restype = ctypes.c_int
     lib.kda_debug_chunk_stall.argtypes = [ctypes.POINTER(ChunkArgs), ctypes.c_void_p]
     lib.kda_debug_chunk_stall.restype = ctypes.c_int
     lib.kda_short_conv.argtypes = [ctypes.POINTER(ConvArgs), ctypes.c_void_p]
@@ -159,7 +180,7 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
                   g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
                   beta_sigmoid_in_kernel=True, gate_in_kernel=True,
                   output_final_state=True, output_transition=False, algo="auto",
-                  o=None, S_T=None, M_T=None, stream=None, _withhold_ready=False):
+                  o=None, S_T=None, M_T=None, S_chunks=None, stream=None, _withhold_ready=False):
     """Chunk-parallel KDA forward.  Returns (o, S_T or None, M_T or None).
 
     (_withhold_ready routes to kda_debug_chunk_stall, the failure-path test hook.)
@@ -167,6 +188,8 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     q, k [B,T,H,Dk]; v [B,T,HV,Dv]; g (log-decay or raw z) [B,T,HV,Dk];
     beta (or logits) [B,T,HV] -- all float32 or all bfloat16, on one CUDA device.
     A_log [HV], dt_bias [HV,Dk], S0 [B,HV,Dk,Dv]: float32.
+    S_chunks: optional float32 [B,HV,ceil(T/chunk),Dk,Dv] that receives the
+    state entering every chunk (the input of kda_chunk_bwd; SIMT kernel only).
     """
     lib = load()
     if not isinstance(q, torch.Tensor) or not q.is_cuda:
@@ -192,6 +215,7 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     if M_T is None and output_transition:
         M_T = torch.empty((B, HV, Dk, Dk), dtype=torch.float32, device=dev)
     _check(M_T, "M_T", (B, HV, Dk, Dk), torch.float32, dev)
+    _check(S_chunks, "S_chunks", (B, HV, -(-T // int(chunk)), Dk, Dv), torch.float32, dev)
     a = ChunkArgs()
     a.B, a.T, a.H, a.HV, a.Dk, a.Dv, a.chunk = B, T, H, HV, Dk, Dv, int(chunk)
     a.dtype, a.algo = _dtype_code(q), ALGOS[algo]
@@ -201,12 +225,66 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     a.gate_in_kernel = int(bool(gate_in_kernel))
     a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
     a.A_log, a.dt_bias, a.S0 = _ptr(A_log), _ptr(dt_bias), _ptr(S0)
-    a.o, a.S_T, a.M_T = _ptr(o), _ptr(S_T), _ptr(M_T)
+    a.o, a.S_T, a.M_T, a.S_chunks = _ptr(o), _ptr(S_T), _ptr(M_T), _ptr(S_chunks)
     if _withhold_ready:
         _raise("kda_debug_chunk_stall", lib.kda_debug_chunk_stall(ctypes.byref(a), _stream(stream, dev)))
     else:
         _raise("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a), _stream(stream, dev)))
     return o, S_T, M_T
+
+
+def kda_chunk_bwd(q, k, v, g, beta, S_chunks, dout, dS_T=None, *, A_log=None, dt_bias=None,
+                  chunk=64, g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
+                  beta_sigmoid_in_kernel=True, gate_in_kernel=True, want_dS0=True, algo="auto",
+                  stream=None):
+    """Gradient of <dout, o> + <dS_T, S_T> for a kda_chunk_fwd call with the
+    same arguments, from the per-chunk states S_chunks that call wrote.
+
+    Returns a dict of float32 tensors: dq, dk [B,T,H,Dk]; dv [B,T,HV,Dv];
+    dg [B,T,HV,Dk] (w.r.t. g, or z with the in-kernel gate); dbeta [B,T,HV]
+    (w.r.t. beta, or its logit); dS0 [B,HV,Dk,Dv] (if want_dS0); dA_log [HV]
+    and ddt_bias [HV,Dk] with the in-kernel gate (ddt_bias only if dt_bias is
+    given).
+    """
+    lib = load()
+    if not isinstance(q, torch.Tensor) or not q.is_cuda:
+        raise ValueError("q must be a CUDA tensor")
+    dev = q.device
+    B, T, H, Dk = q.shape
+    HV, Dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    NC = -(-T // int(chunk))
+    _check(q, "q", (B, T, H, Dk), dt, dev)
+    _check(k, "k", (B, T, H, Dk), dt, dev)
+    _check(v, "v", (B, T, HV, Dv), dt, dev)
+    _check(g, "g", (B, T, HV, Dk), dt, dev)
+    _check(beta, "beta", (B, T, HV), dt, dev)
+    _check(dout, "dout", (B, T, HV, Dv), dt, dev)
+    _check(A_log, "A_log", (HV,), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (HV, Dk), torch.float32, dev)
+    _check(S_chunks, "S_chunks", (B, HV, NC, Dk, Dv), torch.float32, dev)
+    _check(dS_T, "dS_T", (B, HV, Dk, Dv), torch.float32, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dq": torch.empty((B, T, H, Dk), **f32), "dk": torch.empty((B, T, H, Dk), **f32),
+           "dv": torch.empty((B, T, HV, Dv), **f32), "dg": torch.empty((B, T, HV, Dk), **f32),
+           "dbeta": torch.empty((B, T, HV), **f32),
+           "dS0": torch.empty((B, HV, Dk, Dv), **f32) if want_dS0 else None,
+           "dA_log": torch.empty((HV,), **f32) if gate_in_kernel else None,
+           "ddt_bias": torch.empty((HV, Dk), **f32) if (gate_in_kernel and dt_bias is not None) else None}
+    a = ChunkBwdArgs()
+    a.B, a.T, a.H, a.HV, a.Dk, a.Dv, a.chunk = B, T, H, HV, Dk, Dv, int(chunk)
+    a.dtype, a.algo = _dtype_code(q), ALGOS[algo]
+    a.g_min, a.scale, a.l2_eps = float(g_min), float(scale), float(l2_eps)
+    a.qk_l2norm_in_kernel = int(bool(qk_l2norm_in_kernel))
+    a.beta_sigmoid_in_kernel = int(bool(beta_sigmoid_in_kernel))
+    a.gate_in_kernel = int(bool(gate_in_kernel))
+    a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
+    a.A_log, a.dt_bias, a.S_chunks = _ptr(A_log), _ptr(dt_bias), _ptr(S_chunks)
+    a.dout, a.dS_T = _ptr(dout), _ptr(dS_T)
+    for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0", "dA_log", "ddt_bias"):
+        setattr(a, name, _ptr(out[name]))
+    _raise("kda_chunk_bwd", lib.kda_chunk_bwd(ctypes.byref(a), _stream(stream, dev)))
+    return out
 
 
 def kda_step(S, q, k, v, g, beta, *, A_log=None, dt_bias=None, g_min=-5.0, scale=1.0,

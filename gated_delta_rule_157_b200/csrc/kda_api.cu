@@ -53,7 +53,7 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
         for (const void *p : acts)
             if (!aligned(p, es)) return KDA_ERR_ALIGNMENT;
     }
-    const float *fl[] = {a->A_log, a->dt_bias, a->S0, a->S_T, a->M_T};
+    const float *fl[] = {a->A_log, a->dt_bias, a->S0, a->S_T, a->M_T, a->S_chunks};
     for (const float *p : fl)
         if (p && !aligned(p, 4)) return KDA_ERR_ALIGNMENT;
 
@@ -72,11 +72,16 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
     Range r_o = range_of(a->o, ntok ? nv : 0);
     Range r_st = range_of(a->S_T, a->S_T ? ns : 0);
     Range r_mt = range_of(a->M_T, a->M_T ? nm : 0);
+    const size_t nchunks = a->T > 0 ? ((size_t)a->T + a->chunk - 1) / a->chunk : 0;
+    Range r_sc = range_of(a->S_chunks, a->S_chunks ? ns * nchunks : 0);
     for (Range r : r_in) {
-        if (overlaps(r_o, r) || overlaps(r_st, r) || overlaps(r_mt, r)) return KDA_ERR_ALIAS;
+        if (overlaps(r_o, r) || overlaps(r_st, r) || overlaps(r_mt, r) || overlaps(r_sc, r))
+            return KDA_ERR_ALIAS;
     }
     if (overlaps(r_o, r_s0) || overlaps(r_o, r_st) || overlaps(r_o, r_mt) || overlaps(r_st, r_mt) ||
         overlaps(r_mt, r_s0))
+        return KDA_ERR_ALIAS;
+    if (overlaps(r_sc, r_o) || overlaps(r_sc, r_s0) || overlaps(r_sc, r_st) || overlaps(r_sc, r_mt))
         return KDA_ERR_ALIAS;
     if (overlaps(r_st, r_s0) && a->S_T != a->S0) return KDA_ERR_ALIAS;
 
@@ -89,13 +94,14 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
     p.gate_in = a->gate_in_kernel != 0;
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.S0 = a->S0;
-    p.o = a->o; p.S_T = a->S_T; p.M_T = a->M_T;
+    p.o = a->o; p.S_T = a->S_T; p.M_T = a->M_T; p.S_chunks = a->S_chunks;
     p.withhold_ready = withhold_ready ? 1 : 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     if (a->T == 0) return cuda_status(kda::launch_chunk_empty(p, s));
 
-    const bool tc_ok = kda::chunk_tc_supported(p, bf16);
+    // Only the SIMT kernel writes the per-chunk states.
+    const bool tc_ok = kda::chunk_tc_supported(p, bf16) && !a->S_chunks;
     if (withhold_ready && (a->algo != KDA_ALGO_TC || !tc_ok)) return KDA_ERR_UNSUPPORTED;
     if (a->algo == KDA_ALGO_TC) {
         if (!tc_ok) return KDA_ERR_UNSUPPORTED;
@@ -116,6 +122,85 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
 kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) { return chunk_fwd(a, stream, false); }
 
 kda_status kda_debug_chunk_stall(const kda_chunk_args *a, void *stream) { return chunk_fwd(a, stream, true); }
+
+kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARG;
+    if (a->B < 0 || a->T < 0 || a->H < 1 || a->HV < 1 || a->HV % a->H != 0)
+        return KDA_ERR_INVALID_ARG;
+    if (a->Dk < 1 || a->Dv < 1 || a->chunk < 1) return KDA_ERR_INVALID_ARG;
+    if (a->dtype != KDA_DT_F32 && a->dtype != KDA_DT_BF16) return KDA_ERR_INVALID_ARG;
+    if (a->algo != KDA_ALGO_AUTO && a->algo != KDA_ALGO_SIMT && a->algo != KDA_ALGO_TC)
+        return KDA_ERR_INVALID_ARG;
+    if (a->algo == KDA_ALGO_TC) return KDA_ERR_UNSUPPORTED;
+    if (a->Dk > 128 || a->Dv > 128 || a->chunk > 64) return KDA_ERR_UNSUPPORTED;
+    if (!(a->g_min < 0.f) || !(a->l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    if (a->B == 0) return KDA_OK;
+    const bool bf16 = a->dtype == KDA_DT_BF16;
+    const size_t es = bf16 ? 2 : 4;
+    const size_t ntok = (size_t)a->B * a->T;
+    if (ntok > 0) {
+        if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->S_chunks || !a->dout) return KDA_ERR_INVALID_ARG;
+        if (!a->dq || !a->dk || !a->dv || !a->dg || !a->dbeta) return KDA_ERR_INVALID_ARG;
+        if (a->gate_in_kernel && !a->A_log) return KDA_ERR_INVALID_ARG;
+        const void *acts[] = {a->q, a->k, a->v, a->g, a->beta, a->dout};
+        for (const void *p : acts)
+            if (!aligned(p, es)) return KDA_ERR_ALIGNMENT;
+    }
+    const float *fl[] = {a->A_log, a->dt_bias, a->S_chunks, a->dS_T, a->dq, a->dk, a->dv,
+                         a->dg, a->dbeta, a->dS0, a->dA_log, a->ddt_bias};
+    for (const float *p : fl)
+        if (p && !aligned(p, 4)) return KDA_ERR_ALIGNMENT;
+
+    const size_t nq = ntok * a->H * a->Dk, nv = ntok * a->HV * a->Dv;
+    const size_t ng = ntok * a->HV * a->Dk, nb = ntok * a->HV;
+    const size_t ns = (size_t)a->B * a->HV * a->Dk * a->Dv;
+    const size_t nchunks = a->T > 0 ? ((size_t)a->T + a->chunk - 1) / a->chunk : 0;
+    const bool gate = a->gate_in_kernel != 0;
+    Range r_in[] = {range_of(a->q, ntok ? nq * es : 0), range_of(a->k, ntok ? nq * es : 0),
+                    range_of(a->v, ntok ? nv * es : 0), range_of(a->g, ntok ? ng * es : 0),
+                    range_of(a->beta, ntok ? nb * es : 0), range_of(a->dout, ntok ? nv * es : 0),
+                    range_of(a->A_log, a->A_log ? (size_t)a->HV * 4 : 0),
+                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * a->Dk * 4 : 0),
+                    range_of(a->S_chunks, a->S_chunks ? ns * nchunks * 4 : 0),
+                    range_of(a->dS_T, a->dS_T ? ns * 4 : 0)};
+    Range r_out[] = {range_of(a->dq, ntok ? nq * 4 : 0), range_of(a->dk, ntok ? nq * 4 : 0),
+                     range_of(a->dv, ntok ? nv * 4 : 0), range_of(a->dg, ntok ? ng * 4 : 0),
+                     range_of(a->dbeta, ntok ? nb * 4 : 0), range_of(a->dS0, a->dS0 ? ns * 4 : 0),
+                     range_of(gate ? a->dA_log : nullptr, gate && a->dA_log ? (size_t)a->HV * 4 : 0),
+                     range_of(gate ? a->ddt_bias : nullptr, gate && a->ddt_bias ? (size_t)a->HV * a->Dk * 4 : 0)};
+    const int n_out = sizeof(r_out) / sizeof(r_out[0]);
+    for (int i = 0; i < n_out; ++i) {
+        for (Range r : r_in)
+            if (overlaps(r_out[i], r)) return KDA_ERR_ALIAS;
+        for (int j = i + 1; j < n_out; ++j)
+            if (overlaps(r_out[i], r_out[j])) return KDA_ERR_ALIAS;
+    }
+
+    kda::BwdParams p;
+    p.B = a->B; p.T = a->T; p.H = a->H; p.HV = a->HV; p.Dk = a->Dk; p.Dv = a->Dv;
+    p.C = a->chunk; p.group = a->HV / a->H;
+    p.g_min = a->g_min; p.scale = a->scale; p.l2_eps = a->l2_eps;
+    p.l2norm = a->qk_l2norm_in_kernel != 0;
+    p.beta_sigmoid = a->beta_sigmoid_in_kernel != 0;
+    p.gate_in = gate;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+    p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.S_chunks = a->S_chunks;
+    p.dout = a->dout; p.dS_T = a->dS_T;
+    p.dq = a->dq; p.dk = a->dk; p.dv = a->dv; p.dg = a->dg; p.dbeta = a->dbeta; p.dS0 = a->dS0;
+    p.dA_log = gate ? a->dA_log : nullptr;
+    p.ddt_bias = gate ? a->ddt_bias : nullptr;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    // The q/k/g/beta (and parameter) gradients are accumulated with atomics.
+    struct Zero { void *p; size_t bytes; } zeros[] = {
+        {p.dq, ntok ? nq * 4 : 0}, {p.dk, ntok ? nq * 4 : 0}, {p.dg, ntok ? ng * 4 : 0},
+        {p.dbeta, ntok ? nb * 4 : 0}, {p.dA_log, p.dA_log ? (size_t)a->HV * 4 : 0},
+        {p.ddt_bias, p.ddt_bias ? (size_t)a->HV * a->Dk * 4 : 0}};
+    for (const Zero &z : zeros) {
+        if (z.bytes && cudaMemsetAsync(z.p, 0, z.bytes, s) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return cuda_status(kda::launch_chunk_bwd(p, bf16, s));
+}
 
 kda_status kda_step(const kda_step_args *a, void *stream) {
     if (!a) return KDA_ERR_INVALID_ARG;
@@ -246,6 +331,6 @@ const char *kda_status_string(kda_status s) {
     return "KDA_ERR_UNKNOWN";
 }
 
-int kda_version(void) { return 100; }
+int kda_version(void) { return 110; }
 
 }  // extern "C"

@@ -1,0 +1,435 @@
+// FP32 SIMT chunk-parallel KDA backward (CUDA cores only).
+//
+// The gradient of <dO, O> + <dS_T, S_T> through the chunk form of the forward
+// (page "KDA 模块交互式演示" section 1.5, with the decay-weighted UT transform;
+// page "Implémenter KDA", "La forme par blocs"), chunk by chunk in reverse.
+// The pages print no backward; every line below is the derivative of one line
+// of the forward.  Per chunk, with S the state entering it (written by the
+// forward), G the in-chunk cumulative sum of the log-decay and
+// E_c(r, i) = exp(G_rc - G_ic) (r >= i, so every exponential is of a value <= 0):
+//
+//   forward (recomputed)
+//     A[r,i] = sum_c q_rc k_ic E_c(r,i)  (i <= r)    P[r,i] = sum_c k_rc k_ic E_c(r,i)  (i < r)
+//     X = V - (K*exp(G)) S,   U = (I + Diag(beta) P)^-1 Diag(beta) X
+//     O = scale ((Q*exp(G)) S + A U),   S' = Diag(exp(G_last)) S + (K*exp(G_last - G))^T U
+//   reverse, given dO (scaled) and dS' (gradient of the state leaving the chunk)
+//     dU  = A^T dO + (K*exp(G_last - G)) dS'
+//     dZ  = (I + Diag(beta) P)^-T dU                 (back substitution)
+//     dX  = Diag(beta) dZ = dV
+//     dA  = tril(dO U^T),  dP = Diag(beta) tril(-dZ U^T, -1)
+//     dbeta_r = sum_j dZ_rj X_rj + sum_i (-dZ U^T)[r,i] P[r,i]
+//     dS  = (Q*exp(G))^T dO + Diag(exp(G_last)) dS' - (K*exp(G))^T dX
+//   and, per (r, c), the q/k/G gradients of the pairwise sums A and P and of the
+//   elementwise factors exp(G), exp(G_last - G), exp(G_last); dg is the reverse
+//   in-chunk cumulative sum of dG.
+//
+// Parallelisation as the SIMT forward: one CTA per (b, hv, 32-column slice of
+// the value channels).  dV, dS are per column; the q/k/g/beta gradients sum over
+// the columns (and over the value heads of a q/k head), so each CTA adds its
+// share with atomics into zeroed fp32 outputs.  A second pair of kernels takes
+// them through the in-kernel L2 norm, beta sigmoid and bounded gate.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kVT = 32;                       // value columns per CTA
+constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads)
+chunk_bwd_kernel(BwdParams p) {
+    extern __shared__ float smem[];
+    const int C = p.C, Dk = p.Dk, Dv = p.Dv;
+    const int L = Dk | 1;                  // padded row stride of the [C][Dk] tiles
+    float *Qs = smem;                      // [C][L]  q (normalised)
+    float *Ks = Qs + C * L;                // [C][L]  k (normalised)
+    float *Gs = Ks + C * L;                // [C][L]  G, then dG
+    float *Aqk = Gs + C * L;               // [C][C]  A, then dA
+    float *Pkk = Aqk + C * C;              // [C][C]  P, then dP
+    float *Xs = Pkk + C * C;               // [C][kVT] X
+    float *Us = Xs + C * kVT;              // [C][kVT] U
+    float *dOs = Us + C * kVT;             // [C][kVT] scale * dO
+    float *dUs = dOs + C * kVT;            // [C][kVT] dU, then dZ
+    float *Ss = dUs + C * kVT;             // [Dk][kVT] state entering the chunk
+    float *dSs = Ss + Dk * kVT;            // [Dk][kVT] dS of the state leaving, then entering, the chunk
+    float *bet = dSs + Dk * kVT;           // [C]
+    float *dbet = bet + C;                 // [C]
+    float *Glast = dbet + C;               // [Dk]
+    float *dlast = Glast + Dk;             // [Dk]  dG terms of the chunk's last row
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chain = blockIdx.x;
+    const int b = chain / p.HV, hv = chain % p.HV, h = hv / p.group;
+    const int col0 = blockIdx.y * kVT;
+    const int NC = (p.T + C - 1) / C;
+    const Tin *q = static_cast<const Tin *>(p.q);
+    const Tin *k = static_cast<const Tin *>(p.k);
+    const Tin *v = static_cast<const Tin *>(p.v);
+    const Tin *g = static_cast<const Tin *>(p.g);
+    const Tin *bt = static_cast<const Tin *>(p.beta);
+    const Tin *dout = static_cast<const Tin *>(p.dout);
+    const float ea = p.gate_in ? expf(p.A_log[hv]) : 0.f;
+
+    for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
+        const int c = idx / kVT, col = col0 + idx % kVT;
+        dSs[idx] = (p.dS_T && col < Dv) ? p.dS_T[((size_t)chain * Dk + c) * Dv + col] : 0.f;
+    }
+
+    for (int ch = NC - 1; ch >= 0; --ch) {
+        const int t0 = ch * C;
+        const int Cc = min(C, p.T - t0);
+        const size_t tok0 = (size_t)b * p.T + t0;
+        __syncthreads();
+        // ---- 1. load the chunk and the state entering it -------------------
+        for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
+            const int r = idx / Dk, c = idx % Dk;
+            const size_t tok = tok0 + r;
+            Qs[r * L + c] = ld_act(q, (tok * p.H + h) * Dk + c);
+            Ks[r * L + c] = ld_act(k, (tok * p.H + h) * Dk + c);
+            float gz = ld_act(g, (tok * p.HV + hv) * Dk + c);
+            if (p.gate_in) {
+                const float bias = p.dt_bias ? p.dt_bias[(size_t)hv * Dk + c] : 0.f;
+                gz = bounded_gate(gz, bias, ea, p.g_min);
+            }
+            Gs[r * L + c] = gz;
+        }
+        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
+            const int r = idx / kVT, col = col0 + idx % kVT;
+            const size_t tok = tok0 + r;
+            const bool in = col < Dv;
+            Xs[idx] = in ? ld_act(v, (tok * p.HV + hv) * Dv + col) : 0.f;
+            dOs[idx] = in ? p.scale * ld_act(dout, (tok * p.HV + hv) * Dv + col) : 0.f;
+        }
+        for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
+            const int c = idx / kVT, col = col0 + idx % kVT;
+            Ss[idx] = col < Dv ? p.S_chunks[(((size_t)chain * NC + ch) * Dk + c) * Dv + col] : 0.f;
+        }
+        for (int r = tid; r < Cc; r += kThreads) {
+            const float x = ld_act(bt, (tok0 + r) * p.HV + hv);
+            bet[r] = p.beta_sigmoid ? sigmoidf_(x) : x;
+            dbet[r] = 0.f;
+        }
+        __syncthreads();
+        // ---- 2. L2 norms of q, k rows; in-chunk cumulative sum of g ----------
+        if (p.l2norm) {
+            for (int r = warp; r < Cc; r += kThreads / 32) {
+                float sq = 0.f, sk = 0.f;
+                for (int c = lane; c < Dk; c += 32) {
+                    const float a = Qs[r * L + c], bb = Ks[r * L + c];
+                    sq = fmaf(a, a, sq);
+                    sk = fmaf(bb, bb, sk);
+                }
+                for (int off = 16; off > 0; off >>= 1) {
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                }
+                const float rq = rsqrtf(sq + p.l2_eps), rk = rsqrtf(sk + p.l2_eps);
+                for (int c = lane; c < Dk; c += 32) {
+                    Qs[r * L + c] *= rq;
+                    Ks[r * L + c] *= rk;
+                }
+            }
+        }
+        for (int c = tid; c < Dk; c += kThreads) {
+            float run = 0.f;
+            for (int r = 0; r < Cc; ++r) {
+                run += Gs[r * L + c];
+                Gs[r * L + c] = run;
+            }
+            Glast[c] = run;
+        }
+        __syncthreads();
+        // ---- 3. A, P and X = V - (K*exp(G)) S -------------------------------
+        for (int pidx = tid; pidx < Cc * Cc; pidx += kThreads) {
+            const int r = pidx / Cc, i = pidx % Cc;
+            float a = 0.f, pk = 0.f;
+            if (i <= r) {
+                const float *kr = Ks + r * L, *ki = Ks + i * L, *qr = Qs + r * L;
+                const float *gr = Gs + r * L, *gi = Gs + i * L;
+                for (int c = 0; c < Dk; ++c) {
+                    const float kie = ki[c] * expf(gr[c] - gi[c]);
+                    a = fmaf(qr[c], kie, a);
+                    pk = fmaf(kr[c], kie, pk);
+                }
+                if (i == r) pk = 0.f;
+            }
+            Aqk[r * C + i] = a;
+            Pkk[r * C + i] = pk;
+        }
+        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
+            const int r = idx / kVT, jj = idx % kVT;
+            float acc = Xs[idx];
+            const float *kr = Ks + r * L, *gr = Gs + r * L;
+            for (int c = 0; c < Dk; ++c) acc = fmaf(-kr[c] * expf(gr[c]), Ss[c * kVT + jj], acc);
+            Xs[idx] = acc;
+        }
+        __syncthreads();
+        // ---- 4. U = (I + Diag(beta) P)^-1 Diag(beta) X (warp 0); the
+        //         exp(G_last) dS'.S term of the last row's dG (other warps) ----
+        if (warp == 0) {
+            for (int r = 0; r < Cc; ++r) {
+                float acc = Xs[r * kVT + lane];
+                for (int i = 0; i < r; ++i) acc = fmaf(-Pkk[r * C + i], Us[i * kVT + lane], acc);
+                Us[r * kVT + lane] = bet[r] * acc;
+                __syncwarp();
+            }
+        } else {
+            for (int c = tid - 32; c < Dk; c += kThreads - 32) {
+                float acc = 0.f;
+                for (int j = 0; j < kVT; ++j) acc = fmaf(Ss[c * kVT + j], dSs[c * kVT + j], acc);
+                dlast[c] = expf(Glast[c]) * acc;
+            }
+        }
+        __syncthreads();
+        // ---- 5. dU = A^T dO + (K*exp(G_last - G)) dS' ------------------------
+        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
+            const int r = idx / kVT, jj = idx % kVT;
+            float acc = 0.f;
+            for (int rr = r; rr < Cc; ++rr) acc = fmaf(Aqk[rr * C + r], dOs[rr * kVT + jj], acc);
+            const float *kr = Ks + r * L, *gr = Gs + r * L;
+            for (int c = 0; c < Dk; ++c) acc = fmaf(kr[c] * expf(Glast[c] - gr[c]), dSs[c * kVT + jj], acc);
+            dUs[idx] = acc;
+        }
+        __syncthreads();
+        // ---- 6. dZ = (I + Diag(beta) P)^-T dU (warp 0, back substitution) ----
+        if (warp == 0) {
+            for (int r = Cc - 1; r >= 0; --r) {
+                float acc = dUs[r * kVT + lane];
+                for (int rr = r + 1; rr < Cc; ++rr)
+                    acc = fmaf(-bet[rr] * Pkk[rr * C + r], dUs[rr * kVT + lane], acc);
+                dUs[r * kVT + lane] = acc;
+                __syncwarp();
+            }
+        }
+        __syncthreads();
+        // ---- 7. dA, dP, dbeta and dV ------------------------------------------
+        // The column loops start at a lane-dependent offset so that the lanes
+        // of a warp read different shared-memory banks.
+        for (int pidx = tid; pidx < Cc * Cc; pidx += kThreads) {
+            const int r = pidx / Cc, i = pidx % Cc;
+            float da = 0.f, dm = 0.f;
+            if (i <= r) {
+                for (int j0 = 0; j0 < kVT; ++j0) {
+                    const int j = (j0 + lane) & (kVT - 1);
+                    const float u = Us[i * kVT + j];
+                    da = fmaf(dOs[r * kVT + j], u, da);
+                    dm = fmaf(-dUs[r * kVT + j], u, dm);
+                }
+            }
+            if (i < r) {
+                atomicAdd(&dbet[r], dm * Pkk[r * C + i]);
+                Pkk[r * C + i] = bet[r] * dm;
+            } else {
+                Pkk[r * C + i] = 0.f;
+            }
+            Aqk[r * C + i] = da;
+        }
+        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
+            const int r = idx / kVT, col = col0 + idx % kVT;
+            const float dz = dUs[idx];
+            atomicAdd(&dbet[r], dz * Xs[idx]);
+            if (col < Dv) p.dv[((tok0 + r) * p.HV + hv) * Dv + col] = bet[r] * dz;
+        }
+        __syncthreads();
+        // ---- 8. per (r, c): dq, dk (atomics) and dG (registers) --------------
+        float dG[kElemsPerThread];
+#pragma unroll
+        for (int n = 0; n < kElemsPerThread; ++n) {
+            const int idx = tid + n * kThreads;
+            dG[n] = 0.f;
+            if (idx >= Cc * Dk) continue;
+            const int r = idx / Dk, c = idx % Dk;
+            const float qrc = Qs[r * L + c], krc = Ks[r * L + c], grc = Gs[r * L + c];
+            // pairwise sums: row r against earlier tokens, then later tokens against r
+            float aq = 0.f, pr = 0.f;
+            for (int i = 0; i <= r; ++i) {
+                const float kie = Ks[i * L + c] * expf(grc - Gs[i * L + c]);
+                aq = fmaf(Aqk[r * C + i], kie, aq);
+                pr = fmaf(Pkk[r * C + i], kie, pr);
+            }
+            float ak = 0.f, pc = 0.f;
+            for (int rr = r; rr < Cc; ++rr) {
+                const float e = expf(Gs[rr * L + c] - grc);
+                ak = fmaf(Aqk[rr * C + r], Qs[rr * L + c] * e, ak);
+                pc = fmaf(Pkk[rr * C + r], Ks[rr * L + c] * e, pc);
+            }
+            // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T
+            float dqg = 0.f, dkw = 0.f, dkd = 0.f;
+            const float br = bet[r];
+            for (int j0 = 0; j0 < kVT; ++j0) {
+                const int j = (j0 + lane) & (kVT - 1);
+                const float s = Ss[c * kVT + j];
+                dqg = fmaf(dOs[r * kVT + j], s, dqg);
+                dkw = fmaf(-br * dUs[r * kVT + j], s, dkw);
+                dkd = fmaf(Us[r * kVT + j], dSs[c * kVT + j], dkd);
+            }
+            const float eg = expf(grc), ed = expf(Glast[c] - grc);
+            const size_t tq = ((tok0 + r) * p.H + h) * Dk + c;
+            atomicAdd(&p.dq[tq], fmaf(eg, dqg, aq));
+            atomicAdd(&p.dk[tq], ak + pr + pc + eg * dkw + ed * dkd);
+            dG[n] = qrc * aq - krc * ak + krc * pr - krc * pc + eg * (dqg * qrc + dkw * krc) - ed * dkd * krc;
+            atomicAdd(&dlast[c], ed * dkd * krc);
+        }
+        __syncthreads();
+        // ---- 9. dS entering the chunk (in place) -----------------------------
+        for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
+            const int c = idx / kVT, jj = idx % kVT;
+            float acc = expf(Glast[c]) * dSs[idx];
+            for (int r = 0; r < Cc; ++r) {
+                const float e = expf(Gs[r * L + c]);
+                acc = fmaf(e * Qs[r * L + c], dOs[r * kVT + jj], acc);
+                acc = fmaf(-e * Ks[r * L + c] * bet[r], dUs[r * kVT + jj], acc);
+            }
+            dSs[idx] = acc;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int n = 0; n < kElemsPerThread; ++n) {
+            const int idx = tid + n * kThreads;
+            if (idx < Cc * Dk) Gs[(idx / Dk) * L + idx % Dk] = dG[n];
+        }
+        __syncthreads();
+        // ---- 10. dg = reverse cumulative sum of dG; dbeta --------------------
+        for (int c = tid; c < Dk; c += kThreads) {
+            float acc = dlast[c];
+            for (int r = Cc - 1; r >= 0; --r) {
+                acc += Gs[r * L + c];
+                atomicAdd(&p.dg[((tok0 + r) * p.HV + hv) * Dk + c], acc);
+            }
+        }
+        for (int r = tid; r < Cc; r += kThreads) atomicAdd(&p.dbeta[(tok0 + r) * p.HV + hv], dbet[r]);
+    }
+    __syncthreads();
+    if (p.dS0) {
+        for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
+            const int c = idx / kVT, col = col0 + idx % kVT;
+            if (col < Dv) p.dS0[((size_t)chain * Dk + c) * Dv + col] = dSs[idx];
+        }
+    }
+}
+
+// dq, dk through q <- q / sqrt(|q|^2 + eps): warp per (token, head) row.
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads)
+bwd_l2norm_kernel(BwdParams p) {
+    const int lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const long long rows = (long long)p.B * p.T * p.H;
+    if (row >= rows) return;
+    const Tin *xs[2] = {static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k)};
+    float *ds[2] = {p.dq, p.dk};
+    for (int w = 0; w < 2; ++w) {
+        const size_t base = (size_t)row * p.Dk;
+        float xx = 0.f, xy = 0.f;
+        for (int c = lane; c < p.Dk; c += 32) {
+            const float x = ld_act(xs[w], base + c), y = ds[w][base + c];
+            xx = fmaf(x, x, xx);
+            xy = fmaf(x, y, xy);
+        }
+        for (int off = 16; off > 0; off >>= 1) {
+            xx += __shfl_xor_sync(0xffffffffu, xx, off);
+            xy += __shfl_xor_sync(0xffffffffu, xy, off);
+        }
+        const float rn = rsqrtf(xx + p.l2_eps);
+        const float coef = xy * rn * rn * rn;
+        for (int c = lane; c < p.Dk; c += 32) {
+            const float x = ld_act(xs[w], base + c);
+            ds[w][base + c] = fmaf(ds[w][base + c], rn, -x * coef);
+        }
+    }
+}
+
+// dbeta through the sigmoid; dg through the bounded gate, with the sums over
+// tokens of dA_log and ddt_bias.  Block = (value head hv, kGateTokens tokens),
+// thread = key channel.
+constexpr int kGateTokens = 256;
+template <typename Tin>
+__global__ void __launch_bounds__(128)
+bwd_gate_kernel(BwdParams p) {
+    __shared__ float red[4];
+    const int hv = blockIdx.x, c = threadIdx.x;
+    const long long n0 = (long long)blockIdx.y * kGateTokens;
+    const long long ntok = (long long)p.B * p.T;
+    const long long n1 = n0 + kGateTokens < ntok ? n0 + kGateTokens : ntok;
+    const Tin *g = static_cast<const Tin *>(p.g);
+    const Tin *bt = static_cast<const Tin *>(p.beta);
+    if (p.beta_sigmoid) {
+        for (long long n = n0 + c; n < n1; n += blockDim.x) {
+            const size_t i = (size_t)n * p.HV + hv;
+            const float s = sigmoidf_(ld_act(bt, i));
+            p.dbeta[i] *= s * (1.f - s);
+        }
+    }
+    if (!p.gate_in) return;
+    float acc_a = 0.f;
+    if (c < p.Dk) {
+        const float ea = expf(p.A_log[hv]);
+        const float bias = p.dt_bias ? p.dt_bias[(size_t)hv * p.Dk + c] : 0.f;
+        float acc_b = 0.f;
+        for (long long n = n0; n < n1; ++n) {
+            const size_t i = ((size_t)n * p.HV + hv) * p.Dk + c;
+            const float pre = ea * (ld_act(g, i) + bias);
+            const float s = sigmoidf_(pre);
+            const float dpre = p.dg[i] * p.g_min * s * (1.f - s);
+            p.dg[i] = dpre * ea;
+            acc_b = fmaf(dpre, ea, acc_b);
+            acc_a = fmaf(dpre, pre, acc_a);
+        }
+        if (p.ddt_bias) atomicAdd(&p.ddt_bias[(size_t)hv * p.Dk + c], acc_b);
+    }
+    for (int off = 16; off > 0; off >>= 1) acc_a += __shfl_xor_sync(0xffffffffu, acc_a, off);
+    if ((c & 31) == 0) red[c >> 5] = acc_a;
+    __syncthreads();
+    if (c == 0 && p.dA_log) atomicAdd(&p.dA_log[hv], red[0] + red[1] + red[2] + red[3]);
+}
+
+// T == 0: dS0 = dS_T (or 0).
+__global__ void bwd_empty_kernel(BwdParams p) {
+    const size_t n = (size_t)p.B * p.HV * p.Dk * p.Dv;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        p.dS0[i] = p.dS_T ? p.dS_T[i] : 0.f;
+}
+
+}  // namespace
+
+size_t bwd_smem_bytes(int C, int Dk) {
+    const size_t f = (size_t)3 * C * (Dk | 1) + (size_t)2 * C * C + (size_t)4 * C * kVT +
+                     (size_t)2 * Dk * kVT + 2 * C + 2 * Dk;
+    return f * sizeof(float);
+}
+
+template <typename Tin>
+static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s) {
+    const size_t smem = bwd_smem_bytes(p.C, p.Dk);
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.B * p.HV, (p.Dv + kVT - 1) / kVT);
+    chunk_bwd_kernel<Tin><<<grid, kThreads, smem, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.l2norm) {
+        const long long rows = (long long)p.B * p.T * p.H;
+        bwd_l2norm_kernel<Tin><<<(unsigned)((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (p.beta_sigmoid || p.gate_in) {
+        const long long ntok = (long long)p.B * p.T;
+        dim3 g2(p.HV, (unsigned)((ntok + kGateTokens - 1) / kGateTokens));
+        bwd_gate_kernel<Tin><<<g2, 128, 0, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_chunk_bwd(const BwdParams &p, bool bf16, cudaStream_t s) {
+    if (p.T == 0) {
+        if (!p.dS0) return cudaSuccess;
+        bwd_empty_kernel<<<148 * 4, 256, 0, s>>>(p);
+        return cudaGetLastError();
+    }
+    return bf16 ? launch_bwd_t<__nv_bfloat16>(p, s) : launch_bwd_t<float>(p, s);
+}
+
+}  // namespace kda

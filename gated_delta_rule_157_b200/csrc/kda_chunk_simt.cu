@@ -75,6 +75,14 @@ chunk_simt_kernel(ChunkParams p) {
     for (int t0 = 0; t0 < p.T; t0 += C) {
         const int Cc = min(C, p.T - t0);
         __syncthreads();
+        if (p.S_chunks) {
+            // state entering this chunk (state columns only), for the backward
+            const size_t base = ((size_t)chain * ((p.T + C - 1) / C) + t0 / C) * Dk;
+            for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
+                const int c = idx / kVT, col = col0 + idx % kVT;
+                if (col < ncol_state) p.S_chunks[(base + c) * Dv + col] = Ss[idx];
+            }
+        }
         // ---- load and preprocess the chunk --------------------------------
         for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
             int r = idx / Dk, c = idx % Dk;

@@ -36,7 +36,21 @@ struct ChunkParams {
     const float *A_log, *dt_bias, *S0;
     void *o;
     float *S_T, *M_T;
+    float *S_chunks;                 // [B, HV, NC, Dk, Dv]: state entering every chunk, or NULL
     int withhold_ready;              // test hook: the tensor-core kernel's prep warps never hand a chunk over
+};
+
+// Validated arguments of a chunked backward.
+struct BwdParams {
+    int B, T, H, HV, Dk, Dv, C;
+    int group;                       // HV / H
+    float g_min, scale, l2_eps;
+    int l2norm, beta_sigmoid, gate_in;
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias, *S_chunks;
+    const void *dout;
+    const float *dS_T;
+    float *dq, *dk, *dv, *dg, *dbeta, *dS0, *dA_log, *ddt_bias;
 };
 
 struct StepParams {
@@ -71,6 +85,8 @@ cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s);
 bool chunk_tc_supported(const ChunkParams &p, bool bf16);
 cudaError_t launch_chunk_empty(const ChunkParams &p, cudaStream_t s);   // T == 0
+cudaError_t launch_chunk_bwd(const BwdParams &p, bool bf16, cudaStream_t s);
+size_t bwd_smem_bytes(int C, int Dk);
 cudaError_t launch_step(const StepParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s);
 cudaError_t launch_output_gate(const GateParams &p, cudaStream_t s);

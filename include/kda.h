@@ -88,12 +88,17 @@ typedef enum {
  *   S_T     [B, HV, Dk, Dv] fp32 output, or NULL; may be the same buffer as S0
  *           (exactly, not partially overlapping)
  *   M_T     [B, HV, Dk, Dk] fp32 output, or NULL
+ *   S_chunks [B, HV, NC, Dk, Dv] fp32 output, or NULL: the state entering each
+ *           of the NC = ceil(T / chunk) chunks (S_chunks[.., 0, ..] = S0); the
+ *           input kda_chunk_bwd needs.  Only KDA_ALGO_SIMT writes it: with
+ *           S_chunks set, KDA_ALGO_AUTO runs the SIMT kernel and KDA_ALGO_TC
+ *           returns KDA_ERR_UNSUPPORTED.
  *
  * Limits: B, T >= 0; 1 <= H <= HV, HV % H == 0; 1 <= Dk, Dv <= 128;
  * 1 <= chunk <= 64.  q, k, v, g, beta, o must be aligned to their element size;
  * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64 and
- * 16-byte aligned q, k, v, g, o.  o must not overlap any input; S_T and M_T
- * must not overlap each other, o, or any input except S_T == S0.
+ * 16-byte aligned q, k, v, g, o.  o must not overlap any input; S_T, M_T and
+ * S_chunks must not overlap each other, o, or any input except S_T == S0.
  * T == 0 writes S_T = S0 (or 0) and M_T = I.
  */
 typedef struct {
@@ -110,9 +115,59 @@ typedef struct {
     void *o;
     float *S_T;
     float *M_T;
+    float *S_chunks;
 } kda_chunk_args;
 
 kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
+
+/*
+ * kda_chunk_bwd -- gradient of the chunk forward.
+ *
+ * For the loss <dout, o> + <dS_T, S_T> of a kda_chunk_fwd call with the same
+ * arguments, writes the gradients with respect to every input: q, k, v, g
+ * (the raw gate input z when gate_in_kernel), beta (its logit when
+ * beta_sigmoid_in_kernel), the initial state, and A_log, dt_bias when the gate
+ * runs in the kernel.  The pages print no backward; this is the exact
+ * derivative of the forward's chunk form (page "KDA 模块交互式演示" section 1.5
+ * with the decay-weighted UT transform), chunk by chunk in reverse, through
+ * the three in-kernel switches, computed in FP32 on the CUDA cores.
+ *
+ * Inputs: q, k, v, g, beta, A_log, dt_bias and the switches exactly as given
+ * to the forward; S_chunks as the forward wrote it with the same `chunk`
+ * (the forward's S0 is S_chunks[.., 0, ..]); dout [B, T, HV, Dv] dtype;
+ * dS_T [B, HV, Dk, Dv] fp32 or NULL (zeros).
+ * Outputs (fp32, every element written): dq, dk [B, T, H, Dk] (summed over
+ * the value heads that share a q/k head); dv [B, T, HV, Dv]; dg [B, T, HV, Dk];
+ * dbeta [B, T, HV]; dS0 [B, HV, Dk, Dv] or NULL; dA_log [HV] and ddt_bias
+ * [HV, Dk] when gate_in_kernel (else not touched; either may be NULL).
+ *
+ * Limits as kda_chunk_fwd (1 <= Dk, Dv <= 128, 1 <= chunk <= 64); algo must be
+ * KDA_ALGO_AUTO or KDA_ALGO_SIMT.  Activation pointers aligned to their
+ * element size, fp32 pointers to 4 bytes.  No output may overlap an input or
+ * another output.  The q/k/g/beta gradients are sums of fp32 atomic adds, so
+ * their last bits depend on the order the CTAs run in.
+ */
+typedef struct {
+    int B, T, H, HV, Dk, Dv, chunk;
+    int dtype;                 /* kda_dtype of q, k, v, g, beta and dout */
+    int algo;                  /* KDA_ALGO_AUTO or KDA_ALGO_SIMT */
+    float g_min, scale, l2_eps;
+    int qk_l2norm_in_kernel, beta_sigmoid_in_kernel, gate_in_kernel;
+    const void *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias;
+    const float *S_chunks;     /* [B, HV, NC, Dk, Dv] fp32, NC = ceil(T / chunk) */
+    const void *dout;          /* [B, T, HV, Dv] */
+    const float *dS_T;         /* [B, HV, Dk, Dv] or NULL */
+    float *dq, *dk;            /* [B, T, H, Dk] */
+    float *dv;                 /* [B, T, HV, Dv] */
+    float *dg;                 /* [B, T, HV, Dk] */
+    float *dbeta;              /* [B, T, HV] */
+    float *dS0;                /* [B, HV, Dk, Dv] or NULL */
+    float *dA_log;             /* [HV] or NULL */
+    float *ddt_bias;           /* [HV, Dk] or NULL */
+} kda_chunk_bwd_args;
+
+kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);
 
 /*
  * kda_step -- one decode token for B*HV independent chains against a resident

@@ -1,0 +1,143 @@
+"""Host emulation of the library's SIMT chunk kernels -- TEST INFRASTRUCTURE.
+
+Compiles the CUDA sources of the SIMT forward (kda_chunk_simt.cu) and of the
+backward (kda_chunk_bwd.cu) as host C++ with g++ and AddressSanitizer: the
+stand-in headers in fakeinc/ map the CUDA keywords and intrinsics the kernels
+use onto C++, emu_rt.cpp runs every CUDA thread of a block as a std::thread
+(__syncthreads and __syncwarp are std::barriers, a thread that returns drops
+out of them as an exited GPU thread does), and the dynamic shared memory is an
+array whose bytes past the launch's size are poisoned.  A kernel that reads or
+writes outside its buffers, global or shared, stops with an AddressSanitizer
+report.  Only the kernels are compiled: the source is cut before its host
+launchers.  The library never uses any of this; the GPU tests are the parity
+tests proper.
+"""
+import os
+import re
+import subprocess
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(os.path.dirname(HERE))
+CSRC = os.path.join(ROOT, "gated_delta_rule_157_b200", "csrc")
+OUT = os.path.join(HERE, "_build")
+LIB = os.path.join(OUT, "libkda_host_emu.so")
+SMEM_FLOATS = 65536
+
+# extern "C" runners appended to each unit: the grid and block of the
+# library's launchers, with the shared-memory bytes poisoned past the size the
+# kernel asks for.
+_POISON = r'''
+#include <sanitizer/asan_interface.h>
+namespace kda { namespace {
+void emu_poison(size_t used) {
+    ASAN_UNPOISON_MEMORY_REGION(smem, sizeof(smem));
+    ASAN_POISON_MEMORY_REGION(reinterpret_cast<char *>(smem) + used, sizeof(smem) - used);
+}
+} }
+'''
+_RUN_FWD = _POISON + r'''
+extern "C" int emu_sizeof_chunk_params(void) { return (int)sizeof(kda::ChunkParams); }
+extern "C" int emu_offsetof_withhold_ready(void) { return (int)offsetof(kda::ChunkParams, withhold_ready); }
+extern "C" int emu_chunk_fwd(kda::ChunkParams *pp, int bf16) {
+    using namespace kda;
+    const ChunkParams p = *pp;
+    const int ncol = p.Dv + (p.M_T ? p.Dk : 0);
+    const size_t bytes = simt_smem_bytes(p.C, p.Dk);
+    if (bytes > sizeof(smem)) return 1;
+    emu_poison(bytes);
+    const dim3 grid(p.B * p.HV, (ncol + kVT - 1) / kVT);
+    if (bf16) emu_launch(grid, dim3(kThreads), [&] { chunk_simt_kernel<__nv_bfloat16>(p); });
+    else emu_launch(grid, dim3(kThreads), [&] { chunk_simt_kernel<float>(p); });
+    return 0;
+}
+'''
+_RUN_BWD = _POISON + r'''
+extern "C" int emu_sizeof_bwd_params(void) { return (int)sizeof(kda::BwdParams); }
+extern "C" int emu_offsetof_ddt_bias(void) { return (int)offsetof(kda::BwdParams, ddt_bias); }
+template <typename Tin>
+static void run_bwd(const kda::BwdParams &p) {
+    using namespace kda;
+    emu_launch(dim3(p.B * p.HV, (p.Dv + kVT - 1) / kVT), dim3(kThreads), [&] { chunk_bwd_kernel<Tin>(p); });
+    emu_poison(0);
+    if (p.l2norm) {
+        const long long rows = (long long)p.B * p.T * p.H;
+        emu_launch(dim3((unsigned)((rows + kThreads / 32 - 1) / (kThreads / 32))), dim3(kThreads),
+                   [&] { bwd_l2norm_kernel<Tin>(p); });
+    }
+    if (p.beta_sigmoid || p.gate_in) {
+        const long long ntok = (long long)p.B * p.T;
+        emu_launch(dim3(p.HV, (unsigned)((ntok + kGateTokens - 1) / kGateTokens)), dim3(128),
+                   [&] { bwd_gate_kernel<Tin>(p); });
+    }
+}
+// The outputs the library zeroes before these kernels must arrive zeroed.
+extern "C" int emu_chunk_bwd(kda::BwdParams *pp, int bf16) {
+    using namespace kda;
+    const BwdParams p = *pp;
+    const size_t bytes = bwd_smem_bytes(p.C, p.Dk);
+    if (bytes > sizeof(smem)) return 1;
+    emu_poison(bytes);
+    if (p.T == 0) {
+        emu_poison(0);
+        emu_launch(dim3(2), dim3(64), [&] { bwd_empty_kernel(p); });
+        return 0;
+    }
+    if (bf16) run_bwd<__nv_bfloat16>(p);
+    else run_bwd<float>(p);
+    return 0;
+}
+'''
+
+
+def _unit(src_name, runner):
+    s = open(os.path.join(CSRC, src_name)).read()
+    m = re.search(r"^(template <typename Tin>\nstatic )?cudaError_t launch_", s, re.M)
+    if not m:
+        raise RuntimeError("no host launcher found in " + src_name)
+    s = s[: m.start()] + "\n}  // namespace kda\n"
+    # static __shared__ arrays are block-wide: function statics (the blocks of
+    # a grid run one after another); the dynamic one is the array declared below
+    s = s.replace("extern __shared__", "extern").replace("__shared__", "static")
+    head = ('#include <functional>\n#include "cuda_runtime.h"\n'
+            "void emu_launch(dim3 grid, dim3 block, const std::function<void()> &fn);\n"
+            "namespace kda { namespace { alignas(16) float smem[%d]; } }\n" % SMEM_FLOATS)
+    return head + "#line 1 \"%s\"\n" % src_name + s + runner
+
+
+def _deps():
+    return [os.path.join(CSRC, f) for f in ("kda_chunk_simt.cu", "kda_chunk_bwd.cu", "kda_internal.cuh")] + \
+        [os.path.join(HERE, f) for f in ("emu_build.py", "emu_rt.cpp", "fakeinc/cuda_runtime.h", "fakeinc/cuda_bf16.h")] + \
+        [os.path.join(ROOT, "include", "kda.h")]
+
+
+def asan_runtime():
+    return subprocess.run(["g++", "-print-file-name=libasan.so"], check=True, capture_output=True,
+                          text=True).stdout.strip()
+
+
+def build(force=False):
+    """Compile libkda_host_emu.so (skipped when newer than its sources)."""
+    if not force and os.path.exists(LIB) and all(os.path.getmtime(d) <= os.path.getmtime(LIB) for d in _deps()):
+        return LIB
+    os.makedirs(OUT, exist_ok=True)
+    units = {"emu_fwd.cpp": _unit("kda_chunk_simt.cu", _RUN_FWD),
+             "emu_bwd.cpp": _unit("kda_chunk_bwd.cu", _RUN_BWD)}
+    objs = []
+    flags = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address", "-fno-omit-frame-pointer", "-fPIC",
+             "-I", os.path.join(HERE, "fakeinc"), "-I", CSRC, "-Wno-unknown-pragmas", "-c"]
+    for name, text in units.items():
+        path = os.path.join(OUT, name)
+        with open(path, "w") as f:
+            f.write(text)
+        objs.append(path[:-4] + ".o")
+        subprocess.run(flags + [path, "-o", objs[-1]], check=True)
+    objs.append(os.path.join(OUT, "emu_rt.o"))
+    subprocess.run(flags + [os.path.join(HERE, "emu_rt.cpp"), "-o", objs[-1]], check=True)
+    tmp = LIB + ".tmp.%d" % os.getpid()
+    subprocess.run(["g++", "-shared", "-fsanitize=address", "-o", tmp, *objs, "-pthread"], check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force=True))

@@ -1,0 +1,35 @@
+// Host stand-in for the CUDA runtime header: just enough for kernel source to
+// compile as C++ and run one CUDA thread per std::thread (see emu_rt.cpp).
+#pragma once
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+#define __global__
+#define __device__
+#define __host__
+#define __forceinline__ inline
+#define __launch_bounds__(...)
+#define __shared__
+#define __grid_constant__
+typedef int cudaError_t;
+typedef void *cudaStream_t;
+enum { cudaSuccess = 0 };
+struct uint3 { unsigned x, y, z; };
+struct dim3 {
+    unsigned x, y, z;
+    dim3(unsigned a = 1, unsigned b = 1, unsigned c = 1) : x(a), y(b), z(c) {}
+};
+extern thread_local uint3 threadIdx, blockIdx;
+extern thread_local dim3 blockDim, gridDim;
+void __syncthreads();
+void __syncwarp(unsigned mask = 0xffffffffu);
+float __shfl_xor_sync(unsigned mask, float v, int off);
+inline float atomicAdd(float *a, float v) { return std::atomic_ref<float>(*a).fetch_add(v); }
+inline float rsqrtf(float x) { return 1.0f / std::sqrt(x); }
+inline float __expf(float x) { return std::exp(x); }
+inline float __fdividef(float a, float b) { return a / b; }
+using std::max;
+using std::min;

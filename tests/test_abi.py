@@ -253,3 +253,103 @@ def test_layer_valid_calls_reach_the_launch_without_a_gpu():
     """Valid arguments pass validation and the launch itself fails without a GPU."""
     assert kda.load().kda_short_conv(ctypes.byref(_conv_args()), None) == 5      # KDA_ERR_CUDA
     assert kda.load().kda_output_gate(ctypes.byref(_gate_args()), None) == 5
+
+
+# --- struct layouts: ctypes mirrors against the C header ---------------------
+_STRUCTS = {"kda_chunk_args": _lib.ChunkArgs, "kda_chunk_bwd_args": _lib.ChunkBwdArgs,
+            "kda_step_args": _lib.StepArgs, "kda_conv_args": _lib.ConvArgs,
+            "kda_gate_args": _lib.GateArgs}
+
+
+def test_ctypes_structs_match_the_header(tmp_path):
+    """Every field of every argument struct sits at the offset the C compiler
+    gives it, and the sizes agree (a mismatch would make the library read a
+    pointer from the wrong place)."""
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "kda.h"', "int main(void) {"]
+    for cname, py in _STRUCTS.items():
+        lines.append('printf("%s sizeof %%zu\\n", sizeof(%s));' % (cname, cname))
+        for fname, _ in py._fields_:
+            lines.append('printf("%s %s %%zu\\n", offsetof(%s, %s));' % (cname, fname, cname, fname))
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for cname, py in _STRUCTS.items():
+        assert got[(cname, "sizeof")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+# --- chunk states (forward output) and the backward entry point --------------
+@no_gpu_only
+def test_chunk_states_validation():
+    a = _chunk_args()
+    sc = 0x7f0000000000 + (12 << 20)
+    assert _fwd(_chunk_args(S_chunks=sc + 2)) == ALIGN
+    assert _fwd(_chunk_args(S_chunks=a.q)) == ALIAS
+    assert _fwd(_chunk_args(S_chunks=a.o + 4)) == ALIAS
+    assert _fwd(_chunk_args(S_chunks=a.S0)) == ALIAS
+    # only the SIMT kernel writes them
+    assert _fwd(_chunk_args(S_chunks=sc, algo=2)) == UNSUPPORTED
+
+
+def _bwd_args(**kw):
+    a = _lib.ChunkBwdArgs()
+    a.B, a.T, a.H, a.HV, a.Dk, a.Dv, a.chunk = 1, 64, 2, 4, 16, 16, 16
+    a.dtype, a.algo = 0, 0
+    a.g_min, a.scale, a.l2_eps = -5.0, 1.0, 1e-6
+    a.qk_l2norm_in_kernel = a.beta_sigmoid_in_kernel = a.gate_in_kernel = 1
+    base = 0x7f3000000000
+    names = ["q", "k", "v", "g", "beta", "A_log", "dt_bias", "S_chunks", "dout", "dS_T",
+             "dq", "dk", "dv", "dg", "dbeta", "dS0", "dA_log", "ddt_bias"]
+    for i, name in enumerate(names):
+        setattr(a, name, base + (i + 1) * (1 << 20))
+    for key, val in kw.items():
+        setattr(a, key, val)
+    return a
+
+
+def _bwd(a):
+    return kda.load().kda_chunk_bwd(ctypes.byref(a), None)
+
+
+def test_bwd_null_and_empty():
+    assert kda.load().kda_chunk_bwd(None, None) == INVALID
+    assert _bwd(_bwd_args(B=0)) == OK
+
+
+@no_gpu_only
+@pytest.mark.parametrize("field,value,expected", [
+    ("H", 3, INVALID),
+    ("Dk", 129, UNSUPPORTED),
+    ("chunk", 65, UNSUPPORTED),
+    ("chunk", 0, INVALID),
+    ("algo", 2, UNSUPPORTED),        # no tensor-core backward
+    ("algo", 7, INVALID),
+    ("dtype", 3, INVALID),
+    ("g_min", 1.0, INVALID),
+    ("S_chunks", None, INVALID),
+    ("dout", None, INVALID),
+    ("dq", None, INVALID),
+    ("A_log", None, INVALID),        # gate_in_kernel needs A_log
+    ("q", 0x7f3000100002, ALIGN),
+    ("dS0", 0x7f3001000001, ALIGN),
+    ("dq", 0x7f3000100000, ALIAS),   # dq over q
+    ("dv", 0x7f3000c00000, ALIAS),   # dv over dk
+    ("dS0", 0x7f3000a00000, ALIAS),  # dS0 over dS_T
+])
+def test_bwd_validation(field, value, expected):
+    assert _bwd(_bwd_args(**{field: value})) == expected
+
+
+@no_gpu_only
+def test_bwd_valid_request_without_gpu_reports_cuda_error():
+    assert _bwd(_bwd_args()) == 5
+    # the parameter gradients are not outputs without the in-kernel gate
+    assert _bwd(_bwd_args(gate_in_kernel=0, A_log=None, dA_log=0x7f3000100000)) == 5
