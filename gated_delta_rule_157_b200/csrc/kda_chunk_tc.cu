@@ -394,7 +394,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             for (int u = 0; u < 4; ++u) {
                 float g;
                 if (p.gate_in) g = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(zz[u], A1, B1[u])));
-                else g = zz[u] * kLog2e;
+                else g = fmaxf(zz[u] * kLog2e, gmin2);   // the exponent bound needs g >= g_min
                 g2[i][u] = (tq + i < Cc) ? g : 0.f;
             }
         }

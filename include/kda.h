@@ -79,7 +79,11 @@ typedef enum {
  * Layouts (element type `dtype` unless stated):
  *   q, k    [B, T, H,  Dk]
  *   v       [B, T, HV, Dv]
- *   g       [B, T, HV, Dk]  log-decay g, or the raw gate input z when gate_in_kernel
+ *   g       [B, T, HV, Dk]  log-decay g, or the raw gate input z when gate_in_kernel;
+ *           a log-decay given directly should lie in [g_min, 0]: the SIMT
+ *           kernel takes any value, the tensor-core kernel (whose exponent
+ *           bound, 16 |g_min| per 16-token tile, rests on it) clamps values
+ *           below g_min up to g_min
  *   beta    [B, T, HV]      write strength, or its logit when beta_sigmoid_in_kernel
  *   A_log   [HV]      fp32  read iff gate_in_kernel (must then be non-NULL)
  *   dt_bias [HV, Dk]  fp32  read iff gate_in_kernel; NULL means 0

@@ -189,6 +189,23 @@ def test_tc_switches_off(cuda_device):
     check(o, S_T, M_T, ref, "bf16", "tc")
 
 
+def test_log_decay_below_g_min(cuda_device):
+    """A log-decay given directly below g_min: the SIMT kernel uses it as is;
+    the tensor-core kernel clamps it to g_min (its exponent bound rests on
+    g >= g_min), so it matches the oracle run on the clamped values."""
+    w = workloads.Workload("tclow", B=1, T=130, H=1, HV=2, Dk=128, Dv=128, chunk=64, dtype="bf16",
+                           seed=42, s0_std=0.05)
+    inp = workloads.activated_inputs(w, g_min=-9.0)
+    assert float(inp["g"].float().min()) < -8.0
+    d = to_device(inp, cuda_device)
+    o, S_T, _ = run_gpu(d, w, "simt", flags=False)
+    check(o, S_T, None, oracle_chunk(inp, flags=False), "bf16", "simt")
+    clamped = dict(inp, g=inp["g"].float().clamp(min=-5.0).to(inp["g"].dtype))
+    o, S_T, _ = run_gpu(d, w, "tc", flags=False)
+    assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(S_T).all())
+    check(o, S_T, None, oracle_chunk(clamped, flags=False), "bf16", "tc")
+
+
 def test_tc_is_the_default_for_its_shape(cuda_device):
     """algo='auto' picks the tensor-core kernel for bf16 / 128 / chunk 64: its
     result equals the explicit 'tc' call bit for bit."""
