@@ -19,8 +19,10 @@ reverse order, for one chain at a time:
       dS    = Diag(alpha) dP
 
 and through the switches: q^ = q / sqrt(|q|^2 + eps) (same for k), beta =
-sigmoid(logit), g = g_min sigmoid(a (z + dt_bias)) with a = exp(A_log).  It is
-pinned by central finite differences of the forward (tests), not by itself.
+sigmoid(logit), and the gate, g = g_min sigmoid(a (z + dt_bias)) (bounded) or
+g = -a softplus(z + dt_bias) (softplus) with a = exp(A_log), per key channel or
+one per (token, head).  It is pinned by central finite differences of the
+forward (tests), not by itself.
 """
 import numpy as np
 
@@ -79,13 +81,23 @@ def chain_backward(q, k, v, g, beta, S0, do, dS_T, scale=1.0):
     return {"q": dq, "k": dk, "v": dv, "g": dg, "beta": dbeta, "S0": dS}
 
 
+def _softplus(x):
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
 def kda_backward(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, do=None, dS_T=None,
-                 g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm=True, beta_sigmoid=True, gate_in=True):
+                 g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm=True, beta_sigmoid=True, gate_in=True,
+                 gate="bounded", per_head=False):
     """Gradients of <do, o> + <dS_T, S_T> for the layouts of the forward
     (q, k [B,T,H,Dk]; v [B,T,HV,Dv]; g or raw z [B,T,HV,Dk]; beta or logits
     [B,T,HV]; A_log [HV]; dt_bias [HV,Dk]; S0 [B,HV,Dk,Dv]).  Returns a dict
     with dq, dk, dv, dg (w.r.t. the g / z input), dbeta (w.r.t. the beta /
-    logit input), dS0, and dA_log, ddt_bias when the gate runs in-kernel."""
+    logit input), dS0, and dA_log, ddt_bias when the gate runs in-kernel.
+
+    gate: the in-kernel gate, "bounded" (g = g_min sigmoid(exp(A_log)(z + dt_bias)))
+    or "softplus" (g = -exp(A_log) softplus(z + dt_bias)).  per_head: g / z is
+    [B,T,HV] and dt_bias [HV], one decay per (token, value head) shared by the
+    key channels (the gradient w.r.t. it sums over the channels)."""
     q, k, v, g, beta = (np.asarray(a, dtype=np.float64) for a in (q, k, v, g, beta))
     B, T, H, Dk = q.shape
     HV, Dv = v.shape[2], v.shape[3]
@@ -94,22 +106,31 @@ def kda_backward(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, do=None
     dS_T = np.zeros((B, HV, Dk, Dv)) if dS_T is None else np.asarray(dS_T, dtype=np.float64)
     S0 = np.zeros((B, HV, Dk, Dv)) if S0 is None else np.asarray(S0, dtype=np.float64)
     A_log = np.zeros(HV) if A_log is None else np.asarray(A_log, dtype=np.float64)
-    dt_bias = np.zeros((HV, Dk)) if dt_bias is None else np.asarray(dt_bias, dtype=np.float64)
+    bshape = (HV,) if per_head else (HV, Dk)
+    dt_bias = np.zeros(bshape) if dt_bias is None else np.asarray(dt_bias, dtype=np.float64)
+    zc = g[..., None] if per_head else g                     # [B,T,HV,1 or Dk]
+    bc = dt_bias[:, None] if per_head else dt_bias           # [HV,1 or Dk]
 
     qh, nq = _l2(q, l2_eps) if qk_l2norm else (q, None)
     kh, nk = _l2(k, l2_eps) if qk_l2norm else (k, None)
     bt = _sig(beta) if beta_sigmoid else beta
-    if gate_in:
-        a = np.exp(A_log)[None, None, :, None]
-        pre = a * (g + dt_bias[None, None])
+    a = np.exp(A_log)[None, None, :, None]
+    if gate_in and gate == "bounded":
+        pre = a * (zc + bc[None, None])
         sg = _sig(pre)
         gg = g_min * sg
+    elif gate_in and gate == "softplus":
+        pre = zc + bc[None, None]
+        gg = -a * _softplus(pre)
+    elif gate_in:
+        raise ValueError("gate must be 'bounded' or 'softplus'")
     else:
-        gg = g
+        gg = zc
+    gg = np.broadcast_to(gg, (B, T, HV, Dk))
     out = {n: np.zeros_like(x) for n, x in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta))}
     out["S0"] = np.zeros_like(S0)
     dqh, dkh = np.zeros_like(qh), np.zeros_like(kh)
-    dgg = np.zeros_like(gg)
+    dgg = np.zeros((B, T, HV, Dk))
     dbt = np.zeros_like(bt)
     for b in range(B):
         for hv in range(HV):
@@ -125,11 +146,18 @@ def kda_backward(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, do=None
     out["q"] = _l2_back(q, nq, dqh) if qk_l2norm else dqh
     out["k"] = _l2_back(k, nk, dkh) if qk_l2norm else dkh
     out["beta"] = dbt * bt * (1 - bt) if beta_sigmoid else dbt
-    if gate_in:
+    if per_head:
+        dgg = dgg.sum(axis=3, keepdims=True)                 # the decay is shared by the channels
+    if gate_in and gate == "bounded":
         dpre = dgg * g_min * sg * (1 - sg)
-        out["g"] = dpre * a
-        out["dt_bias"] = (dpre * a).sum(axis=(0, 1))
-        out["A_log"] = (dpre * pre).sum(axis=(0, 1, 3))   # d pre / d A_log = pre (a = exp(A_log))
+        dz = dpre * a
+        out["A_log"] = (dpre * pre).sum(axis=(0, 1, 3))     # d pre / d A_log = pre (a = exp(A_log))
+    elif gate_in:
+        dz = -dgg * a * _sig(pre)                           # d softplus = sigmoid
+        out["A_log"] = (dgg * gg[..., :dgg.shape[3]]).sum(axis=(0, 1, 3))   # g is linear in exp(A_log)
     else:
-        out["g"] = dgg
+        dz = dgg
+    if gate_in:
+        out["dt_bias"] = dz.sum(axis=(0, 1))[:, 0] if per_head else dz.sum(axis=(0, 1))
+    out["g"] = dz[..., 0] if per_head else dz
     return out

@@ -137,3 +137,42 @@ def test_chunk_backward_equals_the_token_backward(T, chunk):
     got = chunkwise.chunk_backward(q, k, v, g, b, S0, do, dS, chunk=chunk, scale=0.7)
     for name in ref:
         assert np.allclose(got[name], ref[name], rtol=1e-9, atol=1e-10), name
+
+
+def _loss_variant(x, do, dS, gate, per_head):
+    """Forward through the gate variants of oracle/gates.py, then the C oracle
+    with its own gate switched off."""
+    from oracle import gates
+    Dk = x["q"].shape[-1]
+    if per_head:
+        z = x["z"][..., None]
+        bias = x["dt_bias"][:, None]
+    else:
+        z, bias = x["z"], x["dt_bias"]
+    if gate == "bounded":
+        g = gates.bounded_gate(z, x["A_log"], bias)
+    else:
+        g = gates.softplus_gate(z, x["A_log"], bias)
+    g = np.broadcast_to(g, z.shape[:-1] + (Dk,))
+    f = oracle.kda_fwd(x["q"], x["k"], x["v"], np.ascontiguousarray(g), x["beta"], S0=x["S0"], gate_in=False)
+    return float((f["o"] * do).sum() + (f["S_T"] * dS).sum())
+
+
+@pytest.mark.parametrize("gate,per_head", [("softplus", False), ("bounded", True), ("softplus", True)])
+def test_gate_variant_gradients_match_finite_differences(gate, per_head):
+    """Softplus (v1) gate and the per-head (Gated DeltaNet) layout: directional
+    derivatives of every input, including z, A_log and dt_bias."""
+    x, do, dS = _inputs(seed=13)
+    r = np.random.default_rng(14)
+    x["z"] = r.standard_normal(x["g"].shape[:-1]) if per_head else x["g"]
+    if per_head:
+        x["dt_bias"] = 0.5 * r.standard_normal(x["dt_bias"].shape[0])
+    gr = backward.kda_backward(x["q"], x["k"], x["v"], x["z"], x["beta"], A_log=x["A_log"],
+                               dt_bias=x["dt_bias"], S0=x["S0"], do=do, dS_T=dS, gate=gate, per_head=per_head)
+    for name, gname in [("z", "g"), ("A_log", "A_log"), ("dt_bias", "dt_bias"), ("q", "q"), ("beta", "beta")]:
+        U = RNG.standard_normal(x[name].shape)
+        xp = dict(x); xp[name] = x[name] + H_FD * U
+        xm = dict(x); xm[name] = x[name] - H_FD * U
+        fd = (_loss_variant(xp, do, dS, gate, per_head) - _loss_variant(xm, do, dS, gate, per_head)) / (2 * H_FD)
+        an = float((gr[gname] * U).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, fd, an)
