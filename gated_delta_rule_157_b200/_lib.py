@@ -42,7 +42,7 @@ class ChunkArgs(ctypes.Structure):
         ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p),
         ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("S0", ctypes.c_void_p),
         ("o", ctypes.c_void_p), ("S_T", ctypes.c_void_p), ("M_T", ctypes.c_void_p),
-        ("S_chunks", ctypes.c_void_p),
+        ("S_chunks", ctypes.c_void_p), ("g_per_head", ctypes.c_int),
     ]
 
 
@@ -60,7 +60,7 @@ class ChunkBwdArgs(ctypes.Structure):
         ("dout", ctypes.c_void_p), ("dS_T", ctypes.c_void_p),
         ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p),
         ("dg", ctypes.c_void_p), ("dbeta", ctypes.c_void_p), ("dS0", ctypes.c_void_p),
-        ("dA_log", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p),
+        ("dA_log", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p), ("g_per_head", ctypes.c_int),
     ]
 
 
@@ -74,7 +74,7 @@ class StepArgs(ctypes.Structure):
         ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
         ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p),
         ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
-        ("S", ctypes.c_void_p), ("o", ctypes.c_void_p),
+        ("S", ctypes.c_void_p), ("o", ctypes.c_void_p), ("g_per_head", ctypes.c_int),
     ]
 
 
@@ -171,6 +171,16 @@ def _check(t, name, shape, dtype, device):
         raise ValueError("%s must be contiguous" % name)
 
 
+GATES = {"bounded": 1, "softplus": 2}
+
+
+def _gate_code(gate_in_kernel):
+    """True / "bounded" -> 1 (bounded sigmoid gate), "softplus" -> 2, False -> 0."""
+    if isinstance(gate_in_kernel, str):
+        return GATES[gate_in_kernel]
+    return 1 if gate_in_kernel else 0
+
+
 def _raise(fn, status):
     if status != KDA_OK:
         raise KdaError(fn, status)
@@ -180,7 +190,8 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
                   g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
                   beta_sigmoid_in_kernel=True, gate_in_kernel=True,
                   output_final_state=True, output_transition=False, algo="auto",
-                  o=None, S_T=None, M_T=None, S_chunks=None, stream=None, _withhold_ready=False):
+                  o=None, S_T=None, M_T=None, S_chunks=None, g_per_head=False, stream=None,
+                  _withhold_ready=False):
     """Chunk-parallel KDA forward.  Returns (o, S_T or None, M_T or None).
 
     (_withhold_ready routes to kda_debug_chunk_stall, the failure-path test hook.)
@@ -190,6 +201,9 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     A_log [HV], dt_bias [HV,Dk], S0 [B,HV,Dk,Dv]: float32.
     S_chunks: optional float32 [B,HV,ceil(T/chunk),Dk,Dv] that receives the
     state entering every chunk (the input of kda_chunk_bwd; SIMT kernel only).
+    gate_in_kernel: True or "bounded" (g_min sigmoid gate), "softplus"
+    (-exp(A_log) softplus gate, SIMT only) or False.  g_per_head: g [B,T,HV]
+    and dt_bias [HV], one decay per (token, value head) (SIMT only).
     """
     lib = load()
     if not isinstance(q, torch.Tensor) or not q.is_cuda:
@@ -201,10 +215,11 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     _check(q, "q", (B, T, H, Dk), dt, dev)
     _check(k, "k", (B, T, H, Dk), dt, dev)
     _check(v, "v", (B, T, HV, Dv), dt, dev)
-    _check(g, "g", (B, T, HV, Dk), dt, dev)
+    gk = () if g_per_head else (Dk,)
+    _check(g, "g", (B, T, HV) + gk, dt, dev)
     _check(beta, "beta", (B, T, HV), dt, dev)
     _check(A_log, "A_log", (HV,), torch.float32, dev)
-    _check(dt_bias, "dt_bias", (HV, Dk), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (HV,) + gk, torch.float32, dev)
     _check(S0, "S0", (B, HV, Dk, Dv), torch.float32, dev)
     if o is None:
         o = torch.empty((B, T, HV, Dv), dtype=dt, device=dev)
@@ -222,7 +237,8 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     a.g_min, a.scale, a.l2_eps = float(g_min), float(scale), float(l2_eps)
     a.qk_l2norm_in_kernel = int(bool(qk_l2norm_in_kernel))
     a.beta_sigmoid_in_kernel = int(bool(beta_sigmoid_in_kernel))
-    a.gate_in_kernel = int(bool(gate_in_kernel))
+    a.gate_in_kernel = _gate_code(gate_in_kernel)
+    a.g_per_head = int(bool(g_per_head))
     a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
     a.A_log, a.dt_bias, a.S0 = _ptr(A_log), _ptr(dt_bias), _ptr(S0)
     a.o, a.S_T, a.M_T, a.S_chunks = _ptr(o), _ptr(S_T), _ptr(M_T), _ptr(S_chunks)
@@ -236,15 +252,15 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
 def kda_chunk_bwd(q, k, v, g, beta, S_chunks, dout, dS_T=None, *, A_log=None, dt_bias=None,
                   chunk=64, g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
                   beta_sigmoid_in_kernel=True, gate_in_kernel=True, want_dS0=True, algo="auto",
-                  stream=None):
+                  g_per_head=False, stream=None):
     """Gradient of <dout, o> + <dS_T, S_T> for a kda_chunk_fwd call with the
     same arguments, from the per-chunk states S_chunks that call wrote.
 
     Returns a dict of float32 tensors: dq, dk [B,T,H,Dk]; dv [B,T,HV,Dv];
-    dg [B,T,HV,Dk] (w.r.t. g, or z with the in-kernel gate); dbeta [B,T,HV]
-    (w.r.t. beta, or its logit); dS0 [B,HV,Dk,Dv] (if want_dS0); dA_log [HV]
-    and ddt_bias [HV,Dk] with the in-kernel gate (ddt_bias only if dt_bias is
-    given).
+    dg [B,T,HV,Dk] ([B,T,HV] with g_per_head; w.r.t. g, or z with the
+    in-kernel gate); dbeta [B,T,HV] (w.r.t. beta, or its logit); dS0
+    [B,HV,Dk,Dv] (if want_dS0); dA_log [HV] and ddt_bias [HV,Dk] ([HV] with
+    g_per_head) with the in-kernel gate (ddt_bias only if dt_bias is given).
     """
     lib = load()
     if not isinstance(q, torch.Tensor) or not q.is_cuda:
@@ -257,27 +273,29 @@ def kda_chunk_bwd(q, k, v, g, beta, S_chunks, dout, dS_T=None, *, A_log=None, dt
     _check(q, "q", (B, T, H, Dk), dt, dev)
     _check(k, "k", (B, T, H, Dk), dt, dev)
     _check(v, "v", (B, T, HV, Dv), dt, dev)
-    _check(g, "g", (B, T, HV, Dk), dt, dev)
+    gk = () if g_per_head else (Dk,)
+    _check(g, "g", (B, T, HV) + gk, dt, dev)
     _check(beta, "beta", (B, T, HV), dt, dev)
     _check(dout, "dout", (B, T, HV, Dv), dt, dev)
     _check(A_log, "A_log", (HV,), torch.float32, dev)
-    _check(dt_bias, "dt_bias", (HV, Dk), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (HV,) + gk, torch.float32, dev)
     _check(S_chunks, "S_chunks", (B, HV, NC, Dk, Dv), torch.float32, dev)
     _check(dS_T, "dS_T", (B, HV, Dk, Dv), torch.float32, dev)
     f32 = dict(dtype=torch.float32, device=dev)
     out = {"dq": torch.empty((B, T, H, Dk), **f32), "dk": torch.empty((B, T, H, Dk), **f32),
-           "dv": torch.empty((B, T, HV, Dv), **f32), "dg": torch.empty((B, T, HV, Dk), **f32),
+           "dv": torch.empty((B, T, HV, Dv), **f32), "dg": torch.empty((B, T, HV) + gk, **f32),
            "dbeta": torch.empty((B, T, HV), **f32),
            "dS0": torch.empty((B, HV, Dk, Dv), **f32) if want_dS0 else None,
            "dA_log": torch.empty((HV,), **f32) if gate_in_kernel else None,
-           "ddt_bias": torch.empty((HV, Dk), **f32) if (gate_in_kernel and dt_bias is not None) else None}
+           "ddt_bias": torch.empty((HV,) + gk, **f32) if (gate_in_kernel and dt_bias is not None) else None}
     a = ChunkBwdArgs()
     a.B, a.T, a.H, a.HV, a.Dk, a.Dv, a.chunk = B, T, H, HV, Dk, Dv, int(chunk)
     a.dtype, a.algo = _dtype_code(q), ALGOS[algo]
     a.g_min, a.scale, a.l2_eps = float(g_min), float(scale), float(l2_eps)
     a.qk_l2norm_in_kernel = int(bool(qk_l2norm_in_kernel))
     a.beta_sigmoid_in_kernel = int(bool(beta_sigmoid_in_kernel))
-    a.gate_in_kernel = int(bool(gate_in_kernel))
+    a.gate_in_kernel = _gate_code(gate_in_kernel)
+    a.g_per_head = int(bool(g_per_head))
     a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
     a.A_log, a.dt_bias, a.S_chunks = _ptr(A_log), _ptr(dt_bias), _ptr(S_chunks)
     a.dout, a.dS_T = _ptr(dout), _ptr(dS_T)
@@ -289,10 +307,11 @@ def kda_chunk_bwd(q, k, v, g, beta, S_chunks, dout, dS_T=None, *, A_log=None, dt
 
 def kda_step(S, q, k, v, g, beta, *, A_log=None, dt_bias=None, g_min=-5.0, scale=1.0,
              l2_eps=1e-6, qk_l2norm_in_kernel=True, beta_sigmoid_in_kernel=True,
-             gate_in_kernel=True, o=None, stream=None):
+             gate_in_kernel=True, g_per_head=False, o=None, stream=None):
     """One decode step; S [B,HV,Dk,Dv] float32 is updated in place.  Returns o [B,HV,Dv].
 
-    q, k [B,H,Dk]; v [B,HV,Dv]; g [B,HV,Dk]; beta [B,HV] (float32 or bfloat16).
+    q, k [B,H,Dk]; v [B,HV,Dv]; g [B,HV,Dk] ([B,HV] with g_per_head);
+    beta [B,HV] (float32 or bfloat16).  gate_in_kernel as kda_chunk_fwd.
     """
     lib = load()
     if not isinstance(S, torch.Tensor) or not S.is_cuda:
@@ -305,10 +324,11 @@ def kda_step(S, q, k, v, g, beta, *, A_log=None, dt_bias=None, g_min=-5.0, scale
     _check(q, "q", (B, H, Dk), dt, dev)
     _check(k, "k", (B, H, Dk), dt, dev)
     _check(v, "v", (B, HV, Dv), dt, dev)
-    _check(g, "g", (B, HV, Dk), dt, dev)
+    gk = () if g_per_head else (Dk,)
+    _check(g, "g", (B, HV) + gk, dt, dev)
     _check(beta, "beta", (B, HV), dt, dev)
     _check(A_log, "A_log", (HV,), torch.float32, dev)
-    _check(dt_bias, "dt_bias", (HV, Dk), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (HV,) + gk, torch.float32, dev)
     if o is None:
         o = torch.empty((B, HV, Dv), dtype=dt, device=dev)
     _check(o, "o", (B, HV, Dv), dt, dev)
@@ -318,7 +338,8 @@ def kda_step(S, q, k, v, g, beta, *, A_log=None, dt_bias=None, g_min=-5.0, scale
     a.g_min, a.scale, a.l2_eps = float(g_min), float(scale), float(l2_eps)
     a.qk_l2norm_in_kernel = int(bool(qk_l2norm_in_kernel))
     a.beta_sigmoid_in_kernel = int(bool(beta_sigmoid_in_kernel))
-    a.gate_in_kernel = int(bool(gate_in_kernel))
+    a.gate_in_kernel = _gate_code(gate_in_kernel)
+    a.g_per_head = int(bool(g_per_head))
     a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
     a.A_log, a.dt_bias, a.S, a.o = _ptr(A_log), _ptr(dt_bias), _ptr(S), _ptr(o)
     _raise("kda_step", lib.kda_step(ctypes.byref(a), _stream(stream, dev)))

@@ -40,10 +40,11 @@ class KDAChunkFunction(torch.autograd.Function):
 
 def kda_chunk(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=64, g_min=-5.0,
               scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True, beta_sigmoid_in_kernel=True,
-              gate_in_kernel=True):
+              gate_in_kernel=True, g_per_head=False):
     """Differentiable chunk forward: returns (o, S_T); gradients flow to q, k,
-    v, g, beta, A_log, dt_bias and S0 through kda_chunk_bwd."""
+    v, g, beta, A_log, dt_bias and S0 through kda_chunk_bwd.  gate_in_kernel
+    and g_per_head as kda_chunk_fwd."""
     opts = dict(chunk=int(chunk), g_min=g_min, scale=scale, l2_eps=l2_eps,
                 qk_l2norm_in_kernel=qk_l2norm_in_kernel, beta_sigmoid_in_kernel=beta_sigmoid_in_kernel,
-                gate_in_kernel=gate_in_kernel)
+                gate_in_kernel=gate_in_kernel, g_per_head=bool(g_per_head))
     return KDAChunkFunction.apply(q, k, v, g, beta, A_log, dt_bias, S0, opts)

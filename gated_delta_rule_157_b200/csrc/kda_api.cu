@@ -41,9 +41,11 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
         return KDA_ERR_INVALID_ARG;
     if (a->Dk > 128 || a->Dv > 128 || a->chunk > 64) return KDA_ERR_UNSUPPORTED;
     if (!(a->g_min < 0.f) || !(a->l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    if (a->gate_in_kernel < 0 || a->gate_in_kernel > 2) return KDA_ERR_INVALID_ARG;
     const bool bf16 = a->dtype == KDA_DT_BF16;
     const size_t es = bf16 ? 2 : 4;
     const size_t ntok = (size_t)a->B * a->T;
+    const size_t gk = a->g_per_head ? 1 : (size_t)a->Dk;   // gate values per (token, value head)
     if (a->B == 0) return KDA_OK;
 
     if (ntok > 0) {
@@ -60,14 +62,14 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
     // Aliasing: o must not overlap inputs; S_T / M_T must not overlap o, inputs
     // (S_T == S0 exactly is allowed) or each other.
     const size_t nq = ntok * a->H * a->Dk * es, nv = ntok * a->HV * a->Dv * es;
-    const size_t ng = ntok * a->HV * a->Dk * es, nb = ntok * a->HV * es;
+    const size_t ng = ntok * a->HV * gk * es, nb = ntok * a->HV * es;
     const size_t ns = (size_t)a->B * a->HV * a->Dk * a->Dv * 4;
     const size_t nm = (size_t)a->B * a->HV * a->Dk * a->Dk * 4;
     Range r_in[] = {range_of(a->q, ntok ? nq : 0), range_of(a->k, ntok ? nq : 0),
                     range_of(a->v, ntok ? nv : 0), range_of(a->g, ntok ? ng : 0),
                     range_of(a->beta, ntok ? nb : 0),
                     range_of(a->A_log, a->A_log ? (size_t)a->HV * 4 : 0),
-                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * a->Dk * 4 : 0)};
+                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * gk * 4 : 0)};
     Range r_s0 = range_of(a->S0, a->S0 ? ns : 0);
     Range r_o = range_of(a->o, ntok ? nv : 0);
     Range r_st = range_of(a->S_T, a->S_T ? ns : 0);
@@ -91,7 +93,8 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
     p.g_min = a->g_min; p.scale = a->scale; p.l2_eps = a->l2_eps;
     p.l2norm = a->qk_l2norm_in_kernel != 0;
     p.beta_sigmoid = a->beta_sigmoid_in_kernel != 0;
-    p.gate_in = a->gate_in_kernel != 0;
+    p.gate_in = a->gate_in_kernel;
+    p.g_per_head = a->g_per_head != 0;
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.S0 = a->S0;
     p.o = a->o; p.S_T = a->S_T; p.M_T = a->M_T; p.S_chunks = a->S_chunks;
@@ -100,8 +103,11 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
 
     if (a->T == 0) return cuda_status(kda::launch_chunk_empty(p, s));
 
-    // Only the SIMT kernel writes the per-chunk states.
-    const bool tc_ok = kda::chunk_tc_supported(p, bf16) && !a->S_chunks;
+    // Only the SIMT kernel writes the per-chunk states and takes the softplus
+    // gate (unbounded: the tensor-core exponent scheme needs g >= g_min) or
+    // one gate value per head.
+    const bool tc_ok = kda::chunk_tc_supported(p, bf16) && !a->S_chunks && a->gate_in_kernel <= 1 &&
+                       !a->g_per_head;
     if (withhold_ready && (a->algo != KDA_ALGO_TC || !tc_ok)) return KDA_ERR_UNSUPPORTED;
     if (a->algo == KDA_ALGO_TC) {
         if (!tc_ok) return KDA_ERR_UNSUPPORTED;
@@ -134,10 +140,12 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
     if (a->algo == KDA_ALGO_TC) return KDA_ERR_UNSUPPORTED;
     if (a->Dk > 128 || a->Dv > 128 || a->chunk > 64) return KDA_ERR_UNSUPPORTED;
     if (!(a->g_min < 0.f) || !(a->l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    if (a->gate_in_kernel < 0 || a->gate_in_kernel > 2) return KDA_ERR_INVALID_ARG;
     if (a->B == 0) return KDA_OK;
     const bool bf16 = a->dtype == KDA_DT_BF16;
     const size_t es = bf16 ? 2 : 4;
     const size_t ntok = (size_t)a->B * a->T;
+    const size_t gk = a->g_per_head ? 1 : (size_t)a->Dk;
     if (ntok > 0) {
         if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->S_chunks || !a->dout) return KDA_ERR_INVALID_ARG;
         if (!a->dq || !a->dk || !a->dv || !a->dg || !a->dbeta) return KDA_ERR_INVALID_ARG;
@@ -152,7 +160,7 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
         if (p && !aligned(p, 4)) return KDA_ERR_ALIGNMENT;
 
     const size_t nq = ntok * a->H * a->Dk, nv = ntok * a->HV * a->Dv;
-    const size_t ng = ntok * a->HV * a->Dk, nb = ntok * a->HV;
+    const size_t ng = ntok * a->HV * gk, nb = ntok * a->HV;
     const size_t ns = (size_t)a->B * a->HV * a->Dk * a->Dv;
     const size_t nchunks = a->T > 0 ? ((size_t)a->T + a->chunk - 1) / a->chunk : 0;
     const bool gate = a->gate_in_kernel != 0;
@@ -160,14 +168,14 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
                     range_of(a->v, ntok ? nv * es : 0), range_of(a->g, ntok ? ng * es : 0),
                     range_of(a->beta, ntok ? nb * es : 0), range_of(a->dout, ntok ? nv * es : 0),
                     range_of(a->A_log, a->A_log ? (size_t)a->HV * 4 : 0),
-                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * a->Dk * 4 : 0),
+                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * gk * 4 : 0),
                     range_of(a->S_chunks, a->S_chunks ? ns * nchunks * 4 : 0),
                     range_of(a->dS_T, a->dS_T ? ns * 4 : 0)};
     Range r_out[] = {range_of(a->dq, ntok ? nq * 4 : 0), range_of(a->dk, ntok ? nq * 4 : 0),
                      range_of(a->dv, ntok ? nv * 4 : 0), range_of(a->dg, ntok ? ng * 4 : 0),
                      range_of(a->dbeta, ntok ? nb * 4 : 0), range_of(a->dS0, a->dS0 ? ns * 4 : 0),
                      range_of(gate ? a->dA_log : nullptr, gate && a->dA_log ? (size_t)a->HV * 4 : 0),
-                     range_of(gate ? a->ddt_bias : nullptr, gate && a->ddt_bias ? (size_t)a->HV * a->Dk * 4 : 0)};
+                     range_of(gate ? a->ddt_bias : nullptr, gate && a->ddt_bias ? (size_t)a->HV * gk * 4 : 0)};
     const int n_out = sizeof(r_out) / sizeof(r_out[0]);
     for (int i = 0; i < n_out; ++i) {
         for (Range r : r_in)
@@ -182,7 +190,8 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
     p.g_min = a->g_min; p.scale = a->scale; p.l2_eps = a->l2_eps;
     p.l2norm = a->qk_l2norm_in_kernel != 0;
     p.beta_sigmoid = a->beta_sigmoid_in_kernel != 0;
-    p.gate_in = gate;
+    p.gate_in = a->gate_in_kernel;
+    p.g_per_head = a->g_per_head != 0;
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.S_chunks = a->S_chunks;
     p.dout = a->dout; p.dS_T = a->dS_T;
@@ -195,7 +204,7 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
     struct Zero { void *p; size_t bytes; } zeros[] = {
         {p.dq, ntok ? nq * 4 : 0}, {p.dk, ntok ? nq * 4 : 0}, {p.dg, ntok ? ng * 4 : 0},
         {p.dbeta, ntok ? nb * 4 : 0}, {p.dA_log, p.dA_log ? (size_t)a->HV * 4 : 0},
-        {p.ddt_bias, p.ddt_bias ? (size_t)a->HV * a->Dk * 4 : 0}};
+        {p.ddt_bias, p.ddt_bias ? (size_t)a->HV * gk * 4 : 0}};
     for (const Zero &z : zeros) {
         if (z.bytes && cudaMemsetAsync(z.p, 0, z.bytes, s) != cudaSuccess) return KDA_ERR_CUDA;
     }
@@ -209,7 +218,9 @@ kda_status kda_step(const kda_step_args *a, void *stream) {
     if (a->dtype != KDA_DT_F32 && a->dtype != KDA_DT_BF16) return KDA_ERR_INVALID_ARG;
     if (a->Dk > 128 || a->Dv > 128 || a->Dv % 4 != 0) return KDA_ERR_UNSUPPORTED;
     if (!(a->g_min < 0.f) || !(a->l2_eps >= 0.f)) return KDA_ERR_INVALID_ARG;
+    if (a->gate_in_kernel < 0 || a->gate_in_kernel > 2) return KDA_ERR_INVALID_ARG;
     if (a->B == 0) return KDA_OK;
+    const size_t gk = a->g_per_head ? 1 : (size_t)a->Dk;
     if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->S || !a->o) return KDA_ERR_INVALID_ARG;
     if (a->gate_in_kernel && !a->A_log) return KDA_ERR_INVALID_ARG;
     const bool bf16 = a->dtype == KDA_DT_BF16;
@@ -223,10 +234,10 @@ kda_status kda_step(const kda_step_args *a, void *stream) {
 
     const size_t B = a->B;
     Range r_in[] = {range_of(a->q, B * a->H * a->Dk * es), range_of(a->k, B * a->H * a->Dk * es),
-                    range_of(a->v, B * a->HV * a->Dv * es), range_of(a->g, B * a->HV * a->Dk * es),
+                    range_of(a->v, B * a->HV * a->Dv * es), range_of(a->g, B * a->HV * gk * es),
                     range_of(a->beta, B * a->HV * es),
                     range_of(a->A_log, a->A_log ? (size_t)a->HV * 4 : 0),
-                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * a->Dk * 4 : 0)};
+                    range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * gk * 4 : 0)};
     Range r_s = range_of(a->S, B * a->HV * a->Dk * a->Dv * 4);
     Range r_o = range_of(a->o, B * a->HV * a->Dv * es);
     for (Range r : r_in)
@@ -238,7 +249,8 @@ kda_status kda_step(const kda_step_args *a, void *stream) {
     p.g_min = a->g_min; p.scale = a->scale; p.l2_eps = a->l2_eps;
     p.l2norm = a->qk_l2norm_in_kernel != 0;
     p.beta_sigmoid = a->beta_sigmoid_in_kernel != 0;
-    p.gate_in = a->gate_in_kernel != 0;
+    p.gate_in = a->gate_in_kernel;
+    p.g_per_head = a->g_per_head != 0;
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.A_log = a->A_log; p.dt_bias = a->dt_bias; p.S = a->S; p.o = a->o;
     return cuda_status(kda::launch_step(p, bf16, static_cast<cudaStream_t>(stream)));
@@ -331,6 +343,6 @@ const char *kda_status_string(kda_status s) {
     return "KDA_ERR_UNKNOWN";
 }
 
-int kda_version(void) { return 110; }
+int kda_version(void) { return 120; }
 
 }  // extern "C"

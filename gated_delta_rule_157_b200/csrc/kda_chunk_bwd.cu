@@ -26,8 +26,9 @@
 // Parallelisation as the SIMT forward: one CTA per (b, hv, 32-column slice of
 // the value channels).  dV, dS are per column; the q/k/g/beta gradients sum over
 // the columns (and over the value heads of a q/k head), so each CTA adds its
-// share with atomics into zeroed fp32 outputs.  A second pair of kernels takes
-// them through the in-kernel L2 norm, beta sigmoid and bounded gate.
+// share with atomics into zeroed fp32 outputs (with one decay per head, dg also
+// sums over the key channels).  A second pair of kernels takes them through
+// the in-kernel L2 norm, beta sigmoid and gate (bounded or softplus).
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -88,10 +89,10 @@ chunk_bwd_kernel(BwdParams p) {
             const size_t tok = tok0 + r;
             Qs[r * L + c] = ld_act(q, (tok * p.H + h) * Dk + c);
             Ks[r * L + c] = ld_act(k, (tok * p.H + h) * Dk + c);
-            float gz = ld_act(g, (tok * p.HV + hv) * Dk + c);
+            float gz = ld_act(g, gate_index(p.g_per_head, tok, p.HV, hv, Dk, c));
             if (p.gate_in) {
-                const float bias = p.dt_bias ? p.dt_bias[(size_t)hv * Dk + c] : 0.f;
-                gz = bounded_gate(gz, bias, ea, p.g_min);
+                const float bias = p.dt_bias ? p.dt_bias[bias_index(p.g_per_head, hv, Dk, c)] : 0.f;
+                gz = kda_gate(p.gate_in, gz, bias, ea, p.g_min);
             }
             Gs[r * L + c] = gz;
         }
@@ -296,10 +297,21 @@ chunk_bwd_kernel(BwdParams p) {
             float acc = dlast[c];
             for (int r = Cc - 1; r >= 0; --r) {
                 acc += Gs[r * L + c];
-                atomicAdd(&p.dg[((tok0 + r) * p.HV + hv) * Dk + c], acc);
+                if (p.g_per_head) Gs[r * L + c] = acc;
+                else atomicAdd(&p.dg[((tok0 + r) * p.HV + hv) * Dk + c], acc);
             }
         }
         for (int r = tid; r < Cc; r += kThreads) atomicAdd(&p.dbeta[(tok0 + r) * p.HV + hv], dbet[r]);
+        if (p.g_per_head) {
+            // one decay per (token, head): its gradient sums over the key channels
+            __syncthreads();
+            for (int r = warp; r < Cc; r += kThreads / 32) {
+                float sum = 0.f;
+                for (int c = lane; c < Dk; c += 32) sum += Gs[r * L + c];
+                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                if (lane == 0) atomicAdd(&p.dg[(tok0 + r) * p.HV + hv], sum);
+            }
+        }
     }
     __syncthreads();
     if (p.dS0) {
@@ -341,48 +353,77 @@ bwd_l2norm_kernel(BwdParams p) {
     }
 }
 
-// dbeta through the sigmoid; dg through the bounded gate, with the sums over
-// tokens of dA_log and ddt_bias.  Block = (value head hv, kGateTokens tokens),
-// thread = key channel.
+// Backward of the in-kernel gate at one element: returns dz for the upstream
+// gradient dg of the log-decay and adds this element's share of the sums over
+// tokens of dA_log (acc_a) and ddt_bias (acc_b).
+__device__ __forceinline__ float gate_backward(int mode, float z, float bias, float ea, float g_min, float dg,
+                                               float &acc_a, float &acc_b) {
+    float dz;
+    if (mode == 2) {             // g = -ea softplus(x), x = z + bias: dg/dx = -ea sigmoid(x), dg/dA_log = g
+        const float x = z + bias;
+        dz = -dg * ea * sigmoidf_(x);
+        acc_a = fmaf(dg, -ea * softplusf_(x), acc_a);
+    } else {                     // g = g_min sigmoid(pre), pre = ea (z + bias): dpre/dA_log = pre
+        const float pre = ea * (z + bias), s = sigmoidf_(pre);
+        const float dpre = dg * g_min * s * (1.f - s);
+        dz = dpre * ea;
+        acc_a = fmaf(dpre, pre, acc_a);
+    }
+    acc_b += dz;
+    return dz;
+}
+
+__device__ __forceinline__ float block_sum_128(float v, float *red) {
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    const float total = red[0] + red[1] + red[2] + red[3];
+    __syncthreads();
+    return total;
+}
+
+// dbeta through the sigmoid; dg through the in-kernel gate, with the sums over
+// tokens of dA_log and ddt_bias.  Block = (value head hv, kGateTokens tokens)
+// of 128 threads: thread = key channel, or (one decay per head) thread = token.
 constexpr int kGateTokens = 256;
 template <typename Tin>
 __global__ void __launch_bounds__(128)
 bwd_gate_kernel(BwdParams p) {
     __shared__ float red[4];
-    const int hv = blockIdx.x, c = threadIdx.x;
+    const int hv = blockIdx.x, tid = threadIdx.x;
     const long long n0 = (long long)blockIdx.y * kGateTokens;
     const long long ntok = (long long)p.B * p.T;
     const long long n1 = n0 + kGateTokens < ntok ? n0 + kGateTokens : ntok;
     const Tin *g = static_cast<const Tin *>(p.g);
     const Tin *bt = static_cast<const Tin *>(p.beta);
     if (p.beta_sigmoid) {
-        for (long long n = n0 + c; n < n1; n += blockDim.x) {
+        for (long long n = n0 + tid; n < n1; n += blockDim.x) {
             const size_t i = (size_t)n * p.HV + hv;
             const float s = sigmoidf_(ld_act(bt, i));
             p.dbeta[i] *= s * (1.f - s);
         }
     }
     if (!p.gate_in) return;
-    float acc_a = 0.f;
-    if (c < p.Dk) {
-        const float ea = expf(p.A_log[hv]);
-        const float bias = p.dt_bias ? p.dt_bias[(size_t)hv * p.Dk + c] : 0.f;
-        float acc_b = 0.f;
-        for (long long n = n0; n < n1; ++n) {
-            const size_t i = ((size_t)n * p.HV + hv) * p.Dk + c;
-            const float pre = ea * (ld_act(g, i) + bias);
-            const float s = sigmoidf_(pre);
-            const float dpre = p.dg[i] * p.g_min * s * (1.f - s);
-            p.dg[i] = dpre * ea;
-            acc_b = fmaf(dpre, ea, acc_b);
-            acc_a = fmaf(dpre, pre, acc_a);
+    const float ea = expf(p.A_log[hv]);
+    float acc_a = 0.f, acc_b = 0.f;
+    if (p.g_per_head) {
+        const float bias = p.dt_bias ? p.dt_bias[hv] : 0.f;
+        for (long long n = n0 + tid; n < n1; n += blockDim.x) {
+            const size_t i = (size_t)n * p.HV + hv;
+            p.dg[i] = gate_backward(p.gate_in, ld_act(g, i), bias, ea, p.g_min, p.dg[i], acc_a, acc_b);
         }
-        if (p.ddt_bias) atomicAdd(&p.ddt_bias[(size_t)hv * p.Dk + c], acc_b);
+        const float sb = block_sum_128(acc_b, red);
+        if (tid == 0 && p.ddt_bias) atomicAdd(&p.ddt_bias[hv], sb);
+    } else if (tid < p.Dk) {
+        const float bias = p.dt_bias ? p.dt_bias[(size_t)hv * p.Dk + tid] : 0.f;
+        for (long long n = n0; n < n1; ++n) {
+            const size_t i = ((size_t)n * p.HV + hv) * p.Dk + tid;
+            p.dg[i] = gate_backward(p.gate_in, ld_act(g, i), bias, ea, p.g_min, p.dg[i], acc_a, acc_b);
+        }
+        if (p.ddt_bias) atomicAdd(&p.ddt_bias[(size_t)hv * p.Dk + tid], acc_b);
     }
-    for (int off = 16; off > 0; off >>= 1) acc_a += __shfl_xor_sync(0xffffffffu, acc_a, off);
-    if ((c & 31) == 0) red[c >> 5] = acc_a;
-    __syncthreads();
-    if (c == 0 && p.dA_log) atomicAdd(&p.dA_log[hv], red[0] + red[1] + red[2] + red[3]);
+    const float sa = block_sum_128(acc_a, red);
+    if (tid == 0 && p.dA_log) atomicAdd(&p.dA_log[hv], sa);
 }
 
 // T == 0: dS0 = dS_T (or 0).

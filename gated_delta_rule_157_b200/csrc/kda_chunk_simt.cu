@@ -89,10 +89,10 @@ chunk_simt_kernel(ChunkParams p) {
             size_t tok = (size_t)b * p.T + t0 + r;
             Qs[r * L + c] = ld_act(q, (tok * p.H + h) * Dk + c);
             Ks[r * L + c] = ld_act(k, (tok * p.H + h) * Dk + c);
-            float gz = ld_act(g, (tok * p.HV + hv) * Dk + c);
+            float gz = ld_act(g, gate_index(p.g_per_head, tok, p.HV, hv, Dk, c));
             if (p.gate_in) {
-                float bias = p.dt_bias ? p.dt_bias[(size_t)hv * Dk + c] : 0.f;
-                gz = bounded_gate(gz, bias, ea, p.g_min);
+                float bias = p.dt_bias ? p.dt_bias[bias_index(p.g_per_head, hv, Dk, c)] : 0.f;
+                gz = kda_gate(p.gate_in, gz, bias, ea, p.g_min);
             }
             Gs[r * L + c] = gz;
         }

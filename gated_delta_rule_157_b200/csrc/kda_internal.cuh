@@ -26,12 +26,32 @@ __device__ __forceinline__ float bounded_gate(float z, float bias, float ea, flo
     return g_min * sigmoidf_(ea * (z + bias));
 }
 
+// log(1 + e^x) without overflow for large |x|.
+__device__ __forceinline__ float softplusf_(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+
+// The in-kernel gate, by mode: 1 = bounded (above), 2 = softplus,
+// g = -exp(A_log) * softplus(z + dt_bias) (unbounded below).
+__device__ __forceinline__ float kda_gate(int mode, float z, float bias, float ea, float g_min) {
+    return mode == 2 ? -ea * softplusf_(z + bias) : bounded_gate(z, bias, ea, g_min);
+}
+
+// Element offset of the gate input of (token row tok, value head hv, key
+// channel c), and of its dt_bias entry: one value per key channel, or one per
+// value head shared by the channels (g_per_head).
+__device__ __forceinline__ size_t gate_index(int per_head, size_t tok, int HV, int hv, int Dk, int c) {
+    return per_head ? tok * HV + hv : (tok * HV + hv) * Dk + c;
+}
+__device__ __forceinline__ size_t bias_index(int per_head, int hv, int Dk, int c) {
+    return per_head ? (size_t)hv : (size_t)hv * Dk + c;
+}
+
 // Validated arguments of a chunked forward, as the kernels see them.
 struct ChunkParams {
     int B, T, H, HV, Dk, Dv, C;
     int group;                       // HV / H
     float g_min, scale, l2_eps;
-    int l2norm, beta_sigmoid, gate_in;
+    int l2norm, beta_sigmoid, gate_in;   // gate_in: 0 none, 1 bounded, 2 softplus
+    int g_per_head;                      // g / z [B, T, HV], dt_bias [HV]
     const void *q, *k, *v, *g, *beta;
     const float *A_log, *dt_bias, *S0;
     void *o;
@@ -46,6 +66,7 @@ struct BwdParams {
     int group;                       // HV / H
     float g_min, scale, l2_eps;
     int l2norm, beta_sigmoid, gate_in;
+    int g_per_head;
     const void *q, *k, *v, *g, *beta;
     const float *A_log, *dt_bias, *S_chunks;
     const void *dout;
@@ -57,6 +78,7 @@ struct StepParams {
     int B, H, HV, Dk, Dv, group;
     float g_min, scale, l2_eps;
     int l2norm, beta_sigmoid, gate_in;
+    int g_per_head;
     const void *q, *k, *v, *g, *beta;
     const float *A_log, *dt_bias;
     float *S;

@@ -67,10 +67,10 @@ step_kernel(StepParams p) {
     if (tid < Dk) {
         qc = ld_act(q, ((size_t)b * p.H + h) * Dk + tid);
         kc = ld_act(k, ((size_t)b * p.H + h) * Dk + tid);
-        float gz = ld_act(g, ((size_t)b * p.HV + hv) * Dk + tid);
+        float gz = ld_act(g, gate_index(p.g_per_head, (size_t)b, p.HV, hv, Dk, tid));
         if (p.gate_in) {
-            float bias = p.dt_bias ? p.dt_bias[(size_t)hv * Dk + tid] : 0.f;
-            gz = bounded_gate(gz, bias, expf(p.A_log[hv]), p.g_min);
+            float bias = p.dt_bias ? p.dt_bias[bias_index(p.g_per_head, hv, Dk, tid)] : 0.f;
+            gz = kda_gate(p.gate_in, gz, bias, expf(p.A_log[hv]), p.g_min);
         }
         al[tid] = expf(gz);
     }

@@ -14,9 +14,17 @@
  * "KDAAttention 层", section "chunk_kda 内部做了什么"; all three default on):
  *     qk_l2norm_in_kernel:    q <- q / sqrt(|q|^2 + l2_eps), same for k
  *     beta_sigmoid_in_kernel: beta <- 1 / (1 + exp(-beta))
- *     gate_in_kernel:         g <- g_min * sigmoid(exp(A_log[hv]) * (g + dt_bias[hv,:]))
+ *     gate_in_kernel = 1:     g <- g_min * sigmoid(exp(A_log[hv]) * (g + dt_bias[hv,:]))
  *                             (bounded decay; page "KDA 模块交互式演示" section 1.4
  *                             Eq. 5, page "Implémenter KDA" "La décroissance bornée")
+ *     gate_in_kernel = 2:     g <- -exp(A_log[hv]) * softplus(g + dt_bias[hv,:])
+ *                             (the unbounded gate of the first KDA version, page
+ *                             "Implémenter KDA" "La décroissance bornée"; the SIMT
+ *                             kernels only)
+ *     gate_in_kernel = 0:     g is the log-decay itself.
+ * With g_per_head set, g holds one value per (token, value head), shared by
+ * the Dk key channels (the Gated DeltaNet form, page "线性注意力交互式演示"
+ * Eq. 6), and dt_bias one value per value head (SIMT kernels only).
  *
  * Value head hv reads q/k head h = hv / (HV / H) (contiguous groups).
  *
@@ -79,14 +87,15 @@ typedef enum {
  * Layouts (element type `dtype` unless stated):
  *   q, k    [B, T, H,  Dk]
  *   v       [B, T, HV, Dv]
- *   g       [B, T, HV, Dk]  log-decay g, or the raw gate input z when gate_in_kernel;
+ *   g       [B, T, HV, Dk]  ([B, T, HV] with g_per_head) log-decay g, or the raw
+ *           gate input z when gate_in_kernel;
  *           a log-decay given directly should lie in [g_min, 0]: the SIMT
  *           kernel takes any value, the tensor-core kernel (whose exponent
  *           bound, 16 |g_min| per 16-token tile, rests on it) clamps values
  *           below g_min up to g_min
  *   beta    [B, T, HV]      write strength, or its logit when beta_sigmoid_in_kernel
  *   A_log   [HV]      fp32  read iff gate_in_kernel (must then be non-NULL)
- *   dt_bias [HV, Dk]  fp32  read iff gate_in_kernel; NULL means 0
+ *   dt_bias [HV, Dk]  fp32  ([HV] with g_per_head) read iff gate_in_kernel; NULL means 0
  *   S0      [B, HV, Dk, Dv] fp32, or NULL for zeros
  *   o       [B, T, HV, Dv]  output, element type `dtype` (bf16 rounded to nearest even)
  *   S_T     [B, HV, Dk, Dv] fp32 output, or NULL; may be the same buffer as S0
@@ -100,8 +109,10 @@ typedef enum {
  *
  * Limits: B, T >= 0; 1 <= H <= HV, HV % H == 0; 1 <= Dk, Dv <= 128;
  * 1 <= chunk <= 64.  q, k, v, g, beta, o must be aligned to their element size;
- * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64 and
- * 16-byte aligned q, k, v, g, o.  o must not overlap any input; S_T, M_T and
+ * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64,
+ * gate_in_kernel 0 or 1 with one gate value per key channel, and 16-byte
+ * aligned q, k, v, g, o (KDA_ALGO_AUTO takes the SIMT kernel otherwise).
+ * gate_in_kernel must be 0, 1 or 2.  o must not overlap any input; S_T, M_T and
  * S_chunks must not overlap each other, o, or any input except S_T == S0.
  * T == 0 writes S_T = S0 (or 0) and M_T = I.
  */
@@ -120,6 +131,7 @@ typedef struct {
     float *S_T;
     float *M_T;
     float *S_chunks;
+    int g_per_head;            /* g [B, T, HV] and dt_bias [HV]: one decay per head */
 } kda_chunk_args;
 
 kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
@@ -168,7 +180,8 @@ typedef struct {
     float *dbeta;              /* [B, T, HV] */
     float *dS0;                /* [B, HV, Dk, Dv] or NULL */
     float *dA_log;             /* [HV] or NULL */
-    float *ddt_bias;           /* [HV, Dk] or NULL */
+    float *ddt_bias;           /* [HV, Dk] ([HV] with g_per_head) or NULL */
+    int g_per_head;            /* as kda_chunk_fwd; dg is then [B, T, HV] */
 } kda_chunk_bwd_args;
 
 kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);
@@ -181,9 +194,10 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);
  * Layouts:
  *   q, k    [B, H,  Dk]   dtype
  *   v       [B, HV, Dv]   dtype
- *   g       [B, HV, Dk]   dtype (log-decay, or raw z when gate_in_kernel)
+ *   g       [B, HV, Dk]   dtype (log-decay, or raw z when gate_in_kernel);
+ *           [B, HV] with g_per_head
  *   beta    [B, HV]       dtype
- *   A_log   [HV], dt_bias [HV, Dk] fp32 (as in kda_chunk_fwd)
+ *   A_log   [HV], dt_bias [HV, Dk] ([HV] with g_per_head) fp32, as in kda_chunk_fwd
  *   S       [B, HV, Dk, Dv] fp32, read and written in place, 16-byte aligned
  *   o       [B, HV, Dv]   dtype output
  *
@@ -199,6 +213,7 @@ typedef struct {
     const float *A_log, *dt_bias;
     float *S;
     void *o;
+    int g_per_head;            /* g [B, HV] and dt_bias [HV] */
 } kda_step_args;
 
 kda_status kda_step(const kda_step_args *args, void *stream);

@@ -1,7 +1,8 @@
-"""Host emulation of the library's SIMT chunk kernels -- TEST INFRASTRUCTURE.
+"""Host emulation of the library's SIMT kernels -- TEST INFRASTRUCTURE.
 
-Compiles the CUDA sources of the SIMT forward (kda_chunk_simt.cu) and of the
-backward (kda_chunk_bwd.cu) as host C++ with g++ and AddressSanitizer: the
+Compiles the CUDA sources of the SIMT forward (kda_chunk_simt.cu), the
+backward (kda_chunk_bwd.cu) and the decode step (kda_step.cu) as host C++ with
+g++ and AddressSanitizer: the
 stand-in headers in fakeinc/ map the CUDA keywords and intrinsics the kernels
 use onto C++, emu_rt.cpp runs every CUDA thread of a block as a std::thread
 (__syncthreads and __syncwarp are std::barriers, a thread that returns drops
@@ -91,10 +92,13 @@ extern "C" int emu_chunk_bwd(kda::BwdParams *pp, int bf16) {
 
 def _unit(src_name, runner):
     s = open(os.path.join(CSRC, src_name)).read()
-    m = re.search(r"^(template <typename Tin>\nstatic )?cudaError_t launch_", s, re.M)
+    m = re.search(r"^(template <[^>]*>\n(static )?)?cudaError_t launch_", s, re.M)
     if not m:
         raise RuntimeError("no host launcher found in " + src_name)
-    s = s[: m.start()] + "\n}  // namespace kda\n"
+    s = s[: m.start()]
+    if "\n}  // namespace\n" not in s:      # the first launcher sits inside the unnamed namespace
+        s += "\n}  // namespace\n"
+    s += "}  // namespace kda\n"
     # static __shared__ arrays are block-wide: function statics (the blocks of
     # a grid run one after another); the dynamic one is the array declared below
     s = s.replace("extern __shared__", "extern").replace("__shared__", "static")
@@ -104,8 +108,30 @@ def _unit(src_name, runner):
     return head + "#line 1 \"%s\"\n" % src_name + s + runner
 
 
+_RUN_STEP = r'''
+extern "C" int emu_sizeof_step_params(void) { return (int)sizeof(kda::StepParams); }
+template <int RPT>
+static void run_step(const kda::StepParams &p, int bf16) {
+    using namespace kda;
+    if (bf16) emu_launch(dim3(p.B * p.HV), dim3(kThreads), [&] { step_kernel<RPT, __nv_bfloat16>(p); });
+    else emu_launch(dim3(p.B * p.HV), dim3(kThreads), [&] { step_kernel<RPT, float>(p); });
+}
+extern "C" int emu_step(kda::StepParams *pp, int bf16) {
+    const kda::StepParams p = *pp;
+    const int rpt = (p.Dk + kda::kWarps - 1) / kda::kWarps;
+    if (rpt <= 1) run_step<1>(p, bf16);
+    else if (rpt <= 2) run_step<2>(p, bf16);
+    else if (rpt <= 4) run_step<4>(p, bf16);
+    else if (rpt <= 8) run_step<8>(p, bf16);
+    else run_step<16>(p, bf16);
+    return 0;
+}
+'''
+
+
 def _deps():
-    return [os.path.join(CSRC, f) for f in ("kda_chunk_simt.cu", "kda_chunk_bwd.cu", "kda_internal.cuh")] + \
+    return [os.path.join(CSRC, f) for f in ("kda_chunk_simt.cu", "kda_chunk_bwd.cu", "kda_step.cu",
+                                            "kda_internal.cuh")] + \
         [os.path.join(HERE, f) for f in ("emu_build.py", "emu_rt.cpp", "fakeinc/cuda_runtime.h", "fakeinc/cuda_bf16.h")] + \
         [os.path.join(ROOT, "include", "kda.h")]
 
@@ -121,7 +147,8 @@ def build(force=False):
         return LIB
     os.makedirs(OUT, exist_ok=True)
     units = {"emu_fwd.cpp": _unit("kda_chunk_simt.cu", _RUN_FWD),
-             "emu_bwd.cpp": _unit("kda_chunk_bwd.cu", _RUN_BWD)}
+             "emu_bwd.cpp": _unit("kda_chunk_bwd.cu", _RUN_BWD),
+             "emu_step.cpp": _unit("kda_step.cu", _RUN_STEP)}
     objs = []
     flags = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address", "-fno-omit-frame-pointer", "-fPIC",
              "-I", os.path.join(HERE, "fakeinc"), "-I", CSRC, "-Wno-unknown-pragmas", "-c"]

@@ -33,3 +33,7 @@ inline float __expf(float x) { return std::exp(x); }
 inline float __fdividef(float a, float b) { return a / b; }
 using std::max;
 using std::min;
+struct float4 { float x, y, z, w; };
+inline float4 make_float4(float x, float y, float z, float w) { return float4{x, y, z, w}; }
+inline float4 __ldcs(const float4 *p) { return *p; }
+inline void __stcs(float4 *p, float4 v) { *p = v; }

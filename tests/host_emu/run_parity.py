@@ -26,7 +26,7 @@ _P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 class ChunkParams(ctypes.Structure):       # kda::ChunkParams
     _fields_ = [(n, _I) for n in ("B", "T", "H", "HV", "Dk", "Dv", "C", "group")] + \
         [(n, _F) for n in ("g_min", "scale", "l2_eps")] + \
-        [(n, _I) for n in ("l2norm", "beta_sigmoid", "gate_in")] + \
+        [(n, _I) for n in ("l2norm", "beta_sigmoid", "gate_in", "g_per_head")] + \
         [(n, _P) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0", "o", "S_T", "M_T",
                            "S_chunks")] + [("withhold_ready", _I)]
 
@@ -34,22 +34,52 @@ class ChunkParams(ctypes.Structure):       # kda::ChunkParams
 class BwdParams(ctypes.Structure):         # kda::BwdParams
     _fields_ = [(n, _I) for n in ("B", "T", "H", "HV", "Dk", "Dv", "C", "group")] + \
         [(n, _F) for n in ("g_min", "scale", "l2_eps")] + \
-        [(n, _I) for n in ("l2norm", "beta_sigmoid", "gate_in")] + \
+        [(n, _I) for n in ("l2norm", "beta_sigmoid", "gate_in", "g_per_head")] + \
         [(n, _P) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S_chunks", "dout", "dS_T",
                            "dq", "dk", "dv", "dg", "dbeta", "dS0", "dA_log", "ddt_bias")]
 
 
+class StepParams(ctypes.Structure):        # kda::StepParams
+    _fields_ = [(n, _I) for n in ("B", "H", "HV", "Dk", "Dv", "group")] + \
+        [(n, _F) for n in ("g_min", "scale", "l2_eps")] + \
+        [(n, _I) for n in ("l2norm", "beta_sigmoid", "gate_in", "g_per_head")] + \
+        [(n, _P) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S", "o")]
+
+
 GRADS = ("dq", "dk", "dv", "dg", "dbeta", "dS0", "dA_log", "ddt_bias")
+GATE_CODE = {None: 0, "bounded": 1, "softplus": 2}
+
+
+def _gate_np(z, A_log, dt_bias, gate, per_head, Dk):
+    """Log-decay [.., HV, Dk] from the raw gate input, through oracle/gates.py."""
+    from oracle import gates
+    zc = z[..., None] if per_head else z
+    bc = None if dt_bias is None else (dt_bias[:, None] if per_head else dt_bias)
+    fn = gates.bounded_gate if gate == "bounded" else gates.softplus_gate
+    g = fn(zc, A_log, bc)
+    return np.ascontiguousarray(np.broadcast_to(g, zc.shape[:-1] + (Dk,)))
+
+
+def _per_head(inp):
+    """The generator's draws cut to one gate value per (token, head)."""
+    inp = dict(inp)
+    inp["g"] = inp["g"][..., 0].contiguous()
+    if inp["dt_bias"] is not None:
+        inp["dt_bias"] = inp["dt_bias"][:, 0].contiguous()
+    return inp
 
 
 def _ptr(t):
     return None if t is None or t.numel() == 0 else t.data_ptr()
 
 
-def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed):
+def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed, gate="bounded", per_head=False):
     w = workloads.Workload("emu", B=B, T=T, H=H, HV=HV, Dk=Dk, Dv=Dv, chunk=C, dtype=dtype, seed=seed,
                            a_log="uniform", dt_bias_std=0.5, s0_std=0.2)
     inp = workloads.chunk_inputs(w) if flags else workloads.activated_inputs(w)
+    if per_head:
+        inp = _per_head(inp)
+    gcode = GATE_CODE[gate] if flags else 0
     gen = torch.Generator().manual_seed(seed + 7)
     dout = torch.randn((B, T, HV, Dv), generator=gen).to(inp["q"].dtype)
     dS_T = torch.randn((B, HV, Dk, Dv), generator=gen)
@@ -59,34 +89,45 @@ def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed):
     S_T = torch.zeros((B, HV, Dk, Dv))
     S_ch = torch.full((B, HV, NC, Dk, Dv), float("nan"))
     fl = int(flags)
-    fp = ChunkParams(B, T, H, HV, Dk, Dv, C, HV // H, -5.0, scale, 1e-6, fl, fl, fl,
+    fp = ChunkParams(B, T, H, HV, Dk, Dv, C, HV // H, -5.0, scale, 1e-6, fl, fl, gcode, int(per_head),
                      *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0")),
                      _ptr(o), _ptr(S_T), None, _ptr(S_ch), 0)
     if T > 0 and lib.emu_chunk_fwd(ctypes.byref(fp), bf16) != 0:
         raise RuntimeError("forward emulation refused the shape")
+    gk = () if per_head else (Dk,)
     out = {"dq": torch.zeros((B, T, H, Dk)), "dk": torch.zeros((B, T, H, Dk)),
-           "dv": torch.zeros((B, T, HV, Dv)), "dg": torch.zeros((B, T, HV, Dk)), "dbeta": torch.zeros((B, T, HV)),
+           "dv": torch.zeros((B, T, HV, Dv)), "dg": torch.zeros((B, T, HV) + gk), "dbeta": torch.zeros((B, T, HV)),
            "dS0": torch.zeros((B, HV, Dk, Dv)), "dA_log": torch.zeros(HV) if flags else None,
-           "ddt_bias": torch.zeros((HV, Dk)) if flags else None}
-    bp = BwdParams(B, T, H, HV, Dk, Dv, C, HV // H, -5.0, scale, 1e-6, fl, fl, fl,
+           "ddt_bias": torch.zeros((HV,) + gk) if flags else None}
+    bp = BwdParams(B, T, H, HV, Dk, Dv, C, HV // H, -5.0, scale, 1e-6, fl, fl, gcode, int(per_head),
                    *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias")),
                    _ptr(S_ch), _ptr(dout), _ptr(dS_T), *(_ptr(out[n]) for n in GRADS))
     if lib.emu_chunk_bwd(ctypes.byref(bp), bf16) != 0:
         raise RuntimeError("backward emulation refused the shape")
-    sw = dict(scale=scale, qk_l2norm=flags, beta_sigmoid=flags, gate_in=flags)
     args = [to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")]
-    kw = dict(A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]), S0=to_np(inp["S0"]))
+    if flags and (gate != "bounded" or per_head):
+        # the oracle's forward takes the variant gates precomputed (oracle/gates.py)
+        sw = dict(scale=scale, qk_l2norm=True, beta_sigmoid=True, gate_in=False)
+        fargs = args[:3] + [_gate_np(args[3], to_np(inp["A_log"]), to_np(inp["dt_bias"]), gate, per_head, Dk)] + args[4:]
+        kw = dict(S0=to_np(inp["S0"]))
+    else:
+        sw = dict(scale=scale, qk_l2norm=flags, beta_sigmoid=flags, gate_in=flags)
+        fargs = args
+        kw = dict(A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]), S0=to_np(inp["S0"]))
     err = {}            # each entry is held to TOL (o of bf16 inputs rescaled to its own bar)
     if T > 0:
-        ref = oracle.kda_fwd(*args, **kw, **sw)
+        ref = oracle.kda_fwd(*fargs, **kw, **sw)
         # o is stored in the input dtype: bf16 rounding puts it under the bf16 bar
         err["o"] = max_rel(to_np(o), ref["o"]) * (TOL / TOL_BF16 if dtype == "bf16" else 1.0)
         err["S_T"] = max_rel(to_np(S_T), ref["S_T"])
         for c in range(1, NC):
-            pre = oracle.kda_fwd(*(a[:, : c * C] for a in args), **kw, **sw)
+            pre = oracle.kda_fwd(*(a[:, : c * C] for a in fargs), **kw, **sw)
             err["S_chunks"] = max(err.get("S_chunks", 0.0), max_rel(to_np(S_ch[:, :, c]), pre["S_T"]))
         err["S_chunks0"] = max_rel(to_np(S_ch[:, :, 0]), to_np(inp["S0"]))
-    gr = backward.kda_backward(*args, **kw, do=to_np(dout), dS_T=to_np(dS_T), **sw)
+    gr = backward.kda_backward(*args, A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]),
+                               S0=to_np(inp["S0"]), do=to_np(dout), dS_T=to_np(dS_T), scale=scale,
+                               qk_l2norm=flags, beta_sigmoid=flags, gate_in=flags, gate=gate or "bounded",
+                               per_head=per_head)
     names = {"dq": "q", "dk": "k", "dv": "v", "dg": "g", "dbeta": "beta", "dS0": "S0"}
     if flags:
         names.update(dA_log="A_log", ddt_bias="dt_bias")
@@ -94,6 +135,35 @@ def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed):
         err[n] = max_rel(to_np(out[n]), gr[rn])
     return err
 
+
+def run_step_case(lib, B, H, HV, Dk, Dv, dtype, gate, per_head, seed):
+    """One decode step against the oracle's step."""
+    w = workloads.Workload("emustep", B=B, T=1, H=H, HV=HV, Dk=Dk, Dv=Dv, chunk=1, dtype=dtype, seed=seed,
+                           a_log="uniform", dt_bias_std=0.5, s0_std=0.3)
+    inp = workloads.chunk_inputs(w)
+    if per_head:
+        inp = _per_head(inp)
+    S = inp["S0"].clone()
+    x = {n: inp[n][:, 0].contiguous() for n in ("q", "k", "v", "g", "beta")}
+    o = torch.zeros((B, HV, Dv), dtype=x["q"].dtype)
+    sp = StepParams(B, H, HV, Dk, Dv, HV // H, -5.0, 1.0, 1e-6, 1, 1, GATE_CODE[gate], int(per_head),
+                    *(_ptr(x[n]) for n in ("q", "k", "v", "g", "beta")), _ptr(inp["A_log"]),
+                    _ptr(inp["dt_bias"]), _ptr(S), _ptr(o))
+    lib.emu_step(ctypes.byref(sp), int(dtype == "bf16"))
+    g = _gate_np(to_np(x["g"])[:, None], to_np(inp["A_log"]), to_np(inp["dt_bias"]), gate, per_head, Dk)[:, 0]
+    S_ref, o_ref = oracle.kda_step(to_np(inp["S0"]), *(to_np(x[n]) for n in ("q", "k", "v")), g,
+                                   to_np(x["beta"]), gate_in=False)
+    scale_o = TOL / TOL_BF16 if dtype == "bf16" else 1.0
+    return {"o": max_rel(to_np(o), o_ref) * scale_o, "S": max_rel(to_np(S), S_ref)}
+
+
+STEP_CASES = [
+    # B, H, HV, Dk, Dv, dtype, gate, per_head, seed
+    (2, 1, 2, 128, 128, "f32", "bounded", False, 11),
+    (2, 1, 2, 64, 32, "f32", "softplus", False, 12),
+    (3, 2, 4, 128, 64, "bf16", "softplus", True, 13),
+    (1, 1, 1, 32, 16, "f32", "bounded", True, 14),
+]
 
 CASES = [
     # B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed
@@ -103,6 +173,9 @@ CASES = [
     (1, 45, 1, 1, 24, 20, 16, "bf16", True, 1.0, 4),     # bf16 inputs
     (1, 70, 1, 1, 128, 128, 64, "f32", True, 1.0, 5),    # full head size, C = 64, ragged
     (2, 0, 1, 2, 16, 16, 16, "f32", True, 1.0, 6),       # empty sequence
+    (1, 40, 1, 2, 16, 16, 16, "f32", True, 1.0, 7, "softplus", False),   # unbounded gate
+    (1, 40, 1, 2, 16, 16, 16, "f32", True, 1.0, 8, "bounded", True),     # one decay per head
+    (2, 50, 1, 2, 32, 40, 16, "bf16", True, 1.0, 9, "softplus", True),   # both, bf16
 ]
 TOL = TOL_F32
 
@@ -112,7 +185,14 @@ if __name__ == "__main__":
     assert lib.emu_offsetof_withhold_ready() == ChunkParams.withhold_ready.offset
     assert lib.emu_sizeof_bwd_params() == ctypes.sizeof(BwdParams)
     assert lib.emu_offsetof_ddt_bias() == BwdParams.ddt_bias.offset
+    assert lib.emu_sizeof_step_params() == ctypes.sizeof(StepParams)
     bad = 0
+    for case in STEP_CASES:
+        err = run_step_case(lib, *case)
+        worst = max(err.values())
+        bad += worst > TOL
+        print("step", case, "ok" if worst <= TOL else "MISMATCH", " ".join("%s=%.1e" % kv for kv in err.items()),
+              flush=True)
     for case in CASES:
         err = run_case(lib, *case)
         worst = max(err.values()) if err else 0.0
