@@ -176,6 +176,9 @@ CASES = [
     (1, 40, 1, 2, 16, 16, 16, "f32", True, 1.0, 7, "softplus", False),   # unbounded gate
     (1, 40, 1, 2, 16, 16, 16, "f32", True, 1.0, 8, "bounded", True),     # one decay per head
     (2, 50, 1, 2, 32, 40, 16, "bf16", True, 1.0, 9, "softplus", True),   # both, bf16
+    (1, 5, 1, 1, 1, 1, 1, "f32", False, 1.0, 10),      # Dk = Dv = chunk = 1
+    (2, 23, 1, 3, 3, 5, 7, "f32", True, 1.0, 11),      # odd sizes everywhere
+    (1, 1, 1, 1, 8, 8, 16, "f32", True, 1.0, 12),      # one token, shorter than a chunk
 ]
 TOL = TOL_F32
 

@@ -97,7 +97,15 @@ BWD_CASES = [
     (1, 64, 1, 1, 128, 128, 64, "f32", True, 1.0, None, False),   # one whole chunk, zero S0, dS_T
     (2, 130, 2, 4, 64, 48, 64, "bf16", True, 1.0, 0.1, True),     # grouped heads, ragged
     (1, 200, 1, 1, 128, 128, 64, "bf16", True, 0.8, 0.02, True),  # full head size, ragged
+    (1, 5, 1, 1, 1, 1, 1, "f32", False, 1.0, 0.3, True),          # Dk = Dv = chunk = 1 (see below)
+    (2, 23, 1, 3, 3, 5, 7, "f32", True, 1.0, 0.3, True),          # odd sizes everywhere
+    (1, 1, 1, 1, 8, 8, 16, "f32", True, 1.0, 0.3, True),          # one token
+    (1, 64, 1, 1, 128, 1, 64, "f32", True, 1.0, 0.3, True),       # Dv = 1
 ]
+# At Dk = 1 the in-kernel L2 norm is degenerate (q / |q| = +-1): its gradient,
+# eps / |q|^3 times dq, is the difference of two terms of size |dq| / |q|, which
+# FP32 cannot resolve to 1e-4 of the tiny exact value.  That shape runs with
+# the switches off.
 
 
 @pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "x".join(map(str, c[:8])) + ("" if c[8] else "-raw"))
