@@ -273,6 +273,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of the headline workload (small cases for profiling)")
+    ap.add_argument("--train", action="store_true",
+                    help="also time the training path: forward keeping the chunk states (SIMT) + backward")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -378,6 +380,9 @@ def main():
                                        "kcp": line["kcp"]["launches"],
                                        "layer": line["layer"]["launches"]}
 
+    if args.train:
+        line["train"] = bench_train(args, kda, workloads, dev, stream, world, rank)
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -454,6 +459,45 @@ def bench_kcp(args, kda, workloads, dev, stream, world, rank):
     return {"workload": "kcp_bf16: B=1 H=HV=16 T=65536 as 8 x 8192, Dk=Dv=128",
             "value": whole_job_value(w.token_heads, world, ms), "unit": UNIT, "ms_per_step": ms,
             "launches": 3 * k}
+
+
+def bench_train(args, kda, workloads, dev, stream, world, rank):
+    """Training path at the headline workload (or --batch): kda_chunk_fwd
+    keeping the per-chunk states (SIMT kernel) and kda_chunk_bwd, timed apart;
+    throughput in token-heads per second of forward + backward."""
+    import torch
+    w = workloads.workload("gva_bf16") if args.batch is None else workloads.workload("gva_bf16", B=args.batch)
+    inp = workloads.chunk_inputs(w, seed=rank_seed(w, rank), device=dev)
+    g = torch.Generator(device=dev).manual_seed(17 + rank)
+    dout = torch.randn((w.B, w.T, w.HV, w.Dv), device=dev, generator=g).to(torch.bfloat16)
+    S_ch = torch.empty((w.B, w.HV, -(-w.T // w.chunk), w.Dk, w.Dv), device=dev)
+    o = torch.empty((w.B, w.T, w.HV, w.Dv), dtype=torch.bfloat16, device=dev)
+
+    def fwd(_i):
+        kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], A_log=inp["A_log"],
+                          dt_bias=inp["dt_bias"], S0=inp["S0"], chunk=w.chunk, o=o, S_chunks=S_ch,
+                          output_final_state=False, stream=stream)
+
+    def bwd(_i):
+        kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S_ch, dout, None,
+                          A_log=inp["A_log"], dt_bias=inp["dt_bias"], chunk=w.chunk, stream=stream)
+
+    out = {"workload": "gva_bf16 B=%d: forward with chunk states (SIMT) + backward (SIMT)" % w.B}
+    for name, fn in (("forward_with_states", fwd), ("backward", bwd)):
+        for i in range(max(1, min(args.warmup, 2))):
+            fn(i)
+        kda.kda_device_status(stream)
+        barrier(world, dev)
+        k = max(3, min(args.steps, 5))
+        per = time_launches(fn, k, stream)
+        barrier(world, dev)
+        kda.kda_device_status(stream)
+        out[name] = {"ms_per_step": max_over_ranks(sum(per) / len(per), world, dev)}
+    ms = out["forward_with_states"]["ms_per_step"] + out["backward"]["ms_per_step"]
+    out["value"] = whole_job_value(w.token_heads, world, ms)
+    out["unit"] = UNIT
+    out["roofline"] = None   # CUDA-core, SFU-bound path; no roofline figure until profiled
+    return out
 
 
 def bench_layer(args, kda, dev, stream, pk, world):
