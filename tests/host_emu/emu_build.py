@@ -90,8 +90,18 @@ extern "C" int emu_chunk_bwd(kda::BwdParams *pp, int bf16) {
 '''
 
 
-def _unit(src_name, runner):
-    s = open(os.path.join(CSRC, src_name)).read()
+def unit_from_text(text, runner, poison=True):
+    """A unit for kernel source text given directly (namespace kda, unnamed
+    namespace, no host launchers): the checks of the harness itself."""
+    head = ('#include <functional>\n#include "cuda_runtime.h"\n'
+            "void emu_launch(dim3 grid, dim3 block, const std::function<void()> &fn);\n"
+            "namespace kda { namespace { alignas(16) float smem[%d]; } }\n" % SMEM_FLOATS)
+    body = text.replace("extern __shared__", "extern").replace("__shared__", "static")
+    return head + body + (_POISON if poison else "") + runner
+
+
+def _unit(src_name, runner, src_dir=CSRC):
+    s = open(os.path.join(src_dir, src_name)).read()
     m = re.search(r"^(template <[^>]*>\n(static )?)?cudaError_t launch_", s, re.M)
     if not m:
         raise RuntimeError("no host launcher found in " + src_name)
@@ -136,34 +146,52 @@ def _deps():
         [os.path.join(ROOT, "include", "kda.h")]
 
 
-def asan_runtime():
-    return subprocess.run(["g++", "-print-file-name=libasan.so"], check=True, capture_output=True,
+def sanitizer_runtime(sanitizer="address"):
+    """Path of the g++ sanitizer runtime to preload (libasan / libtsan)."""
+    name = {"address": "libasan.so", "thread": "libtsan.so"}[sanitizer]
+    return subprocess.run(["g++", "-print-file-name=" + name], check=True, capture_output=True,
                           text=True).stdout.strip()
 
 
-def build(force=False):
-    """Compile libkda_host_emu.so (skipped when newer than its sources)."""
-    if not force and os.path.exists(LIB) and all(os.path.getmtime(d) <= os.path.getmtime(LIB) for d in _deps()):
-        return LIB
-    os.makedirs(OUT, exist_ok=True)
+def asan_runtime():
+    return sanitizer_runtime("address")
+
+
+def compile_units(units, lib_path, sanitizer="address", src_dir=CSRC):
+    """Compile {file name: C++ text} plus the thread runtime into lib_path."""
+    out = os.path.dirname(lib_path)
+    os.makedirs(out, exist_ok=True)
+    tag = "" if sanitizer == "address" else "." + sanitizer
+    flags = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=" + sanitizer, "-fno-omit-frame-pointer", "-fPIC",
+             "-I", os.path.join(HERE, "fakeinc"), "-I", src_dir, "-I", CSRC, "-Wno-unknown-pragmas", "-c"]
+    objs = []
+    for name, text in units.items():
+        path = os.path.join(out, name)
+        with open(path, "w") as f:
+            f.write(text)
+        objs.append(path[:-4] + tag + ".o")
+        subprocess.run(flags + [path, "-o", objs[-1]], check=True)
+    objs.append(os.path.join(out, "emu_rt%s.o" % tag))
+    subprocess.run(flags + [os.path.join(HERE, "emu_rt.cpp"), "-o", objs[-1]], check=True)
+    tmp = lib_path + ".tmp.%d" % os.getpid()
+    subprocess.run(["g++", "-shared", "-fsanitize=" + sanitizer, "-o", tmp, *objs, "-pthread"], check=True)
+    os.replace(tmp, lib_path)
+    return lib_path
+
+
+def build(force=False, sanitizer="address"):
+    """Compile libkda_host_emu.so (AddressSanitizer) or libkda_host_emu_tsan.so
+    (ThreadSanitizer); skipped when newer than its sources."""
+    lib = LIB if sanitizer == "address" else LIB[:-3] + "_tsan.so"
+    if not force and os.path.exists(lib) and all(os.path.getmtime(d) <= os.path.getmtime(lib) for d in _deps()):
+        return lib
     units = {"emu_fwd.cpp": _unit("kda_chunk_simt.cu", _RUN_FWD),
              "emu_bwd.cpp": _unit("kda_chunk_bwd.cu", _RUN_BWD),
              "emu_step.cpp": _unit("kda_step.cu", _RUN_STEP)}
-    objs = []
-    flags = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address", "-fno-omit-frame-pointer", "-fPIC",
-             "-I", os.path.join(HERE, "fakeinc"), "-I", CSRC, "-Wno-unknown-pragmas", "-c"]
-    for name, text in units.items():
-        path = os.path.join(OUT, name)
-        with open(path, "w") as f:
-            f.write(text)
-        objs.append(path[:-4] + ".o")
-        subprocess.run(flags + [path, "-o", objs[-1]], check=True)
-    objs.append(os.path.join(OUT, "emu_rt.o"))
-    subprocess.run(flags + [os.path.join(HERE, "emu_rt.cpp"), "-o", objs[-1]], check=True)
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    subprocess.run(["g++", "-shared", "-fsanitize=address", "-o", tmp, *objs, "-pthread"], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    if sanitizer != "address":      # the shared-memory poisoning is AddressSanitizer's
+        units = {n: t.replace("#include <sanitizer/asan_interface.h>", "#define ASAN_POISON_MEMORY_REGION(a, b)\n"
+                              "#define ASAN_UNPOISON_MEMORY_REGION(a, b)") for n, t in units.items()}
+    return compile_units(units, lib, sanitizer)
 
 
 if __name__ == "__main__":

@@ -4,6 +4,8 @@ kernels on small seeded problems and compares them with the FP64 oracle.
 TEST INFRASTRUCTURE, started by tests/test_host_emu_cpu.py in a process with
 the AddressSanitizer runtime preloaded.  Prints one line per case and exits
 non-zero on a mismatch (an out-of-bounds access aborts the process first).
+With ``--races LIB`` it runs a few cases through the ThreadSanitizer build
+LIB without the oracle (a data race makes the process exit non-zero).
 """
 import ctypes
 import os
@@ -73,7 +75,7 @@ def _ptr(t):
     return None if t is None or t.numel() == 0 else t.data_ptr()
 
 
-def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed, gate="bounded", per_head=False):
+def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed, gate="bounded", per_head=False, check=True):
     w = workloads.Workload("emu", B=B, T=T, H=H, HV=HV, Dk=Dk, Dv=Dv, chunk=C, dtype=dtype, seed=seed,
                            a_log="uniform", dt_bias_std=0.5, s0_std=0.2)
     inp = workloads.chunk_inputs(w) if flags else workloads.activated_inputs(w)
@@ -104,6 +106,8 @@ def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed, gate="bound
                    _ptr(S_ch), _ptr(dout), _ptr(dS_T), *(_ptr(out[n]) for n in GRADS))
     if lib.emu_chunk_bwd(ctypes.byref(bp), bf16) != 0:
         raise RuntimeError("backward emulation refused the shape")
+    if not check:
+        return {}
     args = [to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")]
     if flags and (gate != "bounded" or per_head):
         # the oracle's forward takes the variant gates precomputed (oracle/gates.py)
@@ -136,7 +140,7 @@ def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed, gate="bound
     return err
 
 
-def run_step_case(lib, B, H, HV, Dk, Dv, dtype, gate, per_head, seed):
+def run_step_case(lib, B, H, HV, Dk, Dv, dtype, gate, per_head, seed, check=True):
     """One decode step against the oracle's step."""
     w = workloads.Workload("emustep", B=B, T=1, H=H, HV=HV, Dk=Dk, Dv=Dv, chunk=1, dtype=dtype, seed=seed,
                            a_log="uniform", dt_bias_std=0.5, s0_std=0.3)
@@ -150,6 +154,8 @@ def run_step_case(lib, B, H, HV, Dk, Dv, dtype, gate, per_head, seed):
                     *(_ptr(x[n]) for n in ("q", "k", "v", "g", "beta")), _ptr(inp["A_log"]),
                     _ptr(inp["dt_bias"]), _ptr(S), _ptr(o))
     lib.emu_step(ctypes.byref(sp), int(dtype == "bf16"))
+    if not check:
+        return {}
     g = _gate_np(to_np(x["g"])[:, None], to_np(inp["A_log"]), to_np(inp["dt_bias"]), gate, per_head, Dk)[:, 0]
     S_ref, o_ref = oracle.kda_step(to_np(inp["S0"]), *(to_np(x[n]) for n in ("q", "k", "v")), g,
                                    to_np(x["beta"]), gate_in=False)
@@ -182,7 +188,22 @@ CASES = [
 ]
 TOL = TOL_F32
 
+def race_run(lib_path):
+    """ThreadSanitizer build: run the kernels (no oracle, one torch thread) so
+    that any report comes from the kernels' own synchronisation."""
+    torch.set_num_threads(1)
+    lib = ctypes.CDLL(lib_path)
+    for case in (CASES[1], CASES[4], CASES[8], CASES[9]):
+        run_case(lib, *case, check=False)
+    for case in STEP_CASES[:2]:
+        run_step_case(lib, *case, check=False)
+    print("race run done", flush=True)
+    return 0
+
+
 if __name__ == "__main__":
+    if len(sys.argv) > 2 and sys.argv[1] == "--races":
+        sys.exit(race_run(sys.argv[2]))
     lib = ctypes.CDLL(os.path.join(HERE, "_build", "libkda_host_emu.so"))
     assert lib.emu_sizeof_chunk_params() == ctypes.sizeof(ChunkParams)
     assert lib.emu_offsetof_withhold_ready() == ChunkParams.withhold_ready.offset
