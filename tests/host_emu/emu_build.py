@@ -1,8 +1,9 @@
 """Host emulation of the library's SIMT kernels -- TEST INFRASTRUCTURE.
 
-Compiles the CUDA sources of the SIMT forward (kda_chunk_simt.cu), the
-backward (kda_chunk_bwd.cu) and the decode step (kda_step.cu) as host C++ with
-g++ and AddressSanitizer: the
+Compiles the CUDA sources of the library's CUDA-core kernels -- the SIMT chunk
+forward (kda_chunk_simt.cu), the backward (kda_chunk_bwd.cu), the decode step
+(kda_step.cu), the segment combine (kda_compose.cu) and the layer prologue and
+epilogue (kda_layer.cu) -- as host C++ with g++ and AddressSanitizer: the
 stand-in headers in fakeinc/ map the CUDA keywords and intrinsics the kernels
 use onto C++, emu_rt.cpp runs every CUDA thread of a block as a std::thread
 (__syncthreads and __syncwarp are std::barriers, a thread that returns drops
@@ -139,9 +140,51 @@ extern "C" int emu_step(kda::StepParams *pp, int bf16) {
 '''
 
 
+_RUN_COMPOSE = _POISON + r'''
+extern "C" int emu_compose(int n_seg, int BH, int Dk, int Dv, const float *M, const float *S_seg,
+                           const float *S_init, float *S_in) {
+    using namespace kda;
+    const size_t bytes = ((size_t)Dk * kVT + (size_t)Dk * Dk) * sizeof(float);
+    if (bytes > sizeof(smem)) return 1;
+    emu_poison(bytes);
+    emu_launch(dim3(BH, (Dv + kVT - 1) / kVT), dim3(kThreads),
+               [&] { compose_kernel(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in); });
+    return 0;
+}
+'''
+_RUN_LAYER = r'''
+extern "C" int emu_sizeof_conv_params(void) { return (int)sizeof(kda::ConvParams); }
+extern "C" int emu_sizeof_gate_params(void) { return (int)sizeof(kda::GateParams); }
+extern "C" int emu_short_conv(kda::ConvParams *pp) {
+    using namespace kda;
+    const ConvParams p = *pp;
+    const long long nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
+    const long long warps = (long long)p.B * (p.C / 128) * nblk;
+    if (warps == 0) return 0;
+    const dim3 grid((unsigned)((warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32)));
+    switch (p.K) {
+        case 1: emu_launch(grid, dim3(kLayerThreads), [&] { short_conv_kernel<1>(p); }); break;
+        case 2: emu_launch(grid, dim3(kLayerThreads), [&] { short_conv_kernel<2>(p); }); break;
+        case 3: emu_launch(grid, dim3(kLayerThreads), [&] { short_conv_kernel<3>(p); }); break;
+        default: emu_launch(grid, dim3(kLayerThreads), [&] { short_conv_kernel<4>(p); }); break;
+    }
+    return 0;
+}
+extern "C" int emu_output_gate(kda::GateParams *pp) {
+    using namespace kda;
+    const GateParams p = *pp;
+    const long long warps = ((long long)p.N * p.HV + kGateRows - 1) / kGateRows;
+    if (warps == 0) return 0;
+    emu_launch(dim3((unsigned)((warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32))), dim3(kLayerThreads),
+               [&] { output_gate_kernel(p); });
+    return 0;
+}
+'''
+
+
 def _deps():
     return [os.path.join(CSRC, f) for f in ("kda_chunk_simt.cu", "kda_chunk_bwd.cu", "kda_step.cu",
-                                            "kda_internal.cuh")] + \
+                                            "kda_compose.cu", "kda_layer.cu", "kda_internal.cuh")] + \
         [os.path.join(HERE, f) for f in ("emu_build.py", "emu_rt.cpp", "fakeinc/cuda_runtime.h", "fakeinc/cuda_bf16.h")] + \
         [os.path.join(ROOT, "include", "kda.h")]
 
@@ -187,7 +230,9 @@ def build(force=False, sanitizer="address"):
         return lib
     units = {"emu_fwd.cpp": _unit("kda_chunk_simt.cu", _RUN_FWD),
              "emu_bwd.cpp": _unit("kda_chunk_bwd.cu", _RUN_BWD),
-             "emu_step.cpp": _unit("kda_step.cu", _RUN_STEP)}
+             "emu_step.cpp": _unit("kda_step.cu", _RUN_STEP),
+             "emu_compose.cpp": _unit("kda_compose.cu", _RUN_COMPOSE),
+             "emu_layer.cpp": _unit("kda_layer.cu", _RUN_LAYER)}
     if sanitizer != "address":      # the shared-memory poisoning is AddressSanitizer's
         units = {n: t.replace("#include <sanitizer/asan_interface.h>", "#define ASAN_POISON_MEMORY_REGION(a, b)\n"
                               "#define ASAN_UNPOISON_MEMORY_REGION(a, b)") for n, t in units.items()}

@@ -10,3 +10,7 @@ inline __nv_bfloat16 __float2bfloat16_rn(float f) {
     u += 0x7FFFu + ((u >> 16) & 1u);
     return __nv_bfloat16{uint16_t(u >> 16)};
 }
+struct __nv_bfloat162 { __nv_bfloat16 x, y; };
+inline __nv_bfloat162 __floats2bfloat162_rn(float a, float b) {
+    return __nv_bfloat162{__float2bfloat16_rn(a), __float2bfloat16_rn(b)};
+}

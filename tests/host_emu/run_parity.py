@@ -48,6 +48,16 @@ class StepParams(ctypes.Structure):        # kda::StepParams
         [(n, _P) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S", "o")]
 
 
+class ConvParams(ctypes.Structure):        # kda::ConvParams
+    _fields_ = [(n, _I) for n in ("B", "T", "C", "K", "head_dim", "silu")] + [("l2_eps", _F)] + \
+        [(n, _P) for n in ("x", "w", "bias", "state_in", "y", "state_out")]
+
+
+class GateParams(ctypes.Structure):        # kda::GateParams
+    _fields_ = [(n, _I) for n in ("N", "HV", "D")] + [("eps", _F)] + \
+        [(n, _P) for n in ("o", "gate", "weight", "y")]
+
+
 GRADS = ("dq", "dk", "dv", "dg", "dbeta", "dS0", "dA_log", "ddt_bias")
 GATE_CODE = {None: 0, "bounded": 1, "softplus": 2}
 
@@ -163,6 +173,58 @@ def run_step_case(lib, B, H, HV, Dk, Dv, dtype, gate, per_head, seed, check=True
     return {"o": max_rel(to_np(o), o_ref) * scale_o, "S": max_rel(to_np(S), S_ref)}
 
 
+def run_compose_case(lib, n_seg, BH, Dk, Dv, with_init, seed):
+    gen = torch.Generator().manual_seed(seed)
+    M = 0.3 * torch.randn((n_seg, BH, Dk, Dk), generator=gen)
+    S_seg = torch.randn((n_seg, BH, Dk, Dv), generator=gen)
+    S_init = torch.randn((BH, Dk, Dv), generator=gen) if with_init else None
+    S_in = torch.full((n_seg + 1, BH, Dk, Dv), float("nan"))
+    lib.emu_compose(n_seg, BH, Dk, Dv, _ptr(M), _ptr(S_seg), _ptr(S_init), _ptr(S_in))
+    ref = oracle.kda_compose(to_np(M), to_np(S_seg), to_np(S_init))
+    return {"S_in": max_rel(to_np(S_in), ref)}
+
+
+def run_layer_case(lib, B, T, C, K, head_dim, silu, with_state, seed):
+    from oracle import layer
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn((B, T, C), generator=gen).to(torch.bfloat16)
+    w = 0.5 * torch.randn((C, K), generator=gen)
+    bias = 0.1 * torch.randn(C, generator=gen)
+    st_in = torch.randn((B, K - 1, C), generator=gen).to(torch.bfloat16) if with_state else None
+    y = torch.zeros((B, T, C), dtype=torch.bfloat16)
+    st_out = torch.zeros((B, K - 1, C), dtype=torch.bfloat16)
+    cp = ConvParams(B, T, C, K, head_dim, int(silu), 1e-6, _ptr(x), _ptr(w), _ptr(bias), _ptr(st_in), _ptr(y),
+                    _ptr(st_out) if K > 1 else None)
+    lib.emu_short_conv(ctypes.byref(cp))
+    y_ref, st_ref = layer.prologue(to_np(x), to_np(w), to_np(bias), to_np(st_in), head_dim=head_dim, act=silu)
+    # bf16 outputs: one rounding, 2^-8 relative, held to 2^-7 of the largest value
+    err = {"y": max_rel(to_np(y), y_ref) * TOL / 2 ** -7}
+    if K > 1:
+        err["state_out"] = max_rel(to_np(st_out), st_ref)   # copied bf16 inputs: exact
+    HV, D = 4, 128
+    o = torch.randn((B * T, HV, D), generator=gen).to(torch.bfloat16)
+    gate = torch.randn((B * T, HV, D), generator=gen).to(torch.bfloat16)
+    wt = 1.0 + 0.1 * torch.randn(D, generator=gen)
+    yo = torch.zeros_like(o)
+    gp = GateParams(B * T, HV, D, 1e-6, _ptr(o), _ptr(gate), _ptr(wt), _ptr(yo))
+    lib.emu_output_gate(ctypes.byref(gp))
+    err["gate"] = max_rel(to_np(yo), layer.output_gate(to_np(o), to_np(gate), to_np(wt))) * TOL / 2 ** -7
+    return err
+
+
+COMPOSE_CASES = [
+    # n_seg, BH, Dk, Dv, with_init, seed
+    (4, 3, 16, 40, True, 21),
+    (3, 2, 128, 128, False, 22),
+    (0, 2, 8, 8, True, 23),
+]
+LAYER_CASES = [
+    # B, T, C, K, head_dim, silu, with_state, seed
+    (2, 100, 256, 4, 128, True, False, 31),
+    (1, 7, 128, 3, 0, False, True, 32),
+    (1, 0, 128, 4, 0, True, True, 33),
+]
+
 STEP_CASES = [
     # B, H, HV, Dk, Dv, dtype, gate, per_head, seed
     (2, 1, 2, 128, 128, "f32", "bounded", False, 11),
@@ -197,6 +259,19 @@ def race_run(lib_path):
         run_case(lib, *case, check=False)
     for case in STEP_CASES[:2]:
         run_step_case(lib, *case, check=False)
+    lib.emu_compose.argtypes = [_I] * 4 + [_P] * 4
+    gen = torch.Generator().manual_seed(5)
+    M, S_seg = torch.randn((3, 2, 16, 16), generator=gen), torch.randn((3, 2, 16, 40), generator=gen)
+    S_in = torch.empty((4, 2, 16, 40))
+    lib.emu_compose(3, 2, 16, 40, _ptr(M), _ptr(S_seg), None, _ptr(S_in))
+    x = torch.randn((1, 70, 256), generator=gen).to(torch.bfloat16)
+    w = torch.randn((256, 4), generator=gen)
+    y, st = torch.empty_like(x), torch.empty((1, 3, 256), dtype=torch.bfloat16)
+    lib.emu_short_conv(ctypes.byref(ConvParams(1, 70, 256, 4, 128, 1, 1e-6, _ptr(x), _ptr(w), None, None,
+                                               _ptr(y), _ptr(st))))
+    o = torch.randn((70, 4, 128), generator=gen).to(torch.bfloat16)
+    yo = torch.empty_like(o)
+    lib.emu_output_gate(ctypes.byref(GateParams(70, 4, 128, 1e-6, _ptr(o), _ptr(o), None, _ptr(yo))))
     print("race run done", flush=True)
     return 0
 
@@ -210,7 +285,17 @@ if __name__ == "__main__":
     assert lib.emu_sizeof_bwd_params() == ctypes.sizeof(BwdParams)
     assert lib.emu_offsetof_ddt_bias() == BwdParams.ddt_bias.offset
     assert lib.emu_sizeof_step_params() == ctypes.sizeof(StepParams)
+    lib.emu_compose.argtypes = [_I] * 4 + [_P] * 4
+    assert lib.emu_sizeof_conv_params() == ctypes.sizeof(ConvParams)
+    assert lib.emu_sizeof_gate_params() == ctypes.sizeof(GateParams)
     bad = 0
+    for name, fn, cases in (("compose", run_compose_case, COMPOSE_CASES), ("layer", run_layer_case, LAYER_CASES)):
+        for case in cases:
+            err = fn(lib, *case)
+            worst = max(err.values())
+            bad += worst > TOL
+            print(name, case, "ok" if worst <= TOL else "MISMATCH",
+                  " ".join("%s=%.1e" % kv for kv in err.items()), flush=True)
     for case in STEP_CASES:
         err = run_step_case(lib, *case)
         worst = max(err.values())

@@ -1,4 +1,5 @@
-"""The SIMT forward (with per-chunk states), backward and decode-step kernels,
+"""The library's CUDA-core kernels (SIMT chunk forward with per-chunk states,
+backward, decode step, segment combine, layer prologue and epilogue),
 compiled for the host by tests/host_emu and run one std::thread per CUDA thread
 under AddressSanitizer against the FP64 oracle (gate variants included), and
 under ThreadSanitizer for data races; two planted probes (CPU only) show that
@@ -24,7 +25,7 @@ def test_simt_kernels_under_host_emulation():
     r = subprocess.run([sys.executable, os.path.join(HERE, "host_emu", "run_parity.py")], env=env,
                        capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-4000:]
-    assert "MISMATCH" not in r.stdout and r.stdout.count(" ok ") == 16, r.stdout
+    assert "MISMATCH" not in r.stdout and r.stdout.count(" ok ") == 22, r.stdout
 
 
 _PROBE = r"""
@@ -93,7 +94,7 @@ def test_harness_reports_a_missing_barrier(tmp_path):
 
 @pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
 def test_simt_kernels_have_no_data_race():
-    """The SIMT forward, backward and decode kernels under ThreadSanitizer."""
+    """The CUDA-core kernels under ThreadSanitizer."""
     import emu_build  # noqa: E402
     lib = emu_build.build(sanitizer="thread")
     env = dict(os.environ, LD_PRELOAD=emu_build.sanitizer_runtime("thread"), TSAN_OPTIONS="halt_on_error=0",
