@@ -22,6 +22,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -84,7 +85,9 @@ class Clocks:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_bench_%d.csv" % os.getpid())
+        # the raw samples; KDA_CLOCKS_DIR keeps them somewhere chosen (default: the temp directory)
+        self.path = os.path.join(os.environ.get("KDA_CLOCKS_DIR", tempfile.gettempdir()),
+                                 "clocks_bench_%d.csv" % os.getpid())
 
     def start(self):
         try:
