@@ -150,3 +150,33 @@ def test_autograd_function_gradients(cuda_device):
     ref = _oracle_grads(inp, True, 1.0)
     for n in leaves:
         assert max_rel(to_np(leaves[n].grad), ref[n]) <= TOL_F32, n
+
+
+def test_backward_gva_workload_sampled(cuda_device):
+    """The full headline shape (B=4, H=16, HV=32, T=8192, Dk=Dv=128, bf16), run
+    whole on the GPU; one q/k head and its two value heads of one batch row are
+    checked against the oracle (per-token gradients and dS0 of those chains)."""
+    w = workloads.workload("gva_bf16")
+    inp = workloads.chunk_inputs(w)
+    gen = torch.Generator().manual_seed(123)
+    dout = torch.randn((w.B, w.T, w.HV, w.Dv), generator=gen).to(torch.bfloat16)
+    d = to_device(inp, cuda_device)
+    d_out = dout.to(cuda_device)
+    S_ch = torch.empty((w.B, w.HV, w.T // w.chunk, w.Dk, w.Dv), device=cuda_device)
+    kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], A_log=d["A_log"], dt_bias=d["dt_bias"],
+                      S0=d["S0"], chunk=w.chunk, S_chunks=S_ch, output_final_state=False)
+    gr = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S_ch, d_out, None,
+                           A_log=d["A_log"], dt_bias=d["dt_bias"], chunk=w.chunk)
+    torch.cuda.synchronize()
+    del S_ch
+    b, h = 1, 5
+    hv = slice(2 * h, 2 * h + 2)                     # the two value heads reading q/k head h
+    sl = {"q": inp["q"][b:b + 1, :, h:h + 1], "k": inp["k"][b:b + 1, :, h:h + 1],
+          "v": inp["v"][b:b + 1, :, hv], "g": inp["g"][b:b + 1, :, hv], "beta": inp["beta"][b:b + 1, :, hv]}
+    ref = backward.kda_backward(*(to_np(sl[n]) for n in ("q", "k", "v", "g", "beta")),
+                                A_log=to_np(inp["A_log"][hv]), dt_bias=to_np(inp["dt_bias"][hv]),
+                                do=to_np(dout[b:b + 1, :, hv]))
+    got = {"q": gr["dq"][b:b + 1, :, h:h + 1], "k": gr["dk"][b:b + 1, :, h:h + 1], "v": gr["dv"][b:b + 1, :, hv],
+           "g": gr["dg"][b:b + 1, :, hv], "beta": gr["dbeta"][b:b + 1, :, hv], "S0": gr["dS0"][b:b + 1, hv]}
+    for n, t in got.items():
+        assert max_rel(to_np(t), ref[n]) <= TOL_F32, n
