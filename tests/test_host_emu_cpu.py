@@ -103,3 +103,16 @@ def test_simt_kernels_have_no_data_race():
                        env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0 and "data race" not in r.stderr, r.stderr[-4000:]
     assert "race run done" in r.stdout
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+def test_autograd_binding_over_the_emulated_kernels():
+    """torch.autograd through kda_chunk, with the library calls served by the
+    host-emulated kernels: gradients of every input equal the oracle's."""
+    import emu_build  # noqa: E402
+    emu_build.build()
+    env = dict(os.environ, LD_PRELOAD=emu_build.asan_runtime(), ASAN_OPTIONS="detect_leaks=0")
+    r = subprocess.run([sys.executable, os.path.join(HERE, "host_emu", "run_autograd.py")], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert r.stdout.count(" ok ") == 2, r.stdout
