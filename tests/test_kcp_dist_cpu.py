@@ -5,7 +5,6 @@ the rerun from the incoming state) runs exactly as on GPUs; the compute steps
 are the FP64 oracle, so every rank's output rows and the final state must
 equal the oracle's single pass over the whole sequence to rounding.
 """
-import json
 import os
 import socket
 import sys

@@ -4,7 +4,6 @@ import json
 import os
 
 import numpy as np
-import pytest
 from scipy.special import expit
 
 import oracle

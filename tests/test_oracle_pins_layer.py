@@ -1,7 +1,6 @@
 """Pins of the layer prologue / epilogue oracle (oracle/layer.py) against what
 the pages and the mathematics fix, each independent of the oracle's own code."""
 import numpy as np
-import pytest
 from scipy.special import expit
 
 from oracle import layer

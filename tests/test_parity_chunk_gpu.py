@@ -5,7 +5,6 @@ max|o| and <= 2e-2 relative Frobenius error of S_T.  The SIMT kernel computes
 in FP32 from the exact inputs, so its fp32 outputs (S_T, M_T) are also held to
 1e-4 when the inputs are bf16.
 """
-import numpy as np
 import pytest
 import torch
 

@@ -1,13 +1,12 @@
 """GPU parity of kda_step (decode) and kda_compose (KCP combine) against the
 FP64 oracle, plus the end-to-end segmented forward."""
-import numpy as np
 import pytest
 import torch
 
 import gated_delta_rule_157_b200 as kda
 import oracle
 import workloads
-from helpers import TOL_BF16, TOL_F32, fro_rel, max_rel, oracle_chunk, to_device, to_np
+from helpers import TOL_BF16, TOL_F32, max_rel, oracle_chunk, to_device, to_np
 
 pytestmark = pytest.mark.gpu
 
