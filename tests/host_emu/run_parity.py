@@ -212,6 +212,30 @@ def run_layer_case(lib, B, T, C, K, head_dim, silu, with_state, seed):
     return err
 
 
+def run_transition_case(lib, B, T, H, HV, Dk, Dv, C, seed):
+    """Forward with the cumulative transition M_T and the chunk states at once
+    (the transition columns ride in extra column slices)."""
+    w = workloads.Workload("emu_m", B=B, T=T, H=H, HV=HV, Dk=Dk, Dv=Dv, chunk=C, dtype="f32", seed=seed,
+                           a_log="uniform", s0_std=0.1)
+    inp = workloads.chunk_inputs(w, z_mean=-3.0)          # slow decay: M_T far from 0
+    o = torch.zeros((B, T, HV, Dv)); S_T = torch.zeros((B, HV, Dk, Dv)); M_T = torch.zeros((B, HV, Dk, Dk))
+    S_ch = torch.zeros((B, HV, -(-T // C), Dk, Dv))
+    fp = ChunkParams(B, T, H, HV, Dk, Dv, C, HV // H, -5.0, 1.0, 1e-6, 1, 1, 1, 0,
+                     *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0")),
+                     _ptr(o), _ptr(S_T), _ptr(M_T), _ptr(S_ch), 0)
+    lib.emu_chunk_fwd(ctypes.byref(fp), 0)
+    ref = oracle.kda_fwd(*(to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")), A_log=to_np(inp["A_log"]),
+                         S0=to_np(inp["S0"]), want_M=True)
+    return {"o": max_rel(to_np(o), ref["o"]), "S_T": max_rel(to_np(S_T), ref["S_T"]),
+            "M_T": max_rel(to_np(M_T), ref["M_T"]), "S_chunks0": max_rel(to_np(S_ch[:, :, 0]), to_np(inp["S0"]))}
+
+
+TRANSITION_CASES = [
+    # B, T, H, HV, Dk, Dv, C, seed
+    (1, 50, 1, 2, 16, 24, 16, 51),
+    (2, 70, 1, 1, 40, 8, 32, 52),
+]
+
 COMPOSE_CASES = [
     # n_seg, BH, Dk, Dv, with_init, seed
     (4, 3, 16, 40, True, 21),
@@ -289,7 +313,8 @@ if __name__ == "__main__":
     assert lib.emu_sizeof_conv_params() == ctypes.sizeof(ConvParams)
     assert lib.emu_sizeof_gate_params() == ctypes.sizeof(GateParams)
     bad = 0
-    for name, fn, cases in (("compose", run_compose_case, COMPOSE_CASES), ("layer", run_layer_case, LAYER_CASES)):
+    for name, fn, cases in (("transition", run_transition_case, TRANSITION_CASES),
+                            ("compose", run_compose_case, COMPOSE_CASES), ("layer", run_layer_case, LAYER_CASES)):
         for case in cases:
             err = fn(lib, *case)
             worst = max(err.values())
