@@ -36,6 +36,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kVT = 32;                       // value columns per CTA
+static_assert(kVT == 32, "the row loops map one lane to one value column");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
 
 template <typename Tin>
@@ -59,6 +60,9 @@ chunk_bwd_kernel(BwdParams p) {
     float *dbet = bet + C;                 // [C]
     float *Glast = dbet + C;               // [Dk]
     float *dlast = Glast + Dk;             // [Dk]  dG terms of the chunk's last row
+    // per-warp row of factors, computed once per row and read by all 32 lanes
+    // (one lane per value column): [warp][2 * 128]
+    float *wb = dlast + Dk + (threadIdx.x >> 5) * 256;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int chain = blockIdx.x;
@@ -159,12 +163,14 @@ chunk_bwd_kernel(BwdParams p) {
             Aqk[r * C + i] = a;
             Pkk[r * C + i] = pk;
         }
-        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
-            const int r = idx / kVT, jj = idx % kVT;
-            float acc = Xs[idx];
-            const float *kr = Ks + r * L, *gr = Gs + r * L;
-            for (int c = 0; c < Dk; ++c) acc = fmaf(-kr[c] * expf(gr[c]), Ss[c * kVT + jj], acc);
-            Xs[idx] = acc;
+        // warp w takes rows w, w + 8, ...; lane = value column
+        for (int r = warp; r < Cc; r += kThreads / 32) {
+            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * expf(Gs[r * L + c]);
+            __syncwarp();
+            float acc = Xs[r * kVT + lane];
+            for (int c = 0; c < Dk; ++c) acc = fmaf(-wb[c], Ss[c * kVT + lane], acc);
+            Xs[r * kVT + lane] = acc;
+            __syncwarp();
         }
         __syncthreads();
         // ---- 4. U = (I + Diag(beta) P)^-1 Diag(beta) X (warp 0); the
@@ -185,13 +191,14 @@ chunk_bwd_kernel(BwdParams p) {
         }
         __syncthreads();
         // ---- 5. dU = A^T dO + (K*exp(G_last - G)) dS' ------------------------
-        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
-            const int r = idx / kVT, jj = idx % kVT;
+        for (int r = warp; r < Cc; r += kThreads / 32) {
+            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * expf(Glast[c] - Gs[r * L + c]);
+            __syncwarp();
             float acc = 0.f;
-            for (int rr = r; rr < Cc; ++rr) acc = fmaf(Aqk[rr * C + r], dOs[rr * kVT + jj], acc);
-            const float *kr = Ks + r * L, *gr = Gs + r * L;
-            for (int c = 0; c < Dk; ++c) acc = fmaf(kr[c] * expf(Glast[c] - gr[c]), dSs[c * kVT + jj], acc);
-            dUs[idx] = acc;
+            for (int rr = r; rr < Cc; ++rr) acc = fmaf(Aqk[rr * C + r], dOs[rr * kVT + lane], acc);
+            for (int c = 0; c < Dk; ++c) acc = fmaf(wb[c], dSs[c * kVT + lane], acc);
+            dUs[r * kVT + lane] = acc;
+            __syncwarp();
         }
         __syncthreads();
         // ---- 6. dZ = (I + Diag(beta) P)^-T dU (warp 0, back substitution) ----
@@ -275,15 +282,21 @@ chunk_bwd_kernel(BwdParams p) {
         }
         __syncthreads();
         // ---- 9. dS entering the chunk (in place) -----------------------------
-        for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
-            const int c = idx / kVT, jj = idx % kVT;
-            float acc = expf(Glast[c]) * dSs[idx];
-            for (int r = 0; r < Cc; ++r) {
+        // warp w takes key channels w, w + 8, ...; lane = value column
+        for (int c = warp; c < Dk; c += kThreads / 32) {
+            for (int r = lane; r < Cc; r += 32) {
                 const float e = expf(Gs[r * L + c]);
-                acc = fmaf(e * Qs[r * L + c], dOs[r * kVT + jj], acc);
-                acc = fmaf(-e * Ks[r * L + c] * bet[r], dUs[r * kVT + jj], acc);
+                wb[r] = e * Qs[r * L + c];
+                wb[128 + r] = -e * Ks[r * L + c] * bet[r];
             }
-            dSs[idx] = acc;
+            __syncwarp();
+            float acc = expf(Glast[c]) * dSs[c * kVT + lane];
+            for (int r = 0; r < Cc; ++r) {
+                acc = fmaf(wb[r], dOs[r * kVT + lane], acc);
+                acc = fmaf(wb[128 + r], dUs[r * kVT + lane], acc);
+            }
+            dSs[c * kVT + lane] = acc;
+            __syncwarp();
         }
         __syncthreads();
 #pragma unroll
@@ -437,7 +450,7 @@ __global__ void bwd_empty_kernel(BwdParams p) {
 
 size_t bwd_smem_bytes(int C, int Dk) {
     const size_t f = (size_t)3 * C * (Dk | 1) + (size_t)2 * C * C + (size_t)4 * C * kVT +
-                     (size_t)2 * Dk * kVT + 2 * C + 2 * Dk;
+                     (size_t)2 * Dk * kVT + 2 * C + 2 * Dk + (size_t)(kThreads / 32) * 256;
     return f * sizeof(float);
 }
 
