@@ -34,7 +34,8 @@
 namespace kda {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;                 // chunk_bwd_kernel: 16 warps, one CTA per SM
+constexpr int kRowThreads = 256;              // bwd_l2norm_kernel
 constexpr int kVT = 32;                       // value columns per CTA
 static_assert(kVT == 32, "the row loops map one lane to one value column");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
@@ -176,10 +177,18 @@ chunk_bwd_kernel(BwdParams p) {
         // ---- 4. U = (I + Diag(beta) P)^-1 Diag(beta) X (warp 0); the
         //         exp(G_last) dS'.S term of the last row's dG (other warps) ----
         if (warp == 0) {
+            // four partial sums shorten the dependent FMA chain of each row
             for (int r = 0; r < Cc; ++r) {
-                float acc = Xs[r * kVT + lane];
-                for (int i = 0; i < r; ++i) acc = fmaf(-Pkk[r * C + i], Us[i * kVT + lane], acc);
-                Us[r * kVT + lane] = bet[r] * acc;
+                float a0 = Xs[r * kVT + lane], a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                int i = 0;
+                for (; i + 3 < r; i += 4) {
+                    a0 = fmaf(-Pkk[r * C + i], Us[i * kVT + lane], a0);
+                    a1 = fmaf(-Pkk[r * C + i + 1], Us[(i + 1) * kVT + lane], a1);
+                    a2 = fmaf(-Pkk[r * C + i + 2], Us[(i + 2) * kVT + lane], a2);
+                    a3 = fmaf(-Pkk[r * C + i + 3], Us[(i + 3) * kVT + lane], a3);
+                }
+                for (; i < r; ++i) a0 = fmaf(-Pkk[r * C + i], Us[i * kVT + lane], a0);
+                Us[r * kVT + lane] = bet[r] * ((a0 + a1) + (a2 + a3));
                 __syncwarp();
             }
         } else {
@@ -204,10 +213,16 @@ chunk_bwd_kernel(BwdParams p) {
         // ---- 6. dZ = (I + Diag(beta) P)^-T dU (warp 0, back substitution) ----
         if (warp == 0) {
             for (int r = Cc - 1; r >= 0; --r) {
-                float acc = dUs[r * kVT + lane];
-                for (int rr = r + 1; rr < Cc; ++rr)
-                    acc = fmaf(-bet[rr] * Pkk[rr * C + r], dUs[rr * kVT + lane], acc);
-                dUs[r * kVT + lane] = acc;
+                float a0 = dUs[r * kVT + lane], a1 = 0.f, a2 = 0.f, a3 = 0.f;
+                int rr = r + 1;
+                for (; rr + 3 < Cc; rr += 4) {
+                    a0 = fmaf(-bet[rr] * Pkk[rr * C + r], dUs[rr * kVT + lane], a0);
+                    a1 = fmaf(-bet[rr + 1] * Pkk[(rr + 1) * C + r], dUs[(rr + 1) * kVT + lane], a1);
+                    a2 = fmaf(-bet[rr + 2] * Pkk[(rr + 2) * C + r], dUs[(rr + 2) * kVT + lane], a2);
+                    a3 = fmaf(-bet[rr + 3] * Pkk[(rr + 3) * C + r], dUs[(rr + 3) * kVT + lane], a3);
+                }
+                for (; rr < Cc; ++rr) a0 = fmaf(-bet[rr] * Pkk[rr * C + r], dUs[rr * kVT + lane], a0);
+                dUs[r * kVT + lane] = (a0 + a1) + (a2 + a3);
                 __syncwarp();
             }
         }
@@ -337,10 +352,10 @@ chunk_bwd_kernel(BwdParams p) {
 
 // dq, dk through q <- q / sqrt(|q|^2 + eps): warp per (token, head) row.
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kRowThreads)
 bwd_l2norm_kernel(BwdParams p) {
     const int lane = threadIdx.x & 31;
-    const long long row = (long long)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const long long row = (long long)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
     const long long rows = (long long)p.B * p.T * p.H;
     if (row >= rows) return;
     const Tin *xs[2] = {static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k)};
@@ -465,7 +480,8 @@ static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.l2norm) {
         const long long rows = (long long)p.B * p.T * p.H;
-        bwd_l2norm_kernel<Tin><<<(unsigned)((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, s>>>(p);
+        bwd_l2norm_kernel<Tin><<<(unsigned)((rows + kRowThreads / 32 - 1) / (kRowThreads / 32)), kRowThreads, 0,
+                                 s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (p.beta_sigmoid || p.gate_in) {

@@ -63,7 +63,7 @@ static void run_bwd(const kda::BwdParams &p) {
     emu_poison(0);
     if (p.l2norm) {
         const long long rows = (long long)p.B * p.T * p.H;
-        emu_launch(dim3((unsigned)((rows + kThreads / 32 - 1) / (kThreads / 32))), dim3(kThreads),
+        emu_launch(dim3((unsigned)((rows + kRowThreads / 32 - 1) / (kRowThreads / 32))), dim3(kRowThreads),
                    [&] { bwd_l2norm_kernel<Tin>(p); });
     }
     if (p.beta_sigmoid || p.gate_in) {
