@@ -353,3 +353,36 @@ def test_bwd_valid_request_without_gpu_reports_cuda_error():
     assert _bwd(_bwd_args()) == 5
     # the parameter gradients are not outputs without the in-kernel gate
     assert _bwd(_bwd_args(gate_in_kernel=0, A_log=None, dA_log=0x7f3000100000)) == 5
+
+
+def test_header_and_library_link_from_plain_c(tmp_path):
+    """A C99 program includes include/kda.h, links libkda_b200.so and calls the
+    entry points that need no device (version, status names, argument checks)."""
+    import subprocess
+    src = tmp_path / "use.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "kda.h"
+int main(void) {
+    kda_chunk_args a;
+    kda_chunk_bwd_args g;
+    memset(&a, 0, sizeof a);
+    memset(&g, 0, sizeof g);
+    if (kda_version() < 100) return 1;
+    if (strcmp(kda_status_string(KDA_ERR_ALIAS), "KDA_ERR_ALIAS") != 0) return 2;
+    if (kda_chunk_fwd(NULL, NULL) != KDA_ERR_INVALID_ARG) return 3;
+    a.H = 1; a.HV = 3;             /* HV % H fine, but sizes zero: invalid */
+    if (kda_chunk_fwd(&a, NULL) != KDA_ERR_INVALID_ARG) return 4;
+    if (kda_chunk_bwd(&g, NULL) != KDA_ERR_INVALID_ARG) return 5;
+    if (kda_compose(-1, 1, 8, 8, NULL, NULL, NULL, NULL, NULL) != KDA_ERR_INVALID_ARG) return 6;
+    puts("c abi ok");
+    return 0;
+}
+""")
+    lib = kda.library_path()
+    exe = tmp_path / "use"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe),
+                    "-L", os.path.dirname(lib), "-lkda_b200", "-Wl,-rpath," + os.path.dirname(lib)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
