@@ -153,9 +153,10 @@ kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
  * (the forward's S0 is S_chunks[.., 0, ..]); dout [B, T, HV, Dv] dtype;
  * dS_T [B, HV, Dk, Dv] fp32 or NULL (zeros).
  * Outputs (fp32, every element written): dq, dk [B, T, H, Dk] (summed over
- * the value heads that share a q/k head); dv [B, T, HV, Dv]; dg [B, T, HV, Dk];
- * dbeta [B, T, HV]; dS0 [B, HV, Dk, Dv] or NULL; dA_log [HV] and ddt_bias
- * [HV, Dk] when gate_in_kernel (else not touched; either may be NULL).
+ * the value heads that share a q/k head); dv [B, T, HV, Dv]; dg [B, T, HV, Dk]
+ * ([B, T, HV] with g_per_head); dbeta [B, T, HV]; dS0 [B, HV, Dk, Dv] or NULL;
+ * dA_log [HV] and ddt_bias [HV, Dk] ([HV] with g_per_head) when gate_in_kernel
+ * (else not touched; either may be NULL).
  *
  * Limits as kda_chunk_fwd (1 <= Dk, Dv <= 128, 1 <= chunk <= 64); algo must be
  * KDA_ALGO_AUTO or KDA_ALGO_SIMT.  Activation pointers aligned to their
