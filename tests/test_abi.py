@@ -386,3 +386,24 @@ int main(void) {
                     "-L", os.path.dirname(lib), "-lkda_b200", "-Wl,-rpath," + os.path.dirname(lib)], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
+
+
+@no_gpu_only
+def test_gate_mode_and_per_head_validation():
+    """gate_in_kernel must be 0, 1 or 2; with g_per_head the gate tensor is
+    [B, T, HV] and dt_bias [HV], and the aliasing checks use those sizes."""
+    assert _fwd(_chunk_args(gate_in_kernel=3)) == INVALID
+    assert _fwd(_chunk_args(gate_in_kernel=-1)) == INVALID
+    assert _bwd(_bwd_args(gate_in_kernel=3)) == INVALID
+    st = _step_args()
+    st.gate_in_kernel = 5
+    assert kda.load().kda_step(ctypes.byref(st), None) == INVALID
+    # the softplus gate on the tensor-core kernel is refused (it needs g >= g_min)
+    a = _chunk_args(gate_in_kernel=2, algo=2)
+    assert _fwd(a) == UNSUPPORTED
+    # per head: an output right after the [B*T*HV] gate tensor does not overlap it,
+    # one inside the per-channel extent of the same tensor would (checked with per head off)
+    base = _chunk_args()
+    g_end_per_head = base.g + 1 * 64 * 4 * 4          # B*T*HV floats
+    assert _fwd(_chunk_args(g_per_head=1, o=g_end_per_head)) == 5      # valid: reaches the launch
+    assert _fwd(_chunk_args(g_per_head=0, o=g_end_per_head)) == ALIAS
