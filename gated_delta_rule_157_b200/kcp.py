@@ -54,13 +54,14 @@ def _group_shape(group):
 
 def kcp_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=64, group=None,
                   g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
-                  beta_sigmoid_in_kernel=True, gate_in_kernel=True, algo="auto", ops=None):
+                  beta_sigmoid_in_kernel=True, gate_in_kernel=True, g_per_head=False, algo="auto", ops=None):
     """Forward of this rank's segment of a sequence split across `group`.
 
     q, k [B,L,H,Dk]; v [B,L,HV,Dv]; g [B,L,HV,Dk]; beta [B,L,HV]: segment
     `rank` of the sequence (segments in rank order, any lengths).  A_log,
     dt_bias and the initial state S0 [B,HV,Dk,Dv] (or None) are the same on
-    every rank.  Returns (o [B,L,HV,Dv] of this segment, S_T [B,HV,Dk,Dv] of
+    every rank.  gate_in_kernel and g_per_head as kda_chunk_fwd (g [B,L,HV]
+    with g_per_head).  Returns (o [B,L,HV,Dv] of this segment, S_T [B,HV,Dk,Dv] of
     the whole sequence).  Every rank must call this collectively.
     """
     ops = ops or _KernelOps
@@ -69,7 +70,7 @@ def kcp_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     HV, Dv = v.shape[2], v.shape[3]
     kw = dict(A_log=A_log, dt_bias=dt_bias, chunk=chunk, g_min=g_min, scale=scale, l2_eps=l2_eps,
               qk_l2norm_in_kernel=qk_l2norm_in_kernel, beta_sigmoid_in_kernel=beta_sigmoid_in_kernel,
-              gate_in_kernel=gate_in_kernel, algo=algo)
+              gate_in_kernel=gate_in_kernel, g_per_head=g_per_head, algo=algo)
     # 1. this segment from the zero state
     _, S_seg, M_seg = ops.forward(q, k, v, g, beta, None, True, **kw)
     # 2. exchange: [world, B*HV, Dk, Dk] and [world, B*HV, Dk, Dv]
