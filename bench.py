@@ -1,6 +1,6 @@
 """Benchmark of the KDA core on B200.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--train]
 
 One step = one kda_chunk_fwd over the grouped-value-head training-shape
 workload (B=4, H=16, HV=32, T=8192, Dk=Dv=128, chunk=64, bf16 activations,
@@ -11,6 +11,9 @@ Python API with host buffers, the decode step (B=256, H=HV=32, D=128, fp32
 state, 512 consecutive steps) in GB/s, the segmented KCP pass, the layer
 prologue / epilogue kernels in GB/s, and the FP64 oracle timed on the host
 cores as a reported baseline.
+
+--train adds the training path (forward keeping the per-chunk states, then
+kda_chunk_bwd) at the same workload, each timed on the device.
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload (weak
 scaling, no collective on the data path); the time is the max over ranks.
