@@ -1,9 +1,11 @@
 """Host emulation of the library's SIMT kernels -- TEST INFRASTRUCTURE.
 
-Compiles the CUDA sources of the library's CUDA-core kernels -- the SIMT chunk
-forward (kda_chunk_simt.cu), the backward (kda_chunk_bwd.cu), the decode step
-(kda_step.cu), the segment combine (kda_compose.cu) and the layer prologue and
-epilogue (kda_layer.cu) -- as host C++ with g++ and AddressSanitizer: the
+Compiles the CUDA sources of the library's kernels -- the SIMT chunk forward
+(kda_chunk_simt.cu), the backward (kda_chunk_bwd.cu), the decode step
+(kda_step.cu), the segment combine (kda_compose.cu), the layer prologue and
+epilogue (kda_layer.cu) and the tensor-core chunk kernel (kda_chunk_tc.cu,
+against tcinc/tc_ptx.cuh, a host model of the tcgen05 / TMA / mbarrier
+instructions it uses) -- as host C++ with g++ and AddressSanitizer: the
 stand-in headers in fakeinc/ map the CUDA keywords and intrinsics the kernels
 use onto C++, emu_rt.cpp runs every CUDA thread of a block as a std::thread
 (__syncthreads and __syncwarp are std::barriers, a thread that returns drops
@@ -89,6 +91,65 @@ extern "C" int emu_chunk_bwd(kda::BwdParams *pp, int bf16) {
     return 0;
 }
 '''
+
+
+_RUN_TC = r'''
+#include <sanitizer/asan_interface.h>
+namespace kda { namespace tc { EmuCta *g_cta = nullptr; EmuTf32Slots g_tf32[32]; } }
+
+// The tensor maps the library's launcher builds (tokens x heads x 128 channels,
+// [64][1][128] boxes; v in two [64][1][64] boxes with the 128-byte swizzle).
+static kda::tc::EmuTensorMap emu_row_map(const void *base, int heads, long long rows, bool sw128) {
+    kda::tc::EmuTensorMap m{};
+    m.base = static_cast<const uint8_t *>(base);
+    m.dims[0] = 128; m.dims[1] = (uint64_t)heads; m.dims[2] = (uint64_t)rows;
+    m.strides[0] = 128 * 2; m.strides[1] = (uint64_t)heads * 128 * 2;
+    m.box[0] = sw128 ? 64 : 128; m.box[1] = 1; m.box[2] = 64;
+    m.swizzle128 = sw128 ? 1 : 0;
+    return m;
+}
+
+extern "C" int emu_chunk_tc(kda::ChunkParams *pp) {
+    using namespace kda;
+    TcParams tp;
+    tp.p = *pp;
+    const long long rows = (long long)tp.p.B * tp.p.T;
+    const tc::EmuTensorMap maps[4] = {emu_row_map(tp.p.q, tp.p.H, rows, false), emu_row_map(tp.p.k, tp.p.H, rows, false),
+                                      emu_row_map(tp.p.g, tp.p.HV, rows, false),
+                                      emu_row_map(tp.p.v, tp.p.HV, rows, true)};
+    for (int i = 0; i < 4; ++i) std::memcpy(&tp.tm[i], &maps[i], sizeof maps[i]);
+    static tc::EmuCta cta;
+    static tc::EmuMBar bars[sizeof smem_raw / 8];
+    cta.smem = smem_raw;
+    cta.smem_bytes = SMEM_BYTES;
+    cta.bars = bars;
+    g_device_error = 0;
+    emu_launch_cb(dim3(tp.p.B * tp.p.HV, tp.p.M_T ? 2 : 1), dim3(kThreads),
+                  [&](unsigned, unsigned) {
+                      ASAN_UNPOISON_MEMORY_REGION(smem_raw, sizeof smem_raw);
+                      std::memset(cta.tmem, 0, sizeof cta.tmem);
+                      std::memset(smem_raw, 0, sizeof smem_raw);
+                      ASAN_POISON_MEMORY_REGION(smem_raw + SMEM_BYTES, sizeof smem_raw - SMEM_BYTES);
+                      tc::g_cta = &cta;
+                  },
+                  [&] { chunk_tc_kernel(tp); });
+    return g_device_error ? 2 : 0;
+}
+'''
+
+
+def _tc_unit(runner=_RUN_TC):
+    """The tensor-core chunk kernel against the host model of its PTX wrappers
+    (tcinc/tc_ptx.cuh, found before the library's own): the source up to its
+    host functions, the 240 KB shared array, and the runner above."""
+    s = open(os.path.join(CSRC, "kda_chunk_tc.cu")).read()
+    s = s[: s.index("bool chunk_tc_supported")] + "}  // namespace kda\n"
+    s = s.replace("extern __shared__", "extern").replace("__shared__", "static")
+    head = ('#include <functional>\n#include "cuda_runtime.h"\n'
+            "void emu_launch_cb(dim3 grid, dim3 block, const std::function<void(unsigned, unsigned)> &on_block,\n"
+            "                   const std::function<void()> &fn);\n"
+            "namespace kda { namespace { alignas(1024) uint8_t smem_raw[240 * 1024]; } }\n")
+    return head + '#line 1 "kda_chunk_tc.cu"\n' + s + runner
 
 
 def unit_from_text(text, runner, poison=True):
@@ -184,8 +245,10 @@ extern "C" int emu_output_gate(kda::GateParams *pp) {
 
 def _deps():
     return [os.path.join(CSRC, f) for f in ("kda_chunk_simt.cu", "kda_chunk_bwd.cu", "kda_step.cu",
-                                            "kda_compose.cu", "kda_layer.cu", "kda_internal.cuh")] + \
-        [os.path.join(HERE, f) for f in ("emu_build.py", "emu_rt.cpp", "fakeinc/cuda_runtime.h", "fakeinc/cuda_bf16.h")] + \
+                                            "kda_compose.cu", "kda_layer.cu", "kda_chunk_tc.cu",
+                                            "kda_internal.cuh")] + \
+        [os.path.join(HERE, f) for f in ("emu_build.py", "emu_rt.cpp", "fakeinc/cuda_runtime.h", "fakeinc/cuda_bf16.h",
+                                         "fakeinc/cuda.h", "tcinc/tc_ptx.cuh")] + \
         [os.path.join(ROOT, "include", "kda.h")]
 
 
@@ -206,7 +269,8 @@ def compile_units(units, lib_path, sanitizer="address", src_dir=CSRC):
     os.makedirs(out, exist_ok=True)
     tag = "" if sanitizer == "address" else "." + sanitizer
     flags = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=" + sanitizer, "-fno-omit-frame-pointer", "-fPIC",
-             "-I", os.path.join(HERE, "fakeinc"), "-I", src_dir, "-I", CSRC, "-Wno-unknown-pragmas", "-c"]
+             "-I", os.path.join(HERE, "fakeinc"), "-I", os.path.join(HERE, "tcinc"), "-I", src_dir, "-I", CSRC,
+             "-Wno-unknown-pragmas", "-c"]
     objs = []
     for name, text in units.items():
         path = os.path.join(out, name)
@@ -232,7 +296,8 @@ def build(force=False, sanitizer="address"):
              "emu_bwd.cpp": _unit("kda_chunk_bwd.cu", _RUN_BWD),
              "emu_step.cpp": _unit("kda_step.cu", _RUN_STEP),
              "emu_compose.cpp": _unit("kda_compose.cu", _RUN_COMPOSE),
-             "emu_layer.cpp": _unit("kda_layer.cu", _RUN_LAYER)}
+             "emu_layer.cpp": _unit("kda_layer.cu", _RUN_LAYER),
+             "emu_tc.cpp": _tc_unit()}
     if sanitizer != "address":      # the shared-memory poisoning is AddressSanitizer's
         units = {n: t.replace("#include <sanitizer/asan_interface.h>", "#define ASAN_POISON_MEMORY_REGION(a, b)\n"
                               "#define ASAN_UNPOISON_MEMORY_REGION(a, b)") for n, t in units.items()}

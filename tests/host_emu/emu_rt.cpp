@@ -29,11 +29,19 @@ float __shfl_xor_sync(unsigned, float v, int off) {
     return r;
 }
 
-// Runs fn(block) on every thread of every block of the grid, blocks in order.
+// Runs fn(block) on every thread of every block of the grid, blocks in order;
+// on_block(bx, by) runs before each block's threads start.
+void emu_launch_cb(dim3 grid, dim3 block, const std::function<void(unsigned, unsigned)> &on_block,
+                   const std::function<void()> &fn);
 void emu_launch(dim3 grid, dim3 block, const std::function<void()> &fn) {
+    emu_launch_cb(grid, block, [](unsigned, unsigned) {}, fn);
+}
+void emu_launch_cb(dim3 grid, dim3 block, const std::function<void(unsigned, unsigned)> &on_block,
+                   const std::function<void()> &fn) {
     const unsigned nt = block.x;
     for (unsigned by = 0; by < grid.y; ++by)
         for (unsigned bx = 0; bx < grid.x; ++bx) {
+            on_block(bx, by);
             g_block = std::make_unique<std::barrier<>>(nt);
             g_warp.clear();
             for (unsigned w = 0; w < (nt + 31) / 32; ++w)

@@ -14,3 +14,8 @@ struct __nv_bfloat162 { __nv_bfloat16 x, y; };
 inline __nv_bfloat162 __floats2bfloat162_rn(float a, float b) {
     return __nv_bfloat162{__float2bfloat16_rn(a), __float2bfloat16_rn(b)};
 }
+inline float __bfloat162float_(uint16_t b) { uint32_t u = uint32_t(b) << 16; float f; std::memcpy(&f, &u, 4); return f; }
+inline __nv_bfloat162 __hmul2(__nv_bfloat162 a, __nv_bfloat162 b) {
+    return __nv_bfloat162{__float2bfloat16_rn(__bfloat162float_(a.x.x) * __bfloat162float_(b.x.x)),
+                          __float2bfloat16_rn(__bfloat162float_(a.y.x) * __bfloat162float_(b.y.x))};
+}

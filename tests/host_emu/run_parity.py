@@ -236,6 +236,38 @@ TRANSITION_CASES = [
     (2, 70, 1, 1, 40, 8, 32, 52),
 ]
 
+def run_tc_case(lib, B, T, H, HV, want_M, s0, z_mean, seed):
+    """The tensor-core chunk kernel (bf16, Dk = Dv = 128, C = 64) over the host
+    model of its instructions, against the oracle at the bf16 bars (o: 2e-2 of
+    max|o|; S_T, M_T: 2e-2 Frobenius), each rescaled to TOL."""
+    from helpers import fro_rel
+    w = workloads.Workload("emu_tc", B=B, T=T, H=H, HV=HV, Dk=128, Dv=128, chunk=64, dtype="bf16", seed=seed,
+                           a_log="uniform", dt_bias_std=0.5, s0_std=s0)
+    inp = workloads.chunk_inputs(w, z_mean=z_mean)
+    o = torch.zeros((B, T, HV, 128), dtype=torch.bfloat16)
+    S_T = torch.zeros((B, HV, 128, 128))
+    M_T = torch.zeros((B, HV, 128, 128)) if want_M else None
+    fp = ChunkParams(B, T, H, HV, 128, 128, 64, HV // H, -5.0, 1.0, 1e-6, 1, 1, 1, 0,
+                     *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0")),
+                     _ptr(o), _ptr(S_T), _ptr(M_T), None, 0)
+    if lib.emu_chunk_tc(ctypes.byref(fp)) != 0:
+        return {"device_error": 1.0}
+    ref = oracle.kda_fwd(*(to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")), A_log=to_np(inp["A_log"]),
+                         dt_bias=to_np(inp["dt_bias"]), S0=to_np(inp["S0"]), want_M=want_M)
+    k = TOL / TOL_BF16
+    err = {"o": max_rel(to_np(o), ref["o"]) * k, "S_T": fro_rel(to_np(S_T), ref["S_T"]) * k}
+    if want_M:
+        err["M_T"] = fro_rel(to_np(M_T), ref["M_T"]) * k
+    return err
+
+
+TC_CASES = [
+    # B, T, H, HV, want_M, s0, z_mean, seed
+    (1, 64, 1, 1, False, None, 0.0, 95),       # one chunk
+    (1, 192, 1, 2, False, 0.02, 0.0, 223),     # three chunks, carried state
+    (1, 256, 1, 2, True, 0.05, -8.0, 287),     # slow decay, with the transition CTAs
+]
+
 COMPOSE_CASES = [
     # n_seg, BH, Dk, Dv, with_init, seed
     (4, 3, 16, 40, True, 21),
@@ -283,6 +315,17 @@ def race_run(lib_path):
         run_case(lib, *case, check=False)
     for case in STEP_CASES[:2]:
         run_step_case(lib, *case, check=False)
+    for case in TC_CASES[:2]:
+        B, T, H, HV, want_M, s0, z_mean, seed = case
+        w = workloads.Workload("race_tc", B=B, T=T, H=H, HV=HV, Dk=128, Dv=128, chunk=64, dtype="bf16", seed=seed,
+                               a_log="uniform", dt_bias_std=0.5, s0_std=s0)
+        inp = workloads.chunk_inputs(w, z_mean=z_mean)
+        o = torch.zeros((B, T, HV, 128), dtype=torch.bfloat16)
+        S_T = torch.zeros((B, HV, 128, 128))
+        fp = ChunkParams(B, T, H, HV, 128, 128, 64, HV // H, -5.0, 1.0, 1e-6, 1, 1, 1, 0,
+                         *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0")),
+                         _ptr(o), _ptr(S_T), None, None, 0)
+        lib.emu_chunk_tc(ctypes.byref(fp))
     lib.emu_compose.argtypes = [_I] * 4 + [_P] * 4
     gen = torch.Generator().manual_seed(5)
     M, S_seg = torch.randn((3, 2, 16, 16), generator=gen), torch.randn((3, 2, 16, 40), generator=gen)
@@ -313,7 +356,7 @@ if __name__ == "__main__":
     assert lib.emu_sizeof_conv_params() == ctypes.sizeof(ConvParams)
     assert lib.emu_sizeof_gate_params() == ctypes.sizeof(GateParams)
     bad = 0
-    for name, fn, cases in (("transition", run_transition_case, TRANSITION_CASES),
+    for name, fn, cases in (("tc", run_tc_case, TC_CASES), ("transition", run_transition_case, TRANSITION_CASES),
                             ("compose", run_compose_case, COMPOSE_CASES), ("layer", run_layer_case, LAYER_CASES)):
         for case in cases:
             err = fn(lib, *case)

@@ -1,6 +1,7 @@
-"""The library's CUDA-core kernels (SIMT chunk forward with per-chunk states,
-backward, decode step, segment combine, layer prologue and epilogue),
-compiled for the host by tests/host_emu and run one std::thread per CUDA thread
+"""The library's kernels (SIMT chunk forward with per-chunk states, backward,
+decode step, segment combine, layer prologue and epilogue, and the tcgen05
+chunk kernel over a host model of its instructions), compiled for the host by
+tests/host_emu and run one std::thread per CUDA thread
 under AddressSanitizer against the FP64 oracle (gate variants included), and
 under ThreadSanitizer for data races; two planted probes (CPU only) show that
 the harness reports a shared-memory overrun and a missing barrier.  No GPU: this checks the kernels'
@@ -25,7 +26,7 @@ def test_simt_kernels_under_host_emulation():
     r = subprocess.run([sys.executable, os.path.join(HERE, "host_emu", "run_parity.py")], env=env,
                        capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-4000:]
-    assert "MISMATCH" not in r.stdout and r.stdout.count(" ok ") == 24, r.stdout
+    assert "MISMATCH" not in r.stdout and r.stdout.count(" ok ") == 27, r.stdout
 
 
 _PROBE = r"""
