@@ -200,10 +200,10 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     beta (or logits) [B,T,HV] -- all float32 or all bfloat16, on one CUDA device.
     A_log [HV], dt_bias [HV,Dk], S0 [B,HV,Dk,Dv]: float32.
     S_chunks: optional float32 [B,HV,ceil(T/chunk),Dk,Dv] that receives the
-    state entering every chunk (the input of kda_chunk_bwd; SIMT kernel only).
+    state entering every chunk (the input of kda_chunk_bwd).
     gate_in_kernel: True or "bounded" (g_min sigmoid gate), "softplus"
     (-exp(A_log) softplus gate, SIMT only) or False.  g_per_head: g [B,T,HV]
-    and dt_bias [HV], one decay per (token, value head) (SIMT only).
+    and dt_bias [HV], one decay per (token, value head).
     """
     lib = load()
     if not isinstance(q, torch.Tensor) or not q.is_cuda:

@@ -103,11 +103,9 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
 
     if (a->T == 0) return cuda_status(kda::launch_chunk_empty(p, s));
 
-    // Only the SIMT kernel writes the per-chunk states and takes the softplus
-    // gate (unbounded: the tensor-core exponent scheme needs g >= g_min) or
-    // one gate value per head.
-    const bool tc_ok = kda::chunk_tc_supported(p, bf16) && !a->S_chunks && a->gate_in_kernel <= 1 &&
-                       !a->g_per_head;
+    // Only the SIMT kernel takes the softplus gate (unbounded: the tensor-core
+    // exponent scheme needs g >= g_min).
+    const bool tc_ok = kda::chunk_tc_supported(p, bf16) && a->gate_in_kernel <= 1;
     if (withhold_ready && (a->algo != KDA_ALGO_TC || !tc_ok)) return KDA_ERR_UNSUPPORTED;
     if (a->algo == KDA_ALGO_TC) {
         if (!tc_ok) return KDA_ERR_UNSUPPORTED;

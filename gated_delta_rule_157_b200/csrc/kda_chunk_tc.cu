@@ -252,7 +252,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
     float B1[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-        B1[u] = (p.gate_in && p.dt_bias) ? p.dt_bias[(size_t)x.hv * D + c0 + u] * A1 : 0.f;
+        B1[u] = (p.gate_in && p.dt_bias) ? p.dt_bias[p.g_per_head ? (size_t)x.hv : (size_t)x.hv * D + c0 + u] * A1
+                                         : 0.f;
     const float gmin2 = p.g_min * kLog2e;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t ph_mma = 0;
@@ -269,8 +270,12 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         const int row0 = x.b * x.T + mc * C;
         if (zv) {
             const uint32_t bar = bar_addr(x, MB_LZV);
-            mbar_arrive_expect_tx(bar, (uint32_t)(C * D * 2));
-            tma_load_3d(x.sbase + OFF_STAGE_Z, &tmaps[2], 0, x.hv, row0, bar);
+            if (p.g_per_head) {          // one gate value per token: read directly by read_z
+                mbar_arrive(bar);
+            } else {
+                mbar_arrive_expect_tx(bar, (uint32_t)(C * D * 2));
+                tma_load_3d(x.sbase + OFF_STAGE_Z, &tmaps[2], 0, x.hv, row0, bar);
+            }
         } else {
             const uint32_t bar = bar_addr(x, MB_LQK);
             mbar_arrive_expect_tx(bar, (uint32_t)(2 * C * D * 2));
@@ -289,7 +294,17 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         tma_load_3d(x.sbase + OFF_VT + 8192u, &tmaps[3], 64, x.hv, row0, bar);
     };
     uint2 qw[4], kw[4], zw[4];
-    auto read_z = [&](int lCc) {
+    auto read_z = [&](int mc, int lCc) {
+        if (p.g_per_head) {              // the token's one value, in all four channel slots
+            const uint16_t *gz = static_cast<const uint16_t *>(p.g);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = tq + i;
+                const uint32_t bits = t < lCc ? gz[((size_t)x.b * x.T + (size_t)mc * C + t) * p.HV + x.hv] : 0u;
+                zw[i] = make_uint2(bits | (bits << 16), bits | (bits << 16));
+            }
+            return;
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = tq + i;
@@ -312,7 +327,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
     int v_issued = 0;                      // chunks whose V tile was requested
     int mi_issued = 0;                     // chunks whose MMA (I) was issued (by this thread)
     if (tid == kPrepThreads - 32)
-        for (int i = 0; i < 4; ++i) prefetch_tensormap(&tmaps[i]);
+        for (int i = 0; i < 4; ++i)
+            if (i != 2 || !p.g_per_head) prefetch_tensormap(&tmaps[i]);
     if (x.nchunks > 0) {
         issue_rows(0, true);
         issue_rows(0, false);
@@ -385,7 +401,7 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
         // The z rows (requested after the previous chunk's solve) arrive while
         // the norms are computed.
         const bool ok_zv = wait_bar(x, bar_addr(x, MB_LZV), (uint32_t)(m & 1));
-        read_z(Cc);
+        read_z(m, Cc);
         float g2[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -825,10 +841,17 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
                                 id_iv, (x.trans && s == 0) ? 0u : 1u);
             mma_commit(bar_addr(x, MB_MMA_S));
         }
-        // Meanwhile: S^T <- S^T Diag(gamma_C) (fp32, in TMEM).
+        // Meanwhile: S^T <- S^T Diag(gamma_C) (fp32, in TMEM); the state entering
+        // this chunk goes to S_chunks first when it is asked for.
+        float *sck = (p.S_chunks && !x.trans) ? p.S_chunks + ((size_t)x.chain * x.nchunks + n) * D * D + j
+                                              : nullptr;
         for (int mm = 0; mm < D / 16; ++mm) {
             float vals[16];
             tmem_ld16(x.tm + lane_base + COL_ST + mm * 16, vals);
+            if (sck) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) sck[(size_t)(mm * 16 + u) * D] = vals[u];
+            }
             const float4 *g4 = reinterpret_cast<const float4 *>(gam_s + buf * D + mm * 16);
 #pragma unroll
             for (int u4 = 0; u4 < 4; ++u4) {
@@ -1025,7 +1048,8 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s) {
     const long long rows = (long long)p.B * p.T;
     if ((e = make_row_map(&tp.tm[0], p.q, p.H, rows)) != cudaSuccess) return e;
     if ((e = make_row_map(&tp.tm[1], p.k, p.H, rows)) != cudaSuccess) return e;
-    if ((e = make_row_map(&tp.tm[2], p.g, p.HV, rows)) != cudaSuccess) return e;
+    if (p.g_per_head) memset(&tp.tm[2], 0, sizeof(tp.tm[2]));      // z is read directly
+    else if ((e = make_row_map(&tp.tm[2], p.g, p.HV, rows)) != cudaSuccess) return e;
     if ((e = make_row_map(&tp.tm[3], p.v, p.HV, rows, /*swizzle128=*/true)) != cudaSuccess) return e;
     dim3 grid(p.B * p.HV, p.M_T ? 2 : 1);
     chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tp);

@@ -24,7 +24,7 @@
  *     gate_in_kernel = 0:     g is the log-decay itself.
  * With g_per_head set, g holds one value per (token, value head), shared by
  * the Dk key channels (the Gated DeltaNet form, page "线性注意力交互式演示"
- * Eq. 6), and dt_bias one value per value head (SIMT kernels only).
+ * Eq. 6), and dt_bias one value per value head.
  *
  * Value head hv reads q/k head h = hv / (HV / H) (contiguous groups).
  *
@@ -103,15 +103,15 @@ typedef enum {
  *   M_T     [B, HV, Dk, Dk] fp32 output, or NULL
  *   S_chunks [B, HV, NC, Dk, Dv] fp32 output, or NULL: the state entering each
  *           of the NC = ceil(T / chunk) chunks (S_chunks[.., 0, ..] = S0); the
- *           input kda_chunk_bwd needs.  Only KDA_ALGO_SIMT writes it: with
- *           S_chunks set, KDA_ALGO_AUTO runs the SIMT kernel and KDA_ALGO_TC
- *           returns KDA_ERR_UNSUPPORTED.
+ *           input kda_chunk_bwd needs.  Both kernels write it: the SIMT kernel
+ *           its fp32 state, the tensor-core kernel the fp32 state it carries
+ *           between its bf16 MMAs (bf16-path accuracy).
  *
  * Limits: B, T >= 0; 1 <= H <= HV, HV % H == 0; 1 <= Dk, Dv <= 128;
  * 1 <= chunk <= 64.  q, k, v, g, beta, o must be aligned to their element size;
  * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64,
- * gate_in_kernel 0 or 1 with one gate value per key channel, and 16-byte
- * aligned q, k, v, g, o (KDA_ALGO_AUTO takes the SIMT kernel otherwise).
+ * gate_in_kernel 0 or 1 (the bounded gate), and 16-byte aligned q, k, v, g, o
+ * (KDA_ALGO_AUTO takes the SIMT kernel otherwise).
  * gate_in_kernel must be 0, 1 or 2.  o must not overlap any input; S_T, M_T and
  * S_chunks must not overlap each other, o, or any input except S_T == S0.
  * T == 0 writes S_T = S0 (or 0) and M_T = I.

@@ -236,28 +236,43 @@ TRANSITION_CASES = [
     (2, 70, 1, 1, 40, 8, 32, 52),
 ]
 
-def run_tc_case(lib, B, T, H, HV, want_M, s0, z_mean, seed):
+def run_tc_case(lib, B, T, H, HV, want_M, s0, z_mean, seed, per_head=False, states=False):
     """The tensor-core chunk kernel (bf16, Dk = Dv = 128, C = 64) over the host
     model of its instructions, against the oracle at the bf16 bars (o: 2e-2 of
-    max|o|; S_T, M_T: 2e-2 Frobenius), each rescaled to TOL."""
+    max|o|; S_T, M_T, chunk states: 2e-2 Frobenius), each rescaled to TOL."""
     from helpers import fro_rel
     w = workloads.Workload("emu_tc", B=B, T=T, H=H, HV=HV, Dk=128, Dv=128, chunk=64, dtype="bf16", seed=seed,
                            a_log="uniform", dt_bias_std=0.5, s0_std=s0)
     inp = workloads.chunk_inputs(w, z_mean=z_mean)
+    if per_head:
+        inp = _per_head(inp)
     o = torch.zeros((B, T, HV, 128), dtype=torch.bfloat16)
     S_T = torch.zeros((B, HV, 128, 128))
     M_T = torch.zeros((B, HV, 128, 128)) if want_M else None
-    fp = ChunkParams(B, T, H, HV, 128, 128, 64, HV // H, -5.0, 1.0, 1e-6, 1, 1, 1, 0,
+    NC = -(-T // 64)
+    S_ch = torch.full((B, HV, NC, 128, 128), float("nan")) if states else None
+    fp = ChunkParams(B, T, H, HV, 128, 128, 64, HV // H, -5.0, 1.0, 1e-6, 1, 1, 1, int(per_head),
                      *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0")),
-                     _ptr(o), _ptr(S_T), _ptr(M_T), None, 0)
+                     _ptr(o), _ptr(S_T), _ptr(M_T), _ptr(S_ch), 0)
     if lib.emu_chunk_tc(ctypes.byref(fp)) != 0:
         return {"device_error": 1.0}
-    ref = oracle.kda_fwd(*(to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")), A_log=to_np(inp["A_log"]),
-                         dt_bias=to_np(inp["dt_bias"]), S0=to_np(inp["S0"]), want_M=want_M)
+    args = [to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")]
+    if per_head:
+        args[3] = _gate_np(args[3], to_np(inp["A_log"]), to_np(inp["dt_bias"]), "bounded", True, 128)
+        kw = dict(S0=to_np(inp["S0"]), gate_in=False)
+    else:
+        kw = dict(A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]), S0=to_np(inp["S0"]))
+    ref = oracle.kda_fwd(*args, want_M=want_M, **kw)
     k = TOL / TOL_BF16
     err = {"o": max_rel(to_np(o), ref["o"]) * k, "S_T": fro_rel(to_np(S_T), ref["S_T"]) * k}
     if want_M:
         err["M_T"] = fro_rel(to_np(M_T), ref["M_T"]) * k
+    if states:
+        worst = fro_rel(to_np(S_ch[:, :, 0]), to_np(inp["S0"]) if inp["S0"] is not None else np.zeros((B, HV, 128, 128)))
+        for c in range(1, NC):
+            pre = oracle.kda_fwd(*(a[:, : c * 64] for a in args), **kw)["S_T"]
+            worst = max(worst, fro_rel(to_np(S_ch[:, :, c]), pre))
+        err["S_chunks"] = worst * k
     return err
 
 
@@ -266,6 +281,8 @@ TC_CASES = [
     (1, 64, 1, 1, False, None, 0.0, 95),       # one chunk
     (1, 192, 1, 2, False, 0.02, 0.0, 223),     # three chunks, carried state
     (1, 256, 1, 2, True, 0.05, -8.0, 287),     # slow decay, with the transition CTAs
+    (1, 200, 1, 2, False, 0.05, 0.0, 5, False, True),   # chunk states written
+    (1, 130, 2, 4, False, 0.05, 0.0, 6, True, False),   # one decay per (token, head)
 ]
 
 COMPOSE_CASES = [

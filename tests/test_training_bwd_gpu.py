@@ -77,17 +77,29 @@ def test_chunk_states_are_the_prefix_states(cuda_device, shape):
         assert max_rel(S_ch[:, :, c], ref) <= TOL_F32, c
 
 
-def test_auto_with_chunk_states_takes_the_simt_kernel(cuda_device):
-    """A shape the tensor-core kernel takes runs on the SIMT kernel once the
-    per-chunk states are asked for (the tensor-core kernel does not write them)."""
-    w, inp = _inputs(1, 128, 1, 1, 128, 128, 64, "bf16", seed=22)
+def test_tensor_core_kernel_writes_chunk_states(cuda_device):
+    """The tensor-core kernel (which AUTO takes for this shape) writes the state
+    entering each chunk: keeping the states changes neither o nor S_T, and the
+    states are the prefix states within the bf16 bar."""
+    from helpers import TOL_BF16, fro_rel
+    w, inp = _inputs(1, 200, 1, 2, 128, 128, 64, "bf16", seed=22, s0=0.05)
     d = to_device(inp, cuda_device)
     a = _forward_with_states(d, w, True, 1.0, algo="auto")
-    b = _forward_with_states(d, w, True, 1.0, algo="simt")
+    b = _forward_with_states(d, w, True, 1.0, algo="tc")
     for x, y in zip(a, b):
         assert torch.equal(x, y)
-    with pytest.raises(kda.KdaError):
-        _forward_with_states(d, w, True, 1.0, algo="tc")
+    o, S_T, _ = kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], A_log=d["A_log"],
+                                  dt_bias=d["dt_bias"], S0=d["S0"], chunk=64, algo="tc")
+    assert torch.equal(o, b[0]) and torch.equal(S_T, b[1])
+    S_ch = to_np(b[2])
+    for c in range(S_ch.shape[2]):
+        if c == 0:
+            ref = to_np(inp["S0"])
+        else:
+            ref = oracle.kda_fwd(*(to_np(inp[n])[:, :c * 64] for n in ("q", "k", "v", "g", "beta")),
+                                 A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]),
+                                 S0=to_np(inp["S0"]))["S_T"]
+        assert fro_rel(S_ch[:, :, c], ref) <= TOL_BF16, c
 
 
 BWD_CASES = [
@@ -164,7 +176,7 @@ def test_backward_gva_workload_sampled(cuda_device):
     d_out = dout.to(cuda_device)
     S_ch = torch.empty((w.B, w.HV, w.T // w.chunk, w.Dk, w.Dv), device=cuda_device)
     kda.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], A_log=d["A_log"], dt_bias=d["dt_bias"],
-                      S0=d["S0"], chunk=w.chunk, S_chunks=S_ch, output_final_state=False)
+                      S0=d["S0"], chunk=w.chunk, S_chunks=S_ch, output_final_state=False, algo="simt")
     gr = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S_ch, d_out, None,
                            A_log=d["A_log"], dt_bias=d["dt_bias"], chunk=w.chunk)
     torch.cuda.synchronize()

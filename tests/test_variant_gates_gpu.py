@@ -1,8 +1,9 @@
 """GPU parity of the gate variants (softplus gate of the first KDA version; one
 decay per (token, head) as in Gated DeltaNet) on the SIMT kernels -- chunk
 forward, decode step and backward -- against the FP64 oracle, which takes the
-variant gates precomputed by oracle/gates.py.  The tensor-core kernel refuses
-them (its exponent bound needs g >= g_min per key channel).
+variant gates precomputed by oracle/gates.py.  The tensor-core kernel takes
+the per-head decay and refuses the softplus gate (its exponent bound needs
+g >= g_min).
 """
 import numpy as np
 import pytest
@@ -66,16 +67,30 @@ def test_chunk_forward_gate_variants(cuda_device, case):
     assert max_rel(to_np(S_T), ref["S_T"]) <= TOL_F32          # SIMT: fp32 state from exact inputs
 
 
-def test_tensor_core_kernel_refuses_the_variants(cuda_device):
-    """algo='tc' returns UNSUPPORTED; 'auto' runs the SIMT kernel (bit for bit)."""
-    for gate, per_head in (("softplus", False), ("bounded", True)):
-        w, inp = _variant_inputs(1, 128, 1, 1, 128, 128, 64, "bf16", seed=70, per_head=per_head)
-        d = to_device(inp, cuda_device)
-        with pytest.raises(kda.KdaError) as e:
-            _fwd(d, w, gate, per_head, algo="tc")
-        assert e.value.status == 2
-        a, b = _fwd(d, w, gate, per_head, algo="auto"), _fwd(d, w, gate, per_head, algo="simt")
-        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+def test_tensor_core_kernel_refuses_the_softplus_gate(cuda_device):
+    """The unbounded gate breaks the tensor-core kernel's exponent bound:
+    algo='tc' returns UNSUPPORTED, 'auto' runs the SIMT kernel (bit for bit)."""
+    w, inp = _variant_inputs(1, 128, 1, 1, 128, 128, 64, "bf16", seed=70, per_head=False)
+    d = to_device(inp, cuda_device)
+    with pytest.raises(kda.KdaError) as e:
+        _fwd(d, w, "softplus", False, algo="tc")
+    assert e.value.status == 2
+    a, b = _fwd(d, w, "softplus", False, algo="auto"), _fwd(d, w, "softplus", False, algo="simt")
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_per_head_gate_on_the_tensor_core_kernel(cuda_device):
+    """One bounded decay per (token, head) on the tensor-core kernel (AUTO takes
+    it for this shape), against the oracle at the bf16 bars."""
+    from helpers import fro_rel
+    w, inp = _variant_inputs(1, 130, 2, 4, 128, 128, 64, "bf16", seed=72, per_head=True)
+    d = to_device(inp, cuda_device)
+    o, S_T, _ = _fwd(d, w, "bounded", True, algo="tc")
+    a = _fwd(d, w, "bounded", True, algo="auto")
+    assert torch.equal(a[0], o) and torch.equal(a[1], S_T)
+    ref = _oracle_fwd(inp, "bounded", True, 128)
+    assert max_rel(to_np(o), ref["o"]) <= TOL_BF16
+    assert fro_rel(to_np(S_T), ref["S_T"]) <= TOL_BF16
 
 
 def test_unbounded_gate_stays_finite_where_the_factorised_form_overflows(cuda_device):
@@ -138,7 +153,7 @@ def test_backward_gate_variants(cuda_device, case):
     dS_T = torch.randn((B, HV, Dk, Dv), generator=gen)
     d = to_device(inp, cuda_device)
     S_ch = torch.empty((B, HV, -(-T // chunk), Dk, Dv), device=cuda_device)
-    _fwd(d, w, gate, per_head, S_chunks=S_ch)
+    _fwd(d, w, gate, per_head, algo="simt", S_chunks=S_ch)
     gr = kda.kda_chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S_ch, dout.to(cuda_device),
                            dS_T.to(cuda_device), A_log=d["A_log"], dt_bias=d["dt_bias"], chunk=chunk,
                            gate_in_kernel=gate, g_per_head=per_head)
