@@ -283,6 +283,8 @@ TC_CASES = [
     (1, 256, 1, 2, True, 0.05, -8.0, 287),     # slow decay, with the transition CTAs
     (1, 200, 1, 2, False, 0.05, 0.0, 5, False, True),   # chunk states written
     (1, 130, 2, 4, False, 0.05, 0.0, 6, True, False),   # one decay per (token, head)
+    (2, 200, 2, 4, True, 0.02, 0.0, 231),      # two batch rows, grouped heads, ragged, transition
+    (1, 1, 1, 1, False, 0.05, 0.0, 32),        # a single token
 ]
 
 COMPOSE_CASES = [
