@@ -469,8 +469,9 @@ def bench_kcp(args, kda, workloads, dev, stream, world, rank):
 
 def bench_train(args, kda, workloads, dev, stream, world, rank):
     """Training path at the headline workload (or --batch): kda_chunk_fwd
-    keeping the per-chunk states (SIMT kernel) and kda_chunk_bwd, timed apart;
-    throughput in token-heads per second of forward + backward."""
+    keeping the per-chunk states (the tensor-core kernel for this shape) and
+    kda_chunk_bwd, timed apart; throughput in token-heads per second of
+    forward + backward."""
     import torch
     w = workloads.workload("gva_bf16") if args.batch is None else workloads.workload("gva_bf16", B=args.batch)
     inp = workloads.chunk_inputs(w, seed=rank_seed(w, rank), device=dev)
@@ -482,13 +483,13 @@ def bench_train(args, kda, workloads, dev, stream, world, rank):
     def fwd(_i):
         kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], A_log=inp["A_log"],
                           dt_bias=inp["dt_bias"], S0=inp["S0"], chunk=w.chunk, o=o, S_chunks=S_ch,
-                          output_final_state=False, stream=stream)
+                          output_final_state=False, algo=args.algo, stream=stream)
 
     def bwd(_i):
         kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S_ch, dout, None,
                           A_log=inp["A_log"], dt_bias=inp["dt_bias"], chunk=w.chunk, stream=stream)
 
-    out = {"workload": "gva_bf16 B=%d: forward with chunk states (SIMT) + backward (SIMT)" % w.B}
+    out = {"workload": "gva_bf16 B=%d: forward with chunk states (algo %s) + backward (SIMT)" % (w.B, args.algo)}
     for name, fn in (("forward_with_states", fwd), ("backward", bwd)):
         for i in range(max(1, min(args.warmup, 2))):
             fn(i)
