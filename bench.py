@@ -280,7 +280,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of the headline workload (small cases for profiling)")
     ap.add_argument("--train", action="store_true",
-                    help="also time the training path: forward keeping the chunk states (SIMT) + backward")
+                    help="also time the training path: forward keeping the chunk states + backward")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
