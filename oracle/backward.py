@@ -92,7 +92,9 @@ def kda_backward(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, do=None
     (q, k [B,T,H,Dk]; v [B,T,HV,Dv]; g or raw z [B,T,HV,Dk]; beta or logits
     [B,T,HV]; A_log [HV]; dt_bias [HV,Dk]; S0 [B,HV,Dk,Dv]).  Returns a dict
     with dq, dk, dv, dg (w.r.t. the g / z input), dbeta (w.r.t. the beta /
-    logit input), dS0, and dA_log, ddt_bias when the gate runs in-kernel.
+    logit input), dS0, and dA_log, ddt_bias when the gate runs in-kernel (with
+    A_log_l1, dt_bias_l1: the sums of the absolute values of the terms they
+    add up, the scale a floating-point sum is accurate to).
 
     gate: the in-kernel gate, "bounded" (g = g_min sigmoid(exp(A_log)(z + dt_bias)))
     or "softplus" (g = -exp(A_log) softplus(z + dt_bias)).  per_head: g / z is
@@ -151,13 +153,17 @@ def kda_backward(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, do=None
     if gate_in and gate == "bounded":
         dpre = dgg * g_min * sg * (1 - sg)
         dz = dpre * a
-        out["A_log"] = (dpre * pre).sum(axis=(0, 1, 3))     # d pre / d A_log = pre (a = exp(A_log))
+        a_terms = dpre * pre                                # d pre / d A_log = pre (a = exp(A_log))
     elif gate_in:
         dz = -dgg * a * _sig(pre)                           # d softplus = sigmoid
-        out["A_log"] = (dgg * gg[..., :dgg.shape[3]]).sum(axis=(0, 1, 3))   # g is linear in exp(A_log)
+        a_terms = dgg * gg[..., :dgg.shape[3]]              # g is linear in exp(A_log)
     else:
         dz = dgg
     if gate_in:
+        out["A_log"] = a_terms.sum(axis=(0, 1, 3))
         out["dt_bias"] = dz.sum(axis=(0, 1))[:, 0] if per_head else dz.sum(axis=(0, 1))
+        # the sums' conditioning: the summed magnitudes (what a float sum is accurate to)
+        out["A_log_l1"] = np.abs(a_terms).sum(axis=(0, 1, 3))
+        out["dt_bias_l1"] = np.abs(dz).sum(axis=(0, 1))[:, 0] if per_head else np.abs(dz).sum(axis=(0, 1))
     out["g"] = dz[..., 0] if per_head else dz
     return out

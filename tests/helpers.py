@@ -36,6 +36,18 @@ def max_rel(x, ref):
     return float(np.max(np.abs(x - ref)) / den)
 
 
+def sum_rel(x, ref, l1):
+    """Error of a gradient that is a sum over tokens (dA_log, ddt_bias): the
+    largest |x - ref| over the largest of max|ref| and the summed magnitudes
+    l1 of the terms -- a sum of terms that cancel is accurate to its l1, not
+    to its own value."""
+    x, ref, l1 = (np.asarray(a, np.float64) for a in (x, ref, l1))
+    if ref.size == 0:
+        return 0.0
+    den = max(float(np.max(np.abs(ref))), float(np.max(l1)), REL_FLOOR)
+    return float(np.max(np.abs(x - ref)) / den)
+
+
 def fro_rel(x, ref):
     x, ref = np.asarray(x, np.float64), np.asarray(ref, np.float64)
     den = max(float(np.linalg.norm(ref)), REL_FLOOR)

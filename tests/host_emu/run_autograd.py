@@ -19,7 +19,7 @@ sys.path.insert(0, HERE)
 import run_parity as R  # noqa: E402
 import workloads  # noqa: E402
 from gated_delta_rule_157_b200 import _lib, autograd  # noqa: E402
-from helpers import TOL_F32, max_rel, to_np  # noqa: E402
+from helpers import TOL_F32, max_rel, sum_rel, to_np  # noqa: E402
 from oracle import backward  # noqa: E402
 
 lib = ctypes.CDLL(os.path.join(HERE, "_build", "libkda_host_emu.so"))
@@ -86,7 +86,8 @@ def main():
                                     A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]),
                                     S0=to_np(inp["S0"]), do=to_np(do), dS_T=to_np(dS), gate=gate,
                                     per_head=per_head)
-        errs = {n: max_rel(to_np(leaves[n].grad), ref[n]) for n in leaves}
+        errs = {n: (sum_rel(to_np(leaves[n].grad), ref[n], ref[n + "_l1"]) if n in ("A_log", "dt_bias")
+                    else max_rel(to_np(leaves[n].grad), ref[n])) for n in leaves}
         worst = max(errs.values())
         bad += worst > TOL_F32
         print(gate, "per_head" if per_head else "per_channel", "ok" if worst <= TOL_F32 else "MISMATCH",

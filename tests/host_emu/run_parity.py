@@ -19,7 +19,7 @@ sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 sys.path.insert(0, os.path.dirname(HERE))
 import oracle  # noqa: E402
 import workloads  # noqa: E402
-from helpers import TOL_BF16, TOL_F32, max_rel, to_np  # noqa: E402
+from helpers import TOL_BF16, TOL_F32, max_rel, sum_rel, to_np  # noqa: E402
 from oracle import backward  # noqa: E402
 
 _P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -146,7 +146,10 @@ def run_case(lib, B, T, H, HV, Dk, Dv, C, dtype, flags, scale, seed, gate="bound
     if flags:
         names.update(dA_log="A_log", ddt_bias="dt_bias")
     for n, rn in names.items():
-        err[n] = max_rel(to_np(out[n]), gr[rn])
+        if rn in ("A_log", "dt_bias"):     # sums over tokens: against their summed magnitudes
+            err[n] = sum_rel(to_np(out[n]), gr[rn], gr[rn + "_l1"])
+        else:
+            err[n] = max_rel(to_np(out[n]), gr[rn])
     return err
 
 
