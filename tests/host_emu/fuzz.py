@@ -1,6 +1,7 @@
 """Randomised shapes through the host-emulated kernels (SIMT chunk forward and
 backward with the gate variants, decode step, tensor-core chunk kernel with
-chunk states / per-head gate / transition) against the FP64 oracle.
+chunk states / per-head gate / transition, segment combine, layer prologue
+and epilogue) against the FP64 oracle.
 
 TEST INFRASTRUCTURE, run by hand (not by pytest), with the AddressSanitizer
 runtime preloaded after emu_build.py has built the library:
@@ -18,11 +19,12 @@ sys.path.insert(0, HERE)
 import run_parity as R  # noqa: E402
 
 lib = ctypes.CDLL(os.path.join(HERE, "_build", "libkda_host_emu.so"))
+lib.emu_compose.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 4
 rng = random.Random(int(sys.argv[1]) if len(sys.argv) > 1 else 0)
 t_end = time.time() + float(sys.argv[2] if len(sys.argv) > 2 else 600)
 n = bad = 0
 while time.time() < t_end:
-    kind = rng.choice(["simt", "simt", "step", "tc"])
+    kind = rng.choice(["simt", "simt", "step", "tc", "compose", "layer"])
     try:
         if kind == "simt":
             H = rng.choice([1, 2]); HV = H * rng.choice([1, 2])
@@ -42,6 +44,14 @@ while time.time() < t_end:
             case = (rng.choice([1, 3]), H, HV, Dk, Dv, rng.choice(["f32", "bf16"]), rng.choice(["bounded", "softplus"]),
                     rng.random() < 0.3, rng.randint(0, 1000))
             e = R.run_step_case(lib, *case)
+        elif kind == "compose":
+            case = (rng.randint(0, 6), rng.randint(1, 3), rng.choice([1, 8, 33, 128]), rng.choice([1, 16, 40, 128]),
+                    rng.random() < 0.5, rng.randint(0, 1000))
+            e = R.run_compose_case(lib, *case)
+        elif kind == "layer":
+            case = (rng.choice([1, 2]), rng.randint(0, 140), 128 * rng.choice([1, 2]), rng.randint(1, 4),
+                    rng.choice([0, 128]), rng.random() < 0.7, rng.random() < 0.5, rng.randint(0, 1000))
+            e = R.run_layer_case(lib, *case)
         else:
             H = rng.choice([1, 2]); HV = H * rng.choice([1, 2])
             case = (rng.choice([1, 2]), rng.randint(1, 200), H, HV, rng.random() < 0.3, rng.choice([None, 0.05]),
