@@ -176,3 +176,69 @@ def test_gate_variant_gradients_match_finite_differences(gate, per_head):
         fd = (_loss_variant(xp, do, dS, gate, per_head) - _loss_variant(xm, do, dS, gate, per_head)) / (2 * H_FD)
         an = float((gr[gname] * U).sum())
         assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (name, fd, an)
+
+
+# --- the summed magnitudes A_log_l1 / dt_bias_l1 ---------------------------
+# They are the denominators the parameter-gradient bars use (a float sum is
+# accurate to the l1 norm of its terms), so they are pinned too: by the
+# triangle inequality on random draws, by their invariance when the loss
+# changes sign, by additivity over independent batch rows, and exactly on
+# inputs built so that every term has one sign.
+
+@pytest.mark.parametrize("gate,per_head", [("bounded", False), ("softplus", False),
+                                           ("bounded", True), ("softplus", True)])
+def test_l1_bounds_the_parameter_gradients(gate, per_head):
+    """|sum of terms| <= sum of |terms|, element by element, and strictly below
+    it somewhere (random draws give terms of both signs)."""
+    x, do, dS = _inputs(B=2, T=7, seed=31)
+    if per_head:
+        r = np.random.default_rng(32)
+        x["g"] = r.standard_normal(x["g"].shape[:-1])
+        x["dt_bias"] = 0.5 * r.standard_normal(x["dt_bias"].shape[0])
+    gr = _grads(x, do, dS, gate=gate, per_head=per_head)
+    for name in ("A_log", "dt_bias"):
+        l1, s = gr[name + "_l1"], gr[name]
+        assert l1.shape == s.shape
+        assert np.all(np.abs(s) <= l1 * (1 + 1e-12))
+        assert np.any(np.abs(s) < 0.999 * l1)
+
+
+@pytest.mark.parametrize("gate", ["bounded", "softplus"])
+def test_l1_is_even_in_the_loss_and_additive_over_batch_rows(gate):
+    """Negating do and dS_T negates every gradient but leaves the summed
+    magnitudes unchanged; two independent batch rows add their magnitudes."""
+    x, do, dS = _inputs(B=2, T=5, seed=33)
+    gp = _grads(x, do, dS, gate=gate)
+    gm = _grads(x, -do, -dS, gate=gate)
+    rows = [_grads({n: (a[b:b + 1] if n in ("q", "k", "v", "g", "beta", "S0") else a) for n, a in x.items()},
+                   do[b:b + 1], dS[b:b + 1], gate=gate) for b in range(2)]
+    for name in ("A_log", "dt_bias"):
+        np.testing.assert_allclose(gm[name], -gp[name], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(gm[name + "_l1"], gp[name + "_l1"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(rows[0][name + "_l1"] + rows[1][name + "_l1"], gp[name + "_l1"],
+                                   rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("gate,per_head", [("bounded", False), ("softplus", False), ("bounded", True)])
+def test_l1_equals_the_sum_when_every_term_has_one_sign(gate, per_head):
+    """With beta = 0 the recurrence is pure decay, S_T = prod(alpha) S0; with
+    S0 >= 0, dS_T >= 0 and do = 0 every dL/dg is >= 0, so every gate term
+    (dz, and for positive pre-activations the A_log terms) has one sign and
+    the sum of magnitudes equals the magnitude of the sum."""
+    r = np.random.default_rng(35)
+    B, T, H, HV, Dk, Dv = 2, 9, 1, 2, 4, 3
+    zshape = (B, T, HV) if per_head else (B, T, HV, Dk)
+    x = dict(q=r.standard_normal((B, T, H, Dk)), k=r.standard_normal((B, T, H, Dk)),
+             v=r.standard_normal((B, T, HV, Dv)),
+             g=np.abs(r.standard_normal(zshape)) + 0.1,               # z > 0
+             beta=np.zeros((B, T, HV)), A_log=0.3 * r.standard_normal(HV),
+             dt_bias=np.abs(r.standard_normal((HV,) if per_head else (HV, Dk))),   # z + dt_bias > 0
+             S0=np.abs(r.standard_normal((B, HV, Dk, Dv))))
+    do = np.zeros((B, T, HV, Dv))
+    dS = np.abs(r.standard_normal((B, HV, Dk, Dv)))
+    gr = backward.kda_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], A_log=x["A_log"],
+                               dt_bias=x["dt_bias"], S0=x["S0"], do=do, dS_T=dS, beta_sigmoid=False,
+                               gate=gate, per_head=per_head)
+    for name in ("A_log", "dt_bias"):
+        assert np.all(np.abs(gr[name]) > 0)
+        np.testing.assert_allclose(gr[name + "_l1"], np.abs(gr[name]), rtol=1e-12)
