@@ -448,8 +448,8 @@ def bench_kcp(args, kda, workloads, dev, stream, world, rank):
 
     def step(_i):
         kda.kda_chunk_fwd(seg["q"], seg["k"], seg["v"], seg["g"], seg["beta"], A_log=inp["A_log"],
-                          chunk=w.chunk, algo=args.algo, o=o, S_T=S_loc, M_T=M_loc,
-                          output_transition=True, stream=stream)
+                          chunk=w.chunk, algo=args.algo, S_T=S_loc, M_T=M_loc,
+                          output_transition=True, output_o=False, stream=stream)
         kda.kda_compose(M_loc, S_loc, S_init, S_in=S_in, stream=stream)
         kda.kda_chunk_fwd(seg["q"], seg["k"], seg["v"], seg["g"], seg["beta"], A_log=inp["A_log"],
                           S0=S_in[:w.n_seg], chunk=w.chunk, algo=args.algo, o=o,

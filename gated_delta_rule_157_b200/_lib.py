@@ -17,7 +17,7 @@ from . import build as _build
 KDA_OK = 0
 STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
                 3: "KDA_ERR_ALIGNMENT", 4: "KDA_ERR_ALIAS", 5: "KDA_ERR_CUDA",
-                6: "KDA_ERR_TIMEOUT"}
+                6: "KDA_ERR_TIMEOUT", 7: "KDA_ERR_RANGE"}
 DT_F32, DT_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tc": 2}
 
@@ -186,13 +186,25 @@ def _raise(fn, status):
         raise KdaError(fn, status)
 
 
+def _call(name, dev, cfn, *args):
+    """Call library entry point `cfn` with `dev` as the current device: the
+    library launches on the current device (and keeps its per-device state
+    there), so tensors on another device would otherwise be handed to kernels
+    on the wrong GPU.  Raises KdaError on a non-OK status."""
+    with torch.cuda.device(dev):
+        _raise(name, cfn(*args))
+
+
 def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=64,
                   g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
                   beta_sigmoid_in_kernel=True, gate_in_kernel=True,
                   output_final_state=True, output_transition=False, algo="auto",
                   o=None, S_T=None, M_T=None, S_chunks=None, g_per_head=False, stream=None,
-                  _withhold_ready=False):
-    """Chunk-parallel KDA forward.  Returns (o, S_T or None, M_T or None).
+                  output_o=True, _withhold_ready=False):
+    """Chunk-parallel KDA forward.  Returns (o or None, S_T or None, M_T or None).
+
+    output_o=False (with o=None) skips the output rows: only the states are
+    computed (the first pass of a segmented run).
 
     (_withhold_ready routes to kda_debug_chunk_stall, the failure-path test hook.)
 
@@ -221,7 +233,7 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     _check(A_log, "A_log", (HV,), torch.float32, dev)
     _check(dt_bias, "dt_bias", (HV,) + gk, torch.float32, dev)
     _check(S0, "S0", (B, HV, Dk, Dv), torch.float32, dev)
-    if o is None:
+    if o is None and output_o:
         o = torch.empty((B, T, HV, Dv), dtype=dt, device=dev)
     _check(o, "o", (B, T, HV, Dv), dt, dev)
     if S_T is None and output_final_state:
@@ -243,9 +255,9 @@ def kda_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     a.A_log, a.dt_bias, a.S0 = _ptr(A_log), _ptr(dt_bias), _ptr(S0)
     a.o, a.S_T, a.M_T, a.S_chunks = _ptr(o), _ptr(S_T), _ptr(M_T), _ptr(S_chunks)
     if _withhold_ready:
-        _raise("kda_debug_chunk_stall", lib.kda_debug_chunk_stall(ctypes.byref(a), _stream(stream, dev)))
+        _call("kda_debug_chunk_stall", dev, lib.kda_debug_chunk_stall, ctypes.byref(a), _stream(stream, dev))
     else:
-        _raise("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a), _stream(stream, dev)))
+        _call("kda_chunk_fwd", dev, lib.kda_chunk_fwd, ctypes.byref(a), _stream(stream, dev))
     return o, S_T, M_T
 
 
@@ -301,7 +313,7 @@ def kda_chunk_bwd(q, k, v, g, beta, S_chunks, dout, dS_T=None, *, A_log=None, dt
     a.dout, a.dS_T = _ptr(dout), _ptr(dS_T)
     for name in ("dq", "dk", "dv", "dg", "dbeta", "dS0", "dA_log", "ddt_bias"):
         setattr(a, name, _ptr(out[name]))
-    _raise("kda_chunk_bwd", lib.kda_chunk_bwd(ctypes.byref(a), _stream(stream, dev)))
+    _call("kda_chunk_bwd", dev, lib.kda_chunk_bwd, ctypes.byref(a), _stream(stream, dev))
     return out
 
 
@@ -342,7 +354,7 @@ def kda_step(S, q, k, v, g, beta, *, A_log=None, dt_bias=None, g_min=-5.0, scale
     a.g_per_head = int(bool(g_per_head))
     a.q, a.k, a.v, a.g, a.beta = map(_ptr, (q, k, v, g, beta))
     a.A_log, a.dt_bias, a.S, a.o = _ptr(A_log), _ptr(dt_bias), _ptr(S), _ptr(o)
-    _raise("kda_step", lib.kda_step(ctypes.byref(a), _stream(stream, dev)))
+    _call("kda_step", dev, lib.kda_step, ctypes.byref(a), _stream(stream, dev))
     return o
 
 
@@ -359,9 +371,8 @@ def kda_compose(M, S_seg, S_init=None, S_in=None, stream=None):
     if S_in is None:
         S_in = torch.empty((n + 1, BH, Dk, Dv), dtype=torch.float32, device=dev)
     _check(S_in, "S_in", (n + 1, BH, Dk, Dv), torch.float32, dev)
-    st = lib.kda_compose(n, BH, Dk, Dv, _ptr(M), _ptr(S_seg), _ptr(S_init), _ptr(S_in),
-                         _stream(stream, dev))
-    _raise("kda_compose", st)
+    _call("kda_compose", dev, lib.kda_compose, n, BH, Dk, Dv, _ptr(M), _ptr(S_seg), _ptr(S_init),
+          _ptr(S_in), _stream(stream, dev))
     return S_in
 
 
@@ -393,7 +404,7 @@ def kda_short_conv(x, w, bias=None, *, head_dim=0, silu=True, l2_eps=1e-6, state
     a.head_dim, a.silu, a.l2_eps = int(head_dim), int(bool(silu)), float(l2_eps)
     a.x, a.w, a.bias, a.state_in = _ptr(x), _ptr(w), _ptr(bias), _ptr(state_in)
     a.y, a.state_out = _ptr(y), _ptr(state_out)
-    _raise("kda_short_conv", lib.kda_short_conv(ctypes.byref(a), _stream(stream, dev)))
+    _call("kda_short_conv", dev, lib.kda_short_conv, ctypes.byref(a), _stream(stream, dev))
     return (y, state_out) if want_state else y
 
 
@@ -415,7 +426,7 @@ def kda_output_gate(o, gate, weight=None, *, eps=1e-6, y=None, stream=None):
     a = GateArgs()
     a.N, a.HV, a.D, a.eps = N, HV, D, float(eps)
     a.o, a.gate, a.weight, a.y = _ptr(o), _ptr(gate), _ptr(weight), _ptr(y)
-    _raise("kda_output_gate", lib.kda_output_gate(ctypes.byref(a), _stream(stream, dev)))
+    _call("kda_output_gate", dev, lib.kda_output_gate, ctypes.byref(a), _stream(stream, dev))
     return y
 
 
@@ -423,7 +434,7 @@ def kda_device_status(stream=None, device=None):
     """Synchronise and read/clear the device error word; raises KdaError if set."""
     lib = load()
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
-    _raise("kda_device_status", lib.kda_device_status(_stream(stream, dev)))
+    _call("kda_device_status", dev, lib.kda_device_status, _stream(stream, dev))
 
 
 def kda_status_string(status: int) -> str:

@@ -49,7 +49,7 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
     if (a->B == 0) return KDA_OK;
 
     if (ntok > 0) {
-        if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o) return KDA_ERR_INVALID_ARG;
+        if (!a->q || !a->k || !a->v || !a->g || !a->beta) return KDA_ERR_INVALID_ARG;   // o may be NULL
         if (a->gate_in_kernel && !a->A_log) return KDA_ERR_INVALID_ARG;
         const void *acts[] = {a->q, a->k, a->v, a->g, a->beta, a->o};
         for (const void *p : acts)
@@ -71,7 +71,7 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
                     range_of(a->A_log, a->A_log ? (size_t)a->HV * 4 : 0),
                     range_of(a->dt_bias, a->dt_bias ? (size_t)a->HV * gk * 4 : 0)};
     Range r_s0 = range_of(a->S0, a->S0 ? ns : 0);
-    Range r_o = range_of(a->o, ntok ? nv : 0);
+    Range r_o = range_of(a->o, (ntok && a->o) ? nv : 0);
     Range r_st = range_of(a->S_T, a->S_T ? ns : 0);
     Range r_mt = range_of(a->M_T, a->M_T ? nm : 0);
     const size_t nchunks = a->T > 0 ? ((size_t)a->T + a->chunk - 1) / a->chunk : 0;
@@ -114,7 +114,10 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
             if (!aligned(ptr, 16)) return KDA_ERR_ALIGNMENT;
         return cuda_status(kda::launch_chunk_tc(p, s));
     }
-    if (a->algo == KDA_ALGO_AUTO && tc_ok) {
+    // A log-decay given directly (no in-kernel gate) may lie below g_min, where
+    // the tensor-core kernel's exponent bound does not hold: AUTO takes the
+    // SIMT kernel, which is exact for any g <= 0.
+    if (a->algo == KDA_ALGO_AUTO && tc_ok && a->gate_in_kernel != 0) {
         bool al16 = true;
         const void *v16[] = {a->q, a->k, a->v, a->g, a->o};
         for (const void *ptr : v16) al16 = al16 && aligned(ptr, 16);
@@ -325,7 +328,8 @@ kda_status kda_device_status(void *stream) {
     unsigned int word = 0;
     cudaError_t e = kda::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &word);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-    return word ? KDA_ERR_TIMEOUT : KDA_OK;
+    if (word & 1u) return KDA_ERR_TIMEOUT;
+    return (word & 2u) ? KDA_ERR_RANGE : KDA_OK;
 }
 
 const char *kda_status_string(kda_status s) {
@@ -337,10 +341,11 @@ const char *kda_status_string(kda_status s) {
         case KDA_ERR_ALIAS: return "KDA_ERR_ALIAS";
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_RANGE: return "KDA_ERR_RANGE";
     }
     return "KDA_ERR_UNKNOWN";
 }
 
-int kda_version(void) { return 120; }
+int kda_version(void) { return 200; }
 
 }  // extern "C"

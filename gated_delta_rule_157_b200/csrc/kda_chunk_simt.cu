@@ -184,8 +184,8 @@ chunk_simt_kernel(ChunkParams p) {
             }
         }
         __syncthreads();
-        // ---- O = (Q*exp(G)) S + A_qk U --------------------------------------
-        if (col0 < ncol_state) {
+        // ---- O = (Q*exp(G)) S + A_qk U (unless o is not asked for) ---------
+        if (o && col0 < ncol_state) {
             for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
                 int r = idx / kVT, jj = idx % kVT, col = col0 + jj;
                 if (col >= ncol_state) continue;

@@ -3,55 +3,96 @@
 //
 //   S_in[0] = S_init (or 0),  S_in[s+1] = M[s] S_in[s] + S_seg[s]
 //
-// One CTA per (bh, 32-column slice); the segments are walked in order inside
-// the CTA with the running slice in shared memory and M[s] staged through
-// shared memory.  FP32 FMA, summation over the inner index in increasing order.
+// The columns of the state are independent, the segments are not: one CTA per
+// (bh, 8-column slice) walks the segments in order with its slice of the
+// running state in shared memory.  Thread (row c, column quad h) computes
+// S_in[s+1][c][4h..4h+3] = S_seg[s][c][..] + sum_m M[s][c][m] S_in[s][m][..]:
+// its row of M[s] streams from global memory (L2: the CTAs of one bh share
+// it), the running slice is read as broadcast float4s.  FP32 FMA, summation
+// over the inner index in increasing order.
 #include "kda_internal.cuh"
 
 namespace kda {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kVT = 32;
+constexpr int kVT = 8;                      // state columns per CTA
 
+template <bool kVec>
 __global__ void __launch_bounds__(kThreads)
 compose_kernel(int n_seg, int BH, int Dk, int Dv, const float *__restrict__ M,
                const float *__restrict__ S_seg, const float *__restrict__ S_init,
                float *__restrict__ S_in) {
-    extern __shared__ float smem[];
-    float *prev = smem;                 // [Dk][kVT]
-    float *Ms = prev + Dk * kVT;        // [Dk][Dk]
+    __shared__ __align__(16) float prev[128 * kVT];      // [Dk][kVT]
     const int bh = blockIdx.x, col0 = blockIdx.y * kVT;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int col = col0 + lane;
+    const int tid = threadIdx.x, c = tid >> 1, h = tid & 1;
+    const int cb = col0 + 4 * h;                         // first column of this thread
+    const bool row = c < Dk;
     const size_t st = (size_t)Dk * Dv, mt = (size_t)Dk * Dk;
 
-    for (int c = warp; c < Dk; c += kThreads / 32) {
-        float x = 0.f;
-        if (col < Dv && S_init) x = S_init[bh * st + (size_t)c * Dv + col];
-        prev[c * kVT + lane] = x;
-        if (col < Dv) S_in[bh * st + (size_t)c * Dv + col] = x;
+    auto ld4 = [&](const float *base) {                  // columns cb .. cb+3 of a row
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (kVec) {
+            if (cb < Dv) v = *reinterpret_cast<const float4 *>(base + cb);
+        } else {
+            if (cb + 0 < Dv) v.x = base[cb + 0];
+            if (cb + 1 < Dv) v.y = base[cb + 1];
+            if (cb + 2 < Dv) v.z = base[cb + 2];
+            if (cb + 3 < Dv) v.w = base[cb + 3];
+        }
+        return v;
+    };
+    auto st4 = [&](float *base, float4 v) {
+        if (kVec) {
+            if (cb < Dv) *reinterpret_cast<float4 *>(base + cb) = v;
+        } else {
+            if (cb + 0 < Dv) base[cb + 0] = v.x;
+            if (cb + 1 < Dv) base[cb + 1] = v.y;
+            if (cb + 2 < Dv) base[cb + 2] = v.z;
+            if (cb + 3 < Dv) base[cb + 3] = v.w;
+        }
+    };
+
+    if (row) {
+        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (S_init) x0 = ld4(S_init + bh * st + (size_t)c * Dv);
+        *reinterpret_cast<float4 *>(prev + c * kVT + 4 * h) = x0;
+        st4(S_in + bh * st + (size_t)c * Dv, x0);
     }
     for (int s = 0; s < n_seg; ++s) {
-        const float *Mg = M + ((size_t)s * BH + bh) * mt;
         __syncthreads();
-        for (int i = tid; i < Dk * Dk; i += kThreads) Ms[i] = Mg[i];
-        __syncthreads();
-        const float *Sg = S_seg + ((size_t)s * BH + bh) * st;
-        float *out = S_in + ((size_t)(s + 1) * BH + bh) * st;
-        float acc[(128 + kThreads / 32 - 1) / (kThreads / 32)];
-        int n = 0;
-        for (int c = warp; c < Dk; c += kThreads / 32, ++n) {
-            float a = (col < Dv) ? Sg[(size_t)c * Dv + col] : 0.f;
-            const float *mr = Ms + c * Dk;
-            for (int m = 0; m < Dk; ++m) a = fmaf(mr[m], prev[m * kVT + lane], a);
-            acc[n] = a;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row) {
+            acc = ld4(S_seg + ((size_t)s * BH + bh) * st + (size_t)c * Dv);
+            const float *mr = M + ((size_t)s * BH + bh) * mt + (size_t)c * Dk;
+            int m = 0;
+            if (kVec) {
+                for (; m + 4 <= Dk; m += 4) {
+                    const float4 mv = *reinterpret_cast<const float4 *>(mr + m);
+                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 pv = *reinterpret_cast<const float4 *>(prev + (m + u) * kVT + 4 * h);
+                        acc.x = fmaf(mm[u], pv.x, acc.x);
+                        acc.y = fmaf(mm[u], pv.y, acc.y);
+                        acc.z = fmaf(mm[u], pv.z, acc.z);
+                        acc.w = fmaf(mm[u], pv.w, acc.w);
+                    }
+                }
+            }
+            for (; m < Dk; ++m) {
+                const float mv = mr[m];
+                const float4 pv = *reinterpret_cast<const float4 *>(prev + m * kVT + 4 * h);
+                acc.x = fmaf(mv, pv.x, acc.x);
+                acc.y = fmaf(mv, pv.y, acc.y);
+                acc.z = fmaf(mv, pv.z, acc.z);
+                acc.w = fmaf(mv, pv.w, acc.w);
+            }
         }
         __syncthreads();
-        n = 0;
-        for (int c = warp; c < Dk; c += kThreads / 32, ++n) {
-            prev[c * kVT + lane] = acc[n];
-            if (col < Dv) out[(size_t)c * Dv + col] = acc[n];
+        if (row) {
+            *reinterpret_cast<float4 *>(prev + c * kVT + 4 * h) = acc;
+            st4(S_in + ((size_t)(s + 1) * BH + bh) * st + (size_t)c * Dv, acc);
         }
     }
 }
@@ -60,12 +101,12 @@ compose_kernel(int n_seg, int BH, int Dk, int Dv, const float *__restrict__ M,
 
 cudaError_t launch_compose(int n_seg, int BH, int Dk, int Dv, const float *M, const float *S_seg,
                            const float *S_init, float *S_in, cudaStream_t s) {
-    dim3 grid(BH, (Dv + kVT - 1) / kVT);
-    size_t smem = ((size_t)Dk * kVT + (size_t)Dk * Dk) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    compose_kernel<<<grid, kThreads, smem, s>>>(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in);
+    const dim3 grid(BH, (Dv + kVT - 1) / kVT);
+    // float4 rows need Dk, Dv multiples of 4 and 16-byte aligned buffers
+    const bool vec = Dk % 4 == 0 && Dv % 4 == 0 && ((uintptr_t)M | (uintptr_t)S_seg | (uintptr_t)S_init |
+                                                    (uintptr_t)S_in) % 16 == 0;
+    if (vec) compose_kernel<true><<<grid, kThreads, 0, s>>>(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in);
+    else compose_kernel<false><<<grid, kThreads, 0, s>>>(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in);
     return cudaGetLastError();
 }
 

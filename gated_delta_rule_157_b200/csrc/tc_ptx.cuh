@@ -254,6 +254,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void *tmap,
         ::"r"(dst_smem), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
         : "memory");
 }
+// Prefetch one box of a tiled 3-D tensor into L2 (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+                 ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
 // Bring a tensor map (kernel parameter) into the descriptor cache ahead of its first use.
 __device__ __forceinline__ void prefetch_tensormap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

@@ -29,8 +29,9 @@ class _KernelOps:
 
     @staticmethod
     def forward(q, k, v, g, beta, S0, want_M, **kw):
+        # the pass with the transition only needs the states: no o
         o, S_T, M_T = _lib.kda_chunk_fwd(q, k, v, g, beta, S0=S0, output_final_state=True,
-                                         output_transition=want_M, **kw)
+                                         output_transition=want_M, output_o=not want_M, **kw)
         return o, S_T, M_T
 
     @staticmethod

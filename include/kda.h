@@ -38,8 +38,9 @@
  *   - Argument errors are detected on the host before anything is launched and
  *     are returned as a kda_status; nothing is written in that case.  A failed
  *     launch returns KDA_ERR_CUDA.  Device-side faults of the tensor-core
- *     kernel (a bounded wait that ran out) are recorded in the device error
- *     word and reported by kda_device_status().
+ *     kernel (a bounded wait that ran out, a caller-given log-decay below
+ *     g_min) are recorded in the device error word and reported by
+ *     kda_device_status().
  *   - No entry point falls back to the CPU.
  */
 #ifndef KDA_B200_H
@@ -56,7 +57,9 @@ typedef enum {
     KDA_ERR_ALIGNMENT = 3,     /* a pointer is not aligned as the layout requires */
     KDA_ERR_ALIAS = 4,         /* an output overlaps an input or another output */
     KDA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
-    KDA_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up (see kda_device_status) */
+    KDA_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (see kda_device_status) */
+    KDA_ERR_RANGE = 7          /* a log-decay given directly to the tensor-core kernel was
+                                  below g_min and was clamped (see kda_device_status) */
 } kda_status;
 
 typedef enum {
@@ -90,14 +93,18 @@ typedef enum {
  *   g       [B, T, HV, Dk]  ([B, T, HV] with g_per_head) log-decay g, or the raw
  *           gate input z when gate_in_kernel;
  *           a log-decay given directly should lie in [g_min, 0]: the SIMT
- *           kernel takes any value, the tensor-core kernel (whose exponent
- *           bound, 16 |g_min| per 16-token tile, rests on it) clamps values
- *           below g_min up to g_min
+ *           kernel takes any value (KDA_ALGO_AUTO picks it for a log-decay
+ *           given directly); the tensor-core kernel, asked for explicitly
+ *           (whose exponent bound, 16 |g_min| per 16-token tile, rests on
+ *           it), clamps values below g_min up to g_min and records
+ *           KDA_ERR_RANGE for kda_device_status()
  *   beta    [B, T, HV]      write strength, or its logit when beta_sigmoid_in_kernel
  *   A_log   [HV]      fp32  read iff gate_in_kernel (must then be non-NULL)
  *   dt_bias [HV, Dk]  fp32  ([HV] with g_per_head) read iff gate_in_kernel; NULL means 0
  *   S0      [B, HV, Dk, Dv] fp32, or NULL for zeros
- *   o       [B, T, HV, Dv]  output, element type `dtype` (bf16 rounded to nearest even)
+ *   o       [B, T, HV, Dv]  output, element type `dtype` (bf16 rounded to nearest even),
+ *           or NULL when only the states are wanted (e.g. the first pass of a
+ *           segmented run, which needs S_T and M_T): the output work is skipped
  *   S_T     [B, HV, Dk, Dv] fp32 output, or NULL; may be the same buffer as S0
  *           (exactly, not partially overlapping)
  *   M_T     [B, HV, Dk, Dk] fp32 output, or NULL
@@ -111,7 +118,7 @@ typedef enum {
  * 1 <= chunk <= 64.  q, k, v, g, beta, o must be aligned to their element size;
  * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64,
  * gate_in_kernel 0 or 1 (the bounded gate), and 16-byte aligned q, k, v, g, o
- * (KDA_ALGO_AUTO takes the SIMT kernel otherwise).
+ * (KDA_ALGO_AUTO takes the SIMT kernel otherwise, and for gate_in_kernel = 0).
  * gate_in_kernel must be 0, 1 or 2.  o must not overlap any input; S_T, M_T and
  * S_chunks must not overlap each other, o, or any input except S_T == S0.
  * T == 0 writes S_T = S0 (or 0) and M_T = I.
@@ -294,7 +301,10 @@ typedef struct {
 kda_status kda_output_gate(const kda_gate_args *args, void *stream);
 
 /* Reads and clears the device error word of the current device after
- * synchronising `stream`.  Returns KDA_OK, KDA_ERR_TIMEOUT or KDA_ERR_CUDA. */
+ * synchronising `stream`.  Returns KDA_OK, KDA_ERR_TIMEOUT (a bounded wait
+ * gave up since the last call; takes precedence), KDA_ERR_RANGE (a
+ * tensor-core call clamped a caller-given log-decay below g_min) or
+ * KDA_ERR_CUDA. */
 kda_status kda_device_status(void *stream);
 
 /* Test hook for the failure path of the tensor-core chunk kernel (no

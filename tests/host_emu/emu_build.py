@@ -97,8 +97,8 @@ _RUN_TC = r'''
 #include <sanitizer/asan_interface.h>
 namespace kda { namespace tc { EmuCta *g_cta = nullptr; EmuTf32Slots g_tf32[32]; } }
 
-// The tensor maps the library's launcher builds (tokens x heads x 128 channels,
-// [64][1][128] boxes; v in two [64][1][64] boxes with the 128-byte swizzle).
+// The tensor maps the library's launcher builds (tokens x heads x 128 channels:
+// z in [64][1][128] boxes; q, k, v in [64][1][64] boxes with the 128-byte swizzle).
 static kda::tc::EmuTensorMap emu_row_map(const void *base, int heads, long long rows, bool sw128) {
     kda::tc::EmuTensorMap m{};
     m.base = static_cast<const uint8_t *>(base);
@@ -114,7 +114,7 @@ extern "C" int emu_chunk_tc(kda::ChunkParams *pp) {
     TcParams tp;
     tp.p = *pp;
     const long long rows = (long long)tp.p.B * tp.p.T;
-    const tc::EmuTensorMap maps[4] = {emu_row_map(tp.p.q, tp.p.H, rows, false), emu_row_map(tp.p.k, tp.p.H, rows, false),
+    const tc::EmuTensorMap maps[4] = {emu_row_map(tp.p.q, tp.p.H, rows, true), emu_row_map(tp.p.k, tp.p.H, rows, true),
                                       emu_row_map(tp.p.g, tp.p.HV, rows, false),
                                       emu_row_map(tp.p.v, tp.p.HV, rows, true)};
     for (int i = 0; i < 4; ++i) std::memcpy(&tp.tm[i], &maps[i], sizeof maps[i]);
@@ -205,11 +205,13 @@ _RUN_COMPOSE = _POISON + r'''
 extern "C" int emu_compose(int n_seg, int BH, int Dk, int Dv, const float *M, const float *S_seg,
                            const float *S_init, float *S_in) {
     using namespace kda;
-    const size_t bytes = ((size_t)Dk * kVT + (size_t)Dk * Dk) * sizeof(float);
-    if (bytes > sizeof(smem)) return 1;
-    emu_poison(bytes);
-    emu_launch(dim3(BH, (Dv + kVT - 1) / kVT), dim3(kThreads),
-               [&] { compose_kernel(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in); });
+    emu_poison(0);     // the kernel's shared memory is static
+    const bool vec = Dk % 4 == 0 && Dv % 4 == 0 && ((uintptr_t)M | (uintptr_t)S_seg | (uintptr_t)S_init |
+                                                    (uintptr_t)S_in) % 16 == 0;
+    emu_launch(dim3(BH, (Dv + kVT - 1) / kVT), dim3(kThreads), [&] {
+        if (vec) compose_kernel<true>(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in);
+        else compose_kernel<false>(n_seg, BH, Dk, Dv, M, S_seg, S_init, S_in);
+    });
     return 0;
 }
 '''

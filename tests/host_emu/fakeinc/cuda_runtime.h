@@ -14,6 +14,7 @@
 #define __launch_bounds__(...)
 #define __shared__
 #define __grid_constant__
+#define __align__(n) __attribute__((aligned(n)))
 typedef int cudaError_t;
 typedef void *cudaStream_t;
 enum { cudaSuccess = 0 };

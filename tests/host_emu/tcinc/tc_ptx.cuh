@@ -273,6 +273,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void *tmap,
     emu_complete_tx(mbar, off);
 }
 __device__ __forceinline__ void prefetch_tensormap(const void *) {}
+__device__ __forceinline__ void tma_prefetch_3d(const void *, int, int, int) {}
 
 // ---- special functions, conversions, warp-level tf32 mma -------------------------------
 __device__ __forceinline__ float ex2_approx(float x) { return std::exp2(x); }

@@ -53,6 +53,7 @@ def test_library_is_in_tree_and_links_no_oracle():
 def test_status_strings_and_version():
     assert kda.kda_status_string(0) == "KDA_OK"
     assert kda.kda_status_string(6) == "KDA_ERR_TIMEOUT"
+    assert kda.kda_status_string(7) == "KDA_ERR_RANGE"
     assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
     assert kda.kda_version() >= 100
 
@@ -104,7 +105,6 @@ def test_empty_batch_is_a_no_op():
     ("T", -1, INVALID),
     ("g_min", 0.5, INVALID),
     ("q", None, INVALID),
-    ("o", None, INVALID),
     ("A_log", None, INVALID),     # gate_in_kernel needs A_log
     ("q", 0x7f0000100002, ALIGN),  # fp32 needs 4-byte alignment
     ("S0", 0x7f0000800001, ALIGN),
@@ -134,6 +134,8 @@ def test_valid_request_without_gpu_reports_cuda_error():
     # Passes validation, so the launch is attempted and fails: no CPU fallback.
     a = _chunk_args(S_T=_chunk_args().S_T)
     assert _fwd(a) == 5
+    # o may be NULL (only the states are wanted): still a valid request
+    assert _fwd(_chunk_args(o=None)) == 5
 
 
 def _step_args(**kw):

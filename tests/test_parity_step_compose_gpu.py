@@ -58,6 +58,33 @@ def test_decode_workload_full_batch(cuda_device):
         assert max_rel(to_np(S), S_ref) <= TOL_F32
 
 
+def test_decode_workload_512_steps_sampled(cuda_device):
+    """The decode workload as the benchmark runs it: B=256, H=HV=32, 512
+    consecutive steps against the resident fp32 state, every chain updated on
+    the GPU; a sample of chains (spread over batch rows and heads) is followed
+    by the oracle through all 512 steps, o checked at every step and the state
+    at the end (the fp32 state must not drift from the FP64 one)."""
+    import numpy as np
+    w = workloads.workload("decode_bf16")
+    S0 = workloads.decode_state(w)
+    chains = [(0, 0), (17, 5), (128, 31), (255, 16), (63, 9), (200, 22)]
+    bi = np.array([c[0] for c in chains]); hi = np.array([c[1] for c in chains])
+    S_ref = to_np(S0)[bi, hi][:, None]                           # [n, 1, Dk, Dv]
+    S = S0.to(cuda_device)
+    bt, ht = torch.from_numpy(bi).to(cuda_device), torch.from_numpy(hi).to(cuda_device)
+    worst_o = 0.0
+    for step in range(w.steps):
+        inp = workloads.decode_step_inputs(w, step, device=cuda_device)
+        o = _gpu_step(S, inp)
+        sub = {n: to_np(inp[n][bt, ht])[:, None] for n in ("q", "k", "v", "g", "beta")}
+        sub["A_log"] = to_np(inp["A_log"])[:1]
+        sub["dt_bias"] = None
+        S_ref, o_ref = _oracle_step(S_ref, sub)
+        worst_o = max(worst_o, max_rel(to_np(o[bt, ht])[:, None], o_ref))
+    assert worst_o <= TOL_BF16, worst_o
+    assert max_rel(to_np(S[bt, ht])[:, None], S_ref) <= TOL_F32
+
+
 def test_step_matches_chunk_forward(cuda_device):
     """T consecutive decode steps equal one chunked forward over the T tokens."""
     w = workloads.Workload("sm", B=2, T=24, H=1, HV=2, Dk=32, Dv=32, chunk=16, dtype="f32",
