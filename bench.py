@@ -39,6 +39,8 @@ METRIC = "chunk_kda fwd tokens·heads/s + % bf16 TC peak; kda_step decode HBM GB
 CHUNK_TC_TRAFFIC_B4 = 4 * (202.115584e6 + 48.679168e6)
 STEP_TRAFFIC = 545.3e6 + 485.3e6
 UNIT = "tokens·heads/s"
+NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e, nominal (the measured copy peak is the roofline)
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # CUDA-core FP32: SMs x FMA lanes x 2 x max clock
 
 
 def peaks():
@@ -211,6 +213,49 @@ def cpu_baseline(w):
                       % (w.B, w.HV, w.T, w.B * w.HV, dt)}
 
 
+def oracle_chunk_timing(w, T_override=None):
+    """The FP64 oracle on a whole chunk workload (or its first T_override
+    tokens of every chain), wall time on the host cores."""
+    import oracle
+    import torch
+    import workloads
+
+    def f64(t):
+        return None if t is None else t.to(torch.float64).numpy()
+
+    ws = w if T_override is None else workloads.workload(w.name, T=T_override)
+    inp = workloads.chunk_inputs(ws)
+    arrays = [f64(inp[n]) for n in ("q", "k", "v", "g", "beta")]
+    kw = dict(A_log=f64(inp["A_log"]), dt_bias=f64(inp["dt_bias"]), S0=f64(inp["S0"]))
+    del inp
+    t0 = time.perf_counter()
+    oracle.kda_fwd(*arrays, **kw)
+    dt = time.perf_counter() - t0
+    return {"value": ws.token_heads / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "seconds": dt,
+            "sample": "FP64 oracle, whole B=%d HV=%d T=%d pass (%d chains)" % (ws.B, ws.HV, ws.T, ws.B * ws.HV)}
+
+
+def oracle_decode_timing(w, n_steps=8):
+    """The FP64 oracle on n_steps consecutive decode steps of the whole batch."""
+    import oracle
+    import torch
+    import workloads
+
+    def f64(t):
+        return None if t is None else t.to(torch.float64).numpy()
+
+    S = f64(workloads.decode_state(w))
+    steps = [workloads.decode_step_inputs(w, i) for i in range(n_steps)]
+    t0 = time.perf_counter()
+    for d in steps:
+        S, _ = oracle.kda_step(S, *(f64(d[n]) for n in ("q", "k", "v", "g", "beta")), A_log=f64(d["A_log"]))
+    dt = (time.perf_counter() - t0) / n_steps
+    return {"value": decode_bytes(w) / dt / 1e9, "unit": "GB/s", "ms_per_step": dt * 1e3,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "FP64 oracle, %d consecutive steps of the whole B=%d HV=%d batch" % (n_steps, w.B, w.HV)}
+
+
 def run_reference(args):
     """--impl reference: the FP64 oracle on rank 0, one bounded sample per step."""
     rank = int(os.environ.get("RANK", "0"))
@@ -280,7 +325,7 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="override B of the headline workload (small cases for profiling)")
     ap.add_argument("--train", action="store_true",
-                    help="also time the training path: forward keeping the chunk states + backward")
+                    help="(kept for compatibility: the training path is always timed with the extras)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -379,15 +424,19 @@ def main():
     del host, dev_in, h_o, h_S
 
     if not args.no_extras:
+        line["small"] = bench_small_configs(args, kda, workloads, dev, stream, pk, world, rank)
         line["decode"] = bench_decode(args, kda, workloads, dev, stream, pk, world, rank)
         line["kcp"] = bench_kcp(args, kda, workloads, dev, stream, world, rank)
         line["layer"] = bench_layer(args, kda, dev, stream, pk, world)
-        line["gpu_launches_extras"] = {"decode": line["decode"]["launches"],
-                                       "kcp": line["kcp"]["launches"],
-                                       "layer": line["layer"]["launches"]}
-
-    if args.train:
         line["train"] = bench_train(args, kda, workloads, dev, stream, world, rank)
+        line["gpu_launches_extras"] = {"small": line["small"]["launches"],
+                                       "decode": line["decode"]["launches"],
+                                       "kcp": line["kcp"]["launches"],
+                                       "layer": line["layer"]["launches"],
+                                       "train": line["train"]["launches"]}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["kcp"]["cpu_baseline_unsegmented"] = oracle_chunk_timing(workloads.workload("kcp_bf16"))
+            line["decode"]["cpu_baseline"] = oracle_decode_timing(workloads.workload("decode_bf16"))
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
@@ -398,6 +447,54 @@ def main():
         dist.barrier(device_ids=[dev.index])
         dist.destroy_process_group()
     return 0
+
+
+def bench_small_configs(args, kda, workloads, dev, stream, pk, world, rank):
+    """tiny_fp32 (B=1 H=HV=2 T=64 D=16 chunk 16, fp32: the SIMT kernel) and
+    prefill_bf16 (B=1 H=HV=16 T=4096 D=128 chunk 64, bf16, S0 ~ N(0, 0.02):
+    16 chains, so 16 of the 148 SMs work), each timed over consecutive
+    launches with inputs resident."""
+    out, launches = {}, 0
+    for name in ("tiny_fp32", "prefill_bf16"):
+        w = workloads.workload(name)
+        inp = workloads.chunk_inputs(w, seed=rank_seed(w, rank), device=dev)
+        o = torch_empty_like_o(w, dev)
+
+        def step(_i):
+            kda.kda_chunk_fwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], A_log=inp["A_log"],
+                              dt_bias=inp["dt_bias"], S0=inp["S0"], chunk=w.chunk, o=o, stream=stream)
+
+        for i in range(args.warmup):
+            step(i)
+        barrier(world, dev)
+        k = max(5, min(args.steps, 20))
+        per = time_launches(step, k, stream)
+        barrier(world, dev)
+        ms_local = sum(per) / len(per)
+        ms = max_over_ranks(ms_local, world, dev)
+        e = {"workload": "%s: B=%d H=%d HV=%d T=%d Dk=Dv=%d chunk=%d %s" % (name, w.B, w.H, w.HV, w.T, w.Dk,
+                                                                         w.chunk, w.dtype),
+             "value": whole_job_value(w.token_heads, world, ms), "unit": UNIT, "ms_per_step": ms,
+             "launches": k, "chains": w.B * w.HV}
+        if name == "prefill_bf16":
+            tfl = w.token_heads * chunk_flops_per_token_head(w.Dk, w.Dv, w.chunk) / (ms_local * 1e-3) / 1e12
+            gbs = chunk_bytes(w) / (ms_local * 1e-3) / 1e9
+            e["tc_peak_frac"] = tfl / pk["bf16_tflops"]
+            e["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / pk["hbm_gbs"], "traffic": None}
+            e["occupancy"] = "%d chains on 148 SMs: one CTA per chain" % (w.B * w.HV)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            e["cpu_baseline"] = oracle_chunk_timing(w)
+        out[name] = e
+        launches += k
+        del inp, o
+    out["launches"] = launches
+    return out
+
+
+def torch_empty_like_o(w, dev):
+    import torch
+    return torch.empty((w.B, w.T, w.HV, w.Dv), dtype=w.torch_dtype, device=dev)
 
 
 def bench_decode(args, kda, workloads, dev, stream, pk, world, rank):
@@ -429,6 +526,7 @@ def bench_decode(args, kda, workloads, dev, stream, pk, world, rank):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / pk["hbm_gbs"], "traffic": STEP_TRAFFIC,
                          "traffic_unit": "bytes per launch (ncu dram read + write)", "kernel": "kda_step"},
+            "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
             "launches": n, "l2": "state 512 MiB > L2"}
 
 
@@ -489,7 +587,11 @@ def bench_train(args, kda, workloads, dev, stream, world, rank):
         kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S_ch, dout, None,
                           A_log=inp["A_log"], dt_bias=inp["dt_bias"], chunk=w.chunk, stream=stream)
 
-    out = {"workload": "gva_bf16 B=%d: forward with chunk states (algo %s) + backward (SIMT)" % (w.B, args.algo)}
+    out = {"workload": "gva_bf16 B=%d: forward with chunk states (algo %s) + backward (SIMT)" % (w.B, args.algo),
+           "launches": 0}
+    # kernels per call: the forward is one launch; the backward three (chunk
+    # kernel, L2-norm and gate/parameter passes) after the output zeroing
+    n_kernels = {"forward_with_states": 1, "backward": 3}
     for name, fn in (("forward_with_states", fwd), ("backward", bwd)):
         for i in range(max(1, min(args.warmup, 2))):
             fn(i)
@@ -500,10 +602,18 @@ def bench_train(args, kda, workloads, dev, stream, world, rank):
         barrier(world, dev)
         kda.kda_device_status(stream)
         out[name] = {"ms_per_step": max_over_ranks(sum(per) / len(per), world, dev)}
+        out["launches"] += k * n_kernels[name]
     ms = out["forward_with_states"]["ms_per_step"] + out["backward"]["ms_per_step"]
     out["value"] = whole_job_value(w.token_heads, world, ms)
     out["unit"] = UNIT
-    out["roofline"] = None   # CUDA-core, SFU-bound path; no roofline figure until profiled
+    # The backward runs on the CUDA cores in fp32: its roofline is the FP32 FMA
+    # rate (148 SMs x 128 lanes x 2 x 1965 MHz), counted on twice the forward's
+    # useful FLOPs (the usual count for the gradient of a product chain).
+    ms_b = out["backward"]["ms_per_step"]
+    tfl = 2 * w.token_heads * chunk_flops_per_token_head(w.Dk, w.Dv, w.chunk) / (ms_b * 1e-3) / 1e12
+    out["backward"]["roofline"] = {"bound": "alu", "achieved": tfl, "peak": FP32_FMA_TFLOPS, "unit": "TFLOP/s",
+                                   "frac": tfl / FP32_FMA_TFLOPS, "traffic": None,
+                                   "flops": "2 x forward useful FLOPs"}
     return out
 
 

@@ -9,9 +9,9 @@
 //   output_gate_kernel  y = sigmoid(gate) * weight * o / sqrt(mean(o^2) + eps)
 //                       per (token, head) of 128 channels.
 //
-// Both are HBM-bound streams: one warp covers 128 channels of a token (lane =
-// 4 channels, 8-byte loads and stores, 256 contiguous bytes per warp), the
-// per-head reductions are warp shuffles, and nothing is read twice.
+// Both are HBM-bound streams: contiguous 8- or 16-byte loads and stores per
+// lane (256 or 512 contiguous bytes per warp and token), per-head reductions
+// by warp shuffles, and nothing read twice.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -41,77 +41,103 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 __device__ __forceinline__ float silu(float u) { return __fdividef(u, 1.f + __expf(-u)); }
 
-// Warp w of the grid: batch b, 128-channel group grp, tokens [t0, t0 + kConvTokens)
-// (only the 3 halo tokens before t0 are read twice).
+// Warp w of the grid: batch b, 256-channel group grp (lane = 8 channels, one
+// 16-byte load per token row; a 128-channel head is a half-warp), tokens
+// [t0, t0 + kConvTokens) (only the K-1 halo tokens before t0 are read twice).
+// A group of 128 channels at the end of a row leaves the upper half-warp idle.
+__host__ __device__ inline long long conv_grid_warps(const ConvParams &p) {
+    const long long nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
+    return (long long)p.B * ((p.C + 255) / 256) * nblk;
+}
+
+__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
+    const uint32_t r[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(r[i] << 16);
+        f[2 * i + 1] = __uint_as_float(r[i] & 0xFFFF0000u);
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        r[i] = *reinterpret_cast<uint32_t *>(&a);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
 template <int K>
-__global__ void __launch_bounds__(kLayerThreads)
+__global__ void __launch_bounds__(kLayerThreads, 2)
 short_conv_kernel(ConvParams p) {
     const int lane = threadIdx.x & 31;
     const long long gw = (long long)blockIdx.x * (kLayerThreads / 32) + (threadIdx.x >> 5);
-    const int ngrp = p.C / 128;
+    const int ngrp = (p.C + 255) / 256;
     const int nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
-    if (gw >= (long long)p.B * ngrp * nblk) return;
+    if (gw >= conv_grid_warps(p)) return;
     // Consecutive warps take consecutive channel groups of the same tokens, so
     // a thread block streams whole contiguous spans of each token row.
     const int grp = (int)(gw % ngrp);
     const int blk = (int)((gw / ngrp) % nblk);
     const int b = (int)(gw / ((long long)nblk * ngrp));
-    const int c0 = grp * 128 + 4 * lane;
+    const int c0 = grp * 256 + 8 * lane;
+    const bool act = c0 < p.C;                   // the upper half-warp of a 128-channel tail group idles
     const int t0 = blk * kConvTokens, t1 = min(p.T, t0 + kConvTokens);
     const __nv_bfloat16 *x = static_cast<const __nv_bfloat16 *>(p.x);
     const __nv_bfloat16 *sin = static_cast<const __nv_bfloat16 *>(p.state_in);
     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.y);
 
-    float w[4][4], bias[4];
+    float w[8][4], bias[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        bias[u] = p.bias ? p.bias[c0 + u] : 0.f;
+    for (int u = 0; u < 8; ++u) {
+        bias[u] = (act && p.bias) ? p.bias[c0 + u] : 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w[u][j] = j < K ? p.w[(size_t)(c0 + u) * K + j] : 0.f;
+        for (int j = 0; j < 4; ++j) w[u][j] = (act && j < K) ? p.w[(size_t)(c0 + u) * K + j] : 0.f;
     }
+    auto row = [&](int tok) { return *reinterpret_cast<const uint4 *>(x + ((size_t)b * p.T + tok) * p.C + c0); };
     // win[s]: token t - 3 + s, s = 0..2 (only the last K-1 slots are used).
-    auto fetch = [&](int tok, float (&f)[4]) {
-        if (tok >= 0) {
-            unpack4(*reinterpret_cast<const uint2 *>(x + ((size_t)b * p.T + tok) * p.C + c0), f);
-        } else if (sin && tok >= -(K - 1)) {
-            unpack4(*reinterpret_cast<const uint2 *>(sin + ((size_t)b * (K - 1) + (K - 1) + tok) * p.C + c0), f);
-        } else {
-            f[0] = f[1] = f[2] = f[3] = 0.f;
-        }
+    auto fetch = [&](int tok, float (&f)[8]) {
+        uint4 r = make_uint4(0, 0, 0, 0);
+        if (act && tok >= 0) r = row(tok);
+        else if (act && sin && tok >= -(K - 1))
+            r = *reinterpret_cast<const uint4 *>(sin + ((size_t)b * (K - 1) + (K - 1) + tok) * p.C + c0);
+        unpack8(r, f);
     };
-    float win[3][4];
+    float win[3][8];
 #pragma unroll
     for (int s = 0; s < 3; ++s) fetch(t0 - 3 + s, win[s]);
 
-    // Groups of 8 tokens, double-buffered: the 8 row loads of the next group
+    // Groups of 2 tokens, double-buffered: the 2 row loads of the next group
     // are in flight while the current group is computed.  Rows past the block
     // are computed from zeros and not stored.  state_out (the last K-1 tokens of
     // state_in ++ x, oldest first) is written at the sequence's last token.
-    constexpr int G = 8;
+    constexpr int G = 2;
     __nv_bfloat16 *so = static_cast<__nv_bfloat16 *>(p.state_out);
-    auto put_state = [&](const float (&s0)[4], const float (&s1)[4], const float (&s2)[4]) {
+    auto put_state = [&](const float (&s0)[8], const float (&s1)[8], const float (&s2)[8]) {
         const float *rows[3] = {s0, s1, s2};
 #pragma unroll
         for (int r = 0; r < K - 1; ++r) {
             const float *src = rows[4 - K + r];
-            const float f[4] = {src[0], src[1], src[2], src[3]};
-            *reinterpret_cast<uint2 *>(so + ((size_t)b * (K - 1) + r) * p.C + c0) = pack4(f);
+            float f[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) f[u] = src[u];
+            if (act) *reinterpret_cast<uint4 *>(so + ((size_t)b * (K - 1) + r) * p.C + c0) = pack8(f);
         }
     };
-    auto load_group = [&](int tg, uint2 (&r)[G]) {
+    auto load_group = [&](int tg, uint4 (&r)[G]) {
 #pragma unroll
-        for (int i = 0; i < G; ++i)
-            r[i] = tg + i < t1 ? *reinterpret_cast<const uint2 *>(x + ((size_t)b * p.T + tg + i) * p.C + c0)
-                               : make_uint2(0, 0);
+        for (int i = 0; i < G; ++i) r[i] = (act && tg + i < t1) ? row(tg + i) : make_uint4(0, 0, 0, 0);
     };
-    auto process = [&](int tg, const uint2 (&r)[G]) {
+    auto process = [&](int tg, const uint4 (&r)[G]) {
 #pragma unroll
         for (int i = 0; i < G; ++i) {
-            float cur[4];
-            unpack4(r[i], cur);
-            float out[4];
+            float cur[8];
+            unpack8(r[i], cur);
+            float out[8];
+            float ss = 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 // taps j = 0..K-2 read win[4 - K + j]; tap K-1 reads the current token
                 float acc = bias[u];
 #pragma unroll
@@ -119,24 +145,27 @@ short_conv_kernel(ConvParams p) {
                     if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
                 acc = fmaf(w[u][K - 1], cur[u], acc);
                 out[u] = p.silu ? silu(acc) : acc;
+                ss = fmaf(out[u], out[u], ss);
             }
             if (p.head_dim) {
-                const float ss = warp_sum(out[0] * out[0] + out[1] * out[1] + out[2] * out[2] + out[3] * out[3]);
+                // the head's 128 channels are this half-warp's 16 lanes
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                 const float rn = rsqrtf(ss + p.l2_eps);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) out[u] *= rn;
+                for (int u = 0; u < 8; ++u) out[u] *= rn;
             }
-            if (tg + i < t1) *reinterpret_cast<uint2 *>(y + ((size_t)b * p.T + tg + i) * p.C + c0) = pack4(out);
+            if (act && tg + i < t1) *reinterpret_cast<uint4 *>(y + ((size_t)b * p.T + tg + i) * p.C + c0) = pack8(out);
             if (so && tg + i + 1 == p.T) put_state(win[1], win[2], cur);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 win[0][u] = win[1][u];
                 win[1][u] = win[2][u];
                 win[2][u] = cur[u];
             }
         }
     };
-    uint2 ra[G], rb[G];
+    uint4 ra[G], rb[G];
     if (t0 < t1) load_group(t0, ra);
     for (int tg = t0; tg < t1; tg += 2 * G) {
         if (tg + G < t1) load_group(tg + G, rb);
@@ -192,8 +221,7 @@ output_gate_kernel(GateParams p) {
 }  // namespace
 
 cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s) {
-    const long long nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
-    const long long warps = (long long)p.B * (p.C / 128) * nblk;
+    const long long warps = conv_grid_warps(p);
     if (warps == 0) return cudaSuccess;
     const long long blocks = (warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32);
     switch (p.K) {

@@ -16,7 +16,8 @@ M S0 plus its run from zero), so each rank
 
 Every rank returns its own segment's o and the final state of the whole
 sequence.  The compute steps run in the library's kernels; the exchange is a
-process-group all-gather (NCCL between GPUs).
+process-group all-gather (NCCL between GPUs; a gloo group exchanges host
+copies of the blocks).
 """
 import torch
 import torch.distributed as dist
@@ -42,9 +43,15 @@ class _KernelOps:
     def all_gather(t, world, group):
         if world == 1:
             return t.unsqueeze(0)
-        parts = [torch.empty_like(t) for _ in range(world)]
-        dist.all_gather(parts, t.contiguous(), group=group)
-        return torch.stack(parts)
+        src = t.contiguous()
+        # a gloo group exchanges host memory: device blocks travel through host copies
+        via_host = src.is_cuda and dist.get_backend(group) == "gloo"
+        if via_host:
+            src = src.cpu()
+        parts = [torch.empty_like(src) for _ in range(world)]
+        dist.all_gather(parts, src, group=group)
+        out = torch.stack(parts)
+        return out.to(t.device) if via_host else out
 
 
 def _group_shape(group):

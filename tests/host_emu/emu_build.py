@@ -221,8 +221,7 @@ extern "C" int emu_sizeof_gate_params(void) { return (int)sizeof(kda::GateParams
 extern "C" int emu_short_conv(kda::ConvParams *pp) {
     using namespace kda;
     const ConvParams p = *pp;
-    const long long nblk = p.T > 0 ? (p.T + kConvTokens - 1) / kConvTokens : 1;
-    const long long warps = (long long)p.B * (p.C / 128) * nblk;
+    const long long warps = conv_grid_warps(p);
     if (warps == 0) return 0;
     const dim3 grid((unsigned)((warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32)));
     switch (p.K) {
