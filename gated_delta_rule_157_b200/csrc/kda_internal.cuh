@@ -117,5 +117,7 @@ cudaError_t launch_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
                            cudaStream_t s);
 // Device error word (set by bounded waits that gave up).  Reads and clears it.
 cudaError_t read_and_clear_device_error(cudaStream_t s, unsigned int *out);
+// The decode kernels' error word (after the stream has been synchronised).
+cudaError_t read_and_clear_step_error(unsigned int *out);
 
 }  // namespace kda

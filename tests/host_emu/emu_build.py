@@ -180,7 +180,9 @@ def _unit(src_name, runner, src_dir=CSRC):
     return head + "#line 1 \"%s\"\n" % src_name + s + runner
 
 
-_RUN_STEP = r'''
+_RUN_STEP = _POISON + r'''
+void emu_launch_cb(dim3 grid, dim3 block, const std::function<void(unsigned, unsigned)> &on_block,
+                   const std::function<void()> &fn);
 extern "C" int emu_sizeof_step_params(void) { return (int)sizeof(kda::StepParams); }
 template <int RPT>
 static void run_step(const kda::StepParams &p, int bf16) {
@@ -188,8 +190,33 @@ static void run_step(const kda::StepParams &p, int bf16) {
     if (bf16) emu_launch(dim3(p.B * p.HV), dim3(kThreads), [&] { step_kernel<RPT, __nv_bfloat16>(p); });
     else emu_launch(dim3(p.B * p.HV), dim3(kThreads), [&] { step_kernel<RPT, float>(p); });
 }
+namespace kda { namespace tc { extern EmuCta *g_cta; } }
+// Dk = Dv = 128: the persistent bulk-copy kernel, on a grid of at most two
+// CTAs so that every CTA walks several chains through its stage ring.
+static void run_step_bulk(const kda::StepParams &p, int bf16) {
+    using namespace kda;
+    static tc::EmuCta cta;
+    static tc::EmuMBar bars[sizeof(smem) / 8];
+    cta.smem = reinterpret_cast<uint8_t *>(smem);
+    cta.smem_bytes = BULK_SMEM;
+    cta.bars = bars;
+    const int nchains = p.B * p.HV;
+    const unsigned grid = nchains < 2 ? (unsigned)nchains : 2u;
+    emu_launch_cb(dim3(grid), dim3(kThreads), [&](unsigned, unsigned) {
+        emu_poison(BULK_SMEM);
+        std::memset(smem, 0, BULK_SMEM);
+        tc::g_cta = &cta;
+    }, [&] {
+        if (bf16) step_bulk_kernel<__nv_bfloat16>(p);
+        else step_bulk_kernel<float>(p);
+    });
+}
 extern "C" int emu_step(kda::StepParams *pp, int bf16) {
     const kda::StepParams p = *pp;
+    if (p.Dk == 128 && p.Dv == 128) {
+        run_step_bulk(p, bf16);
+        return 0;
+    }
     const int rpt = (p.Dk + kda::kWarps - 1) / kda::kWarps;
     if (rpt <= 1) run_step<1>(p, bf16);
     else if (rpt <= 2) run_step<2>(p, bf16);

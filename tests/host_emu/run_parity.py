@@ -309,6 +309,7 @@ STEP_CASES = [
     (2, 1, 2, 64, 32, "f32", "softplus", False, 12),
     (3, 2, 4, 128, 64, "bf16", "softplus", True, 13),
     (1, 1, 1, 32, 16, "f32", "bounded", True, 14),
+    (3, 1, 3, 128, 128, "bf16", "bounded", False, 15),   # 9 chains: stage reuse in the bulk-copy kernel
 ]
 
 CASES = [

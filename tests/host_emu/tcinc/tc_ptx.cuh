@@ -274,6 +274,19 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void *tmap,
 }
 __device__ __forceinline__ void prefetch_tensormap(const void *) {}
 __device__ __forceinline__ void tma_prefetch_3d(const void *, int, int, int) {}
+// Bulk copies complete at once (the load's mbarrier arrival follows).
+__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes, uint32_t mbar) {
+    std::memcpy(shared_ptr(dst_smem), src, bytes);
+    emu_complete_tx(mbar, bytes);
+}
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes) {
+    std::memcpy(dst, shared_ptr(src_smem), bytes);
+}
+__device__ __forceinline__ void bulk_commit() {}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {}
 
 // ---- special functions, conversions, warp-level tf32 mma -------------------------------
 __device__ __forceinline__ float ex2_approx(float x) { return std::exp2(x); }

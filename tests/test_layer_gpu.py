@@ -95,7 +95,17 @@ def test_output_gate(cuda_device, N, HV, with_w):
 def test_layer_core_composition(cuda_device):
     """Prologue -> core -> epilogue (the layer without its projections) against the
     oracle's composition: q, k, v from the short convolutions, the core with its
-    in-kernel gate and beta, the output gate on o."""
+    in-kernel gate and beta, the output gate on o.
+
+    Each stage is held to its own bar on the previous stage's actual output:
+    the prologue to 2^-7 of max|ref| (bf16 output), the core to the bf16 core
+    bar 2e-2 of max|o| on the prologue's bf16 rows, the epilogue to 2^-7 on the
+    core's o.  The composed output is also compared with the oracle's whole
+    composition on the rows whose RMS is at least a tenth of the largest: the
+    epilogue divides every row by its own RMS, so a row far below the tensor's
+    largest carries the core's absolute error (bounded relative to max|o|)
+    amplified by that ratio, which no max-relative bar on the composition
+    covers."""
     import workloads
     from helpers import oracle_chunk, to_device
     rng = np.random.default_rng(9)
@@ -111,15 +121,23 @@ def test_layer_core_composition(cuda_device):
                                 chunk=64, algo="tc")
     gate = _bf16(rng.standard_normal((B, T, 2, 128)), cuda_device)
     y = kda.kda_output_gate(o, gate)
-    # oracle: prologue in FP64 on the same bf16 inputs, rounded to bf16 like the kernel's output,
-    # then the core oracle (its q/k norm is idempotent on normalised rows), then the gate
+    # prologue stage: FP64 on the same bf16 inputs
     qr, _ = layer.prologue(_np(inp["q"]).reshape(B, T, 128), wq, head_dim=128)
     kr, _ = layer.prologue(_np(inp["k"]).reshape(B, T, 128), wk, head_dim=128)
     vr, _ = layer.prologue(_np(inp["v"]).reshape(B, T, 256), wv)
-    rnd = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).float().numpy()
-    core_in = {"q": rnd(qr).reshape(B, T, 1, 128), "k": rnd(kr).reshape(B, T, 1, 128),
-               "v": rnd(vr).reshape(B, T, 2, 128), "g": _np(inp["g"]), "beta": _np(inp["beta"]),
+    for got, want in ((q, qr), (k, kr), (v, vr)):
+        assert _rel(_np(got).reshape(want.shape), want) <= 2.0 ** -7
+    # core stage: the oracle on the prologue's own bf16 rows (its q/k norm is
+    # idempotent on normalised rows)
+    core_in = {"q": _np(q), "k": _np(k), "v": _np(v), "g": _np(inp["g"]), "beta": _np(inp["beta"]),
                "A_log": _np(inp["A_log"]), "dt_bias": _np(inp["dt_bias"]), "S0": None}
     o_ref = oracle_chunk(core_in)["o"]
+    assert _rel(_np(o), o_ref) <= 2e-2
+    # epilogue stage: the oracle gate on the core's own o
+    assert _rel(_np(y), layer.output_gate(_np(o), _np(gate))) <= 2.0 ** -7
+    # the whole composition on the rows the RMS division does not amplify
     ref = layer.output_gate(o_ref, _np(gate))
-    assert _rel(_np(y), ref) <= 2e-2
+    rms = np.sqrt((o_ref ** 2).mean(-1))
+    keep = rms >= 0.1 * rms.max()
+    assert keep.sum() >= keep.size // 2
+    assert _rel(_np(y)[keep], ref[keep]) <= 2e-2
