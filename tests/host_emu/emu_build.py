@@ -97,8 +97,8 @@ _RUN_TC = r'''
 #include <sanitizer/asan_interface.h>
 namespace kda { namespace tc { EmuCta *g_cta = nullptr; EmuTf32Slots g_tf32[32]; } }
 
-// The tensor maps the library's launcher builds (tokens x heads x 128 channels:
-// z in [64][1][128] boxes; q, k, v in [64][1][64] boxes with the 128-byte swizzle).
+// The tensor maps the library's launcher builds (tokens x heads x 128 channels,
+// [64][1][128] boxes; v in two [64][1][64] boxes with the 128-byte swizzle).
 static kda::tc::EmuTensorMap emu_row_map(const void *base, int heads, long long rows, bool sw128) {
     kda::tc::EmuTensorMap m{};
     m.base = static_cast<const uint8_t *>(base);
@@ -114,7 +114,7 @@ extern "C" int emu_chunk_tc(kda::ChunkParams *pp) {
     TcParams tp;
     tp.p = *pp;
     const long long rows = (long long)tp.p.B * tp.p.T;
-    const tc::EmuTensorMap maps[4] = {emu_row_map(tp.p.q, tp.p.H, rows, true), emu_row_map(tp.p.k, tp.p.H, rows, true),
+    const tc::EmuTensorMap maps[4] = {emu_row_map(tp.p.q, tp.p.H, rows, false), emu_row_map(tp.p.k, tp.p.H, rows, false),
                                       emu_row_map(tp.p.g, tp.p.HV, rows, false),
                                       emu_row_map(tp.p.v, tp.p.HV, rows, true)};
     for (int i = 0; i < 4; ++i) std::memcpy(&tp.tm[i], &maps[i], sizeof maps[i]);
