@@ -37,7 +37,7 @@ METRIC = "chunk_kda fwd tokens·heads/s + % bf16 TC peak; kda_step decode HBM GB
 # (profiles/chunk_tc_kernel_gva_b1.md: one B=1 launch, 32 chains, scaled by 4 to
 # the 128 chains of the B=4 launch; profiles/step_kernel_decode_bf16.md).
 CHUNK_TC_TRAFFIC_B4 = 4 * (202.115584e6 + 48.679168e6)
-STEP_TRAFFIC = 545.3e6 + 485.3e6
+STEP_TRAFFIC = 545.3e6 + 480.8e6
 UNIT = "tokens·heads/s"
 NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e, nominal (the measured copy peak is the roofline)
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # CUDA-core FP32: SMs x FMA lanes x 2 x max clock
@@ -50,10 +50,10 @@ def peaks():
             p = json.load(f)
         return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
                 "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
-                "source": "measured"}
+                "source": "measured (MEASURED_PEAKS.json)"}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-                "source": "fallback"}
+                "source": "fallback (MEASURED_PEAKS.json absent: earlier copy/cuBLAS measurement on B200)"}
 
 
 def chunk_flops_per_token_head(Dk, Dv, C):
@@ -389,7 +389,7 @@ def main():
                          "traffic": CHUNK_TC_TRAFFIC_B4 if (w.B == 4 and args.algo != "simt") else None,
                          "traffic_unit": "bytes per launch (ncu dram read + write)",
                          "kernel": "kda_chunk_fwd (%s)" % args.algo,
-                         "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst)"},
+                         "peak_source": pk["source"] + ", hbm_gbs burst"},
             "gpu_launches": args.steps}
     if clk is not None:
         line["clocks"] = clk
