@@ -81,13 +81,13 @@ constexpr uint32_t OFF_TB = 106496;       // [64 rows][K=64]    T Diag(beta)
 constexpr uint32_t OFF_QG = 114688;       // 2 x [64 rows][K=128]  Q Gamma
 constexpr uint32_t OFF_KP = 147456;       // 2 x K', token-major (MN-major B of (VI): N = 128 channels, K = 64)
 constexpr uint32_t OFF_AQK = 180224;      // 2 x [64 rows][K=64]   A_qk (lower, diagonal kept)
-constexpr uint32_t OFF_W = 196608;        // [128 K-rows][N=64] MN-major, -W
+constexpr uint32_t OFF_W = 196608;        // [128 K-rows][N=64] MN-major, -W; after (IV): o rows [64][128] bf16
 constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_RK = 0;           // float[64]
 constexpr uint32_t MISC_BETA = 256;       // float[64]
 constexpr uint32_t MISC_QSUM = 512;       // float[16 quarters][128] (log2 units)
 constexpr uint32_t MISC_GAM = 8704;       // float[2][128] gamma_C per buffer
-constexpr uint32_t MISC_RQ = 9728;        // float[64]
+constexpr uint32_t MISC_RQ = 9728;        // float[64] q norm factor times the output scale
 constexpr uint32_t MISC_TSUM = 9984;      // float[4][128] tile sums (log2 units)
 constexpr uint32_t MISC_BAR = 12032;      // 14 mbarriers
 constexpr uint32_t MISC_TMEM = 12144;     // uint32
@@ -117,11 +117,12 @@ constexpr uint32_t TMEM_COLS = 512;
 __host__ __device__ constexpr int kr_off(int r) { return 8 * r * (r + 1); }
 
 // Kernel parameters: the chunk arguments plus tensor maps of q, k (per key head)
-// and z, v (per value head), each viewed as [B*T tokens][heads][128 channels]
+// and z, v, o (per value head), each viewed as [B*T tokens][heads][128 channels]
 // with a [64 tokens][1][128] box.
 struct TcParams {
     ChunkParams p;
-    CUtensorMap tm[4];   // q, k, z, v
+    CUtensorMap tm[5];   // q, k, z, v, o
+    int o_tma;           // o rows of whole chunks leave by tensor store through tm[4]
 };
 
 struct Ctx {
@@ -395,11 +396,11 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
             // Lane l holds token ((l >> 4) & 1) * 2 + ((l >> 3) & 1) of this thread's four.
             if ((lane & 7) == 0) {
                 const int t = tq + ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-                rq_s[t] = rsqrtf(sq[0] + p.l2_eps);
+                rq_s[t] = rsqrtf(sq[0] + p.l2_eps) * p.scale;
                 rk_s[t] = rsqrtf(sk[0] + p.l2_eps);
             }
         } else if (lane < 4) {
-            rq_s[tq + lane] = 1.f;
+            rq_s[tq + lane] = p.scale;
             rk_s[tq + lane] = 1.f;
         }
         // The z rows (requested after the previous chunk's solve) arrive while
@@ -755,7 +756,8 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
 // =====================================================================
 // State role: warps 16-19, thread j <-> TMEM lane j <-> value channel j.
 // =====================================================================
-__device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, int tid) {
+__device__ __forceinline__ void state_role(const ChunkParams &p, const CUtensorMap *tmaps, bool o_tma, const Ctx &x,
+                                           int tid) {
     uint8_t *sm = x.sm;
     const int ts = tid - kPrepThreads;      // 0..127
     const int warp = tid >> 5;
@@ -815,6 +817,8 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
             }
         }
         if (ok) ok = wait_bar(x, bar_addr(x, MB_MMA_W + buf), (uint32_t)((n >> 1) & 1));
+        // The previous chunk's o rows in the -W tile have been read by their tensor store.
+        if (ts == 0) bulk_wait_read<0>();
         if (named_bar_any(BAR_STATE, kStateThreads, !ok)) break;
         fence_after_sync();
 
@@ -855,20 +859,21 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
         float *sck = (p.S_chunks && !x.trans) ? p.S_chunks + ((size_t)x.chain * x.nchunks + n) * D * D + j
                                               : nullptr;
         for (int mm = 0; mm < D / 16; ++mm) {
+            // gamma_C of these 16 columns (a broadcast read) is in flight with the TMEM load
+            const float4 *g4p = reinterpret_cast<const float4 *>(gam_s + buf * D + mm * 16);
+            const float4 g4[4] = {g4p[0], g4p[1], g4p[2], g4p[3]};
             float vals[16];
             tmem_ld16(x.tm + lane_base + COL_ST + mm * 16, vals);
             if (sck) {
 #pragma unroll
                 for (int u = 0; u < 16; ++u) sck[(size_t)(mm * 16 + u) * D] = vals[u];
             }
-            const float4 *g4 = reinterpret_cast<const float4 *>(gam_s + buf * D + mm * 16);
 #pragma unroll
             for (int u4 = 0; u4 < 4; ++u4) {
-                const float4 g = g4[u4];
-                vals[4 * u4 + 0] *= g.x;
-                vals[4 * u4 + 1] *= g.y;
-                vals[4 * u4 + 2] *= g.z;
-                vals[4 * u4 + 3] *= g.w;
+                vals[4 * u4 + 0] *= g4[u4].x;
+                vals[4 * u4 + 1] *= g4[u4].y;
+                vals[4 * u4 + 2] *= g4[u4].z;
+                vals[4 * u4 + 3] *= g4[u4].w;
             }
             tmem_st16(x.tm + lane_base + COL_ST + mm * 16, vals);
         }
@@ -931,9 +936,27 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
             for (int u = 0; u < 8; ++u) pk[u] = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
             tmem_st8(x.tm + lane_base + COL_SBF + mm * 8, pk);
         }
-        if (x.want_o) {
-            // o rows of this chunk: thread j writes value channel j of each token.
-            const int t0 = n * C, Cc = min(C, x.T - t0);
+        // o rows of this chunk (the output scale is in q's norm factor): thread j
+        // holds value channel j of each token.  A whole chunk goes through the -W
+        // tile (free since (IV) completed) as [64 tokens][128 channels] bf16 rows
+        // and leaves in one tensor store; a partial last chunk is stored directly.
+        const int t0 = n * C, Cc = min(C, x.T - t0);
+        const bool o_staged = x.want_o && o_tma && Cc == C;
+        if (o_staged) {
+#pragma unroll 1
+            for (int mm = 0; mm < C / 16; ++mm) {
+                float vals[16];
+                tmem_ld16(x.tm + lane_base + col_ut + mm * 16, vals);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t w = pack_bf16x2(vals[2 * u], vals[2 * u + 1]);
+                    uint8_t *row = sm + OFF_W + (uint32_t)(mm * 16 + 2 * u) * 256u + 2u * (uint32_t)j;
+                    *reinterpret_cast<uint16_t *>(row) = (uint16_t)(w & 0xFFFFu);
+                    *reinterpret_cast<uint16_t *>(row + 256) = (uint16_t)(w >> 16);
+                }
+            }
+            fence_async_smem();
+        } else if (x.want_o) {
             __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) +
                                   (((size_t)x.b * x.T + t0) * p.HV + x.hv) * D + j;
             const size_t tstride = (size_t)p.HV * D;
@@ -942,19 +965,26 @@ __device__ __forceinline__ void state_role(const ChunkParams &p, const Ctx &x, i
                 tmem_ld16(x.tm + lane_base + col_ut + mm * 16, vals);
 #pragma unroll
                 for (int u = 0; u < 16; ++u)
-                    if (mm * 16 + u < Cc) orow[(mm * 16 + u) * tstride] = __float2bfloat16_rn(p.scale * vals[u]);
+                    if (mm * 16 + u < Cc) orow[(mm * 16 + u) * tstride] = __float2bfloat16_rn(vals[u]);
             }
         }
         tmem_st_wait();
         fence_before_sync();
         named_bar(BAR_STATE, kStateThreads);
-        if (ts == 0) mbar_arrive(bar_addr(x, MB_FREE + buf));
+        if (ts == 0) {
+            if (o_staged) {
+                tma_store_3d(&tmaps[4], 0, x.hv, x.b * x.T + t0, x.sbase + OFF_W);
+                bulk_commit();
+            }
+            mbar_arrive(bar_addr(x, MB_FREE + buf));
+        }
     }
 
     // Every MMA this role issued ((II)-(VI)) must be complete before the TMEM
     // can be freed, after an abort too: one more commit arrives once all of
     // them are (at once if none is in flight); wait for it (bounded).
     if (ts == 0) {
+        bulk_wait<0>();                    // o tensor stores complete (shared rows read, global written)
         mma_commit(bar_addr(x, MB_DRAIN));
         for (uint32_t i = 0; i < kWaitTries; ++i)
             if (mbar_try_wait_suspend(bar_addr(x, MB_DRAIN), 0u, kSuspendNs)) break;
@@ -1009,7 +1039,7 @@ chunk_tc_kernel(const __grid_constant__ TcParams tp) {
     x.tm = *tmem_slot;
 
     if (warp < kPrepThreads / 32) prep_role(p, tp.tm, x, tid);
-    else state_role(p, x, tid);
+    else state_role(p, tp.tm, tp.o_tma != 0, x, tid);
 
     fence_before_sync();
     __syncthreads();
@@ -1067,6 +1097,9 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s) {
     if (p.g_per_head) memset(&tp.tm[2], 0, sizeof(tp.tm[2]));      // z is read directly
     else if ((e = make_row_map(&tp.tm[2], p.g, p.HV, rows)) != cudaSuccess) return e;
     if ((e = make_row_map(&tp.tm[3], p.v, p.HV, rows, /*swizzle128=*/true)) != cudaSuccess) return e;
+    // o by tensor stores when its map can be made (16-byte aligned base), else by plain stores
+    tp.o_tma = (p.o && make_row_map(&tp.tm[4], p.o, p.HV, rows) == cudaSuccess) ? 1 : 0;
+    if (!tp.o_tma) memset(&tp.tm[4], 0, sizeof(tp.tm[4]));
     dim3 grid(p.B * p.HV, p.M_T ? 2 : 1);
     chunk_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tp);
     return cudaGetLastError();

@@ -254,6 +254,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void *tmap,
         ::"r"(dst_smem), "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(mbar)
         : "memory");
 }
+// Tiled 3-D tensor store of one box from shared memory, in the executing
+// thread's current bulk group (commit, then wait with bulk_wait_read / bulk_wait).
+// Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, int c0, int c1, int c2, uint32_t src_smem) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+                 ::"l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(src_smem)
+                 : "memory");
+}
 // Contiguous bulk copies (no tensor map): global -> shared, completion counted
 // on `mbar` in bytes; shared -> global in a bulk group.  Addresses 16-byte
 // aligned, size a multiple of 16.
@@ -314,11 +322,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// fp32 -> tf32 (round to nearest, ties away), kept in a 32-bit register.
+// fp32 -> tf32 (round to nearest, ties away from zero), kept in a 32-bit
+// register: add half a unit in the last of the 10 kept mantissa bits to the
+// sign-magnitude word, then clear the 13 dropped bits.  Two integer-pipe
+// instructions instead of a conversion on the special-function pipe (a finite
+// value whose rounded magnitude overflows the format becomes infinite).
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
+    return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
 }
 
 // Warp-level D = A B + D with A 16x8 (row-major), B 8x8 (column-major), tf32

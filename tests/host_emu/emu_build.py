@@ -118,6 +118,9 @@ extern "C" int emu_chunk_tc(kda::ChunkParams *pp) {
                                       emu_row_map(tp.p.g, tp.p.HV, rows, false),
                                       emu_row_map(tp.p.v, tp.p.HV, rows, true)};
     for (int i = 0; i < 4; ++i) std::memcpy(&tp.tm[i], &maps[i], sizeof maps[i]);
+    const tc::EmuTensorMap omap = emu_row_map(tp.p.o, tp.p.HV, rows, false);
+    std::memcpy(&tp.tm[4], &omap, sizeof omap);
+    tp.o_tma = tp.p.o ? 1 : 0;
     static tc::EmuCta cta;
     static tc::EmuMBar bars[sizeof smem_raw / 8];
     cta.smem = smem_raw;

@@ -272,6 +272,25 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const void *tmap,
             }
     emu_complete_tx(mbar, off);
 }
+// Tensor store of one box: shared rows -> the tensor, elements outside it skipped
+// (completes at once; the bulk-group waits below are then no-ops).
+__device__ __forceinline__ void tma_store_3d(const void *tmap, int c0, int c1, int c2, uint32_t src_smem) {
+    EmuTensorMap m;
+    std::memcpy(&m, tmap, sizeof m);
+    uint32_t off = 0;
+    for (uint32_t z = 0; z < m.box[2]; ++z)
+        for (uint32_t y = 0; y < m.box[1]; ++y)
+            for (uint32_t x = 0; x < m.box[0]; ++x, off += 2) {
+                const long long gx = (long long)c0 + x, gy = (long long)c1 + y, gz = (long long)c2 + z;
+                if (gx < 0 || gy < 0 || gz < 0 || gx >= (long long)m.dims[0] || gy >= (long long)m.dims[1] ||
+                    gz >= (long long)m.dims[2])
+                    continue;
+                uint32_t a = src_smem + off;
+                if (m.swizzle128) a ^= ((a >> 7) & 7u) << 4;
+                std::memcpy(const_cast<uint8_t *>(m.base) + gz * m.strides[1] + gy * m.strides[0] + gx * 2,
+                            shared_ptr(a), 2);
+            }
+}
 __device__ __forceinline__ void prefetch_tensormap(const void *) {}
 __device__ __forceinline__ void tma_prefetch_3d(const void *, int, int, int) {}
 // Bulk copies complete at once (the load's mbarrier arrival follows).
