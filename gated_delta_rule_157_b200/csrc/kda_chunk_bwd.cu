@@ -138,13 +138,15 @@ chunk_bwd_kernel(BwdParams p) {
                 }
             }
         }
+        // G is kept in log2 units from here on: every use below is a power
+        // 2^(G_a - G_b) (or 2^G), one special-function instruction each.
         for (int c = tid; c < Dk; c += kThreads) {
             float run = 0.f;
             for (int r = 0; r < Cc; ++r) {
                 run += Gs[r * L + c];
-                Gs[r * L + c] = run;
+                Gs[r * L + c] = run * kLog2E;
             }
-            Glast[c] = run;
+            Glast[c] = run * kLog2E;
         }
         __syncthreads();
         // ---- 3. A, P and X = V - (K*exp(G)) S -------------------------------
@@ -155,7 +157,7 @@ chunk_bwd_kernel(BwdParams p) {
                 const float *kr = Ks + r * L, *ki = Ks + i * L, *qr = Qs + r * L;
                 const float *gr = Gs + r * L, *gi = Gs + i * L;
                 for (int c = 0; c < Dk; ++c) {
-                    const float kie = ki[c] * expf(gr[c] - gi[c]);
+                    const float kie = ki[c] * ex2f_(gr[c] - gi[c]);
                     a = fmaf(qr[c], kie, a);
                     pk = fmaf(kr[c], kie, pk);
                 }
@@ -166,7 +168,7 @@ chunk_bwd_kernel(BwdParams p) {
         }
         // warp w takes rows w, w + 8, ...; lane = value column
         for (int r = warp; r < Cc; r += kThreads / 32) {
-            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * expf(Gs[r * L + c]);
+            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * ex2f_(Gs[r * L + c]);
             __syncwarp();
             float acc = Xs[r * kVT + lane];
             for (int c = 0; c < Dk; ++c) acc = fmaf(-wb[c], Ss[c * kVT + lane], acc);
@@ -174,34 +176,58 @@ chunk_bwd_kernel(BwdParams p) {
             __syncwarp();
         }
         __syncthreads();
-        // ---- 4. U = (I + Diag(beta) P)^-1 Diag(beta) X (warp 0); the
-        //         exp(G_last) dS'.S term of the last row's dG (other warps) ----
-        if (warp == 0) {
-            // four partial sums shorten the dependent FMA chain of each row
-            for (int r = 0; r < Cc; ++r) {
-                float a0 = Xs[r * kVT + lane], a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                int i = 0;
-                for (; i + 3 < r; i += 4) {
-                    a0 = fmaf(-Pkk[r * C + i], Us[i * kVT + lane], a0);
-                    a1 = fmaf(-Pkk[r * C + i + 1], Us[(i + 1) * kVT + lane], a1);
-                    a2 = fmaf(-Pkk[r * C + i + 2], Us[(i + 2) * kVT + lane], a2);
-                    a3 = fmaf(-Pkk[r * C + i + 3], Us[(i + 3) * kVT + lane], a3);
-                }
-                for (; i < r; ++i) a0 = fmaf(-Pkk[r * C + i], Us[i * kVT + lane], a0);
-                Us[r * kVT + lane] = bet[r] * ((a0 + a1) + (a2 + a3));
-                __syncwarp();
-            }
-        } else {
-            for (int c = tid - 32; c < Dk; c += kThreads - 32) {
-                float acc = 0.f;
-                for (int j = 0; j < kVT; ++j) acc = fmaf(Ss[c * kVT + j], dSs[c * kVT + j], acc);
-                dlast[c] = expf(Glast[c]) * acc;
-            }
+        // ---- 4. U = (I + Diag(beta) P)^-1 Diag(beta) X by 16-row tiles: the
+        //         diagonal block by forward substitution (warp 0, lane = value
+        //         column), then its contribution taken off every later row (all
+        //         threads); U is built in place over a copy of X ------------------
+        for (int idx = tid; idx < Cc * kVT; idx += kThreads) Us[idx] = Xs[idx];
+        // the exp(G_last) dS'.S term of the last row's dG (independent of U)
+        for (int c = tid; c < Dk; c += kThreads) {
+            float acc = 0.f;
+            for (int j = 0; j < kVT; ++j) acc = fmaf(Ss[c * kVT + j], dSs[c * kVT + j], acc);
+            dlast[c] = ex2f_(Glast[c]) * acc;
         }
         __syncthreads();
+        for (int R0 = 0; R0 < Cc; R0 += 16) {
+            const int R1 = min(R0 + 16, Cc);
+            if (warp == 0) {
+                // the block's column lane in registers; row a takes the finished
+                // rows above it (row of P contiguous, two partial sums)
+                float u[16];
+#pragma unroll
+                for (int a = 0; a < 16; ++a) u[a] = (R0 + a < R1) ? Us[(R0 + a) * kVT + lane] : 0.f;
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    if (R0 + a >= R1) break;
+                    const float *pr = Pkk + (R0 + a) * C + R0;
+                    float acc0 = u[a], acc1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < a; ++i) {
+                        if (i & 1) acc1 = fmaf(-pr[i], u[i], acc1);
+                        else acc0 = fmaf(-pr[i], u[i], acc0);
+                    }
+                    u[a] = bet[R0 + a] * (acc0 + acc1);
+                }
+#pragma unroll
+                for (int a = 0; a < 16; ++a)
+                    if (R0 + a < R1) Us[(R0 + a) * kVT + lane] = u[a];
+            }
+            __syncthreads();
+            if (R1 < Cc) {
+                for (int idx = tid; idx < (Cc - R1) * kVT; idx += kThreads) {
+                    const int r = R1 + idx / kVT, jj = idx % kVT;
+                    float acc = Us[r * kVT + jj];
+#pragma unroll
+                    for (int a = 0; a < 16; ++a)
+                        if (R0 + a < R1) acc = fmaf(-Pkk[r * C + R0 + a], Us[(R0 + a) * kVT + jj], acc);
+                    Us[r * kVT + jj] = acc;
+                }
+                __syncthreads();
+            }
+        }
         // ---- 5. dU = A^T dO + (K*exp(G_last - G)) dS' ------------------------
         for (int r = warp; r < Cc; r += kThreads / 32) {
-            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * expf(Glast[c] - Gs[r * L + c]);
+            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * ex2f_(Glast[c] - Gs[r * L + c]);
             __syncwarp();
             float acc = 0.f;
             for (int rr = r; rr < Cc; ++rr) acc = fmaf(Aqk[rr * C + r], dOs[rr * kVT + lane], acc);
@@ -210,23 +236,42 @@ chunk_bwd_kernel(BwdParams p) {
             __syncwarp();
         }
         __syncthreads();
-        // ---- 6. dZ = (I + Diag(beta) P)^-T dU (warp 0, back substitution) ----
-        if (warp == 0) {
-            for (int r = Cc - 1; r >= 0; --r) {
-                float a0 = dUs[r * kVT + lane], a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                int rr = r + 1;
-                for (; rr + 3 < Cc; rr += 4) {
-                    a0 = fmaf(-bet[rr] * Pkk[rr * C + r], dUs[rr * kVT + lane], a0);
-                    a1 = fmaf(-bet[rr + 1] * Pkk[(rr + 1) * C + r], dUs[(rr + 1) * kVT + lane], a1);
-                    a2 = fmaf(-bet[rr + 2] * Pkk[(rr + 2) * C + r], dUs[(rr + 2) * kVT + lane], a2);
-                    a3 = fmaf(-bet[rr + 3] * Pkk[(rr + 3) * C + r], dUs[(rr + 3) * kVT + lane], a3);
+        // ---- 6. dZ = (I + Diag(beta) P)^-T dU in place, by 16-row tiles from
+        //         the last: the diagonal block by back substitution (warp 0), then
+        //         its contribution taken off every earlier row (all threads) ----
+        for (int T = (Cc - 1) >> 4; T >= 0; --T) {
+            const int R0 = 16 * T, R1 = min(R0 + 16, Cc);
+            if (warp == 0) {
+                // right-looking from the bottom: once dZ_b is final every earlier
+                // row of the block takes its term
+                float z[16];
+#pragma unroll
+                for (int a = 0; a < 16; ++a) z[a] = (R0 + a < R1) ? dUs[(R0 + a) * kVT + lane] : 0.f;
+#pragma unroll
+                for (int b = 15; b >= 0; --b) {
+                    if (R0 + b >= R1) continue;
+                    const float zb = bet[R0 + b] * z[b];
+#pragma unroll
+                    for (int a = 0; a < b; ++a) z[a] = fmaf(-Pkk[(R0 + b) * C + R0 + a], zb, z[a]);
                 }
-                for (; rr < Cc; ++rr) a0 = fmaf(-bet[rr] * Pkk[rr * C + r], dUs[rr * kVT + lane], a0);
-                dUs[r * kVT + lane] = (a0 + a1) + (a2 + a3);
-                __syncwarp();
+#pragma unroll
+                for (int a = 0; a < 16; ++a)
+                    if (R0 + a < R1) dUs[(R0 + a) * kVT + lane] = z[a];
+            }
+            __syncthreads();
+            if (R0 > 0) {
+                for (int idx = tid; idx < R0 * kVT; idx += kThreads) {
+                    const int r = idx / kVT, jj = idx % kVT;
+                    float acc = dUs[idx];
+#pragma unroll
+                    for (int a = 0; a < 16; ++a)
+                        if (R0 + a < R1)
+                            acc = fmaf(-bet[R0 + a] * Pkk[(R0 + a) * C + r], dUs[(R0 + a) * kVT + jj], acc);
+                    dUs[idx] = acc;
+                }
+                __syncthreads();
             }
         }
-        __syncthreads();
         // ---- 7. dA, dP, dbeta and dV ------------------------------------------
         // The column loops start at a lane-dependent offset so that the lanes
         // of a warp read different shared-memory banks.
@@ -268,13 +313,13 @@ chunk_bwd_kernel(BwdParams p) {
             // pairwise sums: row r against earlier tokens, then later tokens against r
             float aq = 0.f, pr = 0.f;
             for (int i = 0; i <= r; ++i) {
-                const float kie = Ks[i * L + c] * expf(grc - Gs[i * L + c]);
+                const float kie = Ks[i * L + c] * ex2f_(grc - Gs[i * L + c]);
                 aq = fmaf(Aqk[r * C + i], kie, aq);
                 pr = fmaf(Pkk[r * C + i], kie, pr);
             }
             float ak = 0.f, pc = 0.f;
             for (int rr = r; rr < Cc; ++rr) {
-                const float e = expf(Gs[rr * L + c] - grc);
+                const float e = ex2f_(Gs[rr * L + c] - grc);
                 ak = fmaf(Aqk[rr * C + r], Qs[rr * L + c] * e, ak);
                 pc = fmaf(Pkk[rr * C + r], Ks[rr * L + c] * e, pc);
             }
@@ -288,7 +333,7 @@ chunk_bwd_kernel(BwdParams p) {
                 dkw = fmaf(-br * dUs[r * kVT + j], s, dkw);
                 dkd = fmaf(Us[r * kVT + j], dSs[c * kVT + j], dkd);
             }
-            const float eg = expf(grc), ed = expf(Glast[c] - grc);
+            const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
             const size_t tq = ((tok0 + r) * p.H + h) * Dk + c;
             atomicAdd(&p.dq[tq], fmaf(eg, dqg, aq));
             atomicAdd(&p.dk[tq], ak + pr + pc + eg * dkw + ed * dkd);
@@ -300,12 +345,12 @@ chunk_bwd_kernel(BwdParams p) {
         // warp w takes key channels w, w + 8, ...; lane = value column
         for (int c = warp; c < Dk; c += kThreads / 32) {
             for (int r = lane; r < Cc; r += 32) {
-                const float e = expf(Gs[r * L + c]);
+                const float e = ex2f_(Gs[r * L + c]);
                 wb[r] = e * Qs[r * L + c];
                 wb[128 + r] = -e * Ks[r * L + c] * bet[r];
             }
             __syncwarp();
-            float acc = expf(Glast[c]) * dSs[c * kVT + lane];
+            float acc = ex2f_(Glast[c]) * dSs[c * kVT + lane];
             for (int r = 0; r < Cc; ++r) {
                 acc = fmaf(wb[r], dOs[r * kVT + lane], acc);
                 acc = fmaf(wb[128 + r], dUs[r * kVT + lane], acc);

@@ -21,6 +21,19 @@ __device__ __forceinline__ void st_act(__nv_bfloat16 *p, size_t i, float x) {
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 
+// 2^x on the special-function unit (PTX ex2.approx, relative error of a few ulp;
+// results below the normal range flush to 0); the plain library call on the host.
+constexpr float kLog2E = 1.4426950408889634f;
+__device__ __forceinline__ float ex2f_(float x) {
+#ifdef __CUDA_ARCH__
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+#else
+    return exp2f(x);
+#endif
+}
+
 // Bounded log-decay g = g_min * sigmoid(exp(A_log) * (z + dt_bias)); `ea` is exp(A_log).
 __device__ __forceinline__ float bounded_gate(float z, float bias, float ea, float g_min) {
     return g_min * sigmoidf_(ea * (z + bias));
