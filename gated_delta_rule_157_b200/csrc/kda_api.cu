@@ -325,11 +325,12 @@ kda_status kda_output_gate(const kda_gate_args *a, void *stream) {
 }
 
 kda_status kda_device_status(void *stream) {
-    unsigned int word = 0, step_word = 0;
+    unsigned int word = 0, step_word = 0, conv_word = 0;
     cudaError_t e = kda::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &word);
     if (e == cudaSuccess) e = kda::read_and_clear_step_error(&step_word);
+    if (e == cudaSuccess) e = kda::read_and_clear_conv_error(&conv_word);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
-    word |= step_word;
+    word |= step_word | conv_word;
     if (word & 1u) return KDA_ERR_TIMEOUT;
     return (word & 2u) ? KDA_ERR_RANGE : KDA_OK;
 }

@@ -132,5 +132,7 @@ cudaError_t launch_compose(int n_seg, int BH, int Dk, int Dv, const float *M,
 cudaError_t read_and_clear_device_error(cudaStream_t s, unsigned int *out);
 // The decode kernels' error word (after the stream has been synchronised).
 cudaError_t read_and_clear_step_error(unsigned int *out);
+// Layer prologue: bit 0 = a stage wait of the tiled short convolution gave up.
+cudaError_t read_and_clear_conv_error(unsigned int *out);
 
 }  // namespace kda

@@ -11,11 +11,17 @@
 //
 // Both are HBM-bound streams: contiguous 8- or 16-byte loads and stores per
 // lane (256 or 512 contiguous bytes per warp and token), per-head reductions
-// by warp shuffles, and nothing read twice.
+// by warp shuffles, and nothing read twice.  For rows of a multiple of 256
+// channels the short convolution streams [128 tokens x 256 channels] tiles
+// through shared memory by tensor-map copies (short_conv_tma_kernel).
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "kda_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace kda {
 namespace {
@@ -218,9 +224,220 @@ output_gate_kernel(GateParams p) {
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// short_conv_tma_kernel: the same convolution for C a multiple of 256, as a
+// stream of tiles (batch row b, 256 channels, 128 tokens) through shared
+// memory.  Persistent CTAs of 512 threads, one per SM; each takes a contiguous
+// range of tiles in the order channel group, batch row, token block (the
+// weights are reloaded only when the group changes).
+// Each tile arrives as one [131 rows x 256 channels] box of a 3-D tensor map
+// (tokens t0-3 .. t0+127; rows before the sequence or past its end read as
+// zeros) in a three-stage ring, two tiles (134 KB) ahead of the one computed,
+// enough bytes in flight per SM to cover the memory latency at full
+// bandwidth; output rows go straight from registers to global memory, 512
+// contiguous bytes per warp and token.  Warp w computes tokens t0 + 8w .. +7 with
+// its 3-token window in registers (16 warps per SM keep enough independent
+// work in flight for the per-token latency chain: taps, tanh, head-norm
+// shuffles, rsqrt), lane = 8 channels (16-byte shared loads,
+// a 128-channel head is a half-warp).  SiLU(u) = u sigmoid(u) with
+// sigmoid(u) = (1 + tanh(u/2)) / 2 on one special-function instruction.
+constexpr int kConvThreads = 512;                        // 16 warps
+constexpr int kTokPerWarp = 8;                           // kTT / 16
+constexpr int kTT = 128;                                 // tokens per tile
+static_assert(kTT == kTokPerWarp * (kConvThreads / 32), "the warps cover a tile");
+constexpr int kTC = 256;                                 // channels per tile
+constexpr int kHalo = 3;                                 // K - 1 <= 3 earlier tokens
+constexpr uint32_t kRowBytes = kTC * 2;                  // 512
+constexpr uint32_t kInBytes = (kTT + kHalo) * kRowBytes; // 67,072
+constexpr int kStages = 3;
+constexpr uint32_t TS_IN = 0;                            // kStages input tiles (128-byte aligned)
+constexpr uint32_t TS_BAR = kStages * kInBytes;          // kStages mbarriers
+constexpr uint32_t TS_SMEM = TS_BAR + 64;
+constexpr long long kConvWaitCycles = 4000000000LL;      // about two seconds of SM clock
+
+__device__ unsigned int g_conv_error = 0;                // bit 0: a stage wait gave up
+
+struct ConvTmaParams {
+    ConvParams p;
+    CUtensorMap tx;          // x as [B][T][C]: boxes of [1][131][256]
+};
+
+__device__ __forceinline__ float silu_tanh(float u) {
+    const float h = 0.5f * u;
+    float th;
+#ifdef __CUDA_ARCH__
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(h));
+#else
+    th = tanhf(h);
+#endif
+    return fmaf(h, th, h);
+}
+
+template <int K>
+__global__ void __launch_bounds__(kConvThreads, 1)
+short_conv_tma_kernel(const __grid_constant__ ConvTmaParams tp) {
+    const ConvParams &p = tp.p;
+    extern __shared__ __align__(1024) float smem[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(smem);
+    const uint32_t sbase = tc::smem_addr(sm);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nblk = (p.T + kTT - 1) / kTT;
+    const int ntiles = p.B * (p.C / kTC) * nblk;      // below 2^31 (checked by the launcher)
+    // This CTA's tiles are the contiguous range [n0, n1) of the order channel
+    // group (slowest), batch row, token block (fastest): moving to the next
+    // tile is an increment, and the weights change only at a group boundary.
+    const int n0 = (int)((long long)ntiles * blockIdx.x / gridDim.x);
+    const int my = (int)((long long)ntiles * (blockIdx.x + 1) / gridDim.x) - n0;
+    struct Cursor {
+        int g, b, blk;
+    };
+    auto first = [&]() {
+        Cursor c;
+        const int rows = p.B * nblk;
+        c.g = n0 / rows;
+        c.b = (n0 % rows) / nblk;
+        c.blk = n0 % nblk;
+        return c;
+    };
+    auto advance = [&](Cursor &c) {
+        if (++c.blk == nblk) {
+            c.blk = 0;
+            if (++c.b == p.B) {
+                c.b = 0;
+                ++c.g;
+            }
+        }
+    };
+    auto bar = [&](int st) { return sbase + TS_BAR + 8u * (uint32_t)st; };
+    Cursor ic = first();                              // the next tile to request (thread 0)
+    int ii = 0;
+    auto issue = [&]() {
+        const int st = ii % kStages;
+        tc::mbar_arrive_expect_tx(bar(st), kInBytes);
+        tc::tma_load_3d(sbase + TS_IN + (uint32_t)st * kInBytes, &tp.tx, ic.g * kTC, ic.blk * kTT - kHalo, ic.b,
+                        bar(st));
+        advance(ic);
+        ++ii;
+    };
+    if (tid == 0) {
+        for (int st = 0; st < kStages; ++st) tc::mbar_init(bar(st), 1);
+        tc::fence_mbar_init();
+        tc::prefetch_tensormap(&tp.tx);
+    }
+    __syncthreads();
+    if (tid == 0)
+        while (ii < my && ii < kStages - 1) issue();
+    const __nv_bfloat16 *sin = static_cast<const __nv_bfloat16 *>(p.state_in);
+    __nv_bfloat16 *so = static_cast<__nv_bfloat16 *>(p.state_out);
+    float w[8][4], bias[8];
+    int wg = -1;                                      // channel group whose weights are loaded
+    int i = 0;
+    bool aborted = false;
+    Cursor cc = first();                              // the tile computed
+    for (; i < my; ++i, advance(cc)) {
+        const int b = cc.b, g = cc.g, blk = cc.blk;
+        const int st = i % kStages;
+        // its stage was read by tile i - 1, finished before the barrier that ended it
+        if (tid == 0 && ii < my) issue();
+        bool ok = tc::mbar_try_wait(bar(st), (uint32_t)((i / kStages) & 1));
+        if (!ok) {
+            const long long c0 = clock64();
+            while (!(ok = tc::mbar_try_wait(bar(st), (uint32_t)((i / kStages) & 1))))
+                if (clock64() - c0 > kConvWaitCycles) break;
+        }
+        if (__syncthreads_or(!ok)) {
+            aborted = true;
+            break;
+        }
+        if (g != wg) {
+            wg = g;
+            const int c = g * kTC + 8 * lane;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                bias[u] = p.bias ? p.bias[c + u] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) w[u][j] = j < K ? p.w[(size_t)(c + u) * K + j] : 0.f;
+            }
+        }
+        const int t0 = blk * kTT, t1 = min(p.T, t0 + kTT);
+        uint8_t *in = sm + TS_IN + (uint32_t)st * kInBytes;            // row r: token t0 - 3 + r
+        const int tw = kTokPerWarp * warp;
+        __nv_bfloat16 *yr = static_cast<__nv_bfloat16 *>(p.y) + ((size_t)b * p.T + t0 + tw) * p.C + g * kTC + 8 * lane;
+        if (t0 == 0 && sin) {
+            // the window before the sequence: the carried K-1 tokens (oldest first)
+            for (int idx = tid; idx < (K - 1) * (kTC / 8); idx += kConvThreads) {
+                const int r = idx / (kTC / 8), l8 = idx % (kTC / 8);
+                *reinterpret_cast<uint4 *>(in + (uint32_t)(kHalo - (K - 1) + r) * kRowBytes + 16u * l8) =
+                    *reinterpret_cast<const uint4 *>(sin + ((size_t)b * (K - 1) + r) * p.C + g * kTC + 8 * l8);
+            }
+            __syncthreads();
+        }
+        float win[3][8];
+#pragma unroll
+        for (int s = 0; s < 3; ++s)
+            unpack8(*reinterpret_cast<const uint4 *>(in + (uint32_t)(tw + s) * kRowBytes + 16u * lane), win[s]);
+#pragma unroll
+        for (int k = 0; k < kTokPerWarp; ++k) {
+            float cur[8];
+            unpack8(*reinterpret_cast<const uint4 *>(in + (uint32_t)(tw + kHalo + k) * kRowBytes + 16u * lane), cur);
+            float o[8];
+            float ss = 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                // taps j = 0..K-2 read win[4 - K + j]; tap K-1 reads the current token
+                float acc = bias[u];
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
+                acc = fmaf(w[u][K - 1], cur[u], acc);
+                o[u] = p.silu ? silu_tanh(acc) : acc;
+                ss = fmaf(o[u], o[u], ss);
+            }
+            if (p.head_dim) {
+#pragma unroll
+                for (int m = 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                const float rn = rsqrtf(ss + p.l2_eps);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) o[u] *= rn;
+            }
+            if (t0 + tw + k < t1) *reinterpret_cast<uint4 *>(yr + (size_t)k * p.C) = pack8(o);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                win[0][u] = win[1][u];
+                win[1][u] = win[2][u];
+                win[2][u] = cur[u];
+            }
+        }
+        // state_out: the last K-1 tokens of state_in ++ x, still in the input tile
+        if (so && t1 == p.T && warp == 0) {
+            for (int r = 0; r < K - 1; ++r) {
+                const int row = p.T - t0 + kHalo - (K - 1) + r;
+                *reinterpret_cast<uint4 *>(so + ((size_t)b * (K - 1) + r) * p.C + g * kTC + 8 * lane) =
+                    *reinterpret_cast<const uint4 *>(in + (uint32_t)row * kRowBytes + 16u * lane);
+            }
+        }
+        __syncthreads();                              // stage st is free for tile i + kStages
+    }
+    if (tid == 0 && aborted) {
+        atomicOr(&g_conv_error, 1u);
+        // tiles i .. i + kStages - 2 may still be arriving: let them land (bounded)
+        for (int j = i; j < ii; ++j)
+            for (int tries = 0; tries < 4000; ++tries)
+                if (tc::mbar_try_wait_suspend(bar((int)(j % kStages)), (uint32_t)((j / kStages) & 1), 500000u))
+                    break;
+    }
+}
+
 }  // namespace
 
+// The tiled kernel, when the shape and buffers allow it (defined below).
+cudaError_t launch_short_conv_tma(const ConvParams &p, cudaStream_t s, bool &launched);
+
 cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s) {
+    bool launched = false;
+    const cudaError_t e0 = launch_short_conv_tma(p, s, launched);
+    if (e0 != cudaSuccess || launched) return e0;
     const long long warps = conv_grid_warps(p);
     if (warps == 0) return cudaSuccess;
     const long long blocks = (warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32);
@@ -239,6 +456,73 @@ cudaError_t launch_output_gate(const GateParams &p, cudaStream_t s) {
     const long long blocks = (warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32);
     output_gate_kernel<<<(unsigned)blocks, kLayerThreads, 0, s>>>(p);
     return cudaGetLastError();
+}
+
+// Tensor map of a bf16 [B][T][C] tensor (channels innermost) with a box of
+// [1][rows][256] channels.
+static bool make_conv_map(CUtensorMap *map, const void *base, const ConvParams &p, int rows) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return false;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)p.C, (cuuint64_t)p.T, (cuuint64_t)p.B};
+    const cuuint64_t strides[2] = {(cuuint64_t)p.C * 2, (cuuint64_t)p.T * p.C * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)kTC, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The tiled kernel takes rows of a multiple of 256 channels, K <= 4, at least
+// one token, and 16-byte aligned state buffers; everything else the warp kernel.
+static bool conv_tma_eligible(const ConvParams &p) {
+    return p.C % kTC == 0 && p.T > 0 && p.K >= 1 && p.K <= 4 && (p.head_dim == 0 || p.head_dim == 128) &&
+           ((uintptr_t)p.state_in % 16 == 0) && ((uintptr_t)p.state_out % 16 == 0);
+}
+
+cudaError_t launch_short_conv_tma(const ConvParams &p, cudaStream_t s, bool &launched) {
+    launched = false;
+    if (!conv_tma_eligible(p)) return cudaSuccess;
+    ConvTmaParams tp;
+    tp.p = p;
+    if (!make_conv_map(&tp.tx, p.x, p, kTT + kHalo) || (uintptr_t)p.y % 16 != 0) return cudaSuccess;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long ntiles = (long long)p.B * (p.C / kTC) * ((p.T + kTT - 1) / kTT);
+    if (ntiles >= (1LL << 31)) return cudaSuccess;                 // the warp kernel takes it
+    const long long grid = ntiles < sms ? ntiles : sms;
+    switch (p.K) {
+#define KDA_CONV_TMA(KK)                                                                                      \
+    case KK:                                                                                                  \
+        if ((e = cudaFuncSetAttribute(short_conv_tma_kernel<KK>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                                      (int)TS_SMEM)) != cudaSuccess)                                          \
+            return e;                                                                                         \
+        short_conv_tma_kernel<KK><<<(unsigned)grid, kConvThreads, TS_SMEM, s>>>(tp);                         \
+        break;
+        KDA_CONV_TMA(1)
+        KDA_CONV_TMA(2)
+        KDA_CONV_TMA(3)
+        default: KDA_CONV_TMA(4)
+#undef KDA_CONV_TMA
+    }
+    launched = true;
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_conv_error(unsigned int *out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_conv_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_conv_error, &zero, sizeof(unsigned int));
 }
 
 }  // namespace kda

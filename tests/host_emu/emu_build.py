@@ -245,12 +245,56 @@ extern "C" int emu_compose(int n_seg, int BH, int Dk, int Dv, const float *M, co
     return 0;
 }
 '''
-_RUN_LAYER = r'''
+_RUN_LAYER = _POISON + r'''
+void emu_launch_cb(dim3 grid, dim3 block, const std::function<void(unsigned, unsigned)> &on_block,
+                   const std::function<void()> &fn);
 extern "C" int emu_sizeof_conv_params(void) { return (int)sizeof(kda::ConvParams); }
 extern "C" int emu_sizeof_gate_params(void) { return (int)sizeof(kda::GateParams); }
+namespace kda { namespace tc { extern EmuCta *g_cta; } }
+// The tiled kernel's tensor maps ([B][T][C], boxes of [1][rows][256]), run on
+// a grid of at most three CTAs so that every CTA walks several tiles through
+// its stage ring (and, with two or more channel groups, changes groups).
+static kda::tc::EmuTensorMap emu_conv_map(const void *base, const kda::ConvParams &p, int rows) {
+    kda::tc::EmuTensorMap m{};
+    m.base = static_cast<const uint8_t *>(base);
+    m.dims[0] = (uint64_t)p.C; m.dims[1] = (uint64_t)p.T; m.dims[2] = (uint64_t)p.B;
+    m.strides[0] = (uint64_t)p.C * 2; m.strides[1] = (uint64_t)p.T * p.C * 2;
+    m.box[0] = 256; m.box[1] = (uint32_t)rows; m.box[2] = 1;
+    return m;
+}
+template <int K>
+static void run_conv_tma(const kda::ConvParams &p) {
+    using namespace kda;
+    ConvTmaParams tp;
+    tp.p = p;
+    const tc::EmuTensorMap mx = emu_conv_map(p.x, p, kTT + kHalo);
+    std::memcpy(&tp.tx, &mx, sizeof mx);
+    static tc::EmuCta cta;
+    static tc::EmuMBar bars[sizeof(smem) / 8];
+    cta.smem = reinterpret_cast<uint8_t *>(smem);
+    cta.smem_bytes = TS_SMEM;
+    cta.bars = bars;
+    const long long ntiles = (long long)p.B * (p.C / kTC) * ((p.T + kTT - 1) / kTT);
+    const unsigned grid = ntiles < 3 ? (unsigned)ntiles : 3u;
+    emu_launch_cb(dim3(grid), dim3(kConvThreads), [&](unsigned, unsigned) {
+        emu_poison(TS_SMEM);
+        std::memset(smem, 0, TS_SMEM);
+        tc::g_cta = &cta;
+    }, [&] { short_conv_tma_kernel<K>(tp); });
+}
 extern "C" int emu_short_conv(kda::ConvParams *pp) {
     using namespace kda;
     const ConvParams p = *pp;
+    if (p.C % kTC == 0 && p.T > 0 && p.K >= 1 && p.K <= 4 && (p.head_dim == 0 || p.head_dim == 128) &&
+        (uintptr_t)p.state_in % 16 == 0 && (uintptr_t)p.state_out % 16 == 0 && (uintptr_t)p.y % 16 == 0) {
+        switch (p.K) {
+            case 1: run_conv_tma<1>(p); break;
+            case 2: run_conv_tma<2>(p); break;
+            case 3: run_conv_tma<3>(p); break;
+            default: run_conv_tma<4>(p); break;
+        }
+        return 0;
+    }
     const long long warps = conv_grid_warps(p);
     if (warps == 0) return 0;
     const dim3 grid((unsigned)((warps + kLayerThreads / 32 - 1) / (kLayerThreads / 32)));

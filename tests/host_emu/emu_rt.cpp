@@ -1,6 +1,7 @@
 // One CUDA block = blockDim.x std::threads; __syncthreads / __syncwarp are
 // std::barriers, a thread that leaves the kernel drops out of them (as an
 // exited GPU thread does), __shfl_xor_sync exchanges through per-warp slots.
+#include <atomic>
 #include <barrier>
 #include <functional>
 #include <memory>
@@ -19,6 +20,20 @@ float g_slots[32][32];
 }
 
 void __syncthreads() { g_block->arrive_and_wait(); }
+// Barrier with an OR of the threads' predicates.  Call k (counted per thread,
+// the same k in every thread of the block) accumulates in slot k % 3; after
+// the barrier thread 0 clears slot (k + 2) % 3, whose last reads were before
+// this barrier and whose next writes come after the next one.
+static std::atomic<int> g_or_acc[3];
+thread_local unsigned g_or_calls = 0;
+int __syncthreads_or(int pred) {
+    const unsigned k = g_or_calls++ % 3;
+    if (pred) g_or_acc[k].fetch_or(1);
+    g_block->arrive_and_wait();
+    const int r = g_or_acc[k].load();
+    if (threadIdx.x == 0) g_or_acc[(k + 2) % 3].store(0);
+    return r;
+}
 void __syncwarp(unsigned) { g_warp[threadIdx.x / 32]->arrive_and_wait(); }
 float __shfl_xor_sync(unsigned, float v, int off) {
     const int w = threadIdx.x / 32, l = threadIdx.x % 32;
@@ -42,6 +57,7 @@ void emu_launch_cb(dim3 grid, dim3 block, const std::function<void(unsigned, uns
     for (unsigned by = 0; by < grid.y; ++by)
         for (unsigned bx = 0; bx < grid.x; ++bx) {
             on_block(bx, by);
+            for (auto &a : g_or_acc) a.store(0);
             g_block = std::make_unique<std::barrier<>>(nt);
             g_warp.clear();
             for (unsigned w = 0; w < (nt + 31) / 32; ++w)

@@ -26,6 +26,7 @@ struct dim3 {
 extern thread_local uint3 threadIdx, blockIdx;
 extern thread_local dim3 blockDim, gridDim;
 void __syncthreads();
+int __syncthreads_or(int pred);
 void __syncwarp(unsigned mask = 0xffffffffu);
 float __shfl_xor_sync(unsigned mask, float v, int off);
 inline float atomicAdd(float *a, float v) { return std::atomic_ref<float>(*a).fetch_add(v); }

@@ -301,6 +301,8 @@ LAYER_CASES = [
     (2, 100, 256, 4, 128, True, False, 31),
     (1, 7, 128, 3, 0, False, True, 32),
     (1, 0, 128, 4, 0, True, True, 33),
+    (2, 150, 512, 3, 128, True, True, 34),
+    (3, 1, 256, 4, 0, True, True, 35),
 ]
 
 STEP_CASES = [
