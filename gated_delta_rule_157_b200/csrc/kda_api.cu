@@ -285,9 +285,10 @@ kda_status kda_short_conv(const kda_conv_args *a, void *stream) {
     if (a->B == 0) return KDA_OK;
     const size_t ntok = (size_t)a->B * a->T, es = 2;
     if (!a->w || (ntok > 0 && (!a->x || !a->y))) return KDA_ERR_INVALID_ARG;
-    const void *p8[] = {a->x, a->y, a->state_in, a->state_out};
-    for (const void *p : p8)
-        if (p && !aligned(p, 8)) return KDA_ERR_ALIGNMENT;
+    // the kernels move 8 channels (16 bytes) per lane
+    const void *p16[] = {a->x, a->y, a->state_in, a->state_out};
+    for (const void *p : p16)
+        if (p && !aligned(p, 16)) return KDA_ERR_ALIGNMENT;
     if (!aligned(a->w, 4) || (a->bias && !aligned(a->bias, 4))) return KDA_ERR_ALIGNMENT;
     const size_t nx = ntok * a->C * es, ns = (size_t)a->B * (a->K - 1) * a->C * es;
     Range r_y = range_of(a->y, ntok ? nx : 0), r_so = range_of(a->state_out, a->state_out ? ns : 0);

@@ -277,8 +277,11 @@ typedef struct {
 } kda_conv_args;
 
 /* Runs the prologue above.  T may be 0 (only state_out is written).  x, y,
- * state_in and state_out must be 8-byte aligned; y and state_out must not
- * overlap any input or each other.  Errors as for kda_chunk_fwd. */
+ * state_in and state_out must be 16-byte aligned (KDA_ERR_ALIGNMENT
+ * otherwise); y and state_out must not overlap any input or each other.
+ * Errors as for kda_chunk_fwd; rows of a multiple of 256 channels are
+ * streamed through shared memory with clock-bounded waits, and a wait that
+ * gives up is reported by kda_device_status as KDA_ERR_TIMEOUT. */
 kda_status kda_short_conv(const kda_conv_args *args, void *stream);
 
 /* Output gate of the layer (the epilogue before the output projection):
@@ -300,9 +303,10 @@ typedef struct {
  * overlap o or gate.  Errors as for kda_chunk_fwd. */
 kda_status kda_output_gate(const kda_gate_args *args, void *stream);
 
-/* Reads and clears the device error word of the current device after
- * synchronising `stream`.  Returns KDA_OK, KDA_ERR_TIMEOUT (a bounded wait
- * gave up since the last call; takes precedence), KDA_ERR_RANGE (a
+/* Reads and clears the device error words of the current device (chunk
+ * kernel, decode step, layer prologue) after synchronising `stream`.
+ * Returns KDA_OK, KDA_ERR_TIMEOUT (a bounded wait gave up since the last
+ * call; takes precedence), KDA_ERR_RANGE (a
  * tensor-core call clamped a caller-given log-decay below g_min) or
  * KDA_ERR_CUDA. */
 kda_status kda_device_status(void *stream);

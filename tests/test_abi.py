@@ -228,7 +228,9 @@ def test_layer_null_and_empty():
     ("head_dim", 64, UNSUPPORTED),
     ("w", None, INVALID),
     ("x", None, INVALID),
-    ("x", 0x7f0000100004, ALIGN),     # 8-byte rows
+    ("x", 0x7f0000100004, ALIGN),     # 16-byte rows
+    ("x", 0x7f0000100008, ALIGN),     # 8-byte aligned is not enough
+    ("state_in", 0x7f0000700008, ALIGN),
     ("state_out", 0x7f0000600002, ALIGN),
     ("y", 0x7f0000100000, ALIAS),     # y == x
     ("state_out", 0x7f0000500000, ALIAS),   # state_out == y
