@@ -36,7 +36,7 @@ METRIC = "chunk_kda fwd tokens·heads/s + % bf16 TC peak; kda_step decode HBM GB
 # DRAM bytes (read + write) per launch from ncu captures of the current kernels
 # (profiles/chunk_tc_kernel_gva_b1.md: one B=1 launch, 32 chains, scaled by 4 to
 # the 128 chains of the B=4 launch; profiles/step_kernel_decode_bf16.md).
-CHUNK_TC_TRAFFIC_B4 = 4 * (202.115584e6 + 48.679168e6)
+CHUNK_TC_TRAFFIC_B4 = 4 * (201.954816e6 + 50.557440e6)   # ncu dram read + write of one B=1 launch, x4 chains
 STEP_TRAFFIC = 545.3e6 + 480.8e6
 UNIT = "tokens·heads/s"
 NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e, nominal (the measured copy peak is the roofline)
@@ -326,6 +326,9 @@ def main():
                     help="override B of the headline workload (small cases for profiling)")
     ap.add_argument("--train", action="store_true",
                     help="(kept for compatibility: the training path is always timed with the extras)")
+    ap.add_argument("--only", default=None, choices=["small", "decode", "kcp", "layer", "train"],
+                    help="run one extra entry alone and print its object (for profiling one kernel; "
+                         "not the result line)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -340,6 +343,19 @@ def main():
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     pk = peaks()
+
+    if args.only:
+        entries = {
+            "small": lambda: bench_small_configs(args, kda, workloads, dev, stream, pk, world, rank),
+            "decode": lambda: bench_decode(args, kda, workloads, dev, stream, pk, world, rank),
+            "kcp": lambda: bench_kcp(args, kda, workloads, dev, stream, world, rank),
+            "layer": lambda: bench_layer(args, kda, dev, stream, pk, world),
+            "train": lambda: bench_train(args, kda, workloads, dev, stream, world, rank),
+        }
+        res = entries[args.only]()
+        if rank == 0:
+            print(json.dumps({"entry": args.only, **res}), flush=True)
+        return 0
 
     # ---------------- headline: chunked forward, B=4 HV=32 T=8192 -------------
     w = workloads.workload("gva_bf16")

@@ -54,10 +54,29 @@ def test_short_conv(cuda_device, K, head_dim, act, T, with_state):
     assert np.array_equal(_np(so), ref_st)            # carried tokens are copied exactly
 
 
-def test_short_conv_decode_steps_equal_one_run(cuda_device):
-    """One token at a time with the carried window equals the whole sequence."""
+def test_short_conv_tiled_groups_and_tiles(cuda_device):
+    """Rows of several 256-channel groups and several 128-token tiles (the
+    tiled kernel): ragged last tile, carried window in and out, three taps."""
+    rng = np.random.default_rng(41)
+    B, T, C, K = 3, 300, 768, 3
+    x = _bf16(rng.standard_normal((B, T, C)), cuda_device)
+    w = rng.standard_normal((C, K)).astype(np.float32)
+    bias = rng.standard_normal(C).astype(np.float32) * 0.1
+    st = _bf16(rng.standard_normal((B, K - 1, C)), cuda_device)
+    y, so = kda.kda_short_conv(x, _f32(w, cuda_device), _f32(bias, cuda_device), head_dim=128, state_in=st,
+                               want_state=True)
+    ref, ref_st = layer.prologue(_np(x), w, bias, _np(st), head_dim=128, act=True)
+    assert _rel(_np(y), ref) <= TOL
+    assert np.array_equal(_np(so), ref_st)
+    assert kda.kda_device_status() is None
+
+
+@pytest.mark.parametrize("C", [128, 512])
+def test_short_conv_decode_steps_equal_one_run(cuda_device, C):
+    """One token at a time with the carried window equals the whole sequence
+    (C = 128: the warp kernel; C = 512: the tiled kernel, both ways)."""
     rng = np.random.default_rng(5)
-    B, T, C = 3, 9, 128
+    B, T = 3, 9
     x = _bf16(rng.standard_normal((B, T, C)), cuda_device)
     w = _f32(rng.standard_normal((C, 4)), cuda_device)
     full = kda.kda_short_conv(x, w, head_dim=128)
