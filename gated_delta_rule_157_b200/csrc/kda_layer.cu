@@ -263,8 +263,9 @@ struct ConvTmaParams {
     CUtensorMap tx;          // x as [B][T][C]: boxes of [1][131][256]
 };
 
-__device__ __forceinline__ float silu_tanh(float u) {
-    const float h = 0.5f * u;
+// SiLU(2h) = h + h tanh(h): the tiled kernel keeps its taps and bias halved,
+// so its convolution yields h = u / 2 directly.
+__device__ __forceinline__ float silu_of_half(float h) {
     float th;
 #ifdef __CUDA_ARCH__
     asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(h));
@@ -355,9 +356,10 @@ short_conv_tma_kernel(const __grid_constant__ ConvTmaParams tp) {
             const int c = g * kTC + 8 * lane;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                bias[u] = p.bias ? p.bias[c + u] : 0.f;
+                // halved (exact in binary floating point): the convolution gives u / 2
+                bias[u] = p.bias ? 0.5f * p.bias[c + u] : 0.f;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) w[u][j] = j < K ? p.w[(size_t)(c + u) * K + j] : 0.f;
+                for (int j = 0; j < 4; ++j) w[u][j] = j < K ? 0.5f * p.w[(size_t)(c + u) * K + j] : 0.f;
             }
         }
         const int t0 = blk * kTT, t1 = min(p.T, t0 + kTT);
@@ -391,7 +393,7 @@ short_conv_tma_kernel(const __grid_constant__ ConvTmaParams tp) {
                 for (int j = 0; j < 3; ++j)
                     if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
                 acc = fmaf(w[u][K - 1], cur[u], acc);
-                o[u] = p.silu ? silu_tanh(acc) : acc;
+                o[u] = p.silu ? silu_of_half(acc) : 2.f * acc;
                 ss = fmaf(o[u], o[u], ss);
             }
             if (p.head_dim) {
