@@ -499,6 +499,29 @@ def bench_small_configs(args, kda, workloads, dev, stream, pk, world, rank):
             e["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": gbs / pk["hbm_gbs"], "traffic": None}
             e["occupancy"] = "%d chains on 148 SMs: one CTA per chain" % (w.B * w.HV)
+            # the same forward with each sequence cut into segments run in
+            # parallel (states-only pass with transitions, compose, output pass)
+            nseg = kda.seq_segments(w.B, w.HV, w.T, w.chunk,
+                                    torch_sm_count(dev))
+
+            def step_sp(_i):
+                kda.kda_chunk_fwd_seqpar(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                         A_log=inp["A_log"], dt_bias=inp["dt_bias"], S0=inp["S0"],
+                                         chunk=w.chunk, segments=nseg)
+
+            for i in range(args.warmup):
+                step_sp(i)
+            barrier(world, dev)
+            per_sp = time_launches(step_sp, k, stream)
+            barrier(world, dev)
+            ms_sp_local = sum(per_sp) / len(per_sp)
+            ms_sp = max_over_ranks(ms_sp_local, world, dev)
+            tfl_sp = w.token_heads * chunk_flops_per_token_head(w.Dk, w.Dv, w.chunk) / (ms_sp_local * 1e-3) / 1e12
+            e["seqpar"] = {"segments": nseg, "ms_per_step": ms_sp,
+                           "value": whole_job_value(w.token_heads, world, ms_sp), "unit": UNIT,
+                           "tc_peak_frac": tfl_sp / pk["bf16_tflops"], "speedup": ms / ms_sp,
+                           "launches": 3 * k, "api": "gated_delta_rule_157_b200.kda_chunk_fwd_seqpar"}
+            launches += 3 * k
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             e["cpu_baseline"] = oracle_chunk_timing(w)
         out[name] = e
@@ -506,6 +529,11 @@ def bench_small_configs(args, kda, workloads, dev, stream, pk, world, rank):
         del inp, o
     out["launches"] = launches
     return out
+
+
+def torch_sm_count(dev):
+    import torch
+    return torch.cuda.get_device_properties(dev).multi_processor_count
 
 
 def torch_empty_like_o(w, dev):

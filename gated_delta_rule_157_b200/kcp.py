@@ -40,6 +40,10 @@ class _KernelOps:
         return _lib.kda_compose(M, S_seg, S_init)
 
     @staticmethod
+    def compose_into(M, S_seg, S_init, S_in):
+        _lib.kda_compose(M, S_seg, S_init, S_in=S_in)
+
+    @staticmethod
     def all_gather(t, world, group):
         if world == 1:
             return t.unsqueeze(0)
@@ -90,3 +94,73 @@ def kcp_chunk_fwd(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=
     # 4. this segment's rows from its incoming state
     o, _, _ = ops.forward(q, k, v, g, beta, S_in[rank].reshape(B, HV, Dk, Dv).contiguous(), False, **kw)
     return o, S_in[world].reshape(B, HV, Dk, Dv)
+
+
+def seq_segments(B, HV, T, chunk, sms):
+    """Segments per sequence for kda_chunk_fwd_seqpar: the power of two n
+    (T divisible by n, at least two chunks per segment) that minimises the
+    modelled time, waves x (chunks per segment + 2 for a CTA's start-up and
+    pipeline fill), over the states-only pass (two CTAs per segment and
+    chain: state and transition) and the output pass (one).  1 when the
+    chains alone fill the SMs."""
+    nchunks = -(-T // chunk)
+    best, best_cost = 1, -(-B * HV // sms) * (nchunks + 2)
+    n = 2
+    while n <= 64 and T % n == 0 and -(-(T // n) // chunk) >= 2:
+        seg = -(-(T // n) // chunk)
+        cost = (-(-2 * B * HV * n // sms) + -(-B * HV * n // sms)) * (seg + 2)
+        if cost < best_cost:
+            best, best_cost = n, cost
+        n *= 2
+    return best
+
+
+def kda_chunk_fwd_seqpar(q, k, v, g, beta, *, A_log=None, dt_bias=None, S0=None, chunk=64, segments=None,
+                         g_min=-5.0, scale=1.0, l2_eps=1e-6, qk_l2norm_in_kernel=True,
+                         beta_sigmoid_in_kernel=True, gate_in_kernel=True, g_per_head=False, algo="auto",
+                         ops=None):
+    """Forward of whole sequences on one GPU with every sequence cut into
+    `segments` equal parts that run in parallel (by default seq_segments():
+    when B x HV chains leave SMs idle, as for a single prefill).  The same
+    affine composition as the context-parallel forward (page "Implémenter
+    KDA", the composition test): the segments run from the zero state keeping
+    their final states and transitions, kda_compose chains them into the
+    state entering each segment, and the segments run again from those states
+    for their output rows.  Returns (o [B,T,HV,Dv], S_T [B,HV,Dk,Dv]); S_T is
+    the last segment's final state of the second pass (a view).  T must be
+    divisible by `segments`; no transition output (M_T) on this path.
+    """
+    ops = ops or _KernelOps
+    B, T, H, Dk = q.shape
+    HV, Dv = v.shape[2], v.shape[3]
+    kw = dict(A_log=A_log, dt_bias=dt_bias, chunk=chunk, g_min=g_min, scale=scale, l2_eps=l2_eps,
+              qk_l2norm_in_kernel=qk_l2norm_in_kernel, beta_sigmoid_in_kernel=beta_sigmoid_in_kernel,
+              gate_in_kernel=gate_in_kernel, g_per_head=g_per_head, algo=algo)
+    if segments is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count if q.is_cuda else 1
+        segments = seq_segments(B, HV, T, chunk, sms)
+    n = int(segments)
+    if n <= 1:
+        o, S_T, _ = ops.forward(q, k, v, g, beta, S0, False, **kw)
+        return o, S_T
+    if T % n:
+        raise ValueError("T = %d is not divisible into %d segments" % (T, n))
+    Ts = T // n
+
+    def seg(x):              # [B, T, ...] -> [B*n, T/n, ...]: a view of the contiguous input
+        return x.reshape((B * n, Ts) + tuple(x.shape[2:]))
+
+    # 1. every segment from the zero state: its final state and transition
+    _, S_seg, M = ops.forward(seg(q), seg(k), seg(v), seg(g), seg(beta), None, True, **kw)
+    S_seg = S_seg.reshape(B, n, HV, Dk, Dv)
+    M = M.reshape(B, n, HV, Dk, Dk)
+    # 2. the state entering each segment, written straight into the second
+    #    pass's initial states (the last segment's transition is not needed)
+    S_in = torch.empty((B, n, HV, Dk, Dv), dtype=S_seg.dtype, device=S_seg.device)
+    for b in range(B):
+        ops.compose_into(M[b, :n - 1], S_seg[b, :n - 1], None if S0 is None else S0[b], S_in[b])
+    # 3. every segment from its incoming state: the output rows, and the
+    #    whole sequence's final state as the last segment's
+    o, S_out, _ = ops.forward(seg(q), seg(k), seg(v), seg(g), seg(beta), S_in.reshape(B * n, HV, Dk, Dv),
+                              False, **kw)
+    return o.reshape(B, T, HV, Dv), S_out.reshape(B, n, HV, Dk, Dv)[:, -1]

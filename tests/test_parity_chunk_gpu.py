@@ -311,3 +311,33 @@ def test_states_only_pass_skips_o(cuda_device, algo):
     o2, S2, M2 = run_gpu(d, w, algo, want_M=True, output_o=False)
     assert o2 is None and o1 is not None
     assert torch.equal(S1, S2) and torch.equal(M1, M2)
+
+
+def test_prefill_bf16_seqpar(cuda_device):
+    """The prefill workload (16 chains on 148 SMs) through the sequence-parallel
+    forward: the policy cuts each sequence into 8 segments of 512 tokens; every
+    chain's o and S_T are compared with the oracle's single pass (o element by
+    element, S_T by Frobenius norm), the initial state S0 included."""
+    w = workloads.workload("prefill_bf16")
+    inp = workloads.chunk_inputs(w)
+    d = to_device(inp, cuda_device)
+    assert kda.seq_segments(w.B, w.HV, w.T, w.chunk,
+                            torch.cuda.get_device_properties(cuda_device).multi_processor_count) > 1
+    o, S_T = kda.kda_chunk_fwd_seqpar(d["q"], d["k"], d["v"], d["g"], d["beta"], A_log=d["A_log"],
+                                      dt_bias=d["dt_bias"], S0=d["S0"], chunk=w.chunk)
+    e_o, e_s = _per_chain_errors(o.cpu(), S_T.cpu(), oracle_chunk(inp))
+    assert e_o <= TOL_BF16, e_o
+    assert e_s <= TOL_BF16, e_s
+
+
+@pytest.mark.parametrize("segments", [3, 8])
+def test_seqpar_ragged_batched(cuda_device, segments):
+    """Two batch rows, grouped heads, segments whose length is not a multiple
+    of the chunk (ragged last chunk in every segment), against the oracle."""
+    w = workloads.workload("prefill_bf16", B=2, H=2, HV=4, T=600, seed=91)
+    inp = workloads.chunk_inputs(w)
+    d = to_device(inp, cuda_device)
+    o, S_T = kda.kda_chunk_fwd_seqpar(d["q"], d["k"], d["v"], d["g"], d["beta"], A_log=d["A_log"],
+                                      dt_bias=d["dt_bias"], S0=d["S0"], chunk=w.chunk, segments=segments)
+    ref = oracle_chunk(inp)
+    check(o, S_T, None, ref, "bf16", "tc")
