@@ -40,7 +40,12 @@ constexpr int kVT = 32;                       // value columns per CTA
 static_assert(kVT == 32, "the row loops map one lane to one value column");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
 
-template <typename Tin>
+// kAnchored (Dk = 128, C = 64, the bounded gate with |g_min| <= 5): step 8's
+// pairwise sums use the forward's 16-token tile anchors, so every factor
+// 2^(G_r - G_i) is a product of one per-row and one per-column power, each in
+// [2^-116, 2^116] (16 tokens x 5 x log2 e); otherwise every pair takes its own
+// power of a non-positive difference (any gate).
+template <typename Tin, bool kAnchored>
 __global__ void __launch_bounds__(kThreads)
 chunk_bwd_kernel(BwdParams p) {
     extern __shared__ float smem[];
@@ -303,42 +308,157 @@ chunk_bwd_kernel(BwdParams p) {
         __syncthreads();
         // ---- 8. per (r, c): dq, dk (atomics) and dG (registers) --------------
         float dG[kElemsPerThread];
+        if (kAnchored) {
+            // Thread (tile R, channel c): rows r = 16R + a, a < 16.  Pairwise sums
+            // with tile anchors P_J = G at the row before tile J (0 for J = 0):
+            //   aq_r = 2^(G_r - P_R) sum_{i <= r} dA[r][i] k_i 2^(P_R - G_i)
+            //   ak_r = sum_{J >= R} 2^(P_J - G_r) sum_{rr in J, rr >= r} dA[rr][r] q_rr 2^(G_rr - P_J)
+            // (pr, pc likewise with dP and k).  Entries of dA / dP above the
+            // diagonal are zero, so the sums run over whole tiles.
+            const int R = tid >> 7, c = tid & 127, r0 = 16 * R;
+            const int ntile = (Cc + 15) >> 4;
+            float dq[16], dk[16];
 #pragma unroll
-        for (int n = 0; n < kElemsPerThread; ++n) {
-            const int idx = tid + n * kThreads;
-            dG[n] = 0.f;
-            if (idx >= Cc * Dk) continue;
-            const int r = idx / Dk, c = idx % Dk;
-            const float qrc = Qs[r * L + c], krc = Ks[r * L + c], grc = Gs[r * L + c];
-            // pairwise sums: row r against earlier tokens, then later tokens against r
-            float aq = 0.f, pr = 0.f;
-            for (int i = 0; i <= r; ++i) {
-                const float kie = Ks[i * L + c] * ex2f_(grc - Gs[i * L + c]);
-                aq = fmaf(Aqk[r * C + i], kie, aq);
-                pr = fmaf(Pkk[r * C + i], kie, pr);
+            for (int a = 0; a < 16; ++a) dq[a] = dk[a] = dG[a] = 0.f;
+            float dl = 0.f;                          // this thread's share of dlast[c]
+            if (R < ntile) {
+                const float PR = R == 0 ? 0.f : Gs[(r0 - 1) * L + c];
+                {
+                    float sa[16], sp[16];
+#pragma unroll
+                    for (int a = 0; a < 16; ++a) sa[a] = sp[a] = 0.f;
+                    const int iend = min(r0 + 16, Cc);
+                    for (int i = 0; i < iend; ++i) {
+                        const float kc = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
+#pragma unroll
+                        for (int a = 0; a < 16; ++a) {
+                            sa[a] = fmaf(Aqk[(r0 + a) * C + i], kc, sa[a]);
+                            sp[a] = fmaf(Pkk[(r0 + a) * C + i], kc, sp[a]);
+                        }
+                    }
+#pragma unroll
+                    for (int a = 0; a < 16; ++a) {
+                        if (r0 + a >= Cc) continue;
+                        const int r = r0 + a;
+                        const float fr = ex2f_(Gs[r * L + c] - PR);
+                        const float aq = fr * sa[a], pr = fr * sp[a];
+                        dq[a] = aq;
+                        dk[a] = pr;
+                        dG[a] = Qs[r * L + c] * aq + Ks[r * L + c] * pr;
+                    }
+                }
+                for (int J = R; J < ntile; ++J) {
+                    const float PJ = J == 0 ? 0.f : Gs[(16 * J - 1) * L + c];
+                    float sa[16], sp[16];
+#pragma unroll
+                    for (int a = 0; a < 16; ++a) sa[a] = sp[a] = 0.f;
+                    const int rend = min(16 * J + 16, Cc);
+                    for (int rr = 16 * J; rr < rend; ++rr) {
+                        const float e = ex2f_(Gs[rr * L + c] - PJ);
+                        const float qe = Qs[rr * L + c] * e, ke = Ks[rr * L + c] * e;
+                        const float4 *arow = reinterpret_cast<const float4 *>(Aqk + rr * C + r0);
+                        const float4 *prow = reinterpret_cast<const float4 *>(Pkk + rr * C + r0);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 av = arow[q4], pv = prow[q4];
+                            sa[4 * q4 + 0] = fmaf(av.x, qe, sa[4 * q4 + 0]);
+                            sa[4 * q4 + 1] = fmaf(av.y, qe, sa[4 * q4 + 1]);
+                            sa[4 * q4 + 2] = fmaf(av.z, qe, sa[4 * q4 + 2]);
+                            sa[4 * q4 + 3] = fmaf(av.w, qe, sa[4 * q4 + 3]);
+                            sp[4 * q4 + 0] = fmaf(pv.x, ke, sp[4 * q4 + 0]);
+                            sp[4 * q4 + 1] = fmaf(pv.y, ke, sp[4 * q4 + 1]);
+                            sp[4 * q4 + 2] = fmaf(pv.z, ke, sp[4 * q4 + 2]);
+                            sp[4 * q4 + 3] = fmaf(pv.w, ke, sp[4 * q4 + 3]);
+                        }
+                    }
+#pragma unroll
+                    for (int a = 0; a < 16; ++a) {
+                        if (r0 + a >= Cc) continue;
+                        const int r = r0 + a;
+                        const float f = ex2f_(PJ - Gs[r * L + c]);
+                        const float akpc = f * (sa[a] + sp[a]);     // ak + pc
+                        dk[a] += akpc;
+                        dG[a] -= Ks[r * L + c] * akpc;
+                    }
+                }
+                // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T,
+                // eight rows at a time (the column of S and dS read once per j)
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    float dqg[8], dkw[8], dkd[8];
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) dqg[a] = dkw[a] = dkd[a] = 0.f;
+                    for (int j0 = 0; j0 < kVT; ++j0) {
+                        const int j = (j0 + lane) & (kVT - 1);
+                        const float sv = Ss[c * kVT + j], dsv = dSs[c * kVT + j];
+#pragma unroll
+                        for (int a = 0; a < 8; ++a) {
+                            const int r = r0 + 8 * hb + a;
+                            dqg[a] = fmaf(dOs[r * kVT + j], sv, dqg[a]);
+                            dkw[a] = fmaf(dUs[r * kVT + j], sv, dkw[a]);
+                            dkd[a] = fmaf(Us[r * kVT + j], dsv, dkd[a]);
+                        }
+                    }
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        const int aa = 8 * hb + a, r = r0 + aa;
+                        if (r >= Cc) continue;
+                        const float grc = Gs[r * L + c], qrc = Qs[r * L + c], krc = Ks[r * L + c];
+                        const float kw = -bet[r] * dkw[a];
+                        const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
+                        dq[aa] = fmaf(eg, dqg[a], dq[aa]);
+                        dk[aa] += eg * kw + ed * dkd[a];
+                        dG[aa] += eg * (dqg[a] * qrc + kw * krc) - ed * dkd[a] * krc;
+                        dl = fmaf(ed * dkd[a], krc, dl);
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    if (r0 + a >= Cc) continue;
+                    const size_t tq = ((tok0 + r0 + a) * p.H + h) * Dk + c;
+                    atomicAdd(&p.dq[tq], dq[a]);
+                    atomicAdd(&p.dk[tq], dk[a]);
+                }
+                atomicAdd(&dlast[c], dl);
             }
-            float ak = 0.f, pc = 0.f;
-            for (int rr = r; rr < Cc; ++rr) {
-                const float e = ex2f_(Gs[rr * L + c] - grc);
-                ak = fmaf(Aqk[rr * C + r], Qs[rr * L + c] * e, ak);
-                pc = fmaf(Pkk[rr * C + r], Ks[rr * L + c] * e, pc);
+        } else {
+#pragma unroll
+            for (int n = 0; n < kElemsPerThread; ++n) {
+                const int idx = tid + n * kThreads;
+                dG[n] = 0.f;
+                if (idx >= Cc * Dk) continue;
+                const int r = idx / Dk, c = idx % Dk;
+                const float qrc = Qs[r * L + c], krc = Ks[r * L + c], grc = Gs[r * L + c];
+                // pairwise sums: row r against earlier tokens, then later tokens against r
+                float aq = 0.f, pr = 0.f;
+                for (int i = 0; i <= r; ++i) {
+                    const float kie = Ks[i * L + c] * ex2f_(grc - Gs[i * L + c]);
+                    aq = fmaf(Aqk[r * C + i], kie, aq);
+                    pr = fmaf(Pkk[r * C + i], kie, pr);
+                }
+                float ak = 0.f, pc = 0.f;
+                for (int rr = r; rr < Cc; ++rr) {
+                    const float e = ex2f_(Gs[rr * L + c] - grc);
+                    ak = fmaf(Aqk[rr * C + r], Qs[rr * L + c] * e, ak);
+                    pc = fmaf(Pkk[rr * C + r], Ks[rr * L + c] * e, pc);
+                }
+                // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T
+                float dqg = 0.f, dkw = 0.f, dkd = 0.f;
+                const float br = bet[r];
+                for (int j0 = 0; j0 < kVT; ++j0) {
+                    const int j = (j0 + lane) & (kVT - 1);
+                    const float s = Ss[c * kVT + j];
+                    dqg = fmaf(dOs[r * kVT + j], s, dqg);
+                    dkw = fmaf(-br * dUs[r * kVT + j], s, dkw);
+                    dkd = fmaf(Us[r * kVT + j], dSs[c * kVT + j], dkd);
+                }
+                const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
+                const size_t tq = ((tok0 + r) * p.H + h) * Dk + c;
+                atomicAdd(&p.dq[tq], fmaf(eg, dqg, aq));
+                atomicAdd(&p.dk[tq], ak + pr + pc + eg * dkw + ed * dkd);
+                dG[n] = qrc * aq - krc * ak + krc * pr - krc * pc + eg * (dqg * qrc + dkw * krc) - ed * dkd * krc;
+                atomicAdd(&dlast[c], ed * dkd * krc);
             }
-            // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T
-            float dqg = 0.f, dkw = 0.f, dkd = 0.f;
-            const float br = bet[r];
-            for (int j0 = 0; j0 < kVT; ++j0) {
-                const int j = (j0 + lane) & (kVT - 1);
-                const float s = Ss[c * kVT + j];
-                dqg = fmaf(dOs[r * kVT + j], s, dqg);
-                dkw = fmaf(-br * dUs[r * kVT + j], s, dkw);
-                dkd = fmaf(Us[r * kVT + j], dSs[c * kVT + j], dkd);
-            }
-            const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
-            const size_t tq = ((tok0 + r) * p.H + h) * Dk + c;
-            atomicAdd(&p.dq[tq], fmaf(eg, dqg, aq));
-            atomicAdd(&p.dk[tq], ak + pr + pc + eg * dkw + ed * dkd);
-            dG[n] = qrc * aq - krc * ak + krc * pr - krc * pc + eg * (dqg * qrc + dkw * krc) - ed * dkd * krc;
-            atomicAdd(&dlast[c], ed * dkd * krc);
         }
         __syncthreads();
         // ---- 9. dS entering the chunk (in place) -----------------------------
@@ -359,10 +479,17 @@ chunk_bwd_kernel(BwdParams p) {
             __syncwarp();
         }
         __syncthreads();
+        if (kAnchored) {
+            const int R = tid >> 7, c = tid & 127;
 #pragma unroll
-        for (int n = 0; n < kElemsPerThread; ++n) {
-            const int idx = tid + n * kThreads;
-            if (idx < Cc * Dk) Gs[(idx / Dk) * L + idx % Dk] = dG[n];
+            for (int a = 0; a < 16; ++a)
+                if (16 * R + a < Cc) Gs[(16 * R + a) * L + c] = dG[a];
+        } else {
+#pragma unroll
+            for (int n = 0; n < kElemsPerThread; ++n) {
+                const int idx = tid + n * kThreads;
+                if (idx < Cc * Dk) Gs[(idx / Dk) * L + idx % Dk] = dG[n];
+            }
         }
         __syncthreads();
         // ---- 10. dg = reverse cumulative sum of dG; dbeta --------------------
@@ -508,20 +635,32 @@ __global__ void bwd_empty_kernel(BwdParams p) {
 
 }  // namespace
 
+// The anchored pairwise sums of step 8 need 128 key channels (one thread per
+// channel and 16-row tile), 64-token chunks and a decay of at most 5 per token.
+inline bool bwd_anchored(const BwdParams &p) {
+    return p.Dk == 128 && p.C == 64 && p.gate_in == 1 && p.g_min >= -5.0f;
+}
+
 size_t bwd_smem_bytes(int C, int Dk) {
     const size_t f = (size_t)3 * C * (Dk | 1) + (size_t)2 * C * C + (size_t)4 * C * kVT +
                      (size_t)2 * Dk * kVT + 2 * C + 2 * Dk + (size_t)(kThreads / 32) * 256;
     return f * sizeof(float);
 }
 
-template <typename Tin>
-static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s) {
+template <typename Tin, bool kAnchored>
+static cudaError_t launch_bwd_main(const BwdParams &p, cudaStream_t s) {
     const size_t smem = bwd_smem_bytes(p.C, p.Dk);
-    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<Tin, kAnchored>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.B * p.HV, (p.Dv + kVT - 1) / kVT);
-    chunk_bwd_kernel<Tin><<<grid, kThreads, smem, s>>>(p);
+    chunk_bwd_kernel<Tin, kAnchored><<<grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+static cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s) {
+    cudaError_t e = bwd_anchored(p) ? launch_bwd_main<Tin, true>(p, s) : launch_bwd_main<Tin, false>(p, s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.l2norm) {
         const long long rows = (long long)p.B * p.T * p.H;

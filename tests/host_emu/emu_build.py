@@ -61,7 +61,10 @@ extern "C" int emu_offsetof_ddt_bias(void) { return (int)offsetof(kda::BwdParams
 template <typename Tin>
 static void run_bwd(const kda::BwdParams &p) {
     using namespace kda;
-    emu_launch(dim3(p.B * p.HV, (p.Dv + kVT - 1) / kVT), dim3(kThreads), [&] { chunk_bwd_kernel<Tin>(p); });
+    if (bwd_anchored(p))
+        emu_launch(dim3(p.B * p.HV, (p.Dv + kVT - 1) / kVT), dim3(kThreads), [&] { chunk_bwd_kernel<Tin, true>(p); });
+    else
+        emu_launch(dim3(p.B * p.HV, (p.Dv + kVT - 1) / kVT), dim3(kThreads), [&] { chunk_bwd_kernel<Tin, false>(p); });
     emu_poison(0);
     if (p.l2norm) {
         const long long rows = (long long)p.B * p.T * p.H;

@@ -328,6 +328,7 @@ CASES = [
     (1, 5, 1, 1, 1, 1, 1, "f32", False, 1.0, 10),      # Dk = Dv = chunk = 1
     (2, 23, 1, 3, 3, 5, 7, "f32", True, 1.0, 11),      # odd sizes everywhere
     (1, 1, 1, 1, 8, 8, 16, "f32", True, 1.0, 12),      # one token, shorter than a chunk
+    (1, 150, 1, 2, 128, 128, 64, "bf16", True, 1.0, 13),  # anchored backward: three chunks, grouped heads
 ]
 TOL = TOL_F32
 
