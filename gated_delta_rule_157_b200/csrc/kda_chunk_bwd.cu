@@ -39,6 +39,12 @@ constexpr int kRowThreads = 256;              // bwd_l2norm_kernel
 constexpr int kVT = 32;                       // value columns per CTA
 static_assert(kVT == 32, "the row loops map one lane to one value column");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
+// Anchored A / P: channels staged 8 at a time -- row-anchored q and k of the 64
+// rows, and for every row tile R the column factors of its 16 (R + 1) columns.
+constexpr int kStageCh = 8;
+constexpr int kKcRows = 16 + 32 + 48 + 64;                // 160: columns of tiles 0..3
+constexpr int kStageFloats = (64 + 64 + kKcRows) * kStageCh;
+__host__ __device__ constexpr int kc_off(int R) { return 8 * R * (R + 1); }   // first row of tile R's columns
 
 // kAnchored (Dk = 128, C = 64, the bounded gate with |g_min| <= 5): step 8's
 // pairwise sums use the forward's 16-token tile anchors, so every factor
@@ -69,6 +75,11 @@ chunk_bwd_kernel(BwdParams p) {
     // per-warp row of factors, computed once per row and read by all 32 lanes
     // (one lane per value column): [warp][2 * 128]
     float *wb = dlast + Dk + (threadIdx.x >> 5) * 256;
+    // anchored path only: [kStageCh][64] q and k rows times 2^(G - P_R), and
+    // [kStageCh][kKcRows] columns k_i 2^(P_R - G_i) for every row tile R
+    float *Qa = dlast + Dk + (kThreads / 32) * 256;
+    float *Ka = Qa + kStageCh * 64;
+    float *Kc = Ka + kStageCh * 64;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int chain = blockIdx.x;
@@ -155,21 +166,105 @@ chunk_bwd_kernel(BwdParams p) {
         }
         __syncthreads();
         // ---- 3. A, P and X = V - (K*exp(G)) S -------------------------------
-        for (int pidx = tid; pidx < Cc * Cc; pidx += kThreads) {
-            const int r = pidx / Cc, i = pidx % Cc;
-            float a = 0.f, pk = 0.f;
-            if (i <= r) {
-                const float *kr = Ks + r * L, *ki = Ks + i * L, *qr = Qs + r * L;
-                const float *gr = Gs + r * L, *gi = Gs + i * L;
-                for (int c = 0; c < Dk; ++c) {
-                    const float kie = ki[c] * ex2f_(gr[c] - gi[c]);
-                    a = fmaf(qr[c], kie, a);
-                    pk = fmaf(kr[c], kie, pk);
-                }
-                if (i == r) pk = 0.f;
+        if (kAnchored) {
+            // A[r][i] = sum_c (q_rc 2^(G_rc - P_R)) (k_ic 2^(P_R - G_ic)), R = tile of r
+            // (P likewise with k_rc), every factor within 2^+-116.  Warp w takes
+            // half-blocks (row tile R, column tile J <= R, 8 rows) w and w + 16 of
+            // the 20; lane = (row lane / 4 of the 8, columns 4 (lane % 4) .. +3).
+            const int ntile = (Cc + 15) >> 4;
+            float sa[2][4], sp[2][4];
+            int hb_R[2], hb_J[2], hb_h[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                int hbi = warp + 16 * t;              // 0..19: (R, J) in order, then half
+                const int blk = hbi >> 1;
+                int R = 0;
+                while (blk >= (R + 1) * (R + 2) / 2) ++R;
+                hb_R[t] = R;
+                hb_J[t] = blk - R * (R + 1) / 2;
+                hb_h[t] = hbi & 1;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) sa[t][u] = sp[t][u] = 0.f;
             }
-            Aqk[r * C + i] = a;
-            Pkk[r * C + i] = pk;
+            for (int c0 = 0; c0 < Dk; c0 += kStageCh) {
+                // stage the factors of channels c0 .. c0+7 (rows past Cc hold stale
+                // values whose products are never stored)
+                for (int e = tid; e < 64 * kStageCh; e += kThreads) {
+                    const int r = e & 63, cc = e >> 6, c = c0 + cc, R = r >> 4;
+                    const float PR = R == 0 ? 0.f : Gs[(16 * R - 1) * L + c];
+                    const float f = ex2f_(Gs[r * L + c] - PR);
+                    Qa[cc * 64 + r] = Qs[r * L + c] * f;
+                    Ka[cc * 64 + r] = Ks[r * L + c] * f;
+                }
+                for (int e = tid; e < kKcRows * kStageCh; e += kThreads) {
+                    const int cc = e / kKcRows, row = e - cc * kKcRows, c = c0 + cc;
+                    int R = 0;
+                    while (row >= kc_off(R + 1)) ++R;
+                    const int i = row - kc_off(R);
+                    const float PR = R == 0 ? 0.f : Gs[(16 * R - 1) * L + c];
+                    Kc[cc * kKcRows + row] = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
+                }
+                __syncthreads();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (warp + 16 * t >= 20 || hb_R[t] >= ntile) continue;
+                    const int r = 16 * hb_R[t] + 8 * hb_h[t] + (lane >> 2);
+                    const int krow = kc_off(hb_R[t]) + 16 * hb_J[t] + 4 * (lane & 3);
+#pragma unroll
+                    for (int cc = 0; cc < kStageCh; ++cc) {
+                        const float qa = Qa[cc * 64 + r], ka = Ka[cc * 64 + r];
+                        const float4 kc = *reinterpret_cast<const float4 *>(Kc + cc * kKcRows + krow);
+                        sa[t][0] = fmaf(qa, kc.x, sa[t][0]);
+                        sa[t][1] = fmaf(qa, kc.y, sa[t][1]);
+                        sa[t][2] = fmaf(qa, kc.z, sa[t][2]);
+                        sa[t][3] = fmaf(qa, kc.w, sa[t][3]);
+                        sp[t][0] = fmaf(ka, kc.x, sp[t][0]);
+                        sp[t][1] = fmaf(ka, kc.y, sp[t][1]);
+                        sp[t][2] = fmaf(ka, kc.z, sp[t][2]);
+                        sp[t][3] = fmaf(ka, kc.w, sp[t][3]);
+                    }
+                }
+                __syncthreads();
+            }
+            // stores: A lower with the diagonal, P strictly lower, zeros above
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (warp + 16 * t >= 20 || hb_R[t] >= ntile) continue;
+                const int r = 16 * hb_R[t] + 8 * hb_h[t] + (lane >> 2);
+                if (r >= Cc) continue;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int i = 16 * hb_J[t] + 4 * (lane & 3) + u;
+                    if (i >= Cc) continue;
+                    Aqk[r * C + i] = i <= r ? sa[t][u] : 0.f;
+                    Pkk[r * C + i] = i < r ? sp[t][u] : 0.f;
+                }
+            }
+            // the blocks above the diagonal tiles
+            for (int e = tid; e < Cc * Cc; e += kThreads) {
+                const int r = e / Cc, i = e % Cc;
+                if ((i >> 4) > (r >> 4)) {
+                    Aqk[r * C + i] = 0.f;
+                    Pkk[r * C + i] = 0.f;
+                }
+            }
+        } else {
+            for (int pidx = tid; pidx < Cc * Cc; pidx += kThreads) {
+                const int r = pidx / Cc, i = pidx % Cc;
+                float a = 0.f, pk = 0.f;
+                if (i <= r) {
+                    const float *kr = Ks + r * L, *ki = Ks + i * L, *qr = Qs + r * L;
+                    const float *gr = Gs + r * L, *gi = Gs + i * L;
+                    for (int c = 0; c < Dk; ++c) {
+                        const float kie = ki[c] * ex2f_(gr[c] - gi[c]);
+                        a = fmaf(qr[c], kie, a);
+                        pk = fmaf(kr[c], kie, pk);
+                    }
+                    if (i == r) pk = 0.f;
+                }
+                Aqk[r * C + i] = a;
+                Pkk[r * C + i] = pk;
+            }
         }
         // warp w takes rows w, w + 8, ...; lane = value column
         for (int r = warp; r < Cc; r += kThreads / 32) {
@@ -641,15 +736,16 @@ inline bool bwd_anchored(const BwdParams &p) {
     return p.Dk == 128 && p.C == 64 && p.gate_in == 1 && p.g_min >= -5.0f;
 }
 
-size_t bwd_smem_bytes(int C, int Dk) {
+size_t bwd_smem_bytes(int C, int Dk, bool anchored) {
     const size_t f = (size_t)3 * C * (Dk | 1) + (size_t)2 * C * C + (size_t)4 * C * kVT +
-                     (size_t)2 * Dk * kVT + 2 * C + 2 * Dk + (size_t)(kThreads / 32) * 256;
+                     (size_t)2 * Dk * kVT + 2 * C + 2 * Dk + (size_t)(kThreads / 32) * 256 +
+                     (anchored ? (size_t)kStageFloats : 0);
     return f * sizeof(float);
 }
 
 template <typename Tin, bool kAnchored>
 static cudaError_t launch_bwd_main(const BwdParams &p, cudaStream_t s) {
-    const size_t smem = bwd_smem_bytes(p.C, p.Dk);
+    const size_t smem = bwd_smem_bytes(p.C, p.Dk, kAnchored);
     cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<Tin, kAnchored>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;

@@ -121,7 +121,7 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, cudaStream_t s);
 bool chunk_tc_supported(const ChunkParams &p, bool bf16);
 cudaError_t launch_chunk_empty(const ChunkParams &p, cudaStream_t s);   // T == 0
 cudaError_t launch_chunk_bwd(const BwdParams &p, bool bf16, cudaStream_t s);
-size_t bwd_smem_bytes(int C, int Dk);
+size_t bwd_smem_bytes(int C, int Dk, bool anchored);
 cudaError_t launch_step(const StepParams &p, bool bf16, cudaStream_t s);
 cudaError_t launch_short_conv(const ConvParams &p, cudaStream_t s);
 cudaError_t launch_output_gate(const GateParams &p, cudaStream_t s);

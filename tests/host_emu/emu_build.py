@@ -81,7 +81,7 @@ static void run_bwd(const kda::BwdParams &p) {
 extern "C" int emu_chunk_bwd(kda::BwdParams *pp, int bf16) {
     using namespace kda;
     const BwdParams p = *pp;
-    const size_t bytes = bwd_smem_bytes(p.C, p.Dk);
+    const size_t bytes = bwd_smem_bytes(p.C, p.Dk, bwd_anchored(p));
     if (bytes > sizeof(smem)) return 1;
     emu_poison(bytes);
     if (p.T == 0) {
