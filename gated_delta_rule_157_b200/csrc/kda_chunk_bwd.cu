@@ -57,27 +57,33 @@ chunk_bwd_kernel(BwdParams p) {
     extern __shared__ float smem[];
     const int C = p.C, Dk = p.Dk, Dv = p.Dv;
     const int L = Dk | 1;                  // padded row stride of the [C][Dk] tiles
+    // every array starts on a 16-byte boundary (packed float2 / float4 loads)
+    const int CL = (C * L + 3) & ~3, CC = (C * C + 3) & ~3;
     float *Qs = smem;                      // [C][L]  q (normalised)
-    float *Ks = Qs + C * L;                // [C][L]  k (normalised)
-    float *Gs = Ks + C * L;                // [C][L]  G, then dG
-    float *Aqk = Gs + C * L;               // [C][C]  A, then dA
-    float *Pkk = Aqk + C * C;              // [C][C]  P, then dP
-    float *Xs = Pkk + C * C;               // [C][kVT] X
+    float *Ks = Qs + CL;                   // [C][L]  k (normalised)
+    float *Gs = Ks + CL;                   // [C][L]  G, then dG
+    float *Aqk = Gs + CL;                  // [C][C]  A, then dA
+    float *Pkk = Aqk + CC;                 // [C][C]  P, then dP
+    float *Xs = Pkk + CC;                  // [C][kVT] X
     float *Us = Xs + C * kVT;              // [C][kVT] U
     float *dOs = Us + C * kVT;             // [C][kVT] scale * dO
     float *dUs = dOs + C * kVT;            // [C][kVT] dU, then dZ
-    float *Ss = dUs + C * kVT;             // [Dk][kVT] state entering the chunk
-    float *dSs = Ss + Dk * kVT;            // [Dk][kVT] dS of the state leaving, then entering, the chunk
-    float *bet = dSs + Dk * kVT;           // [C]
-    float *dbet = bet + C;                 // [C]
-    float *Glast = dbet + C;               // [Dk]
-    float *dlast = Glast + Dk;             // [Dk]  dG terms of the chunk's last row
+    // the state and its gradient transposed, [kVT][SL]: value column j major,
+    // key channels contiguous (SL = 4 mod 32: lane = j reads four channels
+    // as one conflict-free float4; lane = c reads one row without conflicts)
+    const int C4 = (C + 3) & ~3, Dk4 = (Dk + 3) & ~3, SL = Dk4 + 4;
+    float *Ss = dUs + C * kVT;             // [kVT][SL] state entering the chunk (transposed)
+    float *dSs = Ss + kVT * SL;            // [kVT][SL] dS of the state leaving, then entering, the chunk
+    float *bet = dSs + kVT * SL;           // [C]
+    float *dbet = bet + C4;                // [C]
+    float *Glast = dbet + C4;              // [Dk]
+    float *dlast = Glast + Dk4;            // [Dk]  dG terms of the chunk's last row
     // per-warp row of factors, computed once per row and read by all 32 lanes
     // (one lane per value column): [warp][2 * 128]
-    float *wb = dlast + Dk + (threadIdx.x >> 5) * 256;
+    float *wb = dlast + Dk4 + (threadIdx.x >> 5) * 256;
     // anchored path only: [kStageCh][64] q and k rows times 2^(G - P_R), and
     // [kStageCh][kKcRows] columns k_i 2^(P_R - G_i) for every row tile R
-    float *Qa = dlast + Dk + (kThreads / 32) * 256;
+    float *Qa = dlast + Dk4 + (kThreads / 32) * 256;
     float *Ka = Qa + kStageCh * 64;
     float *Kc = Ka + kStageCh * 64;
 
@@ -96,7 +102,7 @@ chunk_bwd_kernel(BwdParams p) {
 
     for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
         const int c = idx / kVT, col = col0 + idx % kVT;
-        dSs[idx] = (p.dS_T && col < Dv) ? p.dS_T[((size_t)chain * Dk + c) * Dv + col] : 0.f;
+        dSs[(idx % kVT) * SL + c] = (p.dS_T && col < Dv) ? p.dS_T[((size_t)chain * Dk + c) * Dv + col] : 0.f;
     }
 
     for (int ch = NC - 1; ch >= 0; --ch) {
@@ -126,7 +132,7 @@ chunk_bwd_kernel(BwdParams p) {
         }
         for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
             const int c = idx / kVT, col = col0 + idx % kVT;
-            Ss[idx] = col < Dv ? p.S_chunks[(((size_t)chain * NC + ch) * Dk + c) * Dv + col] : 0.f;
+            Ss[(idx % kVT) * SL + c] = col < Dv ? p.S_chunks[(((size_t)chain * NC + ch) * Dk + c) * Dv + col] : 0.f;
         }
         for (int r = tid; r < Cc; r += kThreads) {
             const float x = ld_act(bt, (tok0 + r) * p.HV + hv);
@@ -266,13 +272,22 @@ chunk_bwd_kernel(BwdParams p) {
                 Pkk[r * C + i] = pk;
             }
         }
-        // warp w takes rows w, w + 8, ...; lane = value column
+        // warp w takes rows w, w + 16, ...; lane = value column; channel pairs
+        // (c, c + 1) in one packed FMA, two chains
         for (int r = warp; r < Cc; r += kThreads / 32) {
-            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * ex2f_(Gs[r * L + c]);
+            for (int c = lane; c < Dk; c += 32) wb[c] = -Ks[r * L + c] * ex2f_(Gs[r * L + c]);
             __syncwarp();
-            float acc = Xs[r * kVT + lane];
-            for (int c = 0; c < Dk; ++c) acc = fmaf(-wb[c], Ss[c * kVT + lane], acc);
-            Xs[r * kVT + lane] = acc;
+            float2 acc0 = make_float2(Xs[r * kVT + lane], 0.f), acc1 = make_float2(0.f, 0.f);
+            const float *srow = Ss + lane * SL;
+            int c = 0;
+            for (; c + 3 < Dk; c += 4) {
+                const float4 w4 = *reinterpret_cast<const float4 *>(wb + c);
+                const float4 s4 = *reinterpret_cast<const float4 *>(srow + c);
+                acc0 = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(s4.x, s4.y), acc0);
+                acc1 = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(s4.z, s4.w), acc1);
+            }
+            for (; c < Dk; ++c) acc0.x = fmaf(wb[c], srow[c], acc0.x);
+            Xs[r * kVT + lane] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
             __syncwarp();
         }
         __syncthreads();
@@ -284,7 +299,7 @@ chunk_bwd_kernel(BwdParams p) {
         // the exp(G_last) dS'.S term of the last row's dG (independent of U)
         for (int c = tid; c < Dk; c += kThreads) {
             float acc = 0.f;
-            for (int j = 0; j < kVT; ++j) acc = fmaf(Ss[c * kVT + j], dSs[c * kVT + j], acc);
+            for (int j = 0; j < kVT; ++j) acc = fmaf(Ss[j * SL + c], dSs[j * SL + c], acc);
             dlast[c] = ex2f_(Glast[c]) * acc;
         }
         __syncthreads();
@@ -331,8 +346,18 @@ chunk_bwd_kernel(BwdParams p) {
             __syncwarp();
             float acc = 0.f;
             for (int rr = r; rr < Cc; ++rr) acc = fmaf(Aqk[rr * C + r], dOs[rr * kVT + lane], acc);
-            for (int c = 0; c < Dk; ++c) acc = fmaf(wb[c], dSs[c * kVT + lane], acc);
-            dUs[r * kVT + lane] = acc;
+            // channels four at a time, two packed chains
+            const float *drow = dSs + lane * SL;
+            float2 acc0 = make_float2(acc, 0.f), acc1 = make_float2(0.f, 0.f);
+            int c = 0;
+            for (; c + 3 < Dk; c += 4) {
+                const float4 w4 = *reinterpret_cast<const float4 *>(wb + c);
+                const float4 d4 = *reinterpret_cast<const float4 *>(drow + c);
+                acc0 = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(d4.x, d4.y), acc0);
+                acc1 = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(d4.z, d4.w), acc1);
+            }
+            for (; c < Dk; ++c) acc0.x = fmaf(wb[c], drow[c], acc0.x);
+            dUs[r * kVT + lane] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
             __syncwarp();
         }
         __syncthreads();
@@ -373,32 +398,36 @@ chunk_bwd_kernel(BwdParams p) {
             }
         }
         // ---- 7. dA, dP, dbeta and dV ------------------------------------------
-        // The column loops start at a lane-dependent offset so that the lanes
-        // of a warp read different shared-memory banks.
-        for (int pidx = tid; pidx < Cc * Cc; pidx += kThreads) {
-            const int r = pidx / Cc, i = pidx % Cc;
-            float da = 0.f, dm = 0.f;
-            if (i <= r) {
-                for (int j0 = 0; j0 < kVT; ++j0) {
-                    const int j = (j0 + lane) & (kVT - 1);
-                    const float u = Us[i * kVT + j];
-                    da = fmaf(dOs[r * kVT + j], u, da);
-                    dm = fmaf(-dUs[r * kVT + j], u, dm);
+        // Warp w takes rows w, w + 16, ...: lane = column i (rounds of 32),
+        // then lane = value column for dV; the row's dbeta is a warp sum.  The
+        // value-column pairs start at a lane-dependent offset so that the lanes
+        // of a half-warp read different shared-memory banks.
+        for (int r = warp; r < Cc; r += kThreads / 32) {
+            float db = 0.f;
+            for (int i = lane; i < Cc; i += 32) {
+                float2 da = make_float2(0.f, 0.f), dm = make_float2(0.f, 0.f);
+                if (i <= r) {
+                    for (int j0 = 0; j0 < kVT; j0 += 2) {
+                        const int j = (j0 + 2 * lane) & (kVT - 1);
+                        const float2 u = *reinterpret_cast<const float2 *>(Us + i * kVT + j);
+                        da = __ffma2_rn(*reinterpret_cast<const float2 *>(dOs + r * kVT + j), u, da);
+                        dm = __ffma2_rn(*reinterpret_cast<const float2 *>(dUs + r * kVT + j), u, dm);
+                    }
                 }
+                const float dms = -(dm.x + dm.y);
+                if (i < r) {
+                    db = fmaf(dms, Pkk[r * C + i], db);
+                    Pkk[r * C + i] = bet[r] * dms;
+                } else {
+                    Pkk[r * C + i] = 0.f;
+                }
+                Aqk[r * C + i] = da.x + da.y;
             }
-            if (i < r) {
-                atomicAdd(&dbet[r], dm * Pkk[r * C + i]);
-                Pkk[r * C + i] = bet[r] * dm;
-            } else {
-                Pkk[r * C + i] = 0.f;
-            }
-            Aqk[r * C + i] = da;
-        }
-        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
-            const int r = idx / kVT, col = col0 + idx % kVT;
-            const float dz = dUs[idx];
-            atomicAdd(&dbet[r], dz * Xs[idx]);
-            if (col < Dv) p.dv[((tok0 + r) * p.HV + hv) * Dv + col] = bet[r] * dz;
+            const float dz = dUs[r * kVT + lane];
+            db = fmaf(dz, Xs[r * kVT + lane], db);
+            if (col0 + lane < Dv) p.dv[((tok0 + r) * p.HV + hv) * Dv + col0 + lane] = bet[r] * dz;
+            for (int off = 16; off > 0; off >>= 1) db += __shfl_xor_sync(0xffffffffu, db, off);
+            if (lane == 0) dbet[r] = db;
         }
         __syncthreads();
         // ---- 8. per (r, c): dq, dk (atomics) and dG (registers) --------------
@@ -413,30 +442,43 @@ chunk_bwd_kernel(BwdParams p) {
             const int R = tid >> 7, c = tid & 127, r0 = 16 * R;
             const int ntile = (Cc + 15) >> 4;
             float dq[16], dk[16];
-#pragma unroll
-            for (int a = 0; a < 16; ++a) dq[a] = dk[a] = dG[a] = 0.f;
             float dl = 0.f;                          // this thread's share of dlast[c]
-            if (R < ntile) {
+            if (R >= ntile) {
+#pragma unroll
+                for (int a = 0; a < 16; ++a) dG[a] = 0.f;
+            } else {
                 const float PR = R == 0 ? 0.f : Gs[(r0 - 1) * L + c];
                 {
-                    float sa[16], sp[16];
+                    // column pairs (i, i + 1) in one packed FMA per row
+                    float2 sa[16], sp[16];
 #pragma unroll
-                    for (int a = 0; a < 16; ++a) sa[a] = sp[a] = 0.f;
+                    for (int a = 0; a < 16; ++a) sa[a] = sp[a] = make_float2(0.f, 0.f);
                     const int iend = min(r0 + 16, Cc);
-                    for (int i = 0; i < iend; ++i) {
+                    int i = 0;
+                    for (; i + 1 < iend; i += 2) {
+                        const float2 kc = make_float2(Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]),
+                                                      Ks[(i + 1) * L + c] * ex2f_(PR - Gs[(i + 1) * L + c]));
+#pragma unroll
+                        for (int a = 0; a < 16; ++a) {
+                            sa[a] = __ffma2_rn(*reinterpret_cast<const float2 *>(Aqk + (r0 + a) * C + i), kc, sa[a]);
+                            sp[a] = __ffma2_rn(*reinterpret_cast<const float2 *>(Pkk + (r0 + a) * C + i), kc, sp[a]);
+                        }
+                    }
+                    if (i < iend) {                  // an odd last column
                         const float kc = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
 #pragma unroll
                         for (int a = 0; a < 16; ++a) {
-                            sa[a] = fmaf(Aqk[(r0 + a) * C + i], kc, sa[a]);
-                            sp[a] = fmaf(Pkk[(r0 + a) * C + i], kc, sp[a]);
+                            sa[a].x = fmaf(Aqk[(r0 + a) * C + i], kc, sa[a].x);
+                            sp[a].x = fmaf(Pkk[(r0 + a) * C + i], kc, sp[a].x);
                         }
                     }
 #pragma unroll
                     for (int a = 0; a < 16; ++a) {
+                        dq[a] = dk[a] = dG[a] = 0.f;
                         if (r0 + a >= Cc) continue;
                         const int r = r0 + a;
                         const float fr = ex2f_(Gs[r * L + c] - PR);
-                        const float aq = fr * sa[a], pr = fr * sp[a];
+                        const float aq = fr * (sa[a].x + sa[a].y), pr = fr * (sp[a].x + sp[a].y);
                         dq[a] = aq;
                         dk[a] = pr;
                         dG[a] = Qs[r * L + c] * aq + Ks[r * L + c] * pr;
@@ -444,26 +486,24 @@ chunk_bwd_kernel(BwdParams p) {
                 }
                 for (int J = R; J < ntile; ++J) {
                     const float PJ = J == 0 ? 0.f : Gs[(16 * J - 1) * L + c];
-                    float sa[16], sp[16];
+                    // rows (2m, 2m + 1) of ak + pc in one packed FMA
+                    float2 s2[8];
 #pragma unroll
-                    for (int a = 0; a < 16; ++a) sa[a] = sp[a] = 0.f;
+                    for (int m = 0; m < 8; ++m) s2[m] = make_float2(0.f, 0.f);
                     const int rend = min(16 * J + 16, Cc);
                     for (int rr = 16 * J; rr < rend; ++rr) {
                         const float e = ex2f_(Gs[rr * L + c] - PJ);
                         const float qe = Qs[rr * L + c] * e, ke = Ks[rr * L + c] * e;
+                        const float2 qe2 = make_float2(qe, qe), ke2 = make_float2(ke, ke);
                         const float4 *arow = reinterpret_cast<const float4 *>(Aqk + rr * C + r0);
                         const float4 *prow = reinterpret_cast<const float4 *>(Pkk + rr * C + r0);
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             const float4 av = arow[q4], pv = prow[q4];
-                            sa[4 * q4 + 0] = fmaf(av.x, qe, sa[4 * q4 + 0]);
-                            sa[4 * q4 + 1] = fmaf(av.y, qe, sa[4 * q4 + 1]);
-                            sa[4 * q4 + 2] = fmaf(av.z, qe, sa[4 * q4 + 2]);
-                            sa[4 * q4 + 3] = fmaf(av.w, qe, sa[4 * q4 + 3]);
-                            sp[4 * q4 + 0] = fmaf(pv.x, ke, sp[4 * q4 + 0]);
-                            sp[4 * q4 + 1] = fmaf(pv.y, ke, sp[4 * q4 + 1]);
-                            sp[4 * q4 + 2] = fmaf(pv.z, ke, sp[4 * q4 + 2]);
-                            sp[4 * q4 + 3] = fmaf(pv.w, ke, sp[4 * q4 + 3]);
+                            s2[2 * q4] = __ffma2_rn(make_float2(av.x, av.y), qe2, s2[2 * q4]);
+                            s2[2 * q4 + 1] = __ffma2_rn(make_float2(av.z, av.w), qe2, s2[2 * q4 + 1]);
+                            s2[2 * q4] = __ffma2_rn(make_float2(pv.x, pv.y), ke2, s2[2 * q4]);
+                            s2[2 * q4 + 1] = __ffma2_rn(make_float2(pv.z, pv.w), ke2, s2[2 * q4 + 1]);
                         }
                     }
 #pragma unroll
@@ -471,40 +511,51 @@ chunk_bwd_kernel(BwdParams p) {
                         if (r0 + a >= Cc) continue;
                         const int r = r0 + a;
                         const float f = ex2f_(PJ - Gs[r * L + c]);
-                        const float akpc = f * (sa[a] + sp[a]);     // ak + pc
+                        const float akpc = f * ((a & 1) ? s2[a >> 1].y : s2[a >> 1].x);     // ak + pc
                         dk[a] += akpc;
                         dG[a] -= Ks[r * L + c] * akpc;
                     }
                 }
                 // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T,
-                // eight rows at a time (the column of S and dS read once per j)
+                // four rows at a time: the value columns j .. j+3 of a row are
+                // one broadcast float4, the column of S one conflict-free load
+                // per j; (even j, odd j) in one packed FMA
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {
-                    float dqg[8], dkw[8], dkd[8];
+                for (int hb = 0; hb < 4; ++hb) {
+                    float2 dqg[4], dkw[4], dkd[4];
 #pragma unroll
-                    for (int a = 0; a < 8; ++a) dqg[a] = dkw[a] = dkd[a] = 0.f;
-                    for (int j0 = 0; j0 < kVT; ++j0) {
-                        const int j = (j0 + lane) & (kVT - 1);
-                        const float sv = Ss[c * kVT + j], dsv = dSs[c * kVT + j];
+                    for (int a = 0; a < 4; ++a) dqg[a] = dkw[a] = dkd[a] = make_float2(0.f, 0.f);
+                    for (int j = 0; j < kVT; j += 4) {
+                        const float2 s01 = make_float2(Ss[j * SL + c], Ss[(j + 1) * SL + c]);
+                        const float2 s23 = make_float2(Ss[(j + 2) * SL + c], Ss[(j + 3) * SL + c]);
+                        const float2 d01 = make_float2(dSs[j * SL + c], dSs[(j + 1) * SL + c]);
+                        const float2 d23 = make_float2(dSs[(j + 2) * SL + c], dSs[(j + 3) * SL + c]);
 #pragma unroll
-                        for (int a = 0; a < 8; ++a) {
-                            const int r = r0 + 8 * hb + a;
-                            dqg[a] = fmaf(dOs[r * kVT + j], sv, dqg[a]);
-                            dkw[a] = fmaf(dUs[r * kVT + j], sv, dkw[a]);
-                            dkd[a] = fmaf(Us[r * kVT + j], dsv, dkd[a]);
+                        for (int a = 0; a < 4; ++a) {
+                            const int r = r0 + 4 * hb + a;
+                            const float4 o4 = *reinterpret_cast<const float4 *>(dOs + r * kVT + j);
+                            const float4 u4 = *reinterpret_cast<const float4 *>(dUs + r * kVT + j);
+                            const float4 v4 = *reinterpret_cast<const float4 *>(Us + r * kVT + j);
+                            dqg[a] = __ffma2_rn(make_float2(o4.x, o4.y), s01, dqg[a]);
+                            dqg[a] = __ffma2_rn(make_float2(o4.z, o4.w), s23, dqg[a]);
+                            dkw[a] = __ffma2_rn(make_float2(u4.x, u4.y), s01, dkw[a]);
+                            dkw[a] = __ffma2_rn(make_float2(u4.z, u4.w), s23, dkw[a]);
+                            dkd[a] = __ffma2_rn(make_float2(v4.x, v4.y), d01, dkd[a]);
+                            dkd[a] = __ffma2_rn(make_float2(v4.z, v4.w), d23, dkd[a]);
                         }
                     }
 #pragma unroll
-                    for (int a = 0; a < 8; ++a) {
-                        const int aa = 8 * hb + a, r = r0 + aa;
+                    for (int a = 0; a < 4; ++a) {
+                        const int aa = 4 * hb + a, r = r0 + aa;
                         if (r >= Cc) continue;
                         const float grc = Gs[r * L + c], qrc = Qs[r * L + c], krc = Ks[r * L + c];
-                        const float kw = -bet[r] * dkw[a];
+                        const float vqg = dqg[a].x + dqg[a].y, vkd = dkd[a].x + dkd[a].y;
+                        const float kw = -bet[r] * (dkw[a].x + dkw[a].y);
                         const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
-                        dq[aa] = fmaf(eg, dqg[a], dq[aa]);
-                        dk[aa] += eg * kw + ed * dkd[a];
-                        dG[aa] += eg * (dqg[a] * qrc + kw * krc) - ed * dkd[a] * krc;
-                        dl = fmaf(ed * dkd[a], krc, dl);
+                        dq[aa] = fmaf(eg, vqg, dq[aa]);
+                        dk[aa] += eg * kw + ed * vkd;
+                        dG[aa] += eg * (vqg * qrc + kw * krc) - ed * vkd * krc;
+                        dl = fmaf(ed * vkd, krc, dl);
                     }
                 }
 #pragma unroll
@@ -540,12 +591,11 @@ chunk_bwd_kernel(BwdParams p) {
                 // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T
                 float dqg = 0.f, dkw = 0.f, dkd = 0.f;
                 const float br = bet[r];
-                for (int j0 = 0; j0 < kVT; ++j0) {
-                    const int j = (j0 + lane) & (kVT - 1);
-                    const float s = Ss[c * kVT + j];
+                for (int j = 0; j < kVT; ++j) {
+                    const float s = Ss[j * SL + c];
                     dqg = fmaf(dOs[r * kVT + j], s, dqg);
                     dkw = fmaf(-br * dUs[r * kVT + j], s, dkw);
-                    dkd = fmaf(Us[r * kVT + j], dSs[c * kVT + j], dkd);
+                    dkd = fmaf(Us[r * kVT + j], dSs[j * SL + c], dkd);
                 }
                 const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
                 const size_t tq = ((tok0 + r) * p.H + h) * Dk + c;
@@ -558,19 +608,26 @@ chunk_bwd_kernel(BwdParams p) {
         __syncthreads();
         // ---- 9. dS entering the chunk (in place) -----------------------------
         // warp w takes key channels w, w + 8, ...; lane = value column
+        // (row r's two factors side by side: one packed FMA per row, two chains)
         for (int c = warp; c < Dk; c += kThreads / 32) {
             for (int r = lane; r < Cc; r += 32) {
                 const float e = ex2f_(Gs[r * L + c]);
-                wb[r] = e * Qs[r * L + c];
-                wb[128 + r] = -e * Ks[r * L + c] * bet[r];
+                wb[2 * r] = e * Qs[r * L + c];
+                wb[2 * r + 1] = -e * Ks[r * L + c] * bet[r];
             }
             __syncwarp();
-            float acc = ex2f_(Glast[c]) * dSs[c * kVT + lane];
-            for (int r = 0; r < Cc; ++r) {
-                acc = fmaf(wb[r], dOs[r * kVT + lane], acc);
-                acc = fmaf(wb[128 + r], dUs[r * kVT + lane], acc);
+            float2 acc0 = make_float2(ex2f_(Glast[c]) * dSs[lane * SL + c], 0.f), acc1 = make_float2(0.f, 0.f);
+            int r = 0;
+            for (; r + 1 < Cc; r += 2) {
+                const float4 w4 = *reinterpret_cast<const float4 *>(wb + 2 * r);
+                acc0 = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(dOs[r * kVT + lane], dUs[r * kVT + lane]), acc0);
+                acc1 = __ffma2_rn(make_float2(w4.z, w4.w),
+                                  make_float2(dOs[(r + 1) * kVT + lane], dUs[(r + 1) * kVT + lane]), acc1);
             }
-            dSs[c * kVT + lane] = acc;
+            if (r < Cc)
+                acc0 = __ffma2_rn(make_float2(wb[2 * r], wb[2 * r + 1]), make_float2(dOs[r * kVT + lane], dUs[r * kVT + lane]),
+                                  acc0);
+            dSs[lane * SL + c] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
             __syncwarp();
         }
         __syncthreads();
@@ -612,7 +669,7 @@ chunk_bwd_kernel(BwdParams p) {
     if (p.dS0) {
         for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
             const int c = idx / kVT, col = col0 + idx % kVT;
-            if (col < Dv) p.dS0[((size_t)chain * Dk + c) * Dv + col] = dSs[idx];
+            if (col < Dv) p.dS0[((size_t)chain * Dk + c) * Dv + col] = dSs[(idx % kVT) * SL + c];
         }
     }
 }
@@ -737,8 +794,11 @@ inline bool bwd_anchored(const BwdParams &p) {
 }
 
 size_t bwd_smem_bytes(int C, int Dk, bool anchored) {
-    const size_t f = (size_t)3 * C * (Dk | 1) + (size_t)2 * C * C + (size_t)4 * C * kVT +
-                     (size_t)2 * Dk * kVT + 2 * C + 2 * Dk + (size_t)(kThreads / 32) * 256 +
+    const size_t CL = ((size_t)C * (Dk | 1) + 3) & ~(size_t)3, CC = ((size_t)C * C + 3) & ~(size_t)3;
+    const size_t Dk4 = ((size_t)Dk + 3) & ~(size_t)3;
+    const size_t f = 3 * CL + 2 * CC + (size_t)4 * C * kVT + (size_t)2 * kVT * (Dk4 + 4) +
+                     2 * (((size_t)C + 3) & ~(size_t)3) + 2 * Dk4 +
+                     (size_t)(kThreads / 32) * 256 +
                      (anchored ? (size_t)kStageFloats : 0);
     return f * sizeof(float);
 }
