@@ -38,7 +38,9 @@ constexpr int kThreads = 512;                 // chunk_bwd_kernel: 16 warps, one
 constexpr int kRowThreads = 256;              // bwd_l2norm_kernel
 constexpr int kVT = 32;                       // value columns per CTA
 static_assert(kVT == 32, "the row loops map one lane to one value column");
+static_assert(kThreads == 4 * 128, "the dS step maps a thread to (key channel, eight value columns)");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
+constexpr int kLoadBatch = 8;                 // global loads in flight per thread in the chunk load
 // Anchored A / P: channels staged 8 at a time -- row-anchored q and k of the 64
 // rows, and for every row tile R the column factors of its 16 (R + 1) columns.
 constexpr int kStageCh = 8;
@@ -111,6 +113,8 @@ chunk_bwd_kernel(BwdParams p) {
         const size_t tok0 = (size_t)b * p.T + t0;
         __syncthreads();
         // ---- 1. load the chunk and the state entering it -------------------
+        // (the state and value rows in batches of kLoadBatch elements per
+        // thread whose loads are all issued before the first shared-memory store)
         for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
             const int r = idx / Dk, c = idx % Dk;
             const size_t tok = tok0 + r;
@@ -123,21 +127,64 @@ chunk_bwd_kernel(BwdParams p) {
             }
             Gs[r * L + c] = gz;
         }
-        for (int idx = tid; idx < Cc * kVT; idx += kThreads) {
-            const int r = idx / kVT, col = col0 + idx % kVT;
-            const size_t tok = tok0 + r;
-            const bool in = col < Dv;
-            Xs[idx] = in ? ld_act(v, (tok * p.HV + hv) * Dv + col) : 0.f;
-            dOs[idx] = in ? p.scale * ld_act(dout, (tok * p.HV + hv) * Dv + col) : 0.f;
+        for (int base = tid; base < Dk * kVT; base += kLoadBatch * kThreads) {
+            float sv[kLoadBatch];
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+                const int idx = base + u * kThreads, c = idx / kVT, col = col0 + idx % kVT;
+                sv[u] = (idx < Dk * kVT && col < Dv) ? p.S_chunks[(((size_t)chain * NC + ch) * Dk + c) * Dv + col] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kLoadBatch; ++u) {
+                const int idx = base + u * kThreads;
+                if (idx < Dk * kVT) Ss[(idx % kVT) * SL + idx / kVT] = sv[u];
+            }
         }
-        for (int idx = tid; idx < Dk * kVT; idx += kThreads) {
-            const int c = idx / kVT, col = col0 + idx % kVT;
-            Ss[(idx % kVT) * SL + c] = col < Dv ? p.S_chunks[(((size_t)chain * NC + ch) * Dk + c) * Dv + col] : 0.f;
+        for (int base = tid; base < Cc * kVT; base += (kLoadBatch / 2) * kThreads) {
+            float vv[kLoadBatch / 2], ov[kLoadBatch / 2];
+#pragma unroll
+            for (int u = 0; u < kLoadBatch / 2; ++u) {
+                const int idx = base + u * kThreads, r = idx / kVT, col = col0 + idx % kVT;
+                const bool in = idx < Cc * kVT && col < Dv;
+                const size_t tok = tok0 + r;
+                vv[u] = in ? ld_act(v, (tok * p.HV + hv) * Dv + col) : 0.f;
+                ov[u] = in ? p.scale * ld_act(dout, (tok * p.HV + hv) * Dv + col) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kLoadBatch / 2; ++u) {
+                const int idx = base + u * kThreads;
+                if (idx < Cc * kVT) {
+                    Xs[idx] = vv[u];
+                    dOs[idx] = ov[u];
+                }
+            }
         }
         for (int r = tid; r < Cc; r += kThreads) {
             const float x = ld_act(bt, (tok0 + r) * p.HV + hv);
             bet[r] = p.beta_sigmoid ? sigmoidf_(x) : x;
             dbet[r] = 0.f;
+        }
+        // the next chunk's (ch - 1) rows into L2 while this one is worked on
+        if (ch > 0) {
+            const size_t ptok = tok0 - C;
+            const int qlines = (Dk * (int)sizeof(Tin) + 127) / 128;
+            for (int e = tid; e < C * qlines; e += kThreads) {
+                const size_t off = ((ptok + e / qlines) * p.H + h) * Dk * sizeof(Tin) + (size_t)(e % qlines) * 128;
+                prefetch_l2(reinterpret_cast<const char *>(q) + off);
+                prefetch_l2(reinterpret_cast<const char *>(k) + off);
+                if (!p.g_per_head)
+                    prefetch_l2(reinterpret_cast<const char *>(g) + ((ptok + e / qlines) * p.HV + hv) * Dk * sizeof(Tin) +
+                                (size_t)(e % qlines) * 128);
+            }
+            for (int e = tid; e < 2 * C + Dk; e += kThreads) {
+                if (e < C) {
+                    prefetch_l2(v + ((ptok + e) * p.HV + hv) * Dv + col0);
+                } else if (e < 2 * C) {
+                    prefetch_l2(dout + ((ptok + e - C) * p.HV + hv) * Dv + col0);
+                } else {
+                    prefetch_l2(p.S_chunks + (((size_t)chain * NC + ch - 1) * Dk + (e - 2 * C)) * Dv + col0);
+                }
+            }
         }
         __syncthreads();
         // ---- 2. L2 norms of q, k rows; in-chunk cumulative sum of g ----------
@@ -607,28 +654,41 @@ chunk_bwd_kernel(BwdParams p) {
         }
         __syncthreads();
         // ---- 9. dS entering the chunk (in place) -----------------------------
-        // warp w takes key channels w, w + 8, ...; lane = value column
-        // (row r's two factors side by side: one packed FMA per row, two chains)
-        for (int c = warp; c < Dk; c += kThreads / 32) {
-            for (int r = lane; r < Cc; r += 32) {
-                const float e = ex2f_(Gs[r * L + c]);
-                wb[2 * r] = e * Qs[r * L + c];
-                wb[2 * r + 1] = -e * Ks[r * L + c] * bet[r];
+        // thread = (key channel c, eight value columns j0 .. j0+7): the factors
+        // e^G q and -e^G k beta of (r, c) once per thread, the value columns of
+        // rows r of dO and dZ as broadcast float4s; each thread reads and then
+        // overwrites only its own entries of dS'
+        {
+            const int c = tid & 127, j0 = 8 * (tid >> 7);
+            if (c < Dk) {
+                const float el = ex2f_(Glast[c]);
+                float2 acc[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    acc[m] = make_float2(el * dSs[(j0 + 2 * m) * SL + c], el * dSs[(j0 + 2 * m + 1) * SL + c]);
+                for (int r = 0; r < Cc; ++r) {
+                    const float e = ex2f_(Gs[r * L + c]);
+                    const float w1 = e * Qs[r * L + c], w2 = -e * Ks[r * L + c] * bet[r];
+                    const float2 w1p = make_float2(w1, w1), w2p = make_float2(w2, w2);
+                    const float4 o0 = *reinterpret_cast<const float4 *>(dOs + r * kVT + j0);
+                    const float4 o1 = *reinterpret_cast<const float4 *>(dOs + r * kVT + j0 + 4);
+                    const float4 z0 = *reinterpret_cast<const float4 *>(dUs + r * kVT + j0);
+                    const float4 z1 = *reinterpret_cast<const float4 *>(dUs + r * kVT + j0 + 4);
+                    acc[0] = __ffma2_rn(make_float2(o0.x, o0.y), w1p, acc[0]);
+                    acc[1] = __ffma2_rn(make_float2(o0.z, o0.w), w1p, acc[1]);
+                    acc[2] = __ffma2_rn(make_float2(o1.x, o1.y), w1p, acc[2]);
+                    acc[3] = __ffma2_rn(make_float2(o1.z, o1.w), w1p, acc[3]);
+                    acc[0] = __ffma2_rn(make_float2(z0.x, z0.y), w2p, acc[0]);
+                    acc[1] = __ffma2_rn(make_float2(z0.z, z0.w), w2p, acc[1]);
+                    acc[2] = __ffma2_rn(make_float2(z1.x, z1.y), w2p, acc[2]);
+                    acc[3] = __ffma2_rn(make_float2(z1.z, z1.w), w2p, acc[3]);
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    dSs[(j0 + 2 * m) * SL + c] = acc[m].x;
+                    dSs[(j0 + 2 * m + 1) * SL + c] = acc[m].y;
+                }
             }
-            __syncwarp();
-            float2 acc0 = make_float2(ex2f_(Glast[c]) * dSs[lane * SL + c], 0.f), acc1 = make_float2(0.f, 0.f);
-            int r = 0;
-            for (; r + 1 < Cc; r += 2) {
-                const float4 w4 = *reinterpret_cast<const float4 *>(wb + 2 * r);
-                acc0 = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(dOs[r * kVT + lane], dUs[r * kVT + lane]), acc0);
-                acc1 = __ffma2_rn(make_float2(w4.z, w4.w),
-                                  make_float2(dOs[(r + 1) * kVT + lane], dUs[(r + 1) * kVT + lane]), acc1);
-            }
-            if (r < Cc)
-                acc0 = __ffma2_rn(make_float2(wb[2 * r], wb[2 * r + 1]), make_float2(dOs[r * kVT + lane], dUs[r * kVT + lane]),
-                                  acc0);
-            dSs[lane * SL + c] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-            __syncwarp();
         }
         __syncthreads();
         if (kAnchored) {

@@ -58,6 +58,15 @@ __device__ __forceinline__ size_t bias_index(int per_head, int hv, int Dk, int c
     return per_head ? (size_t)hv : (size_t)hv * Dk + c;
 }
 
+// Hint: bring the 128-byte line holding p into L2 (no register, no wait).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+#ifdef __CUDA_ARCH__
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+#else
+    (void)p;
+#endif
+}
+
 // Validated arguments of a chunked forward, as the kernels see them.
 struct ChunkParams {
     int B, T, H, HV, Dk, Dv, C;
