@@ -64,6 +64,21 @@ __device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
         f[2 * i + 1] = __uint_as_float(r[i] & 0xFFFF0000u);
     }
 }
+// The same eight channels as four (even, odd) channel pairs.
+__device__ __forceinline__ void unpack8x2(uint4 w, float2 (&f)[4]) {
+    const uint32_t r[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(r[i] << 16), __uint_as_float(r[i] & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint4 pack8x2(const float2 (&f)[4]) {
+    uint32_t r[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(f[i].x, f[i].y);
+        r[i] = *reinterpret_cast<uint32_t *>(&a);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+}
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     uint32_t r[4];
 #pragma unroll
@@ -274,6 +289,17 @@ __device__ __forceinline__ float silu_of_half(float h) {
 #endif
     return fmaf(h, th, h);
 }
+// Both channels of a pair: tanh per channel, the product-add packed.
+__device__ __forceinline__ float2 silu_of_half2(float2 h) {
+    float2 th;
+#ifdef __CUDA_ARCH__
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.x) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(th.y) : "f"(h.y));
+#else
+    th = make_float2(tanhf(h.x), tanhf(h.y));
+#endif
+    return __ffma2_rn(h, th, h);
+}
 
 template <int K>
 __global__ void __launch_bounds__(kConvThreads, 1)
@@ -331,7 +357,7 @@ short_conv_tma_kernel(const __grid_constant__ ConvTmaParams tp) {
         while (ii < my && ii < kStages - 1) issue();
     const __nv_bfloat16 *sin = static_cast<const __nv_bfloat16 *>(p.state_in);
     __nv_bfloat16 *so = static_cast<__nv_bfloat16 *>(p.state_out);
-    float w[8][4], bias[8];
+    float2 w[4][4], bias[4];                          // channel pairs (8 lane, 8 lane + 1), ...
     int wg = -1;                                      // channel group whose weights are loaded
     int i = 0;
     bool aborted = false;
@@ -355,11 +381,15 @@ short_conv_tma_kernel(const __grid_constant__ ConvTmaParams tp) {
             wg = g;
             const int c = g * kTC + 8 * lane;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 // halved (exact in binary floating point): the convolution gives u / 2
-                bias[u] = p.bias ? 0.5f * p.bias[c + u] : 0.f;
+                bias[u] = p.bias ? make_float2(0.5f * p.bias[c + 2 * u], 0.5f * p.bias[c + 2 * u + 1])
+                                 : make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) w[u][j] = j < K ? 0.5f * p.w[(size_t)(c + u) * K + j] : 0.f;
+                for (int j = 0; j < 4; ++j)
+                    w[u][j] = j < K ? make_float2(0.5f * p.w[(size_t)(c + 2 * u) * K + j],
+                                                  0.5f * p.w[(size_t)(c + 2 * u + 1) * K + j])
+                                    : make_float2(0.f, 0.f);
             }
         }
         const int t0 = blk * kTT, t1 = min(p.T, t0 + kTT);
@@ -375,37 +405,39 @@ short_conv_tma_kernel(const __grid_constant__ ConvTmaParams tp) {
             }
             __syncthreads();
         }
-        float win[3][8];
+        // channel pairs in packed FP32x2 arithmetic (one instruction per pair)
+        float2 win[3][4];
 #pragma unroll
         for (int s = 0; s < 3; ++s)
-            unpack8(*reinterpret_cast<const uint4 *>(in + (uint32_t)(tw + s) * kRowBytes + 16u * lane), win[s]);
+            unpack8x2(*reinterpret_cast<const uint4 *>(in + (uint32_t)(tw + s) * kRowBytes + 16u * lane), win[s]);
 #pragma unroll
         for (int k = 0; k < kTokPerWarp; ++k) {
-            float cur[8];
-            unpack8(*reinterpret_cast<const uint4 *>(in + (uint32_t)(tw + kHalo + k) * kRowBytes + 16u * lane), cur);
-            float o[8];
-            float ss = 0.f;
+            float2 cur[4];
+            unpack8x2(*reinterpret_cast<const uint4 *>(in + (uint32_t)(tw + kHalo + k) * kRowBytes + 16u * lane), cur);
+            float2 o[4];
+            float2 ss2 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 // taps j = 0..K-2 read win[4 - K + j]; tap K-1 reads the current token
-                float acc = bias[u];
+                float2 acc = bias[u];
 #pragma unroll
                 for (int j = 0; j < 3; ++j)
-                    if (j < K - 1) acc = fmaf(w[u][j], win[4 - K + j][u], acc);
-                acc = fmaf(w[u][K - 1], cur[u], acc);
-                o[u] = p.silu ? silu_of_half(acc) : 2.f * acc;
-                ss = fmaf(o[u], o[u], ss);
+                    if (j < K - 1) acc = __ffma2_rn(w[u][j], win[4 - K + j][u], acc);
+                acc = __ffma2_rn(w[u][K - 1], cur[u], acc);
+                o[u] = p.silu ? silu_of_half2(acc) : __fadd2_rn(acc, acc);
+                ss2 = __ffma2_rn(o[u], o[u], ss2);
             }
             if (p.head_dim) {
+                float ss = ss2.x + ss2.y;
 #pragma unroll
                 for (int m = 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
                 const float rn = rsqrtf(ss + p.l2_eps);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) o[u] *= rn;
+                for (int u = 0; u < 4; ++u) o[u] = __fmul2_rn(o[u], make_float2(rn, rn));
             }
-            if (t0 + tw + k < t1) *reinterpret_cast<uint4 *>(yr + (size_t)k * p.C) = pack8(o);
+            if (t0 + tw + k < t1) *reinterpret_cast<uint4 *>(yr + (size_t)k * p.C) = pack8x2(o);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 win[0][u] = win[1][u];
                 win[1][u] = win[2][u];
                 win[2][u] = cur[u];

@@ -49,6 +49,8 @@ inline float2 make_float2(float x, float y) { return float2{x, y}; }
 inline float2 __ffma2_rn(float2 a, float2 b, float2 c) {
     return float2{std::fma(a.x, b.x, c.x), std::fma(a.y, b.y, c.y)};
 }
+inline float2 __fadd2_rn(float2 a, float2 b) { return float2{a.x + b.x, a.y + b.y}; }
+inline float2 __fmul2_rn(float2 a, float2 b) { return float2{a.x * b.x, a.y * b.y}; }
 inline unsigned __float_as_uint(float f) { unsigned u; std::memcpy(&u, &f, 4); return u; }
 inline unsigned atomicOr(unsigned *a, unsigned v) { return std::atomic_ref<unsigned>(*a).fetch_or(v); }
 #include <chrono>
