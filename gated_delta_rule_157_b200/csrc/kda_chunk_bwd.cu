@@ -41,12 +41,6 @@ static_assert(kVT == 32, "the row loops map one lane to one value column");
 static_assert(kThreads == 4 * 128, "the dS step maps a thread to (key channel, eight value columns)");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
 constexpr int kLoadBatch = 8;                 // global loads in flight per thread in the chunk load
-// Anchored A / P: channels staged 8 at a time -- row-anchored q and k of the 64
-// rows, and for every row tile R the column factors of its 16 (R + 1) columns.
-constexpr int kStageCh = 8;
-constexpr int kKcRows = 16 + 32 + 48 + 64;                // 160: columns of tiles 0..3
-constexpr int kStageFloats = (64 + 64 + kKcRows) * kStageCh;
-__host__ __device__ constexpr int kc_off(int R) { return 8 * R * (R + 1); }   // first row of tile R's columns
 
 // kAnchored (Dk = 128, C = 64, the bounded gate with |g_min| <= 5): step 8's
 // pairwise sums use the forward's 16-token tile anchors, so every factor
@@ -57,7 +51,9 @@ template <typename Tin, bool kAnchored>
 __global__ void __launch_bounds__(kThreads)
 chunk_bwd_kernel(BwdParams p) {
     extern __shared__ float smem[];
-    const int C = p.C, Dk = p.Dk, Dv = p.Dv;
+    // the anchored shape is fixed (C = 64, Dk = 128): every tile offset and
+    // stride below is then a compile-time constant
+    const int C = kAnchored ? 64 : p.C, Dk = kAnchored ? 128 : p.Dk, Dv = p.Dv;
     const int L = Dk | 1;                  // padded row stride of the [C][Dk] tiles
     // every array starts on a 16-byte boundary (packed float2 / float4 loads)
     const int CL = (C * L + 3) & ~3, CC = (C * C + 3) & ~3;
@@ -83,11 +79,6 @@ chunk_bwd_kernel(BwdParams p) {
     // per-warp row of factors, computed once per row and read by all 32 lanes
     // (one lane per value column): [warp][2 * 128]
     float *wb = dlast + Dk4 + (threadIdx.x >> 5) * 256;
-    // anchored path only: [kStageCh][64] q and k rows times 2^(G - P_R), and
-    // [kStageCh][kKcRows] columns k_i 2^(P_R - G_i) for every row tile R
-    float *Qa = dlast + Dk4 + (kThreads / 32) * 256;
-    float *Ka = Qa + kStageCh * 64;
-    float *Kc = Ka + kStageCh * 64;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int chain = blockIdx.x;
@@ -223,74 +214,63 @@ chunk_bwd_kernel(BwdParams p) {
             // A[r][i] = sum_c (q_rc 2^(G_rc - P_R)) (k_ic 2^(P_R - G_ic)), R = tile of r
             // (P likewise with k_rc), every factor within 2^+-116.  Warp w takes
             // half-blocks (row tile R, column tile J <= R, 8 rows) w and w + 16 of
-            // the 20; lane = (row lane / 4 of the 8, columns 4 (lane % 4) .. +3).
+            // the 20 and stages its own factors, eight channels at a time, in its
+            // scratch row (no CTA barrier): [8 ch][8 rows] of q and k, [8 ch][16
+            // columns]; lane = (row lane / 4, columns 4 (lane % 4) .. +3).
             const int ntile = (Cc + 15) >> 4;
-            float sa[2][4], sp[2][4];
-            int hb_R[2], hb_J[2], hb_h[2];
-#pragma unroll
+            float *Qw = wb, *Kw = wb + 64, *Kcw = wb + 128;
+#pragma unroll 1
             for (int t = 0; t < 2; ++t) {
-                int hbi = warp + 16 * t;              // 0..19: (R, J) in order, then half
+                const int hbi = warp + 16 * t;              // 0..19: (R, J) in order, then half
+                if (hbi >= 20) break;
                 const int blk = hbi >> 1;
                 int R = 0;
                 while (blk >= (R + 1) * (R + 2) / 2) ++R;
-                hb_R[t] = R;
-                hb_J[t] = blk - R * (R + 1) / 2;
-                hb_h[t] = hbi & 1;
+                const int J = blk - R * (R + 1) / 2, rw0 = 16 * R + 8 * (hbi & 1);
+                if (R >= ntile) continue;
+                float2 sa[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, sp[2] = {sa[0], sa[1]};
+                const int rl = lane >> 2, i4 = 4 * (lane & 3);
+                for (int c0 = 0; c0 < Dk; c0 += 8) {
+                    // rows: (cc = e & 7, row e >> 3), two per lane; columns: four per lane
 #pragma unroll
-                for (int u = 0; u < 4; ++u) sa[t][u] = sp[t][u] = 0.f;
-            }
-            for (int c0 = 0; c0 < Dk; c0 += kStageCh) {
-                // stage the factors of channels c0 .. c0+7 (rows past Cc hold stale
-                // values whose products are never stored)
-                for (int e = tid; e < 64 * kStageCh; e += kThreads) {
-                    const int r = e & 63, cc = e >> 6, c = c0 + cc, R = r >> 4;
-                    const float PR = R == 0 ? 0.f : Gs[(16 * R - 1) * L + c];
-                    const float f = ex2f_(Gs[r * L + c] - PR);
-                    Qa[cc * 64 + r] = Qs[r * L + c] * f;
-                    Ka[cc * 64 + r] = Ks[r * L + c] * f;
-                }
-                for (int e = tid; e < kKcRows * kStageCh; e += kThreads) {
-                    const int cc = e / kKcRows, row = e - cc * kKcRows, c = c0 + cc;
-                    int R = 0;
-                    while (row >= kc_off(R + 1)) ++R;
-                    const int i = row - kc_off(R);
-                    const float PR = R == 0 ? 0.f : Gs[(16 * R - 1) * L + c];
-                    Kc[cc * kKcRows + row] = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
-                }
-                __syncthreads();
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (warp + 16 * t >= 20 || hb_R[t] >= ntile) continue;
-                    const int r = 16 * hb_R[t] + 8 * hb_h[t] + (lane >> 2);
-                    const int krow = kc_off(hb_R[t]) + 16 * hb_J[t] + 4 * (lane & 3);
-#pragma unroll
-                    for (int cc = 0; cc < kStageCh; ++cc) {
-                        const float qa = Qa[cc * 64 + r], ka = Ka[cc * 64 + r];
-                        const float4 kc = *reinterpret_cast<const float4 *>(Kc + cc * kKcRows + krow);
-                        sa[t][0] = fmaf(qa, kc.x, sa[t][0]);
-                        sa[t][1] = fmaf(qa, kc.y, sa[t][1]);
-                        sa[t][2] = fmaf(qa, kc.z, sa[t][2]);
-                        sa[t][3] = fmaf(qa, kc.w, sa[t][3]);
-                        sp[t][0] = fmaf(ka, kc.x, sp[t][0]);
-                        sp[t][1] = fmaf(ka, kc.y, sp[t][1]);
-                        sp[t][2] = fmaf(ka, kc.z, sp[t][2]);
-                        sp[t][3] = fmaf(ka, kc.w, sp[t][3]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int e = lane + 32 * u, cc = e & 7, rr = rw0 + (e >> 3), c = c0 + cc;
+                        const float PR = R == 0 ? 0.f : Gs[(16 * R - 1) * L + c];
+                        const float f = ex2f_(Gs[rr * L + c] - PR);
+                        Qw[cc * 8 + (e >> 3)] = Qs[rr * L + c] * f;
+                        Kw[cc * 8 + (e >> 3)] = Ks[rr * L + c] * f;
                     }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int e = lane + 32 * u, cc = e >> 4, i = 16 * J + (e & 15), c = c0 + cc;
+                        const float PR = R == 0 ? 0.f : Gs[(16 * R - 1) * L + c];
+                        Kcw[cc * 16 + (e & 15)] = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const float qa = Qw[cc * 8 + rl], ka = Kw[cc * 8 + rl];
+                        const float4 kc = *reinterpret_cast<const float4 *>(Kcw + cc * 16 + i4);
+                        const float2 qa2 = make_float2(qa, qa), ka2 = make_float2(ka, ka);
+                        sa[0] = __ffma2_rn(qa2, make_float2(kc.x, kc.y), sa[0]);
+                        sa[1] = __ffma2_rn(qa2, make_float2(kc.z, kc.w), sa[1]);
+                        sp[0] = __ffma2_rn(ka2, make_float2(kc.x, kc.y), sp[0]);
+                        sp[1] = __ffma2_rn(ka2, make_float2(kc.z, kc.w), sp[1]);
+                    }
+                    __syncwarp();
                 }
-                __syncthreads();
-            }
-            // stores: A lower with the diagonal, P strictly lower, zeros above
+                // stores: A lower with the diagonal, P strictly lower, zeros above
+                const int r = rw0 + rl;
+                if (r < Cc) {
+                    const float av[4] = {sa[0].x, sa[0].y, sa[1].x, sa[1].y};
+                    const float pv[4] = {sp[0].x, sp[0].y, sp[1].x, sp[1].y};
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                if (warp + 16 * t >= 20 || hb_R[t] >= ntile) continue;
-                const int r = 16 * hb_R[t] + 8 * hb_h[t] + (lane >> 2);
-                if (r >= Cc) continue;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int i = 16 * hb_J[t] + 4 * (lane & 3) + u;
-                    if (i >= Cc) continue;
-                    Aqk[r * C + i] = i <= r ? sa[t][u] : 0.f;
-                    Pkk[r * C + i] = i < r ? sp[t][u] : 0.f;
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = 16 * J + i4 + u;
+                        if (i >= Cc) continue;
+                        Aqk[r * C + i] = i <= r ? av[u] : 0.f;
+                        Pkk[r * C + i] = i < r ? pv[u] : 0.f;
+                    }
                 }
             }
             // the blocks above the diagonal tiles
@@ -858,8 +838,8 @@ size_t bwd_smem_bytes(int C, int Dk, bool anchored) {
     const size_t Dk4 = ((size_t)Dk + 3) & ~(size_t)3;
     const size_t f = 3 * CL + 2 * CC + (size_t)4 * C * kVT + (size_t)2 * kVT * (Dk4 + 4) +
                      2 * (((size_t)C + 3) & ~(size_t)3) + 2 * Dk4 +
-                     (size_t)(kThreads / 32) * 256 +
-                     (anchored ? (size_t)kStageFloats : 0);
+                     (size_t)(kThreads / 32) * 256;
+    (void)anchored;
     return f * sizeof(float);
 }
 
