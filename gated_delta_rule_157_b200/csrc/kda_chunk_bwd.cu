@@ -212,17 +212,20 @@ chunk_bwd_kernel(BwdParams p) {
         // ---- 3. A, P and X = V - (K*exp(G)) S -------------------------------
         if (kAnchored) {
             // A[r][i] = sum_c (q_rc 2^(G_rc - P_R)) (k_ic 2^(P_R - G_ic)), R = tile of r
-            // (P likewise with k_rc), every factor within 2^+-116.  Warp w takes
-            // half-blocks (row tile R, column tile J <= R, 8 rows) w and w + 16 of
-            // the 20 and stages its own factors, eight channels at a time, in its
-            // scratch row (no CTA barrier): [8 ch][8 rows] of q and k, [8 ch][16
-            // columns]; lane = (row lane / 4, columns 4 (lane % 4) .. +3).
+            // (P likewise with k_rc), every factor within 2^+-116.  Of the 20
+            // half-blocks (row tile R, column tile J <= R, 8 rows), warp w takes
+            // half-block w over all channels and a quarter of the channels of
+            // half-block 16 + w % 4 (summed below), 20 eight-channel steps per
+            // warp; it stages its own factors in its scratch row (no CTA
+            // barrier): [8 ch][8 rows] of q and k, [8 ch][16 columns]; lane =
+            // (row lane / 4, columns 4 (lane % 4) .. +3).  The quarter sums go
+            // to the U and dU tiles, free until step 4.
             const int ntile = (Cc + 15) >> 4;
             float *Qw = wb, *Kw = wb + 64, *Kcw = wb + 128;
 #pragma unroll 1
             for (int t = 0; t < 2; ++t) {
-                const int hbi = warp + 16 * t;              // 0..19: (R, J) in order, then half
-                if (hbi >= 20) break;
+                const int hbi = t == 0 ? warp : 16 + (warp & 3);   // (R, J) in order, then half
+                const int cbeg = t == 0 ? 0 : 32 * (warp >> 2), cend = t == 0 ? Dk : cbeg + 32;
                 const int blk = hbi >> 1;
                 int R = 0;
                 while (blk >= (R + 1) * (R + 2) / 2) ++R;
@@ -230,7 +233,7 @@ chunk_bwd_kernel(BwdParams p) {
                 if (R >= ntile) continue;
                 float2 sa[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, sp[2] = {sa[0], sa[1]};
                 const int rl = lane >> 2, i4 = 4 * (lane & 3);
-                for (int c0 = 0; c0 < Dk; c0 += 8) {
+                for (int c0 = cbeg; c0 < cend; c0 += 8) {
                     // rows: (cc = e & 7, row e >> 3), two per lane; columns: four per lane
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
@@ -259,6 +262,13 @@ chunk_bwd_kernel(BwdParams p) {
                     }
                     __syncwarp();
                 }
+                if (t == 1) {                       // a quarter sum: [quarter][half-block][lane][8]
+                    const int q = warp >> 2;
+                    float *part = (q < 2 ? Us + q * 1024 : dUs + (q - 2) * 1024) + ((hbi - 16) * 32 + lane) * 8;
+                    *reinterpret_cast<float4 *>(part) = make_float4(sa[0].x, sa[0].y, sa[1].x, sa[1].y);
+                    *reinterpret_cast<float4 *>(part + 4) = make_float4(sp[0].x, sp[0].y, sp[1].x, sp[1].y);
+                    continue;
+                }
                 // stores: A lower with the diagonal, P strictly lower, zeros above
                 const int r = rw0 + rl;
                 if (r < Cc) {
@@ -279,6 +289,23 @@ chunk_bwd_kernel(BwdParams p) {
                 if ((i >> 4) > (r >> 4)) {
                     Aqk[r * C + i] = 0.f;
                     Pkk[r * C + i] = 0.f;
+                }
+            }
+            __syncthreads();
+            // half-blocks 16..19 (row tile 3, column tiles 2 and 3): the sums of
+            // the four quarters, [half-block][lane][4 A values, 4 P values]
+            if (ntile == 4) {
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const int idx = tid + kThreads * m;
+                    const float v = (Us[idx] + Us[1024 + idx]) + (dUs[idx] + dUs[1024 + idx]);
+                    const int hbi = 16 + (idx >> 8), ln = (idx >> 3) & 31, u = idx & 3;
+                    const int r = 48 + 8 * (hbi & 1) + (ln >> 2);
+                    const int i = 16 * ((hbi >> 1) - 6) + 4 * (ln & 3) + u;
+                    if (r < Cc && i < Cc) {
+                        if ((idx & 4) == 0) Aqk[r * C + i] = i <= r ? v : 0.f;
+                        else Pkk[r * C + i] = i < r ? v : 0.f;
+                    }
                 }
             }
         } else {
