@@ -326,22 +326,37 @@ chunk_bwd_kernel(BwdParams p) {
                 Pkk[r * C + i] = pk;
             }
         }
-        // warp w takes rows w, w + 16, ...; lane = value column; channel pairs
-        // (c, c + 1) in one packed FMA, two chains
-        for (int r = warp; r < Cc; r += kThreads / 32) {
-            for (int c = lane; c < Dk; c += 32) wb[c] = -Ks[r * L + c] * ex2f_(Gs[r * L + c]);
+        // warp w takes the row pairs (r, r + 16), r = w, w + 32, ...; lane = value
+        // column (one load of S^T per lane and four channels for both rows);
+        // channel pairs (c, c + 1) in one packed FMA
+        for (int r = warp; r < Cc; r += 2 * (kThreads / 32)) {
+            const int r2 = r + kThreads / 32;
+            const bool has2 = r2 < Cc;
+            const int rb = has2 ? r2 : r;
+            for (int c = lane; c < Dk; c += 32) {
+                wb[c] = -Ks[r * L + c] * ex2f_(Gs[r * L + c]);
+                wb[128 + c] = -Ks[rb * L + c] * ex2f_(Gs[rb * L + c]);
+            }
             __syncwarp();
-            float2 acc0 = make_float2(Xs[r * kVT + lane], 0.f), acc1 = make_float2(0.f, 0.f);
+            float2 a0 = make_float2(Xs[r * kVT + lane], 0.f), a1 = make_float2(0.f, 0.f);
+            float2 b0 = make_float2(Xs[rb * kVT + lane], 0.f), b1 = make_float2(0.f, 0.f);
             const float *srow = Ss + lane * SL;
             int c = 0;
             for (; c + 3 < Dk; c += 4) {
-                const float4 w4 = *reinterpret_cast<const float4 *>(wb + c);
                 const float4 s4 = *reinterpret_cast<const float4 *>(srow + c);
-                acc0 = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(s4.x, s4.y), acc0);
-                acc1 = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(s4.z, s4.w), acc1);
+                const float4 wa = *reinterpret_cast<const float4 *>(wb + c);
+                const float4 wc = *reinterpret_cast<const float4 *>(wb + 128 + c);
+                a0 = __ffma2_rn(make_float2(wa.x, wa.y), make_float2(s4.x, s4.y), a0);
+                a1 = __ffma2_rn(make_float2(wa.z, wa.w), make_float2(s4.z, s4.w), a1);
+                b0 = __ffma2_rn(make_float2(wc.x, wc.y), make_float2(s4.x, s4.y), b0);
+                b1 = __ffma2_rn(make_float2(wc.z, wc.w), make_float2(s4.z, s4.w), b1);
             }
-            for (; c < Dk; ++c) acc0.x = fmaf(wb[c], srow[c], acc0.x);
-            Xs[r * kVT + lane] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+            for (; c < Dk; ++c) {
+                a0.x = fmaf(wb[c], srow[c], a0.x);
+                b0.x = fmaf(wb[128 + c], srow[c], b0.x);
+            }
+            Xs[r * kVT + lane] = (a0.x + a0.y) + (a1.x + a1.y);
+            if (has2) Xs[r2 * kVT + lane] = (b0.x + b0.y) + (b1.x + b1.y);
             __syncwarp();
         }
         __syncthreads();
@@ -395,23 +410,41 @@ chunk_bwd_kernel(BwdParams p) {
             }
         }
         // ---- 5. dU = A^T dO + (K*exp(G_last - G)) dS' ------------------------
-        for (int r = warp; r < Cc; r += kThreads / 32) {
-            for (int c = lane; c < Dk; c += 32) wb[c] = Ks[r * L + c] * ex2f_(Glast[c] - Gs[r * L + c]);
+        // row pairs (r, r + 16) as in X: A^T dO with (A[rr][r], A[rr][r + 16])
+        // in one packed FMA (A is zero above the diagonal), then the dS' terms
+        for (int r = warp; r < Cc; r += 2 * (kThreads / 32)) {
+            const int r2 = r + kThreads / 32;
+            const bool has2 = r2 < Cc;
+            const int rb = has2 ? r2 : r;
+            for (int c = lane; c < Dk; c += 32) {
+                wb[c] = Ks[r * L + c] * ex2f_(Glast[c] - Gs[r * L + c]);
+                wb[128 + c] = Ks[rb * L + c] * ex2f_(Glast[c] - Gs[rb * L + c]);
+            }
             __syncwarp();
-            float acc = 0.f;
-            for (int rr = r; rr < Cc; ++rr) acc = fmaf(Aqk[rr * C + r], dOs[rr * kVT + lane], acc);
-            // channels four at a time, two packed chains
+            float2 ab = make_float2(0.f, 0.f);
+            for (int rr = r; rr < Cc; ++rr) {
+                const float o = dOs[rr * kVT + lane];
+                ab = __ffma2_rn(make_float2(Aqk[rr * C + r], Aqk[rr * C + rb]), make_float2(o, o), ab);
+            }
             const float *drow = dSs + lane * SL;
-            float2 acc0 = make_float2(acc, 0.f), acc1 = make_float2(0.f, 0.f);
+            float2 a0 = make_float2(ab.x, 0.f), a1 = make_float2(0.f, 0.f);
+            float2 b0 = make_float2(ab.y, 0.f), b1 = make_float2(0.f, 0.f);
             int c = 0;
             for (; c + 3 < Dk; c += 4) {
-                const float4 w4 = *reinterpret_cast<const float4 *>(wb + c);
                 const float4 d4 = *reinterpret_cast<const float4 *>(drow + c);
-                acc0 = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(d4.x, d4.y), acc0);
-                acc1 = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(d4.z, d4.w), acc1);
+                const float4 wa = *reinterpret_cast<const float4 *>(wb + c);
+                const float4 wc = *reinterpret_cast<const float4 *>(wb + 128 + c);
+                a0 = __ffma2_rn(make_float2(wa.x, wa.y), make_float2(d4.x, d4.y), a0);
+                a1 = __ffma2_rn(make_float2(wa.z, wa.w), make_float2(d4.z, d4.w), a1);
+                b0 = __ffma2_rn(make_float2(wc.x, wc.y), make_float2(d4.x, d4.y), b0);
+                b1 = __ffma2_rn(make_float2(wc.z, wc.w), make_float2(d4.z, d4.w), b1);
             }
-            for (; c < Dk; ++c) acc0.x = fmaf(wb[c], drow[c], acc0.x);
-            dUs[r * kVT + lane] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+            for (; c < Dk; ++c) {
+                a0.x = fmaf(wb[c], drow[c], a0.x);
+                b0.x = fmaf(wb[128 + c], drow[c], b0.x);
+            }
+            dUs[r * kVT + lane] = (a0.x + a0.y) + (a1.x + a1.y);
+            if (has2) dUs[r2 * kVT + lane] = (b0.x + b0.y) + (b1.x + b1.y);
             __syncwarp();
         }
         __syncthreads();
