@@ -12,8 +12,9 @@ state, 512 consecutive steps) in GB/s, the segmented KCP pass, the layer
 prologue / epilogue kernels in GB/s, and the FP64 oracle timed on the host
 cores as a reported baseline.
 
---train adds the training path (forward keeping the per-chunk states, then
-kda_chunk_bwd) at the same workload, each timed on the device.
+The extras include the training path (forward keeping the per-chunk states,
+then kda_chunk_bwd) at the same workload, each timed on the device; --train is
+accepted for compatibility and changes nothing.
 
 Multi-GPU (torchrun): every rank runs its own batch of the same workload (weak
 scaling, no collective on the data path); the time is the max over ranks.
