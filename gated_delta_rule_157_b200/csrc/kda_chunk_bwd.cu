@@ -98,15 +98,37 @@ chunk_bwd_kernel(BwdParams p) {
         dSs[(idx % kVT) * SL + c] = (p.dS_T && col < Dv) ? p.dS_T[((size_t)chain * Dk + c) * Dv + col] : 0.f;
     }
 
+    // Anchored shape with bf16 inputs, one decay per key channel and 16-byte
+    // aligned rows: the raw q, k, g rows of chunk ch - 1 are copied into the A,
+    // P, X and U tiles (free after step 8 of chunk ch) by asynchronous copies
+    // that run during steps 9 and 10.
+    const bool can_stage = kAnchored && sizeof(Tin) == 2 && !p.g_per_head &&
+                           ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                             reinterpret_cast<uintptr_t>(g)) & 15) == 0;
+    const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(Aqk);   // [3][C][Dk] q, k, g
+
     for (int ch = NC - 1; ch >= 0; --ch) {
         const int t0 = ch * C;
         const int Cc = min(C, p.T - t0);
         const size_t tok0 = (size_t)b * p.T + t0;
+        const bool staged = can_stage && ch < NC - 1;
+        if (staged) cp_async_wait_all();
         __syncthreads();
         // ---- 1. load the chunk and the state entering it -------------------
         // (the state and value rows in batches of kLoadBatch elements per
         // thread whose loads are all issued before the first shared-memory store)
-        for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
+        if (staged) {
+            // full chunk (only the last chunk can be ragged, and it is never staged)
+            const int c = tid & 127;
+            const float bias = (p.gate_in && p.dt_bias) ? p.dt_bias[bias_index(0, hv, 128, c)] : 0.f;
+#pragma unroll 4
+            for (int r = tid >> 7; r < C; r += kThreads / 128) {
+                const float gz = __bfloat162float(raw[(2 * C + r) * Dk + c]);
+                Qs[r * L + c] = __bfloat162float(raw[r * Dk + c]);
+                Ks[r * L + c] = __bfloat162float(raw[(C + r) * Dk + c]);
+                Gs[r * L + c] = p.gate_in ? kda_gate(p.gate_in, gz, bias, ea, p.g_min) : gz;
+            }
+        } else for (int idx = tid; idx < Cc * Dk; idx += kThreads) {
             const int r = idx / Dk, c = idx % Dk;
             const size_t tok = tok0 + r;
             Qs[r * L + c] = ld_act(q, (tok * p.H + h) * Dk + c);
@@ -131,6 +153,7 @@ chunk_bwd_kernel(BwdParams p) {
                 if (idx < Dk * kVT) Ss[(idx % kVT) * SL + idx / kVT] = sv[u];
             }
         }
+        if (staged) __syncthreads();       // the staged g rows lie under X, written next
         for (int base = tid; base < Cc * kVT; base += (kLoadBatch / 2) * kThreads) {
             float vv[kLoadBatch / 2], ov[kLoadBatch / 2];
 #pragma unroll
@@ -693,6 +716,22 @@ chunk_bwd_kernel(BwdParams p) {
             }
         }
         __syncthreads();
+        if (can_stage && ch > 0) {
+            // q, k, g rows of chunk ch - 1 (full: C rows of 256 bytes) into the
+            // free A/P/X/U tiles, 16 bytes per copy
+            const size_t ptok = tok0 - C;
+            uint8_t *dst = reinterpret_cast<uint8_t *>(Aqk);
+            for (int e = tid; e < 3 * C * 16; e += kThreads) {
+                const int tsr = e / (C * 16), rest = e % (C * 16), r = rest >> 4, q16 = rest & 15;
+                const size_t tok = ptok + r;
+                const uint8_t *src =
+                    tsr == 0   ? reinterpret_cast<const uint8_t *>(q + (tok * p.H + h) * 128)
+                    : tsr == 1 ? reinterpret_cast<const uint8_t *>(k + (tok * p.H + h) * 128)
+                               : reinterpret_cast<const uint8_t *>(g + (tok * p.HV + hv) * 128);
+                cp_async16(dst + ((size_t)(tsr * C + r) * 128) * 2 + 16 * q16, src + 16 * q16);
+            }
+            cp_async_commit();
+        }
         // ---- 9. dS entering the chunk (in place) -----------------------------
         // thread = (key channel c, eight value columns j0 .. j0+7): the factors
         // e^G q and -e^G k beta of (r, c) once per thread, the value columns of

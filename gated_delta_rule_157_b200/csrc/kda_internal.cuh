@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <cstring>
 
 #include "../../include/kda.h"
 
@@ -56,6 +57,27 @@ __device__ __forceinline__ size_t gate_index(int per_head, size_t tok, int HV, i
 }
 __device__ __forceinline__ size_t bias_index(int per_head, int hv, int Dk, int c) {
     return per_head ? (size_t)hv : (size_t)hv * Dk + c;
+}
+
+// Asynchronous 16-byte global -> shared copy (both addresses 16-byte aligned),
+// its commit, and the wait for every committed copy of this thread.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
+#ifdef __CUDA_ARCH__
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst_smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+#else
+    std::memcpy(dst_smem, src, 16);
+#endif
+}
+__device__ __forceinline__ void cp_async_commit() {
+#ifdef __CUDA_ARCH__
+    asm volatile("cp.async.commit_group;" ::: "memory");
+#endif
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+#ifdef __CUDA_ARCH__
+    asm volatile("cp.async.wait_all;" ::: "memory");
+#endif
 }
 
 // Hint: bring the 128-byte line holding p into L2 (no register, no wait).
