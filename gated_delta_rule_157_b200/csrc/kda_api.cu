@@ -103,9 +103,10 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
 
     if (a->T == 0) return cuda_status(kda::launch_chunk_empty(p, s));
 
-    // Only the SIMT kernel takes the softplus gate (unbounded: the tensor-core
-    // exponent scheme needs g >= g_min).
-    const bool tc_ok = kda::chunk_tc_supported(p, bf16) && a->gate_in_kernel <= 1;
+    // The tensor-core kernel's exponent scheme needs g >= g_min: with a
+    // caller-given decay or the (unbounded) softplus gate it clamps g there
+    // and reports the clamp, so AUTO sends both to the exact SIMT kernel.
+    const bool tc_ok = kda::chunk_tc_supported(p, bf16);
     if (withhold_ready && (a->algo != KDA_ALGO_TC || !tc_ok)) return KDA_ERR_UNSUPPORTED;
     if (a->algo == KDA_ALGO_TC) {
         if (!tc_ok) return KDA_ERR_UNSUPPORTED;
@@ -117,7 +118,7 @@ static kda_status chunk_fwd(const kda_chunk_args *a, void *stream, bool withhold
     // A log-decay given directly (no in-kernel gate) may lie below g_min, where
     // the tensor-core kernel's exponent bound does not hold: AUTO takes the
     // SIMT kernel, which is exact for any g <= 0.
-    if (a->algo == KDA_ALGO_AUTO && tc_ok && a->gate_in_kernel != 0) {
+    if (a->algo == KDA_ALGO_AUTO && tc_ok && a->gate_in_kernel == 1) {
         bool al16 = true;
         const void *v16[] = {a->q, a->k, a->v, a->g, a->o};
         for (const void *ptr : v16) al16 = al16 && aligned(ptr, 16);

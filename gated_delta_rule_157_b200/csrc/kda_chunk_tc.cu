@@ -66,6 +66,7 @@ constexpr int D = 128;
 constexpr int BAR_PREP = 1;
 constexpr int BAR_STATE = 2;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // Shared-memory map (bytes from a 1024-aligned base).
 constexpr uint32_t OFF_AINTRA = 0;        // [128 rows][K=128]  K e^L (rows 0-63), Q e^L (64-127)
@@ -251,13 +252,16 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
     float *Tm = reinterpret_cast<float *>(sm + OFF_TINV);
     const __nv_bfloat16 *bl = static_cast<const __nv_bfloat16 *>(p.beta);
 
-    // Gate in log2 units: g2 = g_min log2(e) / (1 + 2^-(A1 z + B1)), A1 = exp(A_log) log2(e).
+    // Gate in log2 units, A1 = exp(A_log) log2(e): bounded, g2 = g_min log2(e) /
+    // (1 + 2^-(A1 z + B1)) with B1 = A1 dt_bias; softplus, g2 = -A1 softplus(z + B1)
+    // with B1 = dt_bias.
     const float A1 = p.gate_in ? expf(p.A_log[x.hv]) * kLog2e : 0.f;
     float B1[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-        B1[u] = (p.gate_in && p.dt_bias) ? p.dt_bias[p.g_per_head ? (size_t)x.hv : (size_t)x.hv * D + c0 + u] * A1
-                                         : 0.f;
+        B1[u] = (p.gate_in && p.dt_bias)
+                    ? p.dt_bias[p.g_per_head ? (size_t)x.hv : (size_t)x.hv * D + c0 + u] * (p.gate_in == 1 ? A1 : 1.f)
+                    : 0.f;
     const float gmin2 = p.g_min * kLog2e;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     uint32_t ph_mma = 0;
@@ -414,11 +418,17 @@ __device__ __forceinline__ void prep_role(const ChunkParams &p, const CUtensorMa
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 float g;
-                if (p.gate_in) {
+                if (p.gate_in == 1) {
                     g = gmin2 * rcp_approx(1.f + ex2_approx(-fmaf(zz[u], A1, B1[u])));
                 } else {
+                    if (p.gate_in == 2) {
+                        // softplus(x) = max(x, 0) + ln(1 + e^-|x|), unbounded below
+                        const float xx = zz[u] + B1[u];
+                        g = -A1 * (fmaxf(xx, 0.f) + kLn2 * lg2_approx(1.f + ex2_approx(-fabsf(xx) * kLog2e)));
+                    } else {
+                        g = zz[u] * kLog2e;
+                    }
                     // the exponent bound needs g >= g_min: clamped, and reported
-                    g = zz[u] * kLog2e;
                     below_gmin = below_gmin || (tq + i < Cc && g < gmin2);
                     g = fmaxf(g, gmin2);
                 }

@@ -116,9 +116,13 @@ typedef enum {
  *
  * Limits: B, T >= 0; 1 <= H <= HV, HV % H == 0; 1 <= Dk, Dv <= 128;
  * 1 <= chunk <= 64.  q, k, v, g, beta, o must be aligned to their element size;
- * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64,
- * gate_in_kernel 0 or 1 (the bounded gate), and 16-byte aligned q, k, v, g, o
- * (KDA_ALGO_AUTO takes the SIMT kernel otherwise, and for gate_in_kernel = 0).
+ * KDA_ALGO_TC additionally needs dtype = BF16, Dk = Dv = 128, chunk = 64 and
+ * 16-byte aligned q, k, v, g, o.  Its exponent scheme rests on g >= g_min:
+ * with gate_in_kernel = 0 (a caller-given log-decay) or 2 (the softplus gate,
+ * unbounded below) it clamps every g below g_min to g_min and reports the
+ * clamp as KDA_ERR_RANGE through kda_device_status (never silently).
+ * KDA_ALGO_AUTO takes the tensor-core kernel only for the bounded gate
+ * (gate_in_kernel = 1) and the SIMT kernel, exact for any g <= 0, otherwise.
  * gate_in_kernel must be 0, 1 or 2.  o must not overlap any input; S_T, M_T and
  * S_chunks must not overlap each other, o, or any input except S_T == S0.
  * T == 0 writes S_T = S0 (or 0) and M_T = I.

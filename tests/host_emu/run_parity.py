@@ -239,7 +239,7 @@ TRANSITION_CASES = [
     (2, 70, 1, 1, 40, 8, 32, 52),
 ]
 
-def run_tc_case(lib, B, T, H, HV, want_M, s0, z_mean, seed, per_head=False, states=False):
+def run_tc_case(lib, B, T, H, HV, want_M, s0, z_mean, seed, per_head=False, states=False, gate=1):
     """The tensor-core chunk kernel (bf16, Dk = Dv = 128, C = 64) over the host
     model of its instructions, against the oracle at the bf16 bars (o: 2e-2 of
     max|o|; S_T, M_T, chunk states: 2e-2 Frobenius), each rescaled to TOL."""
@@ -249,19 +249,22 @@ def run_tc_case(lib, B, T, H, HV, want_M, s0, z_mean, seed, per_head=False, stat
     inp = workloads.chunk_inputs(w, z_mean=z_mean)
     if per_head:
         inp = _per_head(inp)
+    if gate == 2:      # the softplus gate, kept above g_min (exp(A_log) = 0.22)
+        inp["A_log"] = torch.full_like(inp["A_log"], -1.5)
     o = torch.zeros((B, T, HV, 128), dtype=torch.bfloat16)
     S_T = torch.zeros((B, HV, 128, 128))
     M_T = torch.zeros((B, HV, 128, 128)) if want_M else None
     NC = -(-T // 64)
     S_ch = torch.full((B, HV, NC, 128, 128), float("nan")) if states else None
-    fp = ChunkParams(B, T, H, HV, 128, 128, 64, HV // H, -5.0, 1.0, 1e-6, 1, 1, 1, int(per_head),
+    fp = ChunkParams(B, T, H, HV, 128, 128, 64, HV // H, -5.0, 1.0, 1e-6, 1, 1, gate, int(per_head),
                      *(_ptr(inp[n]) for n in ("q", "k", "v", "g", "beta", "A_log", "dt_bias", "S0")),
                      _ptr(o), _ptr(S_T), _ptr(M_T), _ptr(S_ch), 0)
     if lib.emu_chunk_tc(ctypes.byref(fp)) != 0:
         return {"device_error": 1.0}
     args = [to_np(inp[n]) for n in ("q", "k", "v", "g", "beta")]
-    if per_head:
-        args[3] = _gate_np(args[3], to_np(inp["A_log"]), to_np(inp["dt_bias"]), "bounded", True, 128)
+    if per_head or gate == 2:
+        args[3] = _gate_np(args[3], to_np(inp["A_log"]), to_np(inp["dt_bias"]),
+                           "bounded" if gate == 1 else "softplus", per_head, 128)
         kw = dict(S0=to_np(inp["S0"]), gate_in=False)
     else:
         kw = dict(A_log=to_np(inp["A_log"]), dt_bias=to_np(inp["dt_bias"]), S0=to_np(inp["S0"]))
@@ -288,6 +291,7 @@ TC_CASES = [
     (1, 130, 2, 4, False, 0.05, 0.0, 6, True, False),   # one decay per (token, head)
     (2, 200, 2, 4, True, 0.02, 0.0, 231),      # two batch rows, grouped heads, ragged, transition
     (1, 1, 1, 1, False, 0.05, 0.0, 32),        # a single token
+    (1, 150, 1, 2, False, 0.05, 0.0, 33, False, False, 2),   # the softplus gate above g_min
 ]
 
 COMPOSE_CASES = [

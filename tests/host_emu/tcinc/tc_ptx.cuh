@@ -310,6 +310,7 @@ __device__ __forceinline__ void bulk_wait() {}
 // ---- special functions, conversions, warp-level tf32 mma -------------------------------
 __device__ __forceinline__ float ex2_approx(float x) { return std::exp2(x); }
 __device__ __forceinline__ float rcp_approx(float x) { return 1.0f / x; }
+__device__ __forceinline__ float lg2_approx(float x) { return std::log2(x); }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return ((uint32_t)__float2bfloat16_rn(hi).x << 16) | (uint32_t)__float2bfloat16_rn(lo).x;
 }

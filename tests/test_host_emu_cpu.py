@@ -26,7 +26,7 @@ def test_simt_kernels_under_host_emulation():
     r = subprocess.run([sys.executable, os.path.join(HERE, "host_emu", "run_parity.py")], env=env,
                        capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-4000:] + r.stderr[-4000:]
-    assert "MISMATCH" not in r.stdout and r.stdout.count(" ok ") == 35, r.stdout
+    assert "MISMATCH" not in r.stdout and r.stdout.count(" ok ") == 36, r.stdout
 
 
 _PROBE = r"""

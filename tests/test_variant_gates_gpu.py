@@ -2,8 +2,8 @@
 decay per (token, head) as in Gated DeltaNet) on the SIMT kernels -- chunk
 forward, decode step and backward -- against the FP64 oracle, which takes the
 variant gates precomputed by oracle/gates.py.  The tensor-core kernel takes
-the per-head decay and refuses the softplus gate (its exponent bound needs
-g >= g_min).
+the per-head decay, and the softplus gate under a guard: its exponent bound
+needs g >= g_min, so it clamps there and reports the clamp.
 """
 import numpy as np
 import pytest
@@ -67,14 +67,42 @@ def test_chunk_forward_gate_variants(cuda_device, case):
     assert max_rel(to_np(S_T), ref["S_T"]) <= TOL_F32          # SIMT: fp32 state from exact inputs
 
 
-def test_tensor_core_kernel_refuses_the_softplus_gate(cuda_device):
-    """The unbounded gate breaks the tensor-core kernel's exponent bound:
-    algo='tc' returns UNSUPPORTED, 'auto' runs the SIMT kernel (bit for bit)."""
-    w, inp = _variant_inputs(1, 128, 1, 1, 128, 128, 64, "bf16", seed=70, per_head=False)
+def _clamped_oracle(inp, Dk, g_min=-5.0):
+    g = np.maximum(_log_decay(inp, "softplus", False, Dk), g_min)
+    return oracle.kda_fwd(*(to_np(inp[n]) for n in ("q", "k", "v")), g, to_np(inp["beta"]),
+                          S0=to_np(inp["S0"]), gate_in=False)
+
+
+def test_tensor_core_kernel_guards_the_softplus_gate(cuda_device):
+    """The softplus gate is unbounded below and the tensor-core kernel's
+    exponent bound needs g >= g_min.  Where the gate stays above g_min
+    (small exp(A_log)), algo='tc' matches the oracle at the bf16 bar with no
+    report; where it falls below (large exp(A_log)), the kernel clamps g to
+    g_min, reports KDA_ERR_RANGE and matches the oracle on the clamped decay.
+    'auto' keeps the exact SIMT kernel (bit for bit)."""
+    from helpers import fro_rel
+    w, inp = _variant_inputs(1, 200, 1, 2, 128, 128, 64, "bf16", seed=70, per_head=False)
+    inp["A_log"] = torch.full_like(inp["A_log"], -1.5)          # exp(A_log) = 0.22: g > -2
+    assert float(_log_decay(inp, "softplus", False, 128).min()) > -5.0
     d = to_device(inp, cuda_device)
+    kda.kda_device_status()
+    o, S_T, _ = _fwd(d, w, "softplus", False, algo="tc")
+    kda.kda_device_status()                                     # nothing reported
+    ref = _oracle_fwd(inp, "softplus", False, 128)
+    assert max_rel(to_np(o), ref["o"]) <= TOL_BF16
+    assert fro_rel(to_np(S_T), ref["S_T"]) <= TOL_BF16
+
+    inp["A_log"] = torch.full_like(inp["A_log"], 2.0)           # exp(A_log) = 7.4: g well below -5
+    assert float(_log_decay(inp, "softplus", False, 128).min()) < -8.0
+    d = to_device(inp, cuda_device)
+    o, S_T, _ = _fwd(d, w, "softplus", False, algo="tc")
     with pytest.raises(kda.KdaError) as e:
-        _fwd(d, w, "softplus", False, algo="tc")
-    assert e.value.status == 2
+        kda.kda_device_status()
+    assert e.value.status == 7                                  # KDA_ERR_RANGE
+    kda.kda_device_status()                                     # and cleared
+    ref = _clamped_oracle(inp, 128)
+    assert max_rel(to_np(o), ref["o"]) <= TOL_BF16
+    assert fro_rel(to_np(S_T), ref["S_T"]) <= TOL_BF16
     a, b = _fwd(d, w, "softplus", False, algo="auto"), _fwd(d, w, "softplus", False, algo="simt")
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
