@@ -514,24 +514,41 @@ chunk_bwd_kernel(BwdParams p) {
         // of a half-warp read different shared-memory banks.
         for (int r = warp; r < Cc; r += kThreads / 32) {
             float db = 0.f;
-            for (int i = lane; i < Cc; i += 32) {
-                float2 da = make_float2(0.f, 0.f), dm = make_float2(0.f, 0.f);
-                if (i <= r) {
-                    for (int j0 = 0; j0 < kVT; j0 += 2) {
-                        const int j = (j0 + 2 * lane) & (kVT - 1);
-                        const float2 u = *reinterpret_cast<const float2 *>(Us + i * kVT + j);
-                        da = __ffma2_rn(*reinterpret_cast<const float2 *>(dOs + r * kVT + j), u, da);
-                        dm = __ffma2_rn(*reinterpret_cast<const float2 *>(dUs + r * kVT + j), u, dm);
+            // columns i = lane and i + 32 in one pass over the value columns of
+            // rows r of dO and dZ (the second only where it is on or below the
+            // diagonal: r >= 32)
+            const int i1 = lane + 32;
+            const bool two = r >= 32;
+            float2 da = make_float2(0.f, 0.f), dm = make_float2(0.f, 0.f);
+            float2 da1 = da, dm1 = da;
+            if (lane <= r) {
+                for (int j0 = 0; j0 < kVT; j0 += 2) {
+                    const int j = (j0 + 2 * lane) & (kVT - 1);
+                    const float2 o2 = *reinterpret_cast<const float2 *>(dOs + r * kVT + j);
+                    const float2 z2 = *reinterpret_cast<const float2 *>(dUs + r * kVT + j);
+                    const float2 u = *reinterpret_cast<const float2 *>(Us + lane * kVT + j);
+                    da = __ffma2_rn(o2, u, da);
+                    dm = __ffma2_rn(z2, u, dm);
+                    if (two) {
+                        const float2 u1 = *reinterpret_cast<const float2 *>(Us + i1 * kVT + j);
+                        da1 = __ffma2_rn(o2, u1, da1);
+                        dm1 = __ffma2_rn(z2, u1, dm1);
                     }
                 }
-                const float dms = -(dm.x + dm.y);
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = h ? i1 : lane;
+                if (i >= Cc) continue;
+                const float2 a2 = h ? da1 : da, m2 = h ? dm1 : dm;
+                const float dms = (i <= r) ? -(m2.x + m2.y) : 0.f;
                 if (i < r) {
                     db = fmaf(dms, Pkk[r * C + i], db);
                     Pkk[r * C + i] = bet[r] * dms;
                 } else {
                     Pkk[r * C + i] = 0.f;
                 }
-                Aqk[r * C + i] = da.x + da.y;
+                Aqk[r * C + i] = (i <= r) ? a2.x + a2.y : 0.f;
             }
             const float dz = dUs[r * kVT + lane];
             db = fmaf(dz, Xs[r * kVT + lane], db);
