@@ -560,139 +560,183 @@ chunk_bwd_kernel(BwdParams p) {
         // ---- 8. per (r, c): dq, dk (atomics) and dG (registers) --------------
         float dG[kElemsPerThread];
         if (kAnchored) {
-            // Thread (tile R, channel c): rows r = 16R + a, a < 16.  Pairwise sums
-            // with tile anchors P_J = G at the row before tile J (0 for J = 0):
+            // Thread (tile R, 8-row half h, channels c and c + 64): rows
+            // r = 16R + 8h + a, a < 8, so every row of dA, dP, dO, dZ and U read
+            // by a warp serves two channels.  Pairwise sums with tile anchors
+            // P_J = G at the row before tile J (0 for J = 0):
             //   aq_r = 2^(G_r - P_R) sum_{i <= r} dA[r][i] k_i 2^(P_R - G_i)
             //   ak_r = sum_{J >= R} 2^(P_J - G_r) sum_{rr in J, rr >= r} dA[rr][r] q_rr 2^(G_rr - P_J)
             // (pr, pc likewise with dP and k).  Entries of dA / dP above the
-            // diagonal are zero, so the sums run over whole tiles.
-            const int R = tid >> 7, c = tid & 127, r0 = 16 * R;
+            // diagonal are zero, so the sums run over whole tiles.  dG[8 ch + a].
+            const int R = tid >> 7, hh = (tid >> 6) & 1, cl = tid & 63, r0 = 16 * R, ra = r0 + 8 * hh;
             const int ntile = (Cc + 15) >> 4;
-            float dq[16], dk[16];
-            float dl = 0.f;                          // this thread's share of dlast[c]
-            if (R >= ntile) {
+            float dq[2][8], dk[2][8];
+            float dl[2] = {0.f, 0.f};                // this thread's shares of dlast[c]
+            if (R >= ntile || ra >= Cc) {
 #pragma unroll
-                for (int a = 0; a < 16; ++a) dG[a] = 0.f;
+                for (int n = 0; n < 16; ++n) dG[n] = 0.f;
             } else {
-                const float PR = R == 0 ? 0.f : Gs[(r0 - 1) * L + c];
-                {
-                    // column pairs (i, i + 1) in one packed FMA per row
-                    float2 sa[16], sp[16];
+                float PR[2];
 #pragma unroll
-                    for (int a = 0; a < 16; ++a) sa[a] = sp[a] = make_float2(0.f, 0.f);
+                for (int ch = 0; ch < 2; ++ch) PR[ch] = R == 0 ? 0.f : Gs[(r0 - 1) * L + cl + 64 * ch];
+                {
+                    // column pairs (i, i + 1) in one packed FMA per row and channel
+                    float2 sa[2][8], sp[2][8];
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int a = 0; a < 8; ++a) sa[ch][a] = sp[ch][a] = make_float2(0.f, 0.f);
                     const int iend = min(r0 + 16, Cc);
                     int i = 0;
                     for (; i + 1 < iend; i += 2) {
-                        const float2 kc = make_float2(Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]),
-                                                      Ks[(i + 1) * L + c] * ex2f_(PR - Gs[(i + 1) * L + c]));
+                        float2 kc[2];
 #pragma unroll
-                        for (int a = 0; a < 16; ++a) {
-                            sa[a] = __ffma2_rn(*reinterpret_cast<const float2 *>(Aqk + (r0 + a) * C + i), kc, sa[a]);
-                            sp[a] = __ffma2_rn(*reinterpret_cast<const float2 *>(Pkk + (r0 + a) * C + i), kc, sp[a]);
+                        for (int ch = 0; ch < 2; ++ch) {
+                            const int c = cl + 64 * ch;
+                            kc[ch] = make_float2(Ks[i * L + c] * ex2f_(PR[ch] - Gs[i * L + c]),
+                                                 Ks[(i + 1) * L + c] * ex2f_(PR[ch] - Gs[(i + 1) * L + c]));
+                        }
+#pragma unroll
+                        for (int a = 0; a < 8; ++a) {
+                            const float2 av = *reinterpret_cast<const float2 *>(Aqk + (ra + a) * C + i);
+                            const float2 pv = *reinterpret_cast<const float2 *>(Pkk + (ra + a) * C + i);
+#pragma unroll
+                            for (int ch = 0; ch < 2; ++ch) {
+                                sa[ch][a] = __ffma2_rn(av, kc[ch], sa[ch][a]);
+                                sp[ch][a] = __ffma2_rn(pv, kc[ch], sp[ch][a]);
+                            }
                         }
                     }
                     if (i < iend) {                  // an odd last column
-                        const float kc = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
 #pragma unroll
-                        for (int a = 0; a < 16; ++a) {
-                            sa[a].x = fmaf(Aqk[(r0 + a) * C + i], kc, sa[a].x);
-                            sp[a].x = fmaf(Pkk[(r0 + a) * C + i], kc, sp[a].x);
+                        for (int ch = 0; ch < 2; ++ch) {
+                            const int c = cl + 64 * ch;
+                            const float kc = Ks[i * L + c] * ex2f_(PR[ch] - Gs[i * L + c]);
+#pragma unroll
+                            for (int a = 0; a < 8; ++a) {
+                                sa[ch][a].x = fmaf(Aqk[(ra + a) * C + i], kc, sa[ch][a].x);
+                                sp[ch][a].x = fmaf(Pkk[(ra + a) * C + i], kc, sp[ch][a].x);
+                            }
                         }
                     }
 #pragma unroll
-                    for (int a = 0; a < 16; ++a) {
-                        dq[a] = dk[a] = dG[a] = 0.f;
-                        if (r0 + a >= Cc) continue;
-                        const int r = r0 + a;
-                        const float fr = ex2f_(Gs[r * L + c] - PR);
-                        const float aq = fr * (sa[a].x + sa[a].y), pr = fr * (sp[a].x + sp[a].y);
-                        dq[a] = aq;
-                        dk[a] = pr;
-                        dG[a] = Qs[r * L + c] * aq + Ks[r * L + c] * pr;
-                    }
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int a = 0; a < 8; ++a) {
+                            const int c = cl + 64 * ch, r = ra + a, n = 8 * ch + a;
+                            dq[ch][a] = dk[ch][a] = dG[n] = 0.f;
+                            if (r >= Cc) continue;
+                            const float fr = ex2f_(Gs[r * L + c] - PR[ch]);
+                            const float aq = fr * (sa[ch][a].x + sa[ch][a].y), pr = fr * (sp[ch][a].x + sp[ch][a].y);
+                            dq[ch][a] = aq;
+                            dk[ch][a] = pr;
+                            dG[n] = Qs[r * L + c] * aq + Ks[r * L + c] * pr;
+                        }
                 }
                 for (int J = R; J < ntile; ++J) {
-                    const float PJ = J == 0 ? 0.f : Gs[(16 * J - 1) * L + c];
-                    // rows (2m, 2m + 1) of ak + pc in one packed FMA
-                    float2 s2[8];
+                    float PJ[2];
 #pragma unroll
-                    for (int m = 0; m < 8; ++m) s2[m] = make_float2(0.f, 0.f);
+                    for (int ch = 0; ch < 2; ++ch) PJ[ch] = J == 0 ? 0.f : Gs[(16 * J - 1) * L + cl + 64 * ch];
+                    // rows (2m, 2m + 1) of ak + pc in one packed FMA, per channel
+                    float2 s2[2][4];
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) s2[ch][m] = make_float2(0.f, 0.f);
                     const int rend = min(16 * J + 16, Cc);
                     for (int rr = 16 * J; rr < rend; ++rr) {
-                        const float e = ex2f_(Gs[rr * L + c] - PJ);
-                        const float qe = Qs[rr * L + c] * e, ke = Ks[rr * L + c] * e;
-                        const float2 qe2 = make_float2(qe, qe), ke2 = make_float2(ke, ke);
-                        const float4 *arow = reinterpret_cast<const float4 *>(Aqk + rr * C + r0);
-                        const float4 *prow = reinterpret_cast<const float4 *>(Pkk + rr * C + r0);
+                        const float4 *arow = reinterpret_cast<const float4 *>(Aqk + rr * C + ra);
+                        const float4 *prow = reinterpret_cast<const float4 *>(Pkk + rr * C + ra);
+                        const float4 a0 = arow[0], a1 = arow[1], p0 = prow[0], p1 = prow[1];
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const float4 av = arow[q4], pv = prow[q4];
-                            s2[2 * q4] = __ffma2_rn(make_float2(av.x, av.y), qe2, s2[2 * q4]);
-                            s2[2 * q4 + 1] = __ffma2_rn(make_float2(av.z, av.w), qe2, s2[2 * q4 + 1]);
-                            s2[2 * q4] = __ffma2_rn(make_float2(pv.x, pv.y), ke2, s2[2 * q4]);
-                            s2[2 * q4 + 1] = __ffma2_rn(make_float2(pv.z, pv.w), ke2, s2[2 * q4 + 1]);
+                        for (int ch = 0; ch < 2; ++ch) {
+                            const int c = cl + 64 * ch;
+                            const float e = ex2f_(Gs[rr * L + c] - PJ[ch]);
+                            const float qe = Qs[rr * L + c] * e, ke = Ks[rr * L + c] * e;
+                            const float2 qe2 = make_float2(qe, qe), ke2 = make_float2(ke, ke);
+                            s2[ch][0] = __ffma2_rn(make_float2(a0.x, a0.y), qe2, s2[ch][0]);
+                            s2[ch][1] = __ffma2_rn(make_float2(a0.z, a0.w), qe2, s2[ch][1]);
+                            s2[ch][2] = __ffma2_rn(make_float2(a1.x, a1.y), qe2, s2[ch][2]);
+                            s2[ch][3] = __ffma2_rn(make_float2(a1.z, a1.w), qe2, s2[ch][3]);
+                            s2[ch][0] = __ffma2_rn(make_float2(p0.x, p0.y), ke2, s2[ch][0]);
+                            s2[ch][1] = __ffma2_rn(make_float2(p0.z, p0.w), ke2, s2[ch][1]);
+                            s2[ch][2] = __ffma2_rn(make_float2(p1.x, p1.y), ke2, s2[ch][2]);
+                            s2[ch][3] = __ffma2_rn(make_float2(p1.z, p1.w), ke2, s2[ch][3]);
                         }
                     }
 #pragma unroll
-                    for (int a = 0; a < 16; ++a) {
-                        if (r0 + a >= Cc) continue;
-                        const int r = r0 + a;
-                        const float f = ex2f_(PJ - Gs[r * L + c]);
-                        const float akpc = f * ((a & 1) ? s2[a >> 1].y : s2[a >> 1].x);     // ak + pc
-                        dk[a] += akpc;
-                        dG[a] -= Ks[r * L + c] * akpc;
-                    }
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int a = 0; a < 8; ++a) {
+                            const int c = cl + 64 * ch, r = ra + a;
+                            if (r >= Cc) continue;
+                            const float f = ex2f_(PJ[ch] - Gs[r * L + c]);
+                            const float akpc = f * ((a & 1) ? s2[ch][a >> 1].y : s2[ch][a >> 1].x);   // ak + pc
+                            dk[ch][a] += akpc;
+                            dG[8 * ch + a] -= Ks[r * L + c] * akpc;
+                        }
                 }
                 // elementwise factors: dQg = dO S^T, dKw = -dX S^T, dKd = U dS'^T,
-                // four rows at a time: the value columns j .. j+3 of a row are
-                // one broadcast float4, the column of S one conflict-free load
-                // per j; (even j, odd j) in one packed FMA
+                // four rows at a time: the value columns j .. j+3 of a row are one
+                // broadcast float4 serving both channels; the two channels' S and
+                // dS' entries are one conflict-free load each
 #pragma unroll
-                for (int hb = 0; hb < 4; ++hb) {
-                    float2 dqg[4], dkw[4], dkd[4];
+                for (int hb = 0; hb < 2; ++hb) {
+                    float dqg[2][4], dkw[2][4], dkd[2][4];
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) dqg[a] = dkw[a] = dkd[a] = make_float2(0.f, 0.f);
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) dqg[ch][a] = dkw[ch][a] = dkd[ch][a] = 0.f;
                     for (int j = 0; j < kVT; j += 4) {
-                        const float2 s01 = make_float2(Ss[j * SL + c], Ss[(j + 1) * SL + c]);
-                        const float2 s23 = make_float2(Ss[(j + 2) * SL + c], Ss[(j + 3) * SL + c]);
-                        const float2 d01 = make_float2(dSs[j * SL + c], dSs[(j + 1) * SL + c]);
-                        const float2 d23 = make_float2(dSs[(j + 2) * SL + c], dSs[(j + 3) * SL + c]);
+                        float sv[2][4], dv[2][4];
+#pragma unroll
+                        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                sv[ch][u] = Ss[(j + u) * SL + cl + 64 * ch];
+                                dv[ch][u] = dSs[(j + u) * SL + cl + 64 * ch];
+                            }
 #pragma unroll
                         for (int a = 0; a < 4; ++a) {
-                            const int r = r0 + 4 * hb + a;
+                            const int r = ra + 4 * hb + a;
                             const float4 o4 = *reinterpret_cast<const float4 *>(dOs + r * kVT + j);
                             const float4 u4 = *reinterpret_cast<const float4 *>(dUs + r * kVT + j);
                             const float4 v4 = *reinterpret_cast<const float4 *>(Us + r * kVT + j);
-                            dqg[a] = __ffma2_rn(make_float2(o4.x, o4.y), s01, dqg[a]);
-                            dqg[a] = __ffma2_rn(make_float2(o4.z, o4.w), s23, dqg[a]);
-                            dkw[a] = __ffma2_rn(make_float2(u4.x, u4.y), s01, dkw[a]);
-                            dkw[a] = __ffma2_rn(make_float2(u4.z, u4.w), s23, dkw[a]);
-                            dkd[a] = __ffma2_rn(make_float2(v4.x, v4.y), d01, dkd[a]);
-                            dkd[a] = __ffma2_rn(make_float2(v4.z, v4.w), d23, dkd[a]);
+#pragma unroll
+                            for (int ch = 0; ch < 2; ++ch) {
+                                dqg[ch][a] = fmaf(o4.x, sv[ch][0], fmaf(o4.y, sv[ch][1], fmaf(o4.z, sv[ch][2], fmaf(o4.w, sv[ch][3], dqg[ch][a]))));
+                                dkw[ch][a] = fmaf(u4.x, sv[ch][0], fmaf(u4.y, sv[ch][1], fmaf(u4.z, sv[ch][2], fmaf(u4.w, sv[ch][3], dkw[ch][a]))));
+                                dkd[ch][a] = fmaf(v4.x, dv[ch][0], fmaf(v4.y, dv[ch][1], fmaf(v4.z, dv[ch][2], fmaf(v4.w, dv[ch][3], dkd[ch][a]))));
+                            }
                         }
                     }
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
-                        const int aa = 4 * hb + a, r = r0 + aa;
-                        if (r >= Cc) continue;
-                        const float grc = Gs[r * L + c], qrc = Qs[r * L + c], krc = Ks[r * L + c];
-                        const float vqg = dqg[a].x + dqg[a].y, vkd = dkd[a].x + dkd[a].y;
-                        const float kw = -bet[r] * (dkw[a].x + dkw[a].y);
-                        const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
-                        dq[aa] = fmaf(eg, vqg, dq[aa]);
-                        dk[aa] += eg * kw + ed * vkd;
-                        dG[aa] += eg * (vqg * qrc + kw * krc) - ed * vkd * krc;
-                        dl = fmaf(ed * vkd, krc, dl);
-                    }
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const int aa = 4 * hb + a, r = ra + aa, c = cl + 64 * ch;
+                            if (r >= Cc) continue;
+                            const float grc = Gs[r * L + c], qrc = Qs[r * L + c], krc = Ks[r * L + c];
+                            const float vqg = dqg[ch][a], vkd = dkd[ch][a];
+                            const float kw = -bet[r] * dkw[ch][a];
+                            const float eg = ex2f_(grc), ed = ex2f_(Glast[c] - grc);
+                            dq[ch][aa] = fmaf(eg, vqg, dq[ch][aa]);
+                            dk[ch][aa] += eg * kw + ed * vkd;
+                            dG[8 * ch + aa] += eg * (vqg * qrc + kw * krc) - ed * vkd * krc;
+                            dl[ch] = fmaf(ed * vkd, krc, dl[ch]);
+                        }
                 }
 #pragma unroll
-                for (int a = 0; a < 16; ++a) {
-                    if (r0 + a >= Cc) continue;
-                    const size_t tq = ((tok0 + r0 + a) * p.H + h) * Dk + c;
-                    atomicAdd(&p.dq[tq], dq[a]);
-                    atomicAdd(&p.dk[tq], dk[a]);
+                for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+                    for (int a = 0; a < 8; ++a) {
+                        if (ra + a >= Cc) continue;
+                        const size_t tq = ((tok0 + ra + a) * p.H + h) * Dk + cl + 64 * ch;
+                        atomicAdd(&p.dq[tq], dq[ch][a]);
+                        atomicAdd(&p.dk[tq], dk[ch][a]);
+                    }
+                    atomicAdd(&dlast[cl + 64 * ch], dl[ch]);
                 }
-                atomicAdd(&dlast[c], dl);
             }
         } else {
 #pragma unroll
@@ -788,10 +832,12 @@ chunk_bwd_kernel(BwdParams p) {
         }
         __syncthreads();
         if (kAnchored) {
-            const int R = tid >> 7, c = tid & 127;
+            const int ra = 16 * (tid >> 7) + 8 * ((tid >> 6) & 1), cl = tid & 63;
 #pragma unroll
-            for (int a = 0; a < 16; ++a)
-                if (16 * R + a < Cc) Gs[(16 * R + a) * L + c] = dG[a];
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    if (ra + a < Cc) Gs[(ra + a) * L + cl + 64 * ch] = dG[8 * ch + a];
         } else {
 #pragma unroll
             for (int n = 0; n < kElemsPerThread; ++n) {
