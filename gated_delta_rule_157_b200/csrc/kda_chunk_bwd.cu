@@ -42,11 +42,12 @@ static_assert(kThreads == 4 * 128, "the dS step maps a thread to (key channel, e
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
 constexpr int kLoadBatch = 8;                 // global loads in flight per thread in the chunk load
 
-// kAnchored (Dk = 128, C = 64, the bounded gate with |g_min| <= 5): step 8's
-// pairwise sums use the forward's 16-token tile anchors, so every factor
-// 2^(G_r - G_i) is a product of one per-row and one per-column power, each in
-// [2^-116, 2^116] (16 tokens x 5 x log2 e); otherwise every pair takes its own
-// power of a non-positive difference (any gate).
+// kAnchored (Dk = 128, C = 64, the bounded gate with |g_min| <= 5): the
+// pairwise sums A and P (step 3) and their gradients (step 8) use the
+// forward's 16-token tile anchors, so every factor 2^(G_r - G_i) is a product
+// of one per-row and one per-column power, each in [2^-116, 2^116] (16 tokens
+// x 5 x log2 e); otherwise every pair takes its own power of a non-positive
+// difference (any gate).
 template <typename Tin, bool kAnchored>
 __global__ void __launch_bounds__(kThreads)
 chunk_bwd_kernel(BwdParams p) {
@@ -989,12 +990,14 @@ __global__ void bwd_empty_kernel(BwdParams p) {
 
 }  // namespace
 
-// The anchored pairwise sums of step 8 need 128 key channels (one thread per
-// channel and 16-row tile), 64-token chunks and a decay of at most 5 per token.
+// The anchored instance needs 128 key channels (thread layouts by channel),
+// 64-token chunks and a decay of at most 5 per token (the anchors' bound).
 inline bool bwd_anchored(const BwdParams &p) {
     return p.Dk == 128 && p.C == 64 && p.gate_in == 1 && p.g_min >= -5.0f;
 }
 
+// Dynamic shared memory of chunk_bwd_kernel (both instances use one layout;
+// the anchored one also reuses the A/P/X/U tiles as its staging area).
 size_t bwd_smem_bytes(int C, int Dk, bool anchored) {
     const size_t CL = ((size_t)C * (Dk | 1) + 3) & ~(size_t)3, CC = ((size_t)C * C + 3) & ~(size_t)3;
     const size_t Dk4 = ((size_t)Dk + 3) & ~(size_t)3;
