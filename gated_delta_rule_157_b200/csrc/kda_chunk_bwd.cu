@@ -350,6 +350,44 @@ chunk_bwd_kernel(BwdParams p) {
                 Pkk[r * C + i] = pk;
             }
         }
+        if (kAnchored) {
+            __syncthreads();                   // the quarter sums were read from the U and dU tiles
+            // warp w takes rows w, w + 16, w + 32, w + 48 (their factor rows in
+            // its scratch row and in its rows of the U and dU tiles, free until
+            // step 4); lane = value column: one load of S^T per lane and four
+            // channels serves all four rows
+            float *wr[4] = {wb, wb + 128, Us + warp * 128, dUs + warp * 128};
+            int rs[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rs[q] = warp + 16 * q < Cc ? warp + 16 * q : warp;
+            if (warp < Cc) {
+                for (int c = lane; c < Dk; c += 32) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) wr[q][c] = -Ks[rs[q] * L + c] * ex2f_(Gs[rs[q] * L + c]);
+                }
+                __syncwarp();
+                float2 acc[4][2];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[q][0] = make_float2(Xs[rs[q] * kVT + lane], 0.f);
+                    acc[q][1] = make_float2(0.f, 0.f);
+                }
+                const float *srow = Ss + lane * SL;
+                for (int c = 0; c < Dk; c += 4) {
+                    const float4 s4 = *reinterpret_cast<const float4 *>(srow + c);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 w4 = *reinterpret_cast<const float4 *>(wr[q] + c);
+                        acc[q][0] = __ffma2_rn(make_float2(w4.x, w4.y), make_float2(s4.x, s4.y), acc[q][0]);
+                        acc[q][1] = __ffma2_rn(make_float2(w4.z, w4.w), make_float2(s4.z, s4.w), acc[q][1]);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (warp + 16 * q < Cc)
+                        Xs[rs[q] * kVT + lane] = (acc[q][0].x + acc[q][0].y) + (acc[q][1].x + acc[q][1].y);
+            }
+        } else
         // warp w takes the row pairs (r, r + 16), r = w, w + 32, ...; lane = value
         // column (one load of S^T per lane and four channels for both rows);
         // channel pairs (c, c + 1) in one packed FMA
