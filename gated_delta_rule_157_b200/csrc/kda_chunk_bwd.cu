@@ -30,6 +30,7 @@
 // sums over the key channels).  A second pair of kernels takes them through
 // the in-kernel L2 norm, beta sigmoid and gate (bounded or softplus).
 #include "kda_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace kda {
 namespace {
@@ -41,6 +42,21 @@ static_assert(kVT == 32, "the row loops map one lane to one value column");
 static_assert(kThreads == 4 * 128, "the dS step maps a thread to (key channel, eight value columns)");
 constexpr int kElemsPerThread = 64 * 128 / kThreads;   // (r, c) elements of a chunk per thread
 constexpr int kLoadBatch = 8;                 // global loads in flight per thread in the chunk load
+
+// fp32 product on the tensor cores at fp32-level accuracy: each operand split
+// into a tf32 head and a tf32 tail (x = hi + lo, both exact in tf32 up to the
+// tail's rounding), and D += A_lo B_hi + A_hi B_lo + A_hi B_hi (the lo x lo
+// term is below fp32 resolution).
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    hi = tc::to_tf32(x);
+    lo = tc::to_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma3_tf32(float d[4], const uint32_t ah[4], const uint32_t al[4], const uint32_t bh[2],
+                                          const uint32_t bl[2]) {
+    tc::mma_tf32_16x8x8(d, al, bh);
+    tc::mma_tf32_16x8x8(d, ah, bl);
+    tc::mma_tf32_16x8x8(d, ah, bh);
+}
 
 // kAnchored (Dk = 128, C = 64, the bounded gate with |g_min| <= 5): the
 // pairwise sums A and P (step 3) and their gradients (step 8) use the
@@ -241,9 +257,9 @@ chunk_bwd_kernel(BwdParams p) {
             // half-block w over all channels and a quarter of the channels of
             // half-block 16 + w % 4 (summed below), 20 eight-channel steps per
             // warp; it stages its own factors in its scratch row (no CTA
-            // barrier): [8 ch][8 rows] of q and k, [8 ch][16 columns]; lane =
-            // (row lane / 4, columns 4 (lane % 4) .. +3).  The quarter sums go
-            // to the U and dU tiles, free until step 4.
+            // barrier): [8 ch][8 rows] of q and k, [8 ch][16 columns], and
+            // multiplies them on the tensor cores.  The quarter sums go to the
+            // U and dU tiles, free until step 4.
             const int ntile = (Cc + 15) >> 4;
             float *Qw = wb, *Kw = wb + 64, *Kcw = wb + 128;
 #pragma unroll 1
@@ -255,8 +271,12 @@ chunk_bwd_kernel(BwdParams p) {
                 while (blk >= (R + 1) * (R + 2) / 2) ++R;
                 const int J = blk - R * (R + 1) / 2, rw0 = 16 * R + 8 * (hbi & 1);
                 if (R >= ntile) continue;
-                float2 sa[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, sp[2] = {sa[0], sa[1]};
-                const int rl = lane >> 2, i4 = 4 * (lane & 3);
+                // the block product transposed, D[i][r] = sum_c Khat[i][c] Q~[r][c]
+                // (M = 16 columns, N = 8 rows, K = 8 channels per step) on the
+                // tensor cores; lane (g, t) = (lane / 4, lane % 4) holds
+                // D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]
+                float dA[4] = {0.f, 0.f, 0.f, 0.f}, dP[4] = {0.f, 0.f, 0.f, 0.f};
+                const int g8 = lane >> 2, t4 = lane & 3;
                 for (int c0 = cbeg; c0 < cend; c0 += 8) {
                     // rows: (cc = e & 7, row e >> 3), two per lane; columns: four per lane
 #pragma unroll
@@ -274,37 +294,36 @@ chunk_bwd_kernel(BwdParams p) {
                         Kcw[cc * 16 + (e & 15)] = Ks[i * L + c] * ex2f_(PR - Gs[i * L + c]);
                     }
                     __syncwarp();
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        const float qa = Qw[cc * 8 + rl], ka = Kw[cc * 8 + rl];
-                        const float4 kc = *reinterpret_cast<const float4 *>(Kcw + cc * 16 + i4);
-                        const float2 qa2 = make_float2(qa, qa), ka2 = make_float2(ka, ka);
-                        sa[0] = __ffma2_rn(qa2, make_float2(kc.x, kc.y), sa[0]);
-                        sa[1] = __ffma2_rn(qa2, make_float2(kc.z, kc.w), sa[1]);
-                        sp[0] = __ffma2_rn(ka2, make_float2(kc.x, kc.y), sp[0]);
-                        sp[1] = __ffma2_rn(ka2, make_float2(kc.z, kc.w), sp[1]);
+                    {
+                        uint32_t ah[4], al[4], bh[2], bl[2];
+                        split_tf32(Kcw[t4 * 16 + g8], ah[0], al[0]);
+                        split_tf32(Kcw[t4 * 16 + g8 + 8], ah[1], al[1]);
+                        split_tf32(Kcw[(t4 + 4) * 16 + g8], ah[2], al[2]);
+                        split_tf32(Kcw[(t4 + 4) * 16 + g8 + 8], ah[3], al[3]);
+                        split_tf32(Qw[t4 * 8 + g8], bh[0], bl[0]);
+                        split_tf32(Qw[(t4 + 4) * 8 + g8], bh[1], bl[1]);
+                        mma3_tf32(dA, ah, al, bh, bl);
+                        split_tf32(Kw[t4 * 8 + g8], bh[0], bl[0]);
+                        split_tf32(Kw[(t4 + 4) * 8 + g8], bh[1], bl[1]);
+                        mma3_tf32(dP, ah, al, bh, bl);
                     }
                     __syncwarp();
                 }
                 if (t == 1) {                       // a quarter sum: [quarter][half-block][lane][8]
                     const int q = warp >> 2;
                     float *part = (q < 2 ? Us + q * 1024 : dUs + (q - 2) * 1024) + ((hbi - 16) * 32 + lane) * 8;
-                    *reinterpret_cast<float4 *>(part) = make_float4(sa[0].x, sa[0].y, sa[1].x, sa[1].y);
-                    *reinterpret_cast<float4 *>(part + 4) = make_float4(sp[0].x, sp[0].y, sp[1].x, sp[1].y);
+                    *reinterpret_cast<float4 *>(part) = make_float4(dA[0], dA[1], dA[2], dA[3]);
+                    *reinterpret_cast<float4 *>(part + 4) = make_float4(dP[0], dP[1], dP[2], dP[3]);
                     continue;
                 }
-                // stores: A lower with the diagonal, P strictly lower, zeros above
-                const int r = rw0 + rl;
-                if (r < Cc) {
-                    const float av[4] = {sa[0].x, sa[0].y, sa[1].x, sa[1].y};
-                    const float pv[4] = {sp[0].x, sp[0].y, sp[1].x, sp[1].y};
+                // stores: A lower with the diagonal, P strictly lower, zeros above;
+                // value v of the lane is row rw0 + 2t + (v & 1), column 16J + g + 8 (v >> 1)
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = 16 * J + i4 + u;
-                        if (i >= Cc) continue;
-                        Aqk[r * C + i] = i <= r ? av[u] : 0.f;
-                        Pkk[r * C + i] = i < r ? pv[u] : 0.f;
-                    }
+                for (int v = 0; v < 4; ++v) {
+                    const int r = rw0 + 2 * t4 + (v & 1), i = 16 * J + g8 + 8 * (v >> 1);
+                    if (r >= Cc || i >= Cc) continue;
+                    Aqk[r * C + i] = i <= r ? dA[v] : 0.f;
+                    Pkk[r * C + i] = i < r ? dP[v] : 0.f;
                 }
             }
             // the blocks above the diagonal tiles
@@ -324,8 +343,8 @@ chunk_bwd_kernel(BwdParams p) {
                     const int idx = tid + kThreads * m;
                     const float v = (Us[idx] + Us[1024 + idx]) + (dUs[idx] + dUs[1024 + idx]);
                     const int hbi = 16 + (idx >> 8), ln = (idx >> 3) & 31, u = idx & 3;
-                    const int r = 48 + 8 * (hbi & 1) + (ln >> 2);
-                    const int i = 16 * ((hbi >> 1) - 6) + 4 * (ln & 3) + u;
+                    const int r = 48 + 8 * (hbi & 1) + 2 * (ln & 3) + (u & 1);
+                    const int i = 16 * ((hbi >> 1) - 6) + (ln >> 2) + 8 * (u >> 1);
                     if (r < Cc && i < Cc) {
                         if ((idx & 4) == 0) Aqk[r * C + i] = i <= r ? v : 0.f;
                         else Pkk[r * C + i] = i < r ? v : 0.f;
