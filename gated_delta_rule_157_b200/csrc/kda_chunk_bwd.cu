@@ -482,9 +482,21 @@ chunk_bwd_kernel(BwdParams p) {
                 for (int idx = tid; idx < (Cc - R1) * kVT; idx += kThreads) {
                     const int r = R1 + idx / kVT, jj = idx % kVT;
                     float acc = Us[r * kVT + jj];
+                    if ((C & 3) == 0 && R1 == R0 + 16) {     // the row of P as four float4s
+                        const float4 *prow = reinterpret_cast<const float4 *>(Pkk + r * C + R0);
 #pragma unroll
-                    for (int a = 0; a < 16; ++a)
-                        if (R0 + a < R1) acc = fmaf(-Pkk[r * C + R0 + a], Us[(R0 + a) * kVT + jj], acc);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const float4 pv = prow[q4];
+                            acc = fmaf(-pv.x, Us[(R0 + 4 * q4) * kVT + jj], acc);
+                            acc = fmaf(-pv.y, Us[(R0 + 4 * q4 + 1) * kVT + jj], acc);
+                            acc = fmaf(-pv.z, Us[(R0 + 4 * q4 + 2) * kVT + jj], acc);
+                            acc = fmaf(-pv.w, Us[(R0 + 4 * q4 + 3) * kVT + jj], acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int a = 0; a < 16; ++a)
+                            if (R0 + a < R1) acc = fmaf(-Pkk[r * C + R0 + a], Us[(R0 + a) * kVT + jj], acc);
+                    }
                     Us[r * kVT + jj] = acc;
                 }
                 __syncthreads();
