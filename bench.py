@@ -664,7 +664,8 @@ def bench_train(args, kda, workloads, dev, stream, world, rank):
         kda.kda_chunk_bwd(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S_ch, dout, None,
                           A_log=inp["A_log"], dt_bias=inp["dt_bias"], chunk=w.chunk, stream=stream)
 
-    out = {"workload": "gva_bf16 B=%d: forward with chunk states (algo %s) + backward (SIMT)" % (w.B, args.algo),
+    out = {"workload": "gva_bf16 B=%d: forward with chunk states (algo %s) + backward (fp32; A/P products "
+                       "on the tensor cores, the rest on the CUDA cores)" % (w.B, args.algo),
            "launches": 0}
     # kernels per call: the forward is one launch; the backward three (chunk
     # kernel, L2-norm and gate/parameter passes) after the output zeroing
